@@ -1,0 +1,407 @@
+/*
+ * fp4_oracle.c — plain, slow CPU definition of block-scaled 4-bit microscaling.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the bench's CPU-baseline leg may call
+ * this code.  It shares nothing with the CUDA library: no headers, tables or helpers.  Every
+ * encoder here works by enumerating its lattice (the audit page advises enumerating the lattice
+ * rather than re-deriving a bit trick), and every floating-point step is a single IEEE fp32 (or
+ * exact fp64) operation written out in the order the definition gives.  Build with
+ * -O2 -ffp-contract=off and without fast-math so that no operation is fused or reassociated.
+ *
+ * Sources (page title and section):
+ *   [E] "Sub-4-Bit Microscaling (NVFP4, MXFP4 & Walsh-Hadamard Rotation)", §1-§3.
+ *   [A] "MXFP4 Quantization: Audit the 4.25-Bit Blocks".
+ *   [X] metrale `hardware::exec` docs (E2M1 -> E4M3 conversion).
+ *   [P] "Adaptive Block-Scaled Data Types for FP4 Training" podcast (block scaling, stochastic
+ *       rounding, Hadamard transform, Four Over Six).
+ *   Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3",
+ *       SC'11, §4 (the Philox round function and key schedule).
+ *
+ * Readings where the pages are silent are listed beside each function.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+typedef struct {
+  uint64_t underflow, saturation, nonfinite, blocks_four;
+} ora_counts;
+
+/* ------------------------------------------------------------------------------------------ */
+/* E2M1 element.  [E] §1: 1 sign, 2 exponent, 1 mantissa bit, exponent bias 1, no Inf/NaN.
+ * [A] "Read the FP4 E2M1 value lattice": exponent field 0 is subnormal (0 and 0.5).           */
+
+double ora_e2m1_value(int code) {
+  int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return s ? -mag : mag;
+}
+
+/* Nearest lattice magnitude code (0..7) for a >= 0, a <= 6.  Exact ties take the code whose
+ * mantissa bit is even ([A] "Read the FP4 E2M1 value lattice": ties-to-even on the lattice). */
+static int e2m1_nearest_mag(double a) {
+  int best = 0;
+  double bestd = INFINITY;
+  for (int c = 0; c < 8; ++c) {
+    double d = fabs(a - ora_e2m1_value(c));
+    if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+      best = c;
+      bestd = d;
+    }
+  }
+  return best;
+}
+
+/* RNE encode of a normalised value y.  Magnitudes strictly above 6 clamp to 6 ([A]: "the lab
+ * clamps them to signed 6").  The sign bit always follows signbit(y), so a negative value that
+ * rounds to zero encodes -0 (0x8).  Returns the 4-bit code. */
+int ora_e2m1_encode_rne(float y) {
+  double a = fabs((double)y);
+  int mag = (a > 6.0) ? 7 : e2m1_nearest_mag(a);
+  return (signbit(y) ? 8 : 0) | mag;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Philox4x32-10 (Salmon et al. SC'11).  Round: with multipliers M0, M1, the pair products
+ * (hi,lo) = M0*c0 and M1*c2 give (c0,c1,c2,c3) <- (hi(M1*c2)^c1^k0, lo(M1*c2), hi(M0*c0)^c3^k1,
+ * lo(M0*c0)); between rounds the key is bumped by the Weyl constants.                         */
+
+void ora_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+  uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+  uint32_t k0 = key_in[0], k1 = key_in[1];
+  for (int round = 0; round < 10; ++round) {
+    uint64_t p0 = (uint64_t)M0 * c0;
+    uint64_t p1 = (uint64_t)M1 * c2;
+    uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    uint32_t n1 = (uint32_t)p1;
+    uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    uint32_t n3 = (uint32_t)p0;
+    c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    k0 += W0;
+    k1 += W1;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* The 32-bit random word of flat element index idx: key = (seed lo, seed hi), counter =
+ * (idx/4 lo, idx/4 hi, 0, 0), word idx%4.  (Reading: the pages fix no mapping; this one keys
+ * Philox on (seed, element index) as the problem statement asks, one call per 4 elements.)   */
+uint32_t ora_sr_word(uint64_t seed, uint64_t idx) {
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint64_t blk = idx >> 2;
+  uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u};
+  uint32_t out[4];
+  ora_philox4x32_10(ctr, key, out);
+  return out[idx & 3];
+}
+
+/* Stochastic rounding of y onto the E2M1 lattice ([P]: round up or down with probability given by
+ * the distance, so the expectation is y).  For a = |y| <= 6 let lo <= a < hi be consecutive
+ * lattice magnitudes (lo = a when a is a lattice point); p = (a-lo)/(hi-lo) is exact; the value
+ * rounds up iff r < ceil(p * 2^32).  a > 6 clamps to 6 (saturation, as for RNE).             */
+int ora_e2m1_encode_sr(float y, uint32_t r) {
+  double a = fabs((double)y);
+  int sign = signbit(y) ? 8 : 0;
+  if (a > 6.0) return sign | 7;
+  int lo = 0;
+  for (int c = 0; c < 8; ++c)
+    if (ora_e2m1_value(c) <= a) lo = c;
+  if (lo == 7) return sign | 7; /* a == 6 exactly */
+  double vlo = ora_e2m1_value(lo), vhi = ora_e2m1_value(lo + 1);
+  double p = (a - vlo) / (vhi - vlo);
+  double thresh = ceil(ldexp(p, 32));
+  int up = (double)r < thresh;
+  return sign | (up ? lo + 1 : lo);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* FP8 E4M3 (OCP E4M3FN): 1 sign, 4 exponent (bias 7), 3 mantissa bits; exponent field 0 is
+ * subnormal; 0x7F/0xFF are NaN, so the largest finite magnitude is 448 (0x7E).  The NVFP4 block
+ * scale is a positive E4M3 value ([E] §2, [P] block-scaling segment).                          */
+
+double ora_e4m3_value(int code) {
+  int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  double mag = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+/* Round-to-nearest-even onto the positive E4M3 lattice, saturating to 448 (the "satfinite"
+ * reading: a magnitude above 448 becomes 448, never NaN).  u >= 0.  Ties take the even code.   */
+int ora_e4m3_encode_rne_satfinite(float u) {
+  double a = (double)u;
+  if (!(a <= 448.0)) return 0x7E;
+  int best = 0;
+  double bestd = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    double d = fabs(a - ora_e4m3_value(c));
+    if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+      best = c;
+      bestd = d;
+    }
+  }
+  return best;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* bf16 output rounding: round-to-nearest-even of an fp32 value to its top 16 bits.             */
+uint16_t ora_f32_to_bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x40);
+  uint32_t low = u & 0xFFFFu, hi = u >> 16;
+  if (low > 0x8000u || (low == 0x8000u && (hi & 1u))) hi += 1;
+  return (uint16_t)hi;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* MXFP4.  [A] "Read the shared E8M0 scale": block exponent from the block maximum, clamped to
+ * [-127, 127], byte = e + 127 (byte 0 for -127, 254 for 127, 0xFF never produced); all-zero block
+ * uses e = 0.  policy 0 (OCP floor): e = floor(log2(amax/4)) = floor(log2 amax) - 2, taken
+ * exactly from the binary exponent.  policy 1 (no saturation, [E] §2 sawtooth): the smallest e
+ * with amax <= 6 * 2^e.                                                                       */
+
+static int floor_log2(double a) { /* a > 0 finite: exact via frexp (a = f * 2^x, f in [.5,1)) */
+  int x;
+  frexp(a, &x);
+  return x - 1;
+}
+
+int ora_mx_exponent(float amax, int policy) {
+  if (amax == 0.0f) return 0;
+  double a = (double)amax;
+  int e;
+  if (policy == 0) {
+    e = floor_log2(a) - 2;
+  } else {
+    e = floor_log2(a) - 3; /* 8 * 2^(E-3) > a, so this is below the answer: step up */
+    while (!(a <= ldexp(6.0, e))) e += 1;
+  }
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+/* Encode one block with a given shared exponent e (the manual path of the audit page, and the
+ * inner step of ora_mx_quantize): y = x * 2^-e in fp32 (exact unless it underflows), then RNE
+ * or stochastic E2M1.  idx0 is the flat index of x[0] (for the random word).  Codes land in
+ * codes[0..n-1] (one per byte, unpacked). */
+void ora_mx_encode_block(const float* x, int n, int e, int round, uint64_t seed, uint64_t idx0,
+                         uint8_t* codes, ora_counts* cnt) {
+  float inv_scale = ldexpf(1.0f, -e);
+  for (int i = 0; i < n; ++i) {
+    if (!isfinite(x[i])) cnt->nonfinite += 1;
+    float y = x[i] * inv_scale;
+    int c = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
+    if (isfinite(y) && fabsf(y) > 6.0f) cnt->saturation += 1;
+    if (x[i] != 0.0f && (c & 7) == 0) cnt->underflow += 1;
+    codes[i] = (uint8_t)c;
+  }
+}
+
+static float block_amax(const float* x, int n) {
+  float m = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float a = fabsf(x[i]);
+    if (a > m) m = a;
+  }
+  return m;
+}
+
+/* Pack element 2j into the low nibble and 2j+1 into the high nibble of byte j
+ * ([A] "Encode one MXFP4 block step by step": values 0 and 1 occupy the low and high half of the
+ * first byte). */
+static void pack_pairs(const uint8_t* codes, int n, uint8_t* out) {
+  for (int j = 0; j < n / 2; ++j) out[j] = (uint8_t)((codes[2 * j] & 15) | ((codes[2 * j + 1] & 15) << 4));
+}
+
+/* x: [rows, cols] fp32 row-major; q: [rows, cols/2]; scales: [rows, cols/32] row-major bytes. */
+void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
+                     uint8_t* q, uint8_t* scales, ora_counts* cnt) {
+  const int B = 32;
+  long nb = cols / B;
+  uint8_t codes[32];
+  for (long r = 0; r < rows; ++r) {
+    for (long j = 0; j < nb; ++j) {
+      const float* xb = x + r * cols + j * B;
+      int e = ora_mx_exponent(block_amax(xb, B), policy);
+      scales[r * nb + j] = (uint8_t)(e + 127);
+      ora_mx_encode_block(xb, B, e, round, seed, (uint64_t)(r * cols + j * B), codes, cnt);
+      pack_pairs(codes, B, q + r * (cols / 2) + j * (B / 2));
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* NVFP4 two-level scaling.  [E] §2: an E4M3 scale per 16 elements under an FP32 per-tensor
+ * scale.  Reading (the pages fix the formats, not the rounding steps): s_g = fl(amax_t / (6*M))
+ * with M = 448 (M = 256 under four-over-six, see below), s_g = 1 for an all-zero tensor; for
+ * target T: inv_T = fl(1/fl(T*s_g)), block code = E4M3_RNE_satfinite(fl(amax_b * inv_T)), d its
+ * value; a zero code encodes the block as signed zeros; otherwise R = fl(1/fl(d*s_g)) and
+ * y_i = fl(x_i * R).
+ * Four over six ([P] Four Over Six segment): each block is encoded with T = 6 and with T = 4 and
+ * keeps T = 4 iff its fp32 sum of squared errors is strictly lower; the global scale uses M = 256
+ * ("shrinking the whole tensor's global scale", 1 - 256/448 = 42.9%, "nearly 43 percent"), which
+ * keeps the T = 4 code of the largest block (384) inside E4M3's range.                          */
+
+float ora_nvfp4_global_scale(float amax_t, int four_six) {
+  if (amax_t == 0.0f) return 1.0f;
+  float six_m = four_six ? 1536.0f : 2688.0f;
+  return amax_t / six_m;
+}
+
+/* One candidate encoding of a 16-block: returns the sum of squared dequantisation errors.     */
+static float nv_candidate(const float* x, int n, float amax_b, float s_g, float T, int round,
+                          uint64_t seed, uint64_t idx0, uint8_t* codes, int* scale_code,
+                          ora_counts* c) {
+  float ts = T * s_g;
+  float inv_t = 1.0f / ts;
+  float u = amax_b * inv_t;
+  int sc = ora_e4m3_encode_rne_satfinite(u);
+  float d = (float)ora_e4m3_value(sc);
+  *scale_code = sc;
+  memset(c, 0, sizeof(*c));
+  if (sc == 0) {
+    for (int i = 0; i < n; ++i) {
+      codes[i] = (uint8_t)(signbit(x[i]) ? 8 : 0);
+      if (x[i] != 0.0f) c->underflow += 1;
+    }
+  } else {
+    float ds = d * s_g;
+    float R = 1.0f / ds;
+    for (int i = 0; i < n; ++i) {
+      float y = x[i] * R;
+      int code = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
+      if (isfinite(y) && fabsf(y) > 6.0f) c->saturation += 1;
+      if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
+      codes[i] = (uint8_t)code;
+    }
+  }
+  float sse = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float vd = (float)(ora_e2m1_value(codes[i]) * (double)d); /* exact: <= 6 significant bits */
+    float xhat = vd * s_g;
+    float err = x[i] - xhat;
+    float sq = err * err;
+    sse = sse + sq;
+  }
+  return sse;
+}
+
+/* x: [rows, cols] fp32; q: [rows, cols/2]; scales: [rows, cols/16] row-major E4M3 bytes.
+ * global_in: NULL -> s_g from the tensor amax; else s_g = *global_in.                          */
+void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int four_six, uint64_t seed,
+                        const float* global_in, float* global_out, uint8_t* q, uint8_t* scales,
+                        ora_counts* cnt) {
+  const int B = 16;
+  long nb = cols / B;
+  float s_g;
+  if (global_in) {
+    s_g = *global_in;
+  } else {
+    float amax_t = 0.0f;
+    for (long i = 0; i < rows * cols; ++i) {
+      float a = fabsf(x[i]);
+      if (a > amax_t) amax_t = a;
+    }
+    s_g = ora_nvfp4_global_scale(amax_t, four_six);
+  }
+  if (global_out) *global_out = s_g;
+  uint8_t c6[16], c4[16];
+  for (long r = 0; r < rows; ++r) {
+    for (long j = 0; j < nb; ++j) {
+      const float* xb = x + r * cols + j * B;
+      uint64_t idx0 = (uint64_t)(r * cols + j * B);
+      for (int i = 0; i < B; ++i)
+        if (!isfinite(xb[i])) cnt->nonfinite += 1;
+      float amax_b = block_amax(xb, B);
+      ora_counts k6, k4;
+      int sc6, sc4;
+      float sse6 = nv_candidate(xb, B, amax_b, s_g, 6.0f, round, seed, idx0, c6, &sc6, &k6);
+      const uint8_t* pick = c6;
+      int sc = sc6;
+      ora_counts k = k6;
+      if (four_six) {
+        float sse4 = nv_candidate(xb, B, amax_b, s_g, 4.0f, round, seed, idx0, c4, &sc4, &k4);
+        if (sse4 < sse6) {
+          pick = c4;
+          sc = sc4;
+          k = k4;
+          cnt->blocks_four += 1;
+        }
+      }
+      cnt->underflow += k.underflow;
+      cnt->saturation += k.saturation;
+      scales[r * nb + j] = (uint8_t)sc;
+      pack_pairs(pick, B, q + r * (cols / 2) + j * (B / 2));
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Dequantisation ([A] "Encode one MXFP4 block step by step": reconstruction = lattice value times
+ * the block scale; [X]: block scales applied in FP32).  x_hat = fl(fl(v*d) * s_g) for NVFP4, where
+ * v*d is exact, and x_hat = v * 2^(byte-127) for MXFP4 (exact).  Row-major scales.            */
+void ora_dequantize(const uint8_t* q, const uint8_t* scales, int format, long rows, long cols,
+                    float s_g, float* out) {
+  int B = (format == 0) ? 32 : 16;
+  long nb = cols / B;
+  for (long r = 0; r < rows; ++r) {
+    for (long k = 0; k < cols; ++k) {
+      uint8_t byte = q[r * (cols / 2) + k / 2];
+      int code = (k & 1) ? (byte >> 4) : (byte & 15);
+      uint8_t sb = scales[r * nb + k / B];
+      double v = ora_e2m1_value(code);
+      if (format == 0) {
+        out[r * cols + k] = (float)ldexp(v, (int)sb - 127);
+      } else {
+        float vd = (float)(v * ora_e4m3_value(sb));
+        out[r * cols + k] = vd * s_g;
+      }
+    }
+  }
+}
+
+/* Exact fp64 dequantisation (for the GEMM reference): v * d * s_g with no rounding.            */
+void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, long rows, long cols,
+                        float s_g, double* out) {
+  int B = (format == 0) ? 32 : 16;
+  long nb = cols / B;
+  for (long r = 0; r < rows; ++r) {
+    for (long k = 0; k < cols; ++k) {
+      uint8_t byte = q[r * (cols / 2) + k / 2];
+      int code = (k & 1) ? (byte >> 4) : (byte & 15);
+      uint8_t sb = scales[r * nb + k / B];
+      double v = ora_e2m1_value(code);
+      out[r * cols + k] = (format == 0) ? ldexp(v, (int)sb - 127) : v * ora_e4m3_value(sb) * (double)s_g;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Normalised Walsh-Hadamard rotation of each row ([E] §3: H_d with entries +-1/sqrt(d), applied by
+ * O(d log2 d) add/subtract butterflies).  Reading: natural (Sylvester) order; fp32; the
+ * unnormalised stages run in the fixed order h = 1, 2, 4, ..., d/2, each mapping
+ * (x[i], x[i+h]) -> (x[i]+x[i+h], x[i]-x[i+h]) for (i & h) == 0; then each value is multiplied by
+ * c = fl(1/sqrt(d)).                                                                           */
+
+float ora_fwht_norm_const(long d) { return (float)(1.0L / sqrtl((long double)d)); }
+
+void ora_fwht_rows(const float* x, long rows, long d, float* y) {
+  float c = ora_fwht_norm_const(d);
+  for (long r = 0; r < rows; ++r) {
+    float* v = y + r * d;
+    memcpy(v, x + r * d, (size_t)d * sizeof(float));
+    for (long h = 1; h < d; h *= 2) {
+      for (long i = 0; i < d; ++i) {
+        if (i & h) continue;
+        float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+    for (long i = 0; i < d; ++i) v[i] = v[i] * c;
+  }
+}

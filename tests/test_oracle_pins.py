@@ -1,0 +1,425 @@
+"""Pins of the CPU oracle to facts the source pages and mathematics fix (no GPU).
+
+Each test checks the oracle against something other than itself: a worked example or number the
+pages print (fixtures under tests/golden/, each citing its page and section), a closed form, an
+invariant, or a special case that reduces to a library routine (torch's float8/bf16 casts, scipy's
+Hadamard matrix, numpy's fp64 matmul).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.conftest import golden_rows
+
+LATTICE = [float(v) for v in golden_rows("e2m1_lattice.txt")[0]]
+
+
+# ---------------------------------------------------------------------------------------------
+# E2M1
+
+def test_e2m1_decode_table_matches_printed_lattice():
+    for c in range(8):
+        assert O.e2m1_value(c) == LATTICE[c]
+        neg = O.e2m1_value(c | 8)
+        assert neg == -LATTICE[c] and math.copysign(1.0, neg) == -1.0  # includes -0
+
+
+def test_e2m1_to_e4m3_identity_all_codes():
+    """(q & 0x80808080) | ((q & 0x70707070) >> 2) == E4M3(value * 2^-6) for every nibble."""
+    rows = {r[0]: r[1] for r in golden_rows("e2m1_to_e4m3.txt")}
+    ms, mm, sh = int(rows["mask_sign"], 16), int(rows["mask_mag"], 16), int(rows["shift"])
+    f = 2.0 ** int(rows["factor_log2"])
+    for c in range(16):
+        q = (c << 4) * 0x01010101  # the nibble in bits 7..4 of every byte
+        conv = (q & ms) | ((q & mm) >> sh)
+        for byte in range(4):
+            b = (conv >> (8 * byte)) & 0xFF
+            got = O.e4m3_value(b)
+            want = O.e2m1_value(c) * f
+            assert got == want and math.copysign(1, got) == math.copysign(1, want), (c, hex(b))
+
+
+def test_e2m1_rne_worked_values_and_ties():
+    # exact points stay; ties go to the even mantissa code; >6 saturates; -tiny keeps its sign
+    cases = {1.5: 3, 2.5: 4, 0.15: 0, 6.5: 7, 0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 3.5: 6, 5.0: 6,
+             6.0: 7, 100.0: 7, 0.2500001: 1, 0.7499999: 1}
+    for y, code in cases.items():
+        assert O.e2m1_encode_rne(y) == code, y
+        assert O.e2m1_encode_rne(-y) == code | 8, -y
+    assert O.e2m1_encode_rne(-0.0) == 8
+    assert O.e2m1_encode_rne(-1e-30) == 8
+
+
+def test_e2m1_rne_is_nearest_on_dense_grid():
+    """Brute force: the code's value is at minimal distance (a library argmin over the lattice)."""
+    ys = np.linspace(0, 6.0, 60001, dtype=np.float32)
+    lat = np.array(LATTICE)
+    for y in ys[::7]:
+        c = O.e2m1_encode_rne(float(y))
+        d = np.abs(lat - float(y))
+        assert d[c] == d.min()
+
+
+# ---------------------------------------------------------------------------------------------
+# E4M3 and bf16 casts: reduce to torch's library conversions
+
+def test_e4m3_encoder_matches_torch_float8_on_range():
+    rng = np.random.default_rng(0)
+    u = np.concatenate([rng.uniform(0, 448, 20000), 2.0 ** rng.uniform(-12, 8.8, 20000)]).astype(np.float32)
+    # all midpoints between consecutive finite codes (the tie cases)
+    vals = np.array([O.e4m3_value(c) for c in range(0x7F)])
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    u = np.concatenate([u, mids, vals.astype(np.float32)])
+    u = u[u <= 448]
+    ref = torch.from_numpy(u).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([O.e4m3_encode(float(v)) for v in u], dtype=np.uint8)
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_decode_known_points_and_saturation():
+    assert O.e4m3_value(0x7E) == 448.0
+    assert O.e4m3_value(0x38) == 1.0
+    assert O.e4m3_value(0x08) == 2.0 ** -6
+    assert O.e4m3_value(0x01) == 2.0 ** -9
+    assert math.isnan(O.e4m3_value(0x7F))
+    assert O.e4m3_encode(449.0) == 0x7E and O.e4m3_encode(1e30) == 0x7E
+
+
+def test_bf16_rne_matches_torch_cast():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(5000).astype(np.float32),
+                        (rng.integers(0, 2 ** 32, 5000, dtype=np.uint64).astype(np.uint32)).view(np.float32)])
+    x = x[np.isfinite(x)]
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.bf16_bits(x), ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# Philox and stochastic rounding
+
+def test_philox_known_answers():
+    for r in golden_rows("philox4x32_10_kat.txt"):
+        h = [int(v, 16) for v in r]
+        assert list(O.philox4x32_10(h[0:4], h[4:6])) == h[6:10]
+
+
+def test_sr_word_mapping():
+    seed = 0x0123456789ABCDEF
+    for idx in (0, 1, 2, 3, 4, 7, 1 << 33, (1 << 33) + 3):
+        blk = idx >> 2
+        out = O.philox4x32_10([blk & 0xFFFFFFFF, blk >> 32, 0, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        assert O.sr_word(seed, idx) == out[idx & 3]
+
+
+def test_sr_lattice_points_never_move_and_threshold_is_exact():
+    for code in range(16):
+        y = O.e2m1_value(code)
+        for r in (0, 1, 2 ** 31, 2 ** 32 - 1):
+            c = O.e2m1_encode_sr(y, r)
+            assert O.e2m1_value(c) == y
+    # halfway between 2 and 3: up iff r < 2^31
+    assert O.e2m1_encode_sr(2.5, 2 ** 31 - 1) == 5 and O.e2m1_encode_sr(2.5, 2 ** 31) == 4
+    # a quarter of the way from 4 to 6: p = 1/4, up iff r < 2^30
+    assert O.e2m1_encode_sr(4.5, 2 ** 30 - 1) == 7 and O.e2m1_encode_sr(4.5, 2 ** 30) == 6
+    assert O.e2m1_encode_sr(7.0, 0) == 7  # saturates
+
+
+@pytest.mark.parametrize("y", [0.1, 0.3, 1.2, 2.3, 3.9, 5.1])
+def test_sr_is_unbiased(y):
+    n = 1 << 15
+    vals = np.array([O.e2m1_value(O.e2m1_encode_sr(y, O.sr_word(7, i))) for i in range(n)])
+    lat = np.array(LATTICE)
+    lo = lat[lat <= y].max()
+    hi = lat[lat > y].min()
+    p = (y - lo) / (hi - lo)
+    sigma = (hi - lo) * math.sqrt(p * (1 - p) / n)
+    assert abs(vals.mean() - y) < 4 * sigma
+
+
+# ---------------------------------------------------------------------------------------------
+# MXFP4
+
+def test_bits_per_value():
+    B, eb, sb, blk, bpv = golden_rows("bits_per_value.txt")[0]
+    B, eb, sb = int(B), int(eb), int(sb)
+    assert B * eb + sb == int(blk) and (B * eb + sb) / B == float(bpv)
+    x = np.random.default_rng(2).standard_normal((64, 256)).astype(np.float32)
+    q, s, _ = O.mx_quantize(x)
+    assert (q.nbytes + s.nbytes) * 8 / x.size == float(bpv)
+
+
+def test_mx_worked_block_13():
+    rows = golden_rows("mx_worked_block.txt")
+    e_expected = int(rows[0][1])
+    x = np.zeros(32, dtype=np.float32)
+    srcs = [float(r[0]) for r in rows[1:]]
+    x[: len(srcs)] = srcs
+    q, s, c = O.mx_quantize(x[None, :])
+    assert int(s[0, 0]) - 127 == e_expected
+    xh = O.dequantize(q, s, O.MXFP4)[0]
+    for i, r in enumerate(rows[1:]):
+        assert xh[i] == float(np.float32(r[2])), r
+    assert c["underflow"] == 1 and c["saturation"] == 1
+
+
+def test_mx_ramp_fixtures():
+    base = np.array([-2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2] * 4, dtype=np.float32)[:31]
+    for appended, e, last, zeros, maxerr, rmse in golden_rows("mx_ramp_fixtures.txt"):
+        x = np.append(base, np.float32(appended)).astype(np.float32)
+        q, s, _ = O.mx_quantize(x[None, :])
+        xh = O.dequantize(q, s, O.MXFP4)[0].astype(np.float64)
+        err = xh - x
+        assert int(s[0, 0]) - 127 == int(e)
+        assert xh[-1] == float(last)
+        assert int((xh == 0).sum()) == int(zeros)
+        assert np.abs(err).max() == float(maxerr)
+        assert round(math.sqrt((err ** 2).mean()), 6) == float(rmse)
+
+
+def test_e8m0_limits():
+    for e, byte in golden_rows("e8m0_limits.txt"):
+        e, byte = int(e), int(byte)
+        x = np.full(32, 1.0, dtype=np.float32)
+        codes, _ = O.mx_encode_block(x, e)
+        assert e + 127 == byte  # the byte mapping the oracle stores
+    # data-driven exponent clamps at -127 (byte 0) and never yields byte 255
+    tiny = np.full((1, 32), 2.0 ** -140, dtype=np.float32)
+    assert O.mx_quantize(tiny)[1][0, 0] == 0
+    huge = np.full((1, 32), 3.0e38, dtype=np.float32)
+    assert O.mx_quantize(huge)[1][0, 0] == 125 + 127
+    zero = np.zeros((1, 32), dtype=np.float32)
+    assert O.mx_quantize(zero)[1][0, 0] == 127  # all-zero policy: exponent 0
+
+
+def test_mx_exponent_matches_log2_definition():
+    rng = np.random.default_rng(3)
+    for a in np.concatenate([2.0 ** rng.uniform(-120, 120, 2000), [1.0, 4.0, 6.0, 8.0, 6.1, 13.0]]).astype(np.float32):
+        a = float(a)
+        assert O.mx_exponent(a, O.OCP_FLOOR) == max(-127, math.floor(math.log2(a / 4)))
+        e = O.mx_exponent(a, O.NOSAT_CEIL)
+        assert a <= 6 * 2.0 ** e and (e == -127 or a > 6 * 2.0 ** (e - 1))
+
+
+def test_sawtooth_cliff_6_1():
+    """The 6.1-max block: the no-saturation rule doubles the scale (byte 128) and leaves 4 and 6
+    unused; the OCP rule keeps byte 127 and saturates."""
+    rows = {r[1]: r for r in golden_rows("scale_policies.txt")}
+    x = np.linspace(-6.0, 6.1, 32).astype(np.float32)
+    x[-1] = np.float32(6.1)
+    q, s, c = O.mx_quantize(x[None, :], policy=O.NOSAT_CEIL)
+    assert int(s[0, 0]) - 127 == int(rows["nosat_ceil"][2])
+    codes = np.stack([q[0] & 15, q[0] >> 4], 1).ravel()
+    mags = codes & 7
+    assert not np.isin(mags, [6, 7]).any()          # lattice steps 4.0 and 6.0 unused
+    assert np.float32(6.1) / 2 == np.float32(rows["nosat_ceil"][3])
+    assert c["saturation"] == 0
+    q2, s2, c2 = O.mx_quantize(x[None, :], policy=O.OCP_FLOOR)
+    assert int(s2[0, 0]) - 127 == int(rows["ocp_floor"][2]) and c2["saturation"] == 1
+
+
+# ---------------------------------------------------------------------------------------------
+# NVFP4
+
+def test_nvfp4_global_scale_closed_forms():
+    assert O.nvfp4_global_scale(2688.0) == 1.0
+    assert O.nvfp4_global_scale(1536.0, four_six=True) == 1.0
+    assert O.nvfp4_global_scale(0.0) == 1.0
+    assert O.nvfp4_global_scale(448.0 * 6 * 3) == np.float32(3.0)
+
+
+def test_nvfp4_exact_block():
+    """s_g = 1, block max 6: code 1.0 (0x38), every lattice value reproduces exactly."""
+    x = np.array([6, -4, 3, 2, 1.5, 1, 0.5, 0, -0.5, -1, -1.5, -2, -3, 4, 6, -6], dtype=np.float32)[None, :]
+    q, s, sg, c = O.nvfp4_quantize(x, global_in=1.0)
+    assert sg == 1.0 and s[0, 0] == 0x38
+    assert np.array_equal(O.dequantize(q, s, O.NVFP4, sg), x)
+    assert c == {"underflow": 0, "saturation": 0, "nonfinite": 0, "blocks_four": 0}
+
+
+def test_nvfp4_scale_is_amax_over_six_cast_to_e4m3():
+    """The block scale is amax_b/(6 s_g) cast to E4M3 (podcast IF4 segment: "largest value over six,
+    cast to FP8 E4M3"), checked against torch's float8 cast of the fp64 ratio."""
+    x = O._f32(np.random.default_rng(4).standard_normal((64, 256)) * 3)
+    q, s, sg, _ = O.nvfp4_quantize(x)
+    amax_b = np.abs(x.reshape(64, 16, 16)).max(-1)
+    ideal = torch.from_numpy((amax_b / (6.0 * sg)).astype(np.float32)).to(torch.float8_e4m3fn)
+    ideal = ideal.view(torch.uint8).numpy()
+    # fp32 rounding of 1/(6 s_g) may move a value across an E4M3 midpoint: at most one code apart
+    assert np.abs(s.astype(int) - ideal.astype(int)).max() <= 1
+    assert (s == ideal).mean() > 0.99
+    assert s.max() <= 0x7E
+
+
+def test_nvfp4_block_max_normalises_below_six_times_e4m3_step():
+    x = O._f32(np.random.default_rng(5).laplace(size=(128, 512)))
+    q, s, sg, c = O.nvfp4_quantize(x)
+    d = np.array([O.e4m3_value(int(b)) for b in s.ravel()]).reshape(s.shape)
+    top = np.abs(x.reshape(128, 32, 16)).max(-1) / (d * sg)
+    assert top.max() <= 6 * (1 + 2 ** -4) + 1e-6
+
+
+def test_four_over_six_pins():
+    gave, usable, cut = golden_rows("four_over_six.txt")[0]
+    assert round(1 - 256 / 448, 2) == float(cut)           # M = 256 instead of 448
+    assert 2 * 8 - 1 == int(usable)                          # 16 codes, one shared zero
+    # a block lying on the 4-scaled lattice: 4/6 picks T=4 with zero error
+    x = np.array([4, 3, 2, 1.5, 1, 0.5, 0, -4, -3, -2, -1, -0.5, 4, 3, 2, 1], dtype=np.float32)[None, :] * 0.25
+    q, s, sg, c = O.nvfp4_quantize(x, four_six=True, global_in=1.0 / 16)
+    assert c["blocks_four"] == 1
+    assert np.array_equal(O.dequantize(q, s, O.NVFP4, sg), x)
+    # in T=4 blocks the +-6 codes (the two values given up) never appear
+    y = O._f32(np.random.default_rng(6).standard_normal((256, 256)))
+    q, s, sg, c = O.nvfp4_quantize(y, four_six=True)
+    assert c["blocks_four"] > 0
+    q6, s6, _, _ = O.nvfp4_quantize(y, four_six=False, global_in=sg)
+    codes = np.stack([q & 15, q >> 4], -1).reshape(256, 16, 16)
+    four_blocks = (s.reshape(256, 16) != s6.reshape(256, 16)) | np.any(codes != np.stack([q6 & 15, q6 >> 4], -1).reshape(256, 16, 16), -1)
+    assert four_blocks.sum() > 0
+    assert not np.isin(codes[four_blocks] & 7, [7]).any() or int(gave) == 2
+
+
+def test_four_over_six_picks_lower_error_candidate_brute_force():
+    """Independent brute force: per block, both candidates from torch's E4M3 cast and a numpy
+    nearest-lattice search; the oracle's choice must be the lower-SSE one."""
+    rng = np.random.default_rng(7)
+    x = O._f32(rng.standard_normal((8, 64)))
+    q, s, sg, c = O.nvfp4_quantize(x, four_six=True)
+    lat = np.array(LATTICE)
+    xh = O.dequantize(q, s, O.NVFP4, sg)
+    for r in range(8):
+        for b in range(4):
+            blk = x[r, 16 * b:16 * b + 16].astype(np.float64)
+            sse = {}
+            for T in (6.0, 4.0):
+                inv = np.float32(1) / (np.float32(T) * np.float32(sg))
+                u = np.float32(np.abs(blk).max()) * inv
+                code = torch.tensor([u], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).item()
+                d = O.e4m3_value(code)
+                if d == 0:
+                    rec = np.zeros(16)
+                else:
+                    R = np.float32(1) / (np.float32(d) * np.float32(sg))
+                    y = (blk.astype(np.float32) * R).astype(np.float64)
+                    mags = np.array([lat[np.argmin(np.abs(lat - min(abs(v), 6.0)) + (np.arange(8) % 2) * 1e-12)] for v in y])
+                    rec = np.sign(y) * mags * d * sg
+                sse[T] = float(((blk - rec) ** 2).sum())
+            got = float(((blk - xh[r, 16 * b:16 * b + 16]) ** 2).sum())
+            assert got <= min(sse.values()) * (1 + 1e-5) + 1e-30
+
+
+# ---------------------------------------------------------------------------------------------
+# Walsh-Hadamard rotation
+
+def test_fwht_norm_constant():
+    assert O.fwht_norm_const(8192) == np.float32(1 / math.sqrt(8192))
+    assert O.fwht_norm_const(4096) == 2.0 ** -6
+
+
+def test_fwht_matches_sylvester_hadamard_matrix():
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(8)
+    for d in (1024, 2048):
+        x = O._f32(rng.standard_normal((3, d)))
+        ref = (x.astype(np.float64) @ hadamard(d).T.astype(np.float64)) / math.sqrt(d)
+        got = O.fwht(x).astype(np.float64)
+        # fp32 butterflies: normwise error within log2(d) roundings of 2^-24 each (doubled)
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < math.log2(d) * 2.0 ** -23
+
+
+def test_fwht_involution_is_exact_on_small_integers():
+    """H H^T = I: with d = 4^k, c = 2^-k exactly and all sums of small integers are exact."""
+    rng = np.random.default_rng(9)
+    for d in (1024, 4096, 16384):
+        x = rng.integers(-8, 9, size=(2, d)).astype(np.float32)
+        assert np.array_equal(O.fwht(O.fwht(x)), x)
+    x = rng.integers(-8, 9, size=(2, 8192)).astype(np.float32)
+    assert np.allclose(O.fwht(O.fwht(x)), x, rtol=0, atol=1e-5)
+
+
+def test_fwht_spike_damping():
+    d, spike, damp = golden_rows("hadamard_spike.txt")[0]
+    d, spike = int(d), float(spike)
+    x = np.zeros((1, d), dtype=np.float32)
+    x[0, 1234] = spike
+    y = O.fwht(x)[0]
+    c = np.float32(O.fwht_norm_const(d))
+    assert np.all(np.abs(y) == np.float32(spike) * c)
+    assert round(spike / np.abs(y).max(), 1) == float(damp)
+    # sign pattern is column 1234 of the Sylvester matrix: (-1)^popcount(i & 1234)
+    signs = np.array([(-1) ** bin(i & 1234).count("1") for i in range(d)])
+    assert np.array_equal(np.sign(y), signs)
+
+
+def test_fwht_parseval():
+    x = O._f32(np.random.default_rng(10).laplace(size=(4, 8192)))
+    y = O.fwht(x)
+    n0 = np.linalg.norm(x.astype(np.float64), axis=1)
+    n1 = np.linalg.norm(y.astype(np.float64), axis=1)
+    assert np.max(np.abs(n1 / n0 - 1)) < 1e-6
+
+
+# ---------------------------------------------------------------------------------------------
+# Dequantisation and the GEMM reference
+
+def test_dequant_f32_equals_exact_value_when_representable():
+    x = O._f32(np.random.default_rng(11).standard_normal((32, 128)))
+    q, s, sg, _ = O.nvfp4_quantize(x)
+    a = O.dequantize(q, s, O.NVFP4, sg).astype(np.float64)
+    b = O.dequantize_f64(q, s, O.NVFP4, sg)
+    assert np.max(np.abs(a - b) / np.maximum(np.abs(b), 1e-30)) <= 2 ** -24
+    q, s, _ = O.mx_quantize(x)
+    assert np.array_equal(O.dequantize(q, s, O.MXFP4).astype(np.float64), O.dequantize_f64(q, s, O.MXFP4))
+
+
+def test_gemm_reference_closed_forms():
+    M, N, K = 128, 256, 512
+    # every A element = 1 with E8M0 scale 2^1, every B element = 1.5 with 2^-3: C = K * 2 * 1.5/8
+    Aq = np.full((M, K // 2), 0x22, dtype=np.uint8)   # code 2 (1.0) in both nibbles
+    Bq = np.full((N, K // 2), 0x33, dtype=np.uint8)   # code 3 (1.5)
+    As = np.full((M, K // 32), 128, dtype=np.uint8)
+    Bs = np.full((N, K // 32), 124, dtype=np.uint8)
+    C, S = O.gemm_f64(Aq, As, 1.0, Bq, Bs, 1.0, O.MXFP4)
+    assert np.all(C == K * 2 * 1.5 / 8) and np.all(S == C)
+    # one-hot: A row m has a single 6.0 at column (m % K); B row n a single -4 at column (n % K)
+    Aq = np.zeros((M, K // 2), dtype=np.uint8)
+    Bq = np.zeros((N, K // 2), dtype=np.uint8)
+    for m in range(M):
+        k = (3 * m) % K
+        Aq[m, k // 2] |= 7 << (4 * (k & 1))
+    for n in range(N):
+        k = (3 * n) % K
+        Bq[n, k // 2] |= 0xE << (4 * (k & 1))
+    As = np.full((M, K // 16), 0x38, dtype=np.uint8)   # E4M3 1.0
+    Bs = np.full((N, K // 16), 0x40, dtype=np.uint8)   # E4M3 2.0
+    C, _ = O.gemm_f64(Aq, As, 0.5, Bq, Bs, 0.25, O.NVFP4)
+    want = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            if (3 * m) % K == (3 * n) % K:
+                want[m, n] = 6.0 * 1.0 * 0.5 * (-4.0) * 2.0 * 0.25
+    assert np.array_equal(C, want)
+
+
+def test_scale_tile_layout_is_a_bijection_with_the_documented_offsets():
+    rows, nb = 256, 8
+    s = np.arange(rows * nb, dtype=np.int64).reshape(rows, nb) % 251
+    t = O.scales_to_mma_tiled(s.astype(np.uint8))
+    assert np.array_equal(O.scales_from_mma_tiled(t, rows, nb), s.astype(np.uint8))
+    # row 37, block 6: tile (0, 1), in-tile (37 % 32) * 16 + (37 // 32) * 4 + 2
+    assert t[1 * 512 + 5 * 16 + 1 * 4 + 2] == s[37, 6]
+    # row 130, block 1: tile (1, 0) -> 2 * 512, in-tile 2 * 16 + 0 * 4 + 1
+    assert t[2 * 512 + 2 * 16 + 1] == s[130, 1]
+
+
+def test_nvfp4_vs_mxfp4_mse_ratio_reported():
+    """Context only (parity unpinned): the Eluvix page claims ~2.4x lower block MSE for NVFP4 with
+    no data distribution given; on N(0,1) the ratio is reported, asserting only NVFP4 < MXFP4."""
+    x = O._f32(np.random.default_rng(12).standard_normal((128, 1024)))
+    q, s, sg, _ = O.nvfp4_quantize(x)
+    e_nv = ((O.dequantize(q, s, O.NVFP4, sg) - x) ** 2).mean()
+    q, s, _ = O.mx_quantize(x)
+    e_mx = ((O.dequantize(q, s, O.MXFP4) - x) ** 2).mean()
+    assert e_nv < e_mx
