@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Throughput of the block-scaled FP4 hot path on B200.
+
+Headline workload (one step): NVFP4 two-level quantisation of an 8192 x 8192 bf16 activation
+(N(0,1) with 0.1% of the columns x U(50,100), seed 5), once plain and once with adaptive 4/6 —
+each a two-pass call (tensor amax, then per-block E4M3 scale + E2M1 encode + pack).  The value is
+algorithmic GB/s: 4.5625 bytes per element per call (2 amax read + 2 read + 0.5 nibbles + 1/16
+scale) over the device time of the step.  Secondary lines measure the other workloads (MXFP4
+quantise + dequantise, fused Walsh-Hadamard + NVFP4 with stochastic rounding, the NVFP4 and MXFP4
+block-scaled GEMMs and the down_proj quantise + GEMM pipeline).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-secondary]
+
+Under torchrun every rank quantises its own copy of the workload (independent problems, weak
+scaling, no collective on the data path); the step time is the max over ranks.
+Timing: CUDA events on the launching stream per step, L2 flushed (a 256 MiB write) before every
+timed step, outside the events; clocks sampled with nvidia-smi during the timed loop.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import block_scaled_fp4_amax_b200 as fp4  # noqa: E402
+from block_scaled_fp4_amax_b200 import synth  # noqa: E402
+
+METRIC = "FP4 quantize GB/s vs HBM peak; block-scaled FP4 GEMM TFLOPS vs FP4 peak"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NV_BYTES_2PASS = 4.5625     # bytes per element, two-pass NVFP4 (bf16 in)
+NV_BYTES_1PASS = 2.5625     # bytes per element, one quantise launch (bf16 in)
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+# ---------------------------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def profile_traffic(name):
+    """Per-launch DRAM bytes (read + write) recorded in profiles/<name>.md, if any."""
+    path = os.path.join(PROFILE_DIR, name + ".md")
+    if not os.path.exists(path):
+        return None
+    for ln in open(path):
+        if ln.startswith("traffic_bytes_per_launch:"):
+            v = ln.split(":", 1)[1].strip()
+            return None if v in ("", "null") else float(v)
+    return None
+
+
+class Clocks:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "50"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+
+    def stop(self, t0, t1):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = []
+        for ln in open(self.f.name):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        load = [p for ts, p in rows if t0 - 1 <= ts <= t1 + 1] or [p for _, p in rows]
+        if not load:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(p[2]) for p in load if p[2].replace(".", "").isdigit()]
+        mx = [float(p[3]) for p in load if p[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in load for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(load)}
+
+
+def dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as td
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return td, td.get_rank(), ws, local
+    return None, 0, 1, 0
+
+
+def barrier(td):
+    if td is not None:
+        td.barrier()
+
+
+def max_over_ranks(td, v):
+    if td is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, K, W, flush, td, events_per_step=True):
+    """W warm-up calls, then K timed calls, each preceded by an L2 flush outside its events.
+    Returns per-step device milliseconds."""
+    s = torch.cuda.current_stream()
+    for _ in range(W):
+        flush()
+        fn()
+    barrier(td)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        flush()
+        a.record(s)
+        fn()
+        b.record(s)
+    torch.cuda.synchronize()
+    barrier(td)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+# ---------------------------------------------------------------------------------------------
+# Workloads (C-ABI calls on preallocated device buffers)
+
+class NvStep:
+    """One headline step: nvfp4_quantize(x) plain, then with four-over-six (two passes each)."""
+
+    def __init__(self, x, dev):
+        L = fp4.lib()
+        self.L = L
+        self.x = x
+        rows, cols = x.shape
+        self.rows, self.cols = rows, cols
+        self.q = [torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.s = [torch.empty(rows * cols // 16, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.g = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.c = [torch.empty(4, dtype=torch.int64, device=dev) for _ in range(2)]
+        self.ws = torch.empty(fp4.workspace_size(fp4.OP_NVFP4_QUANTIZE), dtype=torch.uint8, device=dev)
+
+    def call(self, i, four_six, global_in=None):
+        st = self.L.nvfp4_quantize(ctypes.c_void_p(self.x.data_ptr()), fp4.BF16, self.rows, self.cols, 16, fp4.RNE,
+                                   int(four_six), 0, fp4.ROWMAJOR,
+                                   None if global_in is None else ctypes.c_void_p(global_in.data_ptr()),
+                                   ctypes.c_void_p(self.g[i].data_ptr()), ctypes.c_void_p(self.q[i].data_ptr()),
+                                   ctypes.c_void_p(self.s[i].data_ptr()), ctypes.c_void_p(self.c[i].data_ptr()),
+                                   ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(self.L.fp4_last_error().decode())
+
+    def __call__(self):
+        self.call(0, False)
+        self.call(1, True)
+
+    launches_per_step = 4  # amax + quantise, twice
+
+
+def run_ours(args, td, rank, world, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    x_cpu = synth.nv_outliers()
+    x = x_cpu.to(dev)
+    n = x.numel()
+    step = NvStep(x, dev)
+
+    clocks = Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                    os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    clocks.start()
+    t0 = time.time()
+    ms = timed(step, args.steps, args.warmup, flush, td)
+    t1 = time.time()
+    clk = clocks.stop(t0, t1)
+    ms_step = max_over_ranks(td, sum(ms) / len(ms))
+    bytes_step = 2 * NV_BYTES_2PASS * n
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+
+    # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g
+    g = step.g[1].clone()
+    kms = timed(lambda: step.call(1, True, global_in=g), args.steps, args.warmup, flush, td)
+    k_ms = max_over_ranks(td, sum(kms) / len(kms))
+    k_bytes = NV_BYTES_1PASS * n
+    achieved = k_bytes / (k_ms * 1e-3) / 1e9
+    roof = {"kernel": "quantize_kernel<bf16, NVFP4, RNE, 4/6> (one launch, 8192x8192)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
+            "traffic": profile_traffic("nvfp4_quantize_8192x8192"),
+            "algorithmic_bytes_per_launch": k_bytes}
+
+    # end to end through the public binding: pinned host input -> device -> both calls -> host
+    host_in = x_cpu.pin_memory()
+    host_q = [torch.empty((8192, 4096), dtype=torch.uint8).pin_memory() for _ in range(2)]
+    host_s = [torch.empty(8192 * 512, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    host_g = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(2)]
+    xd = torch.empty_like(x)
+
+    def e2e_step():
+        xd.copy_(host_in, non_blocking=True)
+        for i, fs in enumerate((False, True)):
+            q, s, gg, c = fp4.nvfp4_quantize(xd, four_six=fs, workspace=step.ws)
+            host_q[i].copy_(q, non_blocking=True)
+            host_s[i].copy_(s, non_blocking=True)
+            host_g[i].copy_(gg, non_blocking=True)
+
+    ems = timed(e2e_step, max(3, args.steps // 10), args.warmup, flush, td)
+    e_ms = max_over_ranks(td, sum(ems) / len(ems))
+    e2e = {"value": round(world * bytes_step / (e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "h2d_bytes_per_step": int(host_in.numel() * 2),
+           "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_q + host_s + host_g)),
+           "ms_per_step": round(e_ms, 4)}
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e2m1 (fp32 arithmetic)",
+            "data": "synthetic (seeded numpy; no dataset)",
+            "config": {"workload": "NVFP4 two-level quantisation 8192x8192 bf16, N(0,1) + 0.1% outlier "
+                                   "columns x U(50,100), seed 5; plain + adaptive 4/6, two passes each",
+                       "rows": 8192, "cols": 8192, "block": 16, "global_scale": "amax/(6*448); 4/6: amax/(6*256)",
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof, "e2e": e2e, "gpu_launches": NvStep.launches_per_step * args.steps,
+            "clocks": clk}
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x_cpu)
+    if not args.no_secondary:
+        line["secondary"] = secondary(args, dev, flush, td, pk)
+    return line
+
+
+def cpu_baseline(x_cpu, rows=4096):
+    """The oracle as it stands, single-threaded, on the first `rows` rows of the workload."""
+    import oracle as O
+    xs = synth.as_f32_numpy(x_cpu[:rows])
+    t = time.perf_counter()
+    O.nvfp4_quantize(xs, four_six=False)
+    O.nvfp4_quantize(xs, four_six=True)
+    dt = time.perf_counter() - t
+    b = 2 * NV_BYTES_2PASS * xs.size
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of 8192 rows (plain + 4/6), {dt:.1f} s single-threaded C oracle"}
+
+
+# ---------------------------------------------------------------------------------------------
+def secondary(args, dev, flush, td, pk):
+    out = []
+    K = max(5, args.steps // 10)
+    W = args.warmup
+    # config 1: MXFP4 quantise + dequantise, 256 x 512 fp32
+    x1 = synth.mx_small().to(dev)
+
+    def c1():
+        q, s, c = fp4.mx_quantize(x1)
+        fp4.fp4_dequantize(q, s, fp4.MXFP4)
+
+    ms = timed(c1, K, W, flush, td)
+    t = statistics.median(ms)
+    b = x1.numel() * (4 + 0.5 + 1 / 32) * 2
+    out.append({"workload": "MXFP4 quantise + dequantise 256x512 fp32 (launch-bound, L2-resident)",
+                "ms": round(t, 5), "GB/s": round(b / (t * 1e-3) / 1e9, 1)})
+    # config 3: fused FWHT + NVFP4 + SR, 16384 x 8192 bf16
+    x3 = synth.fwht_laplace().to(dev)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+
+    def c3():
+        fp4.fwht_quantize(x3, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7, workspace=ws)
+
+    ms = timed(c3, K, W, flush, td)
+    t = statistics.median(ms)
+    b = NV_BYTES_2PASS * x3.numel()
+    out.append({"workload": "FWHT d=8192 + NVFP4 + stochastic rounding, 16384x8192 bf16, two passes",
+                "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
+                "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    del x3
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+def run_reference(args, rank):
+    """The oracle (plain C, single thread) on a bounded sample of the headline workload."""
+    import oracle as O
+    rows = 512
+    x = synth.as_f32_numpy(synth.nv_outliers()[:rows])
+    for _ in range(args.warmup):
+        O.nvfp4_quantize(x[:64], four_six=False)
+    ts = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        O.nvfp4_quantize(x, four_six=False)
+        O.nvfp4_quantize(x, four_six=True)
+        ts.append(time.perf_counter() - t)
+    dt = statistics.mean(ts)
+    b = 2 * NV_BYTES_2PASS * x.size
+    v = round(b / dt / 1e9, 4)
+    sample = f"first {rows} of 8192 rows per step (plain + 4/6), single-threaded C oracle"
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp32 arithmetic (CPU)", "data": "synthetic (seeded numpy; no dataset)",
+            "config": {"workload": "NVFP4 two-level quantisation 8192x8192 bf16, N(0,1) + 0.1% outlier columns "
+                                   "x U(50,100), seed 5; plain + adaptive 4/6, two passes each", "rows_sampled": rows},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": v, "unit": "GB/s"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+CASES = ("nv", "nv46", "nv_amax", "mx", "fwht", "gemm_nv", "gemm_mx", "dequant")
+
+
+def run_case(name, reps):
+    """Run one kernel on its full-size workload `reps` times (for profiler captures)."""
+    dev = torch.device("cuda", 0)
+    if name in ("nv", "nv46", "nv_amax"):
+        x = synth.nv_outliers().to(dev)
+        g = torch.tensor([0.02], device=dev)
+        for _ in range(reps):
+            if name == "nv_amax":
+                fp4.nvfp4_quantize(x)
+            else:
+                fp4.nvfp4_quantize(x, four_six=(name == "nv46"), global_in=g)
+    elif name == "mx":
+        a = synth.swiglu_act().to(dev)
+        for _ in range(reps):
+            fp4.mx_quantize(a, layout=fp4.MMA_TILED)
+    elif name == "fwht":
+        x = synth.fwht_laplace().to(dev)
+        for _ in range(reps):
+            fp4.fwht_quantize(x, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7)
+    elif name == "dequant":
+        x = synth.nv_outliers().to(dev)
+        q, s, g, _ = fp4.nvfp4_quantize(x)
+        for _ in range(reps):
+            fp4.fp4_dequantize(q, s, fp4.NVFP4, g, out_dtype=torch.bfloat16)
+    elif name in ("gemm_nv", "gemm_mx"):
+        if name == "gemm_nv":
+            A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)
+            B = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 2).to(dev), layout=fp4.MMA_TILED)
+            args = (fp4.NVFP4, A[0], A[1], B[0], B[1], A[2], B[2])
+        else:
+            A = fp4.mx_quantize(synth.swiglu_act().to(dev), layout=fp4.MMA_TILED)
+            B = fp4.mx_quantize(synth.weight().to(dev), layout=fp4.MMA_TILED)
+            args = (fp4.MXFP4, A[0], A[1], B[0], B[1])
+        for _ in range(reps):
+            fp4.fp4_block_gemm(*args)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, "reps": reps, "ok": True}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=CASES, help="run one kernel on its workload (profiling)")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.case:
+        run_case(args.case, args.reps)
+        return
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, rank)))
+        return
+    td, rank, world, local = dist()
+    try:
+        line = run_ours(args, td, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line))
+    finally:
+        if td is not None:
+            td.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+"""block_scaled_fp4_amax_b200 — Python binding of libfp4mx.so (block-scaled FP4 microscaling on B200).
+
+Argument marshalling only: every function here checks tensor devices/dtypes/shapes, allocates the
+outputs with torch (device memory is torch's job) and calls the C ABI declared in
+``include/fp4mx.h`` on torch's current CUDA stream.  All arithmetic runs in the CUDA kernels of
+libfp4mx.so; there is no CPU path.  If the shared library is missing or was built for nothing this
+process can load, the first call raises.
+
+    from block_scaled_fp4_amax_b200 import mx_quantize, nvfp4_quantize, fwht_quantize, \
+        fp4_dequantize, fp4_block_gemm
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp4mx.so")
+
+# enums of include/fp4mx.h
+F32, BF16 = 0, 1
+MXFP4, NVFP4 = 0, 1
+RNE, STOCHASTIC = 0, 1
+OCP_FLOOR, NOSAT_CEIL = 0, 1
+ROWMAJOR, MMA_TILED = 0, 1
+OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEMM = range(5)
+STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
+
+# Every symbol include/fp4mx.h declares.
+EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
+           "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error")
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfp4mx.so and declare its C signatures (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m block_scaled_fp4_amax_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, LG, ULL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_ulonglong, ctypes.c_size_t
+    L.mx_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P]
+    L.nvfp4_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P, SZ, P]
+    L.fwht_quantize.argtypes = [P, I, LG, LG, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
+    L.fp4_dequantize.argtypes = [P, P, I, I, I, P, LG, LG, I, P, P]
+    L.fp4_block_gemm.argtypes = [I, I, I, I, P, P, P, P, P, P, P, LG, P, SZ, P]
+    L.fp4_workspace_size.argtypes = [I, LG, LG]
+    L.fp4_workspace_size.restype = SZ
+    L.fp4_gemm_status_word.argtypes = []
+    L.fp4_gemm_status_word.restype = SZ
+    L.fp4_status_str.argtypes = [I]
+    L.fp4_status_str.restype = ctypes.c_char_p
+    L.fp4_last_error.argtypes = []
+    L.fp4_last_error.restype = ctypes.c_char_p
+    for name in ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "fp4_dequantize", "fp4_block_gemm"):
+        getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        raise Fp4Error(status, lib().fp4_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"input dtype must be float32 or bfloat16, got {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def workspace_size(op: int, rows: int = 0, cols: int = 0) -> int:
+    return int(lib().fp4_workspace_size(op, rows, cols))
+
+
+def _workspace(op, device, rows=0, cols=0):
+    n = workspace_size(op, rows, cols)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def _alloc_outputs(rows, cols, block, device):
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    s = torch.empty((rows * cols // block,), dtype=torch.uint8, device=device)
+    c = torch.empty(4, dtype=torch.int64, device=device)  # zeroed by the library on its stream
+    return q, s, c
+
+
+def mx_quantize(x: torch.Tensor, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0,
+                layout: int = ROWMAJOR, block: int = 32, stream=None):
+    """MXFP4: returns (q uint8 [rows, cols/2], scales uint8 [rows*cols/32] in `layout`,
+    counts int64[4] on device: underflow, saturation, nonfinite, blocks_four)."""
+    _need_cuda(x)
+    rows, cols = x.shape
+    q, s, c = _alloc_outputs(rows, cols, 32, x.device)
+    _check(lib().mx_quantize(_ptr(x), _dtype_code(x), rows, cols, block, policy, round, seed, layout,
+                             _ptr(q), _ptr(s), _ptr(c), _stream(stream)))
+    return q, s, c
+
+
+def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
+                   layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
+                   stream=None, workspace: torch.Tensor | None = None):
+    """NVFP4: returns (q, scales, s_g float32[1] on device, counts)."""
+    _need_cuda(x, global_in)
+    rows, cols = x.shape
+    q, s, c = _alloc_outputs(rows, cols, 16, x.device)
+    g = torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else _workspace(OP_NVFP4_QUANTIZE, x.device, rows, cols)
+    _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, round, int(bool(four_six)), seed,
+                                layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c), _ptr(ws),
+                                ws.numel(), _stream(stream)))
+    return q, s, g, c
+
+
+def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
+                  layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, want_rotated: bool = False,
+                  block: int | None = None, stream=None, workspace: torch.Tensor | None = None):
+    """Walsh-Hadamard rotation of each row fused with the quantiser of `fmt`.
+    Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
+    _need_cuda(x, global_in)
+    rows, d = x.shape
+    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, x.device)
+    g = torch.empty(1, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
+    rot = torch.empty((rows, d), dtype=torch.float32, device=x.device) if want_rotated else None
+    ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, x.device, rows, d)
+    _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, fmt, B, round, int(bool(four_six)), seed,
+                               layout, _ptr(global_in), _ptr(g), _ptr(rot), _ptr(q), _ptr(s), _ptr(c),
+                               _ptr(ws), ws.numel(), _stream(stream)))
+    return q, s, g, c, rot
+
+
+def fp4_dequantize(q: torch.Tensor, scales: torch.Tensor, fmt: int, global_scale: torch.Tensor | None = None,
+                   layout: int = ROWMAJOR, out_dtype: torch.dtype = torch.float32, block: int | None = None,
+                   stream=None):
+    """x_hat [rows, 2*q.shape[1]] in out_dtype."""
+    _need_cuda(q, scales, global_scale)
+    rows, half = q.shape
+    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    out = torch.empty((rows, 2 * half), dtype=out_dtype, device=q.device)
+    _check(lib().fp4_dequantize(_ptr(q), _ptr(scales), fmt, B, layout, _ptr(global_scale), rows, 2 * half,
+                                _dtype_code(out), _ptr(out), _stream(stream)))
+    return out
+
+
+def fp4_block_gemm(fmt: int, Aq: torch.Tensor, As: torch.Tensor, Bq: torch.Tensor, Bs: torch.Tensor,
+                   Ag: torch.Tensor | None = None, Bg: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   stream=None, workspace: torch.Tensor | None = None):
+    """C = alpha * A @ B^T in bf16 from packed operands with MMA-tiled scales.  Returns (C, workspace);
+    workspace[0:4] holds the kernel status word (0 = ok)."""
+    _need_cuda(Aq, As, Bq, Bs, Ag, Bg)
+    M, K = Aq.shape[0], Aq.shape[1] * 2
+    N = Bq.shape[0]
+    if Bq.shape[1] * 2 != K:
+        raise ValueError("A and B disagree on K")
+    C = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=Aq.device)
+    ws = workspace if workspace is not None else _workspace(OP_BLOCK_GEMM, Aq.device, M, N)
+    _check(lib().fp4_block_gemm(fmt, M, N, K, _ptr(Aq), _ptr(As), _ptr(Ag), _ptr(Bq), _ptr(Bs), _ptr(Bg),
+                                _ptr(C), C.stride(0), _ptr(ws), ws.numel(), _stream(stream)))
+    return C, ws

@@ -1,0 +1,271 @@
+// fp4_device.cuh — device-side building blocks shared by the quantise / rotate / dequantise
+// kernels of libfp4mx: 16-byte vector loads, the sm_100 FP4/FP8 conversion instructions,
+// Philox4x32-10 and the E2M1 rounding rules.
+//
+// Every floating-point step that decides a code is an explicitly rounded fp32 intrinsic
+// (__fmul_rn, __fadd_rn, __fsub_rn, __frcp_rn, __fdiv_rn) so the compiler cannot contract or
+// reorder it.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace fp4k {
+
+// ---------------------------------------------------------------------------------------------
+// Loads.  16 bytes per lane, read-only path.  `Stream` loads are marked evict-first (data that
+// will not be read again); the default keeps the line in L2 for a following pass.
+template <bool Stream>
+__device__ __forceinline__ uint4 ld16(const void* p) {
+  if (Stream) return __ldcs(reinterpret_cast<const uint4*>(p));
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// Element type traits: E values per 16-byte chunk, unpacked to fp32 (exact).
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ __forceinline__ static void unpack(const uint4& r, float* v) {
+    v[0] = __uint_as_float(r.x); v[1] = __uint_as_float(r.y);
+    v[2] = __uint_as_float(r.z); v[3] = __uint_as_float(r.w);
+  }
+};
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ __forceinline__ static void unpack(const uint4& r, float* v) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+// 32 bytes per lane (sm_100 256-bit load): a warp reads 1 KiB of contiguous memory per
+// instruction.  `Stream` marks the lines evict-first in L2 (last use); otherwise they are kept
+// for a following pass.
+struct U8 {
+  uint32_t w[8];
+};
+template <bool Stream>
+__device__ __forceinline__ U8 ld32(const void* p) {
+  U8 r;
+  if (Stream) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]),
+                   "=r"(r.w[6]), "=r"(r.w[7])
+                 : "l"(p));
+  } else {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_last.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]),
+                   "=r"(r.w[6]), "=r"(r.w[7])
+                 : "l"(p));
+  }
+  return r;
+}
+
+// Element traits for a 32-byte chunk: E values, unpacked to fp32 (exact), and the number of
+// values that are +-0 (from the bit patterns: the magnitude bits of a nonzero value, plus all
+// ones, carry into the top bit of its field).
+template <typename T> struct Vec32;
+template <> struct Vec32<float> {
+  static constexpr int E = 8;
+  __device__ __forceinline__ static void unpack(const U8& r, float* v) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r.w[i]);
+  }
+  __device__ __forceinline__ static int zeros(const U8& r) {
+    int nz = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nz += (r.w[i] & 0x7FFFFFFFu) != 0u;
+    return 8 - nz;
+  }
+};
+template <> struct Vec32<__nv_bfloat16> {
+  static constexpr int E = 16;
+  __device__ __forceinline__ static void unpack(const U8& r, float* v) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(r.w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(r.w[i] & 0xFFFF0000u);
+    }
+  }
+  __device__ __forceinline__ static int zeros(const U8& r) {
+    int nz = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nz += __popc(((r.w[i] & 0x7FFF7FFFu) + 0x7FFF7FFFu) & 0x80008000u);
+    return 16 - nz;
+  }
+};
+
+// Number of +-0 codes among the 8 nibbles of a packed word.
+__device__ __forceinline__ int zero_nibbles(uint32_t p) {
+  return 8 - __popc(((p & 0x77777777u) + 0x77777777u) & 0x88888888u);
+}
+
+// ---------------------------------------------------------------------------------------------
+// E2M1 encode of pairs with the sm_100 conversion (round to nearest even, saturating to +-6).
+// Packs 8 values into one 32-bit word: value i in bits [4i, 4i+4) — element 2j in the low
+// nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(const float* y) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return out;
+}
+__device__ __forceinline__ uint32_t e2m1x4(const float* y) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]));
+  return out;
+}
+template <int E>
+__device__ __forceinline__ uint32_t e2m1_pack(const float* y) {
+  if constexpr (E == 8) return e2m1x8(y); else return e2m1x4(y);
+}
+
+// Two f16 halves of a 32-bit word to fp32 (exact), without type punning.
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+      : "=f"(lo), "=f"(hi) : "r"(h));
+}
+
+// Round two fp32 values to bf16 (RNE) and pack them: `lo` in bits 0-15, `hi` in bits 16-31.
+__device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Decode the low E nibbles of `codes` back to fp32 (exact) through f16x2.
+template <int E>
+__device__ __forceinline__ void e2m1_unpack(uint32_t codes, float* v) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(codes));
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) f16x2_to_f32(h[i], v[2 * i], v[2 * i + 1]);
+}
+
+// E4M3 (E4M3FN) round to nearest even, saturating at 448; u >= 0.  Returns the code byte.
+__device__ __forceinline__ uint32_t e4m3_code(float u) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(u));
+  return r & 0xFFu;
+}
+// Exact fp32 value of an E4M3 code byte.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h;
+  const uint16_t c = (uint16_t)code;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+  float lo, hi;
+  f16x2_to_f32(h, lo, hi);
+  return lo;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64 multiplies with the round
+// keys advanced by the Weyl increments.  Counter (blk lo, blk hi, 0, 0), key (seed lo, seed hi).
+struct Philox4 { uint32_t w[4]; };
+__device__ __forceinline__ Philox4 philox4x32_10(uint64_t blk, uint64_t seed) {
+  uint32_t c0 = (uint32_t)blk, c1 = (uint32_t)(blk >> 32), c2 = 0u, c3 = 0u;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  Philox4 o;
+  o.w[0] = c0; o.w[1] = c1; o.w[2] = c2; o.w[3] = c3;
+  return o;
+}
+
+// Random words for E consecutive elements starting at flat index idx0 (idx0 % 4 == 0).
+template <int E>
+__device__ __forceinline__ void sr_words(uint64_t idx0, uint64_t seed, uint32_t* r) {
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    Philox4 p = philox4x32_10((idx0 >> 2) + k, seed);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[4 * k + i] = p.w[i];
+  }
+}
+
+// Stochastic rounding of y onto the E2M1 lattice, returning the rounded lattice value (with the
+// sign of y).  For a = |y| <= 6: lo = largest lattice point <= a (steps of .5 below 2, 1 below 4,
+// 2 up to 6), p = (a - lo)/step; round up iff r < ceil(p * 2^32).  a - lo is exact (Sterbenz)
+// and the scaling by 2^32/step is a power of two, so the threshold is exact.  a > 6 clamps.
+__device__ __forceinline__ float sr_round(float y, uint32_t r) {
+  const float a = fabsf(y);
+  float lo, scale, step;
+  if (a < 2.0f) {
+    lo = __fmul_rn(floorf(__fmul_rn(a, 2.0f)), 0.5f); step = 0.5f; scale = 8589934592.0f;  // 2^33
+  } else if (a < 4.0f) {
+    lo = floorf(a); step = 1.0f; scale = 4294967296.0f;                                    // 2^32
+  } else {
+    lo = 4.0f; step = 2.0f; scale = 2147483648.0f;                                         // 2^31
+  }
+  float v;
+  if (a > 6.0f) {
+    v = 6.0f;
+  } else {
+    const float t = ceilf(__fmul_rn(__fsub_rn(a, lo), scale));
+    const unsigned long long th = __float2ull_rn(t);
+    v = ((unsigned long long)r < th) ? __fadd_rn(lo, step) : lo;
+  }
+  return copysignf(v, y);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Scale-byte placement.  Row-major: the flat block index.  MMA tile layout: 128 x 4 tiles of
+// 512 bytes, block-column groups fastest (the layout tcgen05.cp 32x128b.warpx4 expects).
+__device__ __forceinline__ uint64_t scale_offset(uint64_t blk, uint32_t nb, bool tiled) {
+  if (!tiled) return blk;
+  const uint32_t r = (uint32_t)(blk / nb), j = (uint32_t)(blk - (uint64_t)r * nb);
+  return ((uint64_t)(r >> 7) * (nb >> 2) + (j >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u +
+         (j & 3u);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Counter reduction: per-thread partial counts -> one atomicAdd per CTA and counter.
+template <int NC>
+__device__ __forceinline__ void flush_counts(uint32_t (&c)[NC], unsigned long long* dst) {
+  __shared__ unsigned long long red[NC];
+  if (threadIdx.x < NC) red[threadIdx.x] = 0ull;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    uint32_t v = c[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if ((threadIdx.x & 31) == 0 && v) atomicAdd(&red[i], (unsigned long long)v);
+  }
+  __syncthreads();
+  if (threadIdx.x < NC && red[threadIdx.x]) atomicAdd(dst + threadIdx.x, red[threadIdx.x]);
+}
+
+}  // namespace fp4k

@@ -1,0 +1,488 @@
+// fwht.cu — online normalised Walsh-Hadamard rotation fused ahead of the FP4 quantisers.
+//
+// "Sub-4-Bit Microscaling" §3: activations are multiplied by H_d (entries +-1/sqrt(d)) with an
+// O(d log2 d) add/subtract butterfly before quantisation, which spreads an outlier channel over
+// all d channels.  The rotation is computed in fp32 in a fixed order — unnormalised radix-2
+// stages h = 1, 2, 4, ..., d/2, each (a, b) -> (a + b, a - b) on pairs (i, i + h) with i & h == 0,
+// then one multiply by c = fl(1/sqrt(d)) — so the rotated values, and therefore every code, are
+// reproducible bit for bit.
+//
+// Data movement (d = 2^LOG_D, 32 values per thread, T = d/32 threads per row):
+//   round A : the thread loads its 32 consecutive values (index bits 0-4) straight from global
+//             memory and runs stages h = 1..16 in registers; writes fp32 to shared memory;
+//   round B : the thread gathers the 32 values that differ in index bits 5-9, stages h=32..512;
+//   last    : the thread gathers the values that differ in the remaining high bits together with
+//             2^L consecutive values (index bits 0..L-1, L = 5 - #high bits) and runs the last
+//             stages, multiplies by c and quantises straight from registers.  A 16-value NVFP4
+//             block then spans 2^(4-L) adjacent lanes (amax = xor-shuffle), a Philox call covers
+//             whole 4-value groups (L >= 2), and the packed nibbles are contiguous across lanes.
+// Shared memory holds one fp32 row per row slot; 16-byte chunks are XOR-swizzled by the low
+// three bits of their 32-value row so that every round's accesses are bank-conflict free.
+#include "fp4_device.cuh"
+#include "launch.h"
+
+namespace fp4k {
+
+template <int LOG_D>
+struct Geom {
+  static constexpr int D = 1 << LOG_D;
+  static constexpr int T = D / 32;                 // threads per row
+  static constexpr int CTA = T < 256 ? 256 : T;    // threads per CTA
+  static constexpr int ROWS = CTA / T;             // row slots per CTA
+  static constexpr int NR = (LOG_D + 4) / 5;       // rounds
+  static constexpr int HI = 5 * (NR - 1);          // first index bit of the last round
+  static constexpr int NH = LOG_D - HI;            // high bits in the last round
+  static constexpr int L = 5 - NH;                 // consecutive low bits held in the last round
+  static_assert(LOG_D >= 10 && LOG_D <= 14, "d must be in [1024, 16384]");
+};
+
+__device__ __forceinline__ int swz(int i) {  // word offset of element i inside its row slot
+  const int row = i >> 5;
+  return (row << 5) | ((((i >> 2) & 7) ^ (row & 7)) << 2) | (i & 3);
+}
+
+template <int BIT>
+__device__ __forceinline__ void stage(float (&v)[32]) {
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    if (!(p & (1 << BIT))) {
+      const float a = v[p], b = v[p | (1 << BIT)];
+      v[p] = __fadd_rn(a, b);
+      v[p | (1 << BIT)] = __fsub_rn(a, b);
+    }
+  }
+}
+template <int LO, int HI_>
+__device__ __forceinline__ void stages(float (&v)[32]) {  // local bits LO..HI_-1 in order
+  if constexpr (LO < HI_) {
+    stage<LO>(v);
+    stages<LO + 1, HI_>(v);
+  }
+}
+
+template <typename T>
+struct RowLoad {
+  static constexpr int NV = 32 * (int)sizeof(T) / 16;  // 16-byte chunks per thread
+};
+
+// Round A + B + last-round rotation of one row into v[32] (last-round order: j = low | h << L).
+// `raw` holds this thread's round-A chunks.  Leaves the values unnormalised.
+template <typename T, int LOG_D>
+__device__ __forceinline__ void rotate_row(const uint4 (&raw)[RowLoad<T>::NV], float* srow, int t,
+                                           float (&v)[32]) {
+  using G = Geom<LOG_D>;
+  // round A: index bits 0-4 local
+#pragma unroll
+  for (int c = 0; c < RowLoad<T>::NV; ++c) Vec<T>::unpack(raw[c], v + c * Vec<T>::E);
+  stages<0, 5>(v);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int i = (t << 5) | (q << 2);
+    *reinterpret_cast<float4*>(srow + swz(i)) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+  __syncthreads();
+  if constexpr (G::NR == 3) {
+    // round B: index bits 5-9 local; lane = bits 0-4, rest = bits 10..
+    const int lo5 = t & 31, hi = t >> 5;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = srow[swz(lo5 | (j << 5) | (hi << 10))];
+    stages<0, 5>(v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) srow[swz(lo5 | (j << 5) | (hi << 10))] = v[j];
+    __syncthreads();
+  }
+  // last round: high bits HI.. plus low bits 0..L-1
+  constexpr int L = G::L, NH = G::NH, HI = G::HI;
+#pragma unroll
+  for (int h = 0; h < (1 << NH); ++h) {
+    const int i0 = (t << L) | (h << HI);
+    if constexpr (L >= 2) {
+#pragma unroll
+      for (int q = 0; q < (1 << L) / 4; ++q) {
+        const float4 f = *reinterpret_cast<const float4*>(srow + swz(i0 + 4 * q));
+        v[(h << L) + 4 * q] = f.x; v[(h << L) + 4 * q + 1] = f.y;
+        v[(h << L) + 4 * q + 2] = f.z; v[(h << L) + 4 * q + 3] = f.w;
+      }
+    } else if constexpr (L == 1) {
+      const float2 f = *reinterpret_cast<const float2*>(srow + swz(i0));
+      v[h << 1] = f.x; v[(h << 1) + 1] = f.y;
+    } else {
+      v[h] = srow[swz(i0)];
+    }
+  }
+  stages<L, 5>(v);
+  __syncthreads();  // shared row free for the next row
+}
+
+template <typename T, int LOG_D>
+__device__ __forceinline__ void load_row(const T* x, long long row, long long rows, int t,
+                                         uint4 (&raw)[RowLoad<T>::NV]) {
+  constexpr int D = 1 << LOG_D;
+  if (row < rows) {
+    const char* p = reinterpret_cast<const char*>(x + row * D + (long long)t * 32);
+#pragma unroll
+    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = ld16<false>(p + 16 * c);
+  } else {
+#pragma unroll
+    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Lattice value of each of N already-normalised values after E2M1 encoding (encode + decode).
+template <int N>
+__device__ __forceinline__ void e2m1_roundtrip(const float* y, float* q) {
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int c = 0; c < N / 8; ++c) e2m1_unpack<8>(e2m1x8(y + 8 * c), q + 8 * c);
+  } else {
+    float t[4], o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) t[i] = (i < N) ? y[i] : 0.0f;
+    e2m1_unpack<4>(e2m1x4(t), o);
+#pragma unroll
+    for (int i = 0; i < N; ++i) q[i] = o[i];
+  }
+}
+
+struct FwhtParams {
+  const void* x;
+  long long rows;
+  float c;            // fl(1/sqrt(d))
+  int tiled;
+  int reverse;
+  unsigned long long seed;
+  const float* global_in;
+  uint32_t* amax_bits;
+  float* global_out;
+  float six_m;
+  float* rotated_out;
+  uint8_t* q;
+  uint8_t* scales;
+  unsigned long long* counts;
+};
+
+// Pass 1 (NVFP4 without a caller scale): amax of the rotated tensor.
+template <typename T, int LOG_D>
+__global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams p) {
+  using G = Geom<LOG_D>;
+  extern __shared__ __align__(16) float smem[];
+  const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
+  float* srow = smem + slot * G::D;
+  const T* x = reinterpret_cast<const T*>(p.x);
+  const long long step = (long long)gridDim.x * G::ROWS;
+  float m = 0.0f;
+  uint4 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  long long row = (long long)blockIdx.x * G::ROWS + slot;
+  load_row<T, LOG_D>(x, row, p.rows, t, raw);
+  for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
+    load_row<T, LOG_D>(x, row + step, p.rows, t, nxt);
+    float v[32];
+    rotate_row<T, LOG_D>(raw, srow, t, v);
+    if (row < p.rows) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+    row += step;
+  }
+  // |fl(c*u)| is monotone in |u|: scale the maximum once.
+  m = __fmul_rn(m, p.c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ float wm[32];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int w = 0; w < G::CTA / 32; ++w) b = fmaxf(b, wm[w]);
+    atomicMax(p.amax_bits, __float_as_uint(b));
+  }
+}
+
+// Pass 2: rotate again, normalise, quantise from registers.
+template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX>
+__global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams p) {
+  using G = Geom<LOG_D>;
+  constexpr int L = G::L, NH = G::NH, HI = G::HI, D = G::D;
+  constexpr int B = NV ? 16 : 32;
+  constexpr int LB = NV ? 4 : 5;                 // log2 block
+  constexpr int GE = 1 << L;                     // elements per group
+  constexpr int GL = (L >= LB) ? 1 : (1 << (LB - L));  // lanes per block
+  constexpr int GA = GE < 4 ? 4 : GE;            // register array size for one group
+  static_assert(L <= LB, "group larger than a block");
+  extern __shared__ __align__(16) float smem[];
+  const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
+  const int lane = threadIdx.x & 31;
+  float* srow = smem + slot * D;
+  const T* x = reinterpret_cast<const T*>(p.x);
+  const long long step = (long long)gridDim.x * G::ROWS;
+  const uint32_t nb = D / B;
+
+  float s_g = 1.0f, inv6 = 1.0f, inv4 = 1.0f;
+  if (NV) {
+    if (p.global_in) {
+      s_g = *p.global_in;
+    } else {
+      const float amax = __uint_as_float(*p.amax_bits);
+      s_g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, p.six_m);
+    }
+    inv6 = __frcp_rn(__fmul_rn(6.0f, s_g));
+    inv4 = __frcp_rn(__fmul_rn(4.0f, s_g));
+    if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = s_g;
+  }
+  uint32_t cnt[4] = {0u, 0u, 0u, 0u};
+  uint4 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  auto phys = [&](long long r) { return p.reverse ? (p.rows - 1 - r) : r; };
+  long long row = (long long)blockIdx.x * G::ROWS + slot;
+  load_row<T, LOG_D>(x, row < p.rows ? phys(row) : row, p.rows, t, raw);
+  for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
+    const long long rn = row + step;
+    load_row<T, LOG_D>(x, rn < p.rows ? phys(rn) : rn, p.rows, t, nxt);
+    float v[32];
+    rotate_row<T, LOG_D>(raw, srow, t, v);
+    const bool valid = row < p.rows;
+    const long long prow = valid ? phys(row) : 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], p.c);
+    if (valid && p.rotated_out) {
+#pragma unroll
+      for (int h = 0; h < (1 << NH); ++h) {
+        float* dst = p.rotated_out + prow * D + ((t << L) | (h << HI));
+        if constexpr (L >= 2) {
+#pragma unroll
+          for (int q = 0; q < GE / 4; ++q)
+            reinterpret_cast<float4*>(dst)[q] = make_float4(v[(h << L) + 4 * q], v[(h << L) + 4 * q + 1],
+                                                            v[(h << L) + 4 * q + 2], v[(h << L) + 4 * q + 3]);
+        } else if constexpr (L == 1) {
+          *reinterpret_cast<float2*>(dst) = make_float2(v[h << 1], v[(h << 1) + 1]);
+        } else {
+          *dst = v[h];
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < (1 << NH); ++h) {
+      const float* g = v + (h << L);
+      const int i0 = (t << L) | (h << HI);                      // index in row of g[0]
+      const unsigned long long idx0 = (unsigned long long)prow * D + i0;
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < GE; ++i) amax = fmaxf(amax, fabsf(g[i]));
+#pragma unroll
+      for (int o = 1; o < GL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      uint32_t rnd[GA];
+      if (SR) {
+        if constexpr (GE >= 4) {
+          sr_words<GE>(idx0, p.seed, rnd);
+        } else {
+          const Philox4 ph = philox4x32_10(idx0 >> 2, p.seed);
+#pragma unroll
+          for (int i = 0; i < GE; ++i) rnd[i] = ph.w[(idx0 + i) & 3];
+        }
+      }
+      float y[GA];
+      uint32_t sc, sat = 0, unf = 0, four = 0;
+      if (!NV) {
+        // MXFP4 OCP rule: e = floor(log2 amax) - 2, clamped, all-zero -> 0
+        const uint32_t bits = __float_as_uint(amax);
+        const int ef = (int)((bits >> 23) & 0xFFu);
+        int e = (amax == 0.0f) ? 0 : (ef == 0 ? -127 : ef - 129);
+        e = e < -127 ? -127 : e;
+        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+        for (int i = 0; i < GE; ++i) {
+          float tt = __fmul_rn(g[i], inv);
+          sat += fabsf(tt) > 6.0f;
+          if (SR) { tt = sr_round(tt, rnd[i]); unf += (g[i] != 0.0f) & (tt == 0.0f); }
+          else unf += (g[i] != 0.0f) & (fabsf(tt) <= 0.25f);
+          y[i] = tt;
+        }
+        sc = (uint32_t)(e + 127);
+      } else {
+        float yy[2][GA], sq[2][GA];
+        uint32_t scs[2], sats[2] = {0u, 0u}, unfs[2] = {0u, 0u};
+        const int ncand = FOUR_SIX ? 2 : 1;
+#pragma unroll
+        for (int k = 0; k < ncand; ++k) {
+          const uint32_t code = e4m3_code(__fmul_rn(amax, k == 0 ? inv6 : inv4));
+          const float d = e4m3_value(code);
+          scs[k] = code;
+          const float R = code ? __frcp_rn(__fmul_rn(d, s_g)) : 0.0f;
+#pragma unroll
+          for (int i = 0; i < GE; ++i) {
+            float tt;
+            if (code == 0) {
+              tt = copysignf(0.0f, g[i]);
+              unfs[k] += g[i] != 0.0f;
+            } else {
+              tt = __fmul_rn(g[i], R);
+              sats[k] += fabsf(tt) > 6.0f;
+              if (SR) { tt = sr_round(tt, rnd[i]); unfs[k] += (g[i] != 0.0f) & (tt == 0.0f); }
+              else unfs[k] += (g[i] != 0.0f) & (fabsf(tt) <= 0.25f);
+            }
+            yy[k][i] = tt;
+          }
+          if (FOUR_SIX) {
+            // exact lattice values: |tt| rounds onto the lattice in the encoder; decode back
+            float qv[GA];
+            e2m1_roundtrip<GE>(yy[k], qv);
+#pragma unroll
+            for (int i = 0; i < GE; ++i) {
+              const float xhat = __fmul_rn(__fmul_rn(qv[i], d), s_g);
+              const float e = __fsub_rn(g[i], xhat);
+              sq[k][i] = __fmul_rn(e, e);
+            }
+          }
+        }
+        int pick = 0;
+        if (FOUR_SIX) {
+          float sse[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            // fp32 sum in element order: every lane of the block adds the broadcast squared
+            // errors of lanes 0..GL-1 of the block, so all of them hold the same sum
+            const int basel = lane & ~(GL - 1);
+            float acc = 0.0f;
+#pragma unroll
+            for (int gg = 0; gg < GL; ++gg) {
+#pragma unroll
+              for (int i = 0; i < GE; ++i) acc = __fadd_rn(acc, __shfl_sync(0xFFFFFFFFu, sq[k][i], basel + gg));
+            }
+            sse[k] = acc;
+          }
+          pick = (sse[1] < sse[0]) ? 1 : 0;
+          four = pick;
+        }
+#pragma unroll
+        for (int i = 0; i < GE; ++i) y[i] = pick ? yy[1][i] : yy[0][i];
+        sc = pick ? scs[1] : scs[0];
+        sat = pick ? sats[1] : sats[0];
+        unf = pick ? unfs[1] : unfs[0];
+      }
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < GE; ++i) cnt[2] += !isfinite(g[i]);
+        cnt[0] += unf;
+        cnt[1] += sat;
+        uint8_t* qrow = p.q + prow * (D / 2);
+        if constexpr (GE == 16) {
+          const uint32_t a = e2m1x8(y), b = e2m1x8(y + 8);
+          *reinterpret_cast<uint2*>(qrow + i0 / 2) = make_uint2(a, b);
+        } else if constexpr (GE == 8) {
+          *reinterpret_cast<uint32_t*>(qrow + i0 / 2) = e2m1x8(y);
+        } else if constexpr (GE == 4) {
+          *reinterpret_cast<uint16_t*>(qrow + i0 / 2) = (uint16_t)e2m1x4(y);
+        } else if constexpr (GE == 2) {
+          float y4[4] = {y[0], y[1], 0.0f, 0.0f};
+          qrow[i0 / 2] = (uint8_t)e2m1x4(y4);
+        }
+        if ((lane & (GL - 1)) == 0) {
+          const unsigned long long blk = (unsigned long long)prow * nb + (i0 >> LB);
+          p.scales[scale_offset(blk, nb, p.tiled)] = (uint8_t)sc;
+          cnt[3] += four;
+        }
+      }
+      if constexpr (GE == 1) {
+        // one value per lane: pair nibbles across neighbouring lanes
+        float y4[4] = {y[0], 0.0f, 0.0f, 0.0f};
+        const uint32_t c1 = e2m1x4(y4) & 0xFu;
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, c1, 1);
+        if (valid && !(lane & 1)) p.q[prow * (D / 2) + i0 / 2] = (uint8_t)(c1 | (other << 4));
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+    row += step;
+  }
+  if (p.counts) flush_counts<4>(cnt, p.counts);
+}
+
+// ---------------------------------------------------------------------------------------------
+template <typename T, int LOG_D>
+static int fwht_grid(long long rows) {
+  using G = Geom<LOG_D>;
+  const int smem = G::ROWS * G::D * 4;
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwht_amax_kernel<T, LOG_D>, G::CTA, smem);
+  if (per_sm < 1) per_sm = 1;
+  const long long want = (rows + G::ROWS - 1) / G::ROWS;
+  const long long cap = (long long)num_sms() * per_sm;
+  return (int)(want < 1 ? 1 : (want < cap ? want : cap));
+}
+
+static FwhtParams make_params(const FwhtLaunch& L) {
+  FwhtParams p;
+  p.x = L.x; p.rows = L.rows;
+  p.c = (float)(1.0 / sqrt((double)L.d));
+  p.tiled = L.tiled; p.reverse = 0; p.seed = L.seed;
+  p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
+  p.six_m = L.four_six ? 1536.0f : 2688.0f;
+  p.rotated_out = L.rotated_out; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
+  return p;
+}
+
+template <typename T, int LOG_D>
+static cudaError_t amax_d(const FwhtParams& p, cudaStream_t s) {
+  using G = Geom<LOG_D>;
+  const int smem = G::ROWS * G::D * 4;
+  cudaFuncSetAttribute(fwht_amax_kernel<T, LOG_D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  fwht_amax_kernel<T, LOG_D><<<fwht_grid<T, LOG_D>(p.rows), G::CTA, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int LOG_D, bool NV, bool SR, bool FS>
+static cudaError_t quant_d(const FwhtParams& p, cudaStream_t s) {
+  using G = Geom<LOG_D>;
+  const int smem = G::ROWS * G::D * 4;
+  auto k = fwht_quant_kernel<T, LOG_D, NV, SR, FS>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  k<<<fwht_grid<T, LOG_D>(p.rows), G::CTA, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int LOG_D>
+static cudaError_t quant_sel(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
+  if (!L.nv) return L.sr ? quant_d<T, LOG_D, false, true, false>(p, s) : quant_d<T, LOG_D, false, false, false>(p, s);
+  if (L.four_six) return L.sr ? quant_d<T, LOG_D, true, true, true>(p, s) : quant_d<T, LOG_D, true, false, true>(p, s);
+  return L.sr ? quant_d<T, LOG_D, true, true, false>(p, s) : quant_d<T, LOG_D, true, false, false>(p, s);
+}
+
+template <typename T>
+static cudaError_t dispatch_amax(const FwhtParams& p, int d, cudaStream_t s) {
+  switch (d) {
+    case 1024: return amax_d<T, 10>(p, s);
+    case 2048: return amax_d<T, 11>(p, s);
+    case 4096: return amax_d<T, 12>(p, s);
+    case 8192: return amax_d<T, 13>(p, s);
+    case 16384: return amax_d<T, 14>(p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t dispatch_quant(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
+  switch (L.d) {
+    case 1024: return quant_sel<T, 10>(p, L, s);
+    case 2048: return quant_sel<T, 11>(p, L, s);
+    case 4096: return quant_sel<T, 12>(p, L, s);
+    case 8192: return quant_sel<T, 13>(p, L, s);
+    case 16384: return quant_sel<T, 14>(p, L, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s) {
+  if (L.rows == 0) return cudaSuccess;
+  FwhtParams p = make_params(L);
+  return L.bf16 ? dispatch_amax<__nv_bfloat16>(p, L.d, s) : dispatch_amax<float>(p, L.d, s);
+}
+
+cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s) {
+  if (L.rows == 0) return cudaSuccess;
+  FwhtParams p = make_params(L);
+  p.reverse = (L.nv && !L.global_in) ? 1 : 0;
+  return L.bf16 ? dispatch_quant<__nv_bfloat16>(p, L, s) : dispatch_quant<float>(p, L, s);
+}
+
+}  // namespace fp4k

@@ -1,0 +1,404 @@
+// gemm_sm100.cu — W4A4 block-scaled GEMM on the sm_100 tensor cores.
+//
+// C[m][n] = alpha * sum_k dA[m][k/B] dB[n][k/B] vA[m][k] vB[n][k], FP32 accumulation in tensor
+// memory, bf16 output.  NVFP4 operands (E4M3 scale per 16, alpha = product of the global scales)
+// run tcgen05.mma kind::mxf4nvf4 with scale_vec::4X; MXFP4 operands (E8M0 scale per 32) the same
+// kind with scale_vec::2X.  ("Sub-4-Bit Microscaling" §2: NVFP4 on the 5th-generation tensor
+// core; metrale `hardware::exec`: NVFP4 activations take the block-scaled FP4 MMA.)
+//
+// Structure: persistent CTAs (one per SM), 128 x 256 output tile, K consumed 256 values (128
+// bytes) per pipeline stage.  Six warps:
+//   warp 0     TMA producer: A/B tiles by 2-D tensor-map loads (128-byte swizzle), the scale
+//              tiles by 1-D bulk copies (they are contiguous in the MMA tile layout);
+//   warp 1     allocates tensor memory and issues, from one lane, tcgen05.cp (scales smem->TMEM)
+//              and tcgen05.mma; tcgen05.commit frees each smem stage and signals the epilogue;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns a 32-lane quarter), scale
+//              by alpha, round to bf16, store.
+// Every mbarrier wait is bounded in time; on expiry the kernel records the site in the caller's
+// status word, tells the other roles to stop, drains what it issued and frees tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "launch.h"
+
+namespace fp4k {
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BKB = 128;  // tile rows, tile cols, K bytes per stage (256 values)
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr int A_BYTES = BM * BKB, B_BYTES = BN * BKB;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COL = 0, SFA_COL = 256, SFB_COL = 288;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+struct Params {
+  int M, N, K;
+  int nv;           // 1: NVFP4 (16-blocks, E4M3), 0: MXFP4 (32-blocks, E8M0)
+  int atoms;        // 512-byte scale atoms per 128 rows per stage (4 NVFP4, 2 MXFP4)
+  int atoms_row;    // scale atoms per 128-row group over the whole K
+  const uint8_t* As;
+  const uint8_t* Bs;
+  const float* Ag;
+  const float* Bg;
+  __nv_bfloat16_raw* C;
+  long long ldc;
+  uint32_t* status;
+};
+
+// ---------------------------------------------------------------------------------------------
+// PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: true when the phase completed; false when this or another role gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status, uint32_t site) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (now_ns() - t0 > kTimeoutNs) {
+      atomicOr(status, 1u << site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// scales: 32 rows x 16 bytes from shared memory, replicated into the four 32-lane quarters
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+template <bool NV>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+  if constexpr (NV) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+  } else {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+  }
+}
+
+#define TC_LD32(taddr, r)                                                                                   \
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                       \
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),        \
+                 "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),      \
+                 "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),      \
+                 "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                           \
+               : "r"(taddr))
+
+// Shared-memory matrix descriptor (sm_100 format, version 1).
+//   K-major operand tile, 128-byte swizzle: 8-row groups 1024 bytes apart (SBO), no LBO.
+//   Scale tile (no swizzle): 8 rows of 16 bytes per core matrix, core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor, kind::mxf4nvf4: E2M1 x E2M1, K-major A and B, M = 128, N = 256,
+// scale type bit 23 (0 = UE4M3, 1 = UE8M0), scale-factor byte ids for A (29-30) and B (4-5).
+__host__ __device__ constexpr uint32_t idesc(bool nv, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((nv ? 0u : 1u) << 23) |
+         ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
+}
+
+// ---------------------------------------------------------------------------------------------
+template <bool NV>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  constexpr int ATOMS = NV ? 4 : 2;           // scale atoms per 128 rows per stage
+  constexpr int SFA_BYTES = ATOMS * 512;
+  constexpr int SFB_BYTES = 2 * ATOMS * 512;  // two 128-row groups
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  constexpr uint32_t TX_BYTES = STAGE_BYTES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                  // STAGES x A_BYTES
+  uint8_t* sB = sA + STAGES * A_BYTES;                 // STAGES x B_BYTES
+  uint8_t* sSFA = sB + STAGES * B_BYTES;               // STAGES x SFA_BYTES
+  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;           // STAGES x SFB_BYTES
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  // bars: full[STAGES], empty[STAGES], tmem_full, tmem_empty, drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+  const uint32_t tmem_full = smem_u32(bars + 2 * STAGES), tmem_empty = smem_u32(bars + 2 * STAGES + 1);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 2);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int tiles_m = p.M / BM, tiles_n = p.N / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kt_count = p.K / 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+      uint32_t g = 0;  // global k-iteration counter
+      uint32_t last_parity[STAGES];
+      bool pending[STAGES];
+      for (int s = 0; s < STAGES; ++s) { pending[s] = false; last_parity[s] = 0; }
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        for (int kt = 0; kt < kt_count; ++kt, ++g) {
+          const int s = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * s;
+          mbar_expect_tx(fb, TX_BYTES);
+          pending[s] = true;
+          last_parity[s] = ph;
+          tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, kt * BKB, tm * BM, fb);
+          tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, kt * BKB, tn * BN, fb);
+          const uint8_t* sfa = p.As + ((size_t)tm * p.atoms_row + (size_t)kt * ATOMS) * 512;
+          bulk_load(smem_u32(sSFA + s * SFA_BYTES), sfa, SFA_BYTES, fb);
+#pragma unroll
+          for (int rg = 0; rg < 2; ++rg) {
+            const uint8_t* sfb = p.Bs + ((size_t)(2 * tn + rg) * p.atoms_row + (size_t)kt * ATOMS) * 512;
+            bulk_load(smem_u32(sSFB + s * SFB_BYTES + rg * ATOMS * 512), sfb, ATOMS * 512, fb);
+          }
+        }
+      }
+      if (!ok) {
+        // drain: every fill issued must land before the CTA's shared memory goes away
+        for (int s = 0; s < STAGES; ++s) {
+          if (!pending[s]) continue;
+          const unsigned long long t0 = now_ns();
+          while (!mbar_try(full0 + 8 * s, last_parity[s]) && now_ns() - t0 < kTimeoutNs) {
+          }
+        }
+      } else {
+        // wait for the MMA side to release the last STAGES fills, so that no tcgen05.commit
+        // arrival is still in flight towards this CTA's barriers when it exits
+        for (int i = 0; i < STAGES; ++i, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait(empty0 + 8 * s, ((g / STAGES) & 1) ^ 1, abort_flag, p.status, 4)) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    uint32_t g = 0, j = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++j) {
+      if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1)) { ok = false; break; }
+      tc_fence_after();
+      for (int kt = 0; kt < kt_count; ++kt, ++g) {
+        const int s = g % STAGES;
+        const uint32_t ph = (g / STAGES) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.status, 2)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + s * A_BYTES), b0 = smem_u32(sB + s * B_BYTES);
+          const uint32_t fa = smem_u32(sSFA + s * SFA_BYTES), fbs = smem_u32(sSFB + s * SFB_BYTES);
+#pragma unroll
+          for (int a = 0; a < ATOMS; ++a) {
+            tc_cp_sf(tmem + SFA_COL + 4 * a, desc_sf(fa + a * 512));
+            tc_cp_sf(tmem + SFB_COL + 8 * a, desc_sf(fbs + a * 512));
+            tc_cp_sf(tmem + SFB_COL + 8 * a + 4, desc_sf(fbs + (ATOMS + a) * 512));
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {  // four K=64 MMAs per 256-value stage
+            const int atom = NV ? t : (t >> 1);
+            const uint32_t sf_id = NV ? 0u : (uint32_t)((t & 1) * 2);
+            tc_mma<NV>(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc(NV, sf_id, sf_id),
+                       tmem + SFA_COL + 4 * atom, tmem + SFB_COL + 8 * atom, (kt > 0 || t > 0) ? 1u : 0u);
+          }
+          tc_commit(empty0 + 8 * s);  // stage free once these MMAs have read it
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(tmem_full);
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      tc_commit(drain);
+      const unsigned long long t0 = now_ns();
+      while (!mbar_try(drain, 0) && now_ns() - t0 < kTimeoutNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const float alpha = p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f;
+    uint32_t j = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3)) break;
+      tc_fence_after();
+      const int row = tm * BM + q * 32 + lane;
+      uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        TC_LD32(tmem + ACC_COL + ((uint32_t)(q * 32) << 16) + c * 32, r);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float lo = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
+          const float hi = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
+          uint32_t b;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b) : "f"(hi), "f"(lo));
+          packed[i] = b;
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          crow[c * 4 + v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+      }
+      tc_fence_before();
+      mbar_arrive(tmem_empty);  // accumulator read out: the next tile may start
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+template <bool NV>
+constexpr int smem_bytes() {
+  constexpr int atoms = NV ? 4 : 2;
+  return 1024 + STAGES * (A_BYTES + B_BYTES + atoms * 512 * 3) + 256;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side: tensor maps through the driver entry point (no link against libcuda).
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)BKB, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace gemm
+
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
+  using namespace gemm;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, L.Aq, (uint64_t)L.K / 2, (uint64_t)L.M, BM) ||
+      !make_map(&tb, L.Bq, (uint64_t)L.K / 2, (uint64_t)L.N, BN))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.M = L.M; p.N = L.N; p.K = L.K; p.nv = L.nv ? 1 : 0;
+  p.atoms = L.nv ? 4 : 2;
+  p.atoms_row = L.K / (L.nv ? 16 : 32) / 4;
+  p.As = L.As; p.Bs = L.Bs; p.Ag = L.Ag; p.Bg = L.Bg;
+  p.C = reinterpret_cast<__nv_bfloat16_raw*>(L.C);
+  p.ldc = L.ldc;
+  p.status = L.status;
+  const int tiles = (L.M / BM) * (L.N / BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  if (L.nv) {
+    auto k = gemm_kernel<true>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<true>());
+    k<<<grid, NUM_THREADS, smem_bytes<true>(), s>>>(ta, tb, p);
+  } else {
+    auto k = gemm_kernel<false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<false>());
+    k<<<grid, NUM_THREADS, smem_bytes<false>(), s>>>(ta, tb, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fp4k

@@ -1,0 +1,78 @@
+// launch.h — internal interface between the C ABI (capi.cu) and the kernel translation units.
+// Arguments arrive here already validated; launchers only configure grids and enqueue.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp4k {
+
+int num_sms();  // SM count of the current device (cached per device)
+
+struct QuantLaunch {
+  const void* x;
+  bool bf16;
+  long long rows, cols;
+  bool nv;        // NVFP4 (block 16, E4M3) vs MXFP4 (block 32, E8M0)
+  int policy;     // MXFP4 exponent rule
+  bool sr;        // stochastic rounding
+  bool four_six;  // NVFP4 4/6
+  unsigned long long seed;
+  int tiled;      // scale layout
+  int reverse;    // walk tiles last-to-first
+  const float* global_in;    // NVFP4: caller-fixed s_g, or NULL to derive from *amax_bits
+  const uint32_t* amax_bits;
+  float* global_out;
+  uint8_t* q;
+  uint8_t* scales;
+  unsigned long long* counts;  // 4 counters or NULL
+};
+
+struct DequantLaunch {
+  const uint8_t* q;
+  const uint8_t* scales;
+  bool nv;
+  int tiled;
+  const float* global;
+  long long rows, cols;
+  bool out_bf16;
+  void* out;
+};
+
+struct FwhtLaunch {
+  const void* x;
+  bool bf16;
+  long long rows;
+  int d;
+  bool nv;
+  bool sr;
+  bool four_six;
+  unsigned long long seed;
+  int tiled;
+  const float* global_in;
+  uint32_t* amax_bits;   // workspace word (pass 1 output / pass 2 input)
+  float* global_out;
+  float* rotated_out;
+  uint8_t* q;
+  uint8_t* scales;
+  unsigned long long* counts;
+};
+
+struct GemmLaunch {
+  bool nv;
+  int M, N, K;
+  const uint8_t *Aq, *As, *Bq, *Bs;
+  const float *Ag, *Bg;
+  void* C;
+  long long ldc;
+  uint32_t* status;  // device status word
+};
+
+cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits, cudaStream_t s);
+cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
+cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);
+cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s);
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s);
+
+}  // namespace fp4k

@@ -1,0 +1,412 @@
+// quantize.cu — MXFP4 / NVFP4 block quantisers, the tensor-amax reduction and the dequantiser.
+//
+// All three are HBM-bound streaming kernels.  The row-major tensor is viewed as a flat array of
+// 32-byte chunks (16 bf16 or 8 fp32 values); a warp reads 32 consecutive chunks (1 KiB, one
+// 256-bit load per lane) per step, kUnroll steps in flight per lane.  A quantisation block of B
+// values is G = B / E adjacent lanes: for the bf16 NVFP4 case G = 1, so a lane owns a whole block
+// (amax, scale, both 4/6 candidates and their error sums without any cross-lane traffic).  Blocks
+// never straddle rows because cols % B == 0.
+//
+// Per-element work is kept to the encode itself: the block amax is an integer max over the
+// magnitude bits (which also exposes Inf/NaN: a block with a non-finite value has amax bits
+// >= 0x7F800000 and only then counts per element); saturation is counted per element only when
+// the block's normalised maximum exceeds 6; underflow = zero codes minus zero inputs, both from
+// popcounts over the packed bits.
+//
+// Sources: "MXFP4 Quantization: Audit the 4.25-Bit Blocks" ("Read the shared E8M0 scale",
+// "Encode one MXFP4 block step by step"); "Sub-4-Bit Microscaling" §1-§2 (E2M1, NVFP4 two-level
+// scaling); podcast "Adaptive Block-Scaled Data Types" (stochastic rounding, Four Over Six).
+#include "fp4_device.cuh"
+#include "launch.h"
+
+namespace fp4k {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+// ---------------------------------------------------------------------------------------------
+// MXFP4 shared exponent from the amax bit pattern (exact): OCP floor(log2 amax) - 2, or the
+// smallest e with amax <= 6 * 2^e; clamped to [-127, 127]; an all-zero block takes e = 0.
+__device__ __forceinline__ int mx_exponent(uint32_t bits, int policy) {
+  const int ef = (int)((bits >> 23) & 0xFFu);
+  if (bits == 0u) return 0;
+  if (ef == 0) return -127;  // subnormal maximum: below 2^-126, clamps
+  const int E = ef - 127;
+  const int e = (policy == 0) ? E - 2 : (((bits & 0x7FFFFFu) <= 0x400000u) ? E - 2 : E - 1);
+  return e < -127 ? -127 : e;
+}
+
+struct NvScale {
+  float s_g, inv6, inv4;
+};
+
+__device__ __forceinline__ NvScale nv_scales(const float* global_in, const uint32_t* amax_bits,
+                                             float six_m) {
+  NvScale s;
+  if (global_in) {
+    s.s_g = *global_in;
+  } else {
+    const float amax = __uint_as_float(*amax_bits);
+    s.s_g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, six_m);
+  }
+  s.inv6 = __frcp_rn(__fmul_rn(6.0f, s.s_g));
+  s.inv4 = __frcp_rn(__fmul_rn(4.0f, s.s_g));
+  return s;
+}
+
+// E values scaled by `R` (a power of two for MXFP4) and E2M1-encoded (RNE or stochastic).
+// Returns the packed nibbles in w[E/8] (E = 8 or 16); adds saturations to `sat`.
+template <int E, bool SR>
+__device__ __forceinline__ void encode(const float* v, float R, float top, const uint32_t* rnd,
+                                       uint32_t* w, uint32_t& sat) {
+  float y[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) y[i] = __fmul_rn(v[i], R);
+  if (top > 6.0f) {  // some |y| > 6 only if the block maximum normalises above 6
+#pragma unroll
+    for (int i = 0; i < E; ++i) sat += fabsf(y[i]) > 6.0f;
+  }
+  if (SR) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) y[i] = sr_round(y[i], rnd[i]);
+  }
+#pragma unroll
+  for (int k = 0; k < E / 8; ++k) w[k] = e2m1x8(y + 8 * k);
+}
+
+// One NVFP4 candidate (target T through inv_t): block scale code, packed nibbles, saturations.
+template <int E, bool SR>
+__device__ __forceinline__ uint32_t nv_candidate(const float* v, float amax, float s_g, float inv_t,
+                                                 const uint32_t* rnd, uint32_t* w, uint32_t& sat,
+                                                 float& d) {
+  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
+  d = e4m3_value(sc);
+  sat = 0;
+  if (sc == 0) {
+    float y[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) y[i] = copysignf(0.0f, v[i]);
+#pragma unroll
+    for (int k = 0; k < E / 8; ++k) w[k] = e2m1x8(y + 8 * k);
+  } else {
+    const float R = __frcp_rn(__fmul_rn(d, s_g));
+    encode<E, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
+  }
+  return sc;
+}
+
+// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2) of the lane's E values.
+template <int E>
+__device__ __forceinline__ void sq_errors(const float* v, const uint32_t* w, float d, float s_g, float* sq) {
+#pragma unroll
+  for (int k = 0; k < E / 8; ++k) {
+    float q[8];
+    e2m1_unpack<8>(w[k], q);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float xhat = __fmul_rn(__fmul_rn(q[i], d), s_g);
+      const float e = __fsub_rn(v[8 * k + i], xhat);
+      sq[8 * k + i] = __fmul_rn(e, e);
+    }
+  }
+}
+
+// fp32 sum of the block's squared errors in element order.  G = 1: the lane owns the block.
+// G > 1: every lane of the block adds the broadcast values of lanes 0..G-1 in order.
+template <int E, int G>
+__device__ __forceinline__ float block_sse(const float* sq, int lane) {
+  float acc = 0.0f;
+  if constexpr (G == 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) acc = __fadd_rn(acc, sq[i]);
+  } else {
+    const int base = lane & ~(G - 1);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) acc = __fadd_rn(acc, __shfl_sync(0xFFFFFFFFu, sq[i], base + g));
+    }
+  }
+  return acc;
+}
+
+struct QuantParams {
+  const void* x;
+  long long n_chunks;  // rows * cols / E
+  uint32_t nb;         // blocks per row
+  int policy;          // MXFP4 exponent rule
+  int tiled;           // scale layout
+  int reverse;         // walk the tiles last-to-first (re-use the tail a previous pass left in L2)
+  unsigned long long seed;
+  const float* global_in;
+  const uint32_t* amax_bits;
+  float* global_out;
+  float six_m;
+  uint8_t* q;
+  uint8_t* scales;
+  unsigned long long* counts;
+};
+
+template <typename T, bool NV, bool SR, bool FOUR_SIX>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
+  constexpr int E = Vec32<T>::E;  // 16 (bf16) or 8 (fp32)
+  constexpr int B = NV ? 16 : 32;
+  constexpr int G = B / E;
+  constexpr int W = E / 8;        // packed words per chunk
+  const int lane = threadIdx.x & 31;
+  const long long warp = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
+  const long long per_tile = 32LL * kUnroll;
+  const long long ntiles = (p.n_chunks + per_tile - 1) / per_tile;
+
+  NvScale ns{1.0f, 1.0f, 1.0f};
+  if (NV) {
+    ns = nv_scales(p.global_in, p.amax_bits, p.six_m);
+    if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = ns.s_g;
+  }
+  uint32_t cnt[4] = {0u, 0u, 0u, 0u};  // underflow, saturation, nonfinite, blocks_four
+  const char* xb = reinterpret_cast<const char*>(p.x);
+
+  for (long long t = warp; t < ntiles; t += nwarps) {
+    const long long tile = p.reverse ? (ntiles - 1 - t) : t;
+    const long long c0 = tile * per_tile + lane;
+    U8 raw[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = c0 + 32LL * u;
+      if (c < p.n_chunks) {
+        raw[u] = ld32<true>(xb + c * 32);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) raw[u].w[i] = 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = c0 + 32LL * u;
+      const bool valid = c < p.n_chunks;
+      float v[E];
+      Vec32<T>::unpack(raw[u], v);
+      uint32_t am = 0u;
+#pragma unroll
+      for (int i = 0; i < E; ++i) am = max(am, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+#pragma unroll
+      for (int o = 1; o < G; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      if (am >= 0x7F800000u && valid) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) cnt[2] += !isfinite(v[i]);
+      }
+      const float amax = __uint_as_float(am);
+      const unsigned long long idx0 = (unsigned long long)c * E;
+      uint32_t rnd[E];
+      if (SR) sr_words<E>(idx0, p.seed, rnd);
+      uint32_t w[W], sc, sat = 0, four = 0;
+      if (!NV) {
+        const int e = mx_exponent(am, p.policy);
+        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+        encode<E, SR>(v, inv, __fmul_rn(amax, inv), rnd, w, sat);
+        sc = (uint32_t)(e + 127);
+      } else if (!FOUR_SIX) {
+        float d;
+        sc = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d);
+      } else {
+        float d6, d4, sq[E];
+        uint32_t w4[W], sat4;
+        const uint32_t sc6 = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d6);
+        const uint32_t sc4 = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv4, rnd, w4, sat4, d4);
+        sq_errors<E>(v, w, d6, ns.s_g, sq);
+        const float sse6 = block_sse<E, G>(sq, lane);
+        sq_errors<E>(v, w4, d4, ns.s_g, sq);
+        const float sse4 = block_sse<E, G>(sq, lane);
+        sc = sc6;
+        if (sse4 < sse6) {
+          sc = sc4;
+          sat = sat4;
+          four = 1;
+#pragma unroll
+          for (int k = 0; k < W; ++k) w[k] = w4[k];
+        }
+      }
+      if (valid) {
+        int zc = 0;
+#pragma unroll
+        for (int k = 0; k < W; ++k) zc += zero_nibbles(w[k]);
+        cnt[0] += (uint32_t)(zc - Vec32<T>::zeros(raw[u]));
+        cnt[1] += sat;
+        if (W == 2) {
+          reinterpret_cast<uint2*>(p.q)[c] = make_uint2(w[0], w[W - 1]);
+        } else {
+          reinterpret_cast<uint32_t*>(p.q)[c] = w[0];
+        }
+        if ((lane & (G - 1)) == 0) {
+          const unsigned long long blk = (unsigned long long)c / G;
+          p.scales[scale_offset(blk, p.nb, p.tiled)] = (uint8_t)sc;
+          cnt[3] += four;
+        }
+      }
+    }
+  }
+  if (p.counts) flush_counts<4>(cnt, p.counts);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Tensor amax (NVFP4 global scale, first pass): max |x| over the whole tensor as an integer max
+// of the magnitude bits (monotone for non-negative floats), one atomicMax per CTA.  Loads keep
+// their L2 lines so the second pass, walking the tiles in reverse, starts on resident data.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long n_chunks,
+                                                        uint32_t* amax_bits) {
+  constexpr int E = Vec32<T>::E;
+  const char* xb = reinterpret_cast<const char*>(x);
+  const long long tid = (long long)blockIdx.x * kThreads + threadIdx.x;
+  const long long stride = (long long)gridDim.x * kThreads;
+  uint32_t m = 0u;
+  long long c = tid;
+  for (; c + 3 * stride < n_chunks; c += 4 * stride) {
+    U8 r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r[u] = ld32<false>(xb + (c + u * stride) * 32);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float v[E];
+      Vec32<T>::unpack(r[u], v);
+#pragma unroll
+      for (int i = 0; i < E; ++i) m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+    }
+  }
+  for (; c < n_chunks; c += stride) {
+    float v[E];
+    Vec32<T>::unpack(ld32<false>(xb + c * 32), v);
+#pragma unroll
+    for (int i = 0; i < E; ++i) m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t wm[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0u;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) b = max(b, wm[w]);
+    atomicMax(amax_bits, b);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Dequantiser: each lane expands 8 packed bytes (16 values).  x_hat = fl(fl(v*d)*s_g) (NVFP4) or
+// v * 2^(byte-127) (MXFP4, exact).  bf16 output is the RNE cast of the fp32 value.
+template <bool NV, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, const uint8_t* scales,
+                                                           const float* global, long long n_groups,
+                                                           uint32_t nb, int tiled, void* out) {
+  constexpr int B = NV ? 16 : 32;
+  const float s_g = NV ? *global : 1.0f;
+  const long long stride = (long long)gridDim.x * kThreads;
+  for (long long g = (long long)blockIdx.x * kThreads + threadIdx.x; g < n_groups; g += stride) {
+    const uint2 w = *reinterpret_cast<const uint2*>(q + g * 8);
+    const unsigned long long blk = (unsigned long long)(g * 16) / B;
+    const uint8_t sb = scales[scale_offset(blk, nb, tiled)];
+    float d;
+    if (NV) d = e4m3_value(sb);
+    else d = __uint_as_float((uint32_t)sb << 23);  // 2^(sb-127); sb = 0 -> 0 (handled below)
+    float v[16];
+    e2m1_unpack<8>(w.x, v);
+    e2m1_unpack<8>(w.y, v + 8);
+    float o[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (NV) {
+        o[i] = __fmul_rn(__fmul_rn(v[i], d), s_g);
+      } else if (sb != 0) {
+        o[i] = __fmul_rn(v[i], d);
+      } else {
+        o[i] = __fmul_rn(__fmul_rn(v[i], 0x1p-64f), 0x1p-63f);  // v * 2^-127, exact (subnormal)
+      }
+    }
+    if (OUT_BF16) {
+      uint32_t pw[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pw[i] = bf16x2_pack(o[2 * i], o[2 * i + 1]);
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + g * 16);
+      dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + g * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Launchers
+
+static int grid_for(long long work_items, int per_cta) {
+  const long long want = (work_items + per_cta - 1) / per_cta;
+  const long long cap = (long long)num_sms() * (2048 / kThreads);
+  return (int)(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+template <typename T, bool NV, bool SR, bool FS>
+static cudaError_t launch_q(const QuantParams& p, cudaStream_t s) {
+  const long long tiles = (p.n_chunks + 32LL * kUnroll - 1) / (32LL * kUnroll);
+  const int grid = grid_for(tiles * 32, kThreads);
+  quantize_kernel<T, NV, SR, FS><<<grid, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t dispatch_q(const QuantParams& p, bool nv, bool sr, bool fs, cudaStream_t s) {
+  if (!nv) return sr ? launch_q<T, false, true, false>(p, s) : launch_q<T, false, false, false>(p, s);
+  if (fs) return sr ? launch_q<T, true, true, true>(p, s) : launch_q<T, true, false, true>(p, s);
+  return sr ? launch_q<T, true, true, false>(p, s) : launch_q<T, true, false, false>(p, s);
+}
+
+cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
+  QuantParams p;
+  const int E = L.bf16 ? 16 : 8;
+  p.x = L.x;
+  p.n_chunks = (long long)(L.rows * L.cols / E);
+  p.nb = (uint32_t)(L.cols / (L.nv ? 16 : 32));
+  p.policy = L.policy;
+  p.tiled = L.tiled;
+  p.reverse = L.reverse;
+  p.seed = L.seed;
+  p.global_in = L.global_in;
+  p.amax_bits = L.amax_bits;
+  p.global_out = L.global_out;
+  p.six_m = L.four_six ? 1536.0f : 2688.0f;
+  p.q = L.q;
+  p.scales = L.scales;
+  p.counts = L.counts;
+  if (p.n_chunks == 0) return cudaSuccess;
+  return L.bf16 ? dispatch_q<__nv_bfloat16>(p, L.nv, L.sr, L.four_six, s)
+                : dispatch_q<float>(p, L.nv, L.sr, L.four_six, s);
+}
+
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits, cudaStream_t s) {
+  const long long chunks = n_elems / (bf16 ? 16 : 8);
+  if (chunks == 0) return cudaSuccess;
+  const int grid = grid_for(chunks / 4 + 1, kThreads);
+  if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits);
+  else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s) {
+  const long long groups = L.rows * L.cols / 16;
+  if (groups == 0) return cudaSuccess;
+  const uint32_t nb = (uint32_t)(L.cols / (L.nv ? 16 : 32));
+  const int grid = grid_for(groups, kThreads);
+  if (L.nv) {
+    if (L.out_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(L.q, L.scales, L.global, groups, nb, L.tiled, L.out);
+    else dequant_kernel<true, false><<<grid, kThreads, 0, s>>>(L.q, L.scales, L.global, groups, nb, L.tiled, L.out);
+  } else {
+    if (L.out_bf16) dequant_kernel<false, true><<<grid, kThreads, 0, s>>>(L.q, L.scales, nullptr, groups, nb, L.tiled, L.out);
+    else dequant_kernel<false, false><<<grid, kThreads, 0, s>>>(L.q, L.scales, nullptr, groups, nb, L.tiled, L.out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fp4k

@@ -1,0 +1,206 @@
+/*
+ * fp4mx.h — C ABI of libfp4mx.so: block-scaled 4-bit (E2M1) microscaling on NVIDIA B200 (sm_100a).
+ *
+ * Every entry point takes plain pointers and sizes.  Pointers documented as "device" must point to
+ * memory the caller allocated on the current CUDA device; the library never allocates, frees or
+ * synchronises.  All work is enqueued on the caller's `stream` (a cudaStream_t passed as void*;
+ * NULL = the legacy default stream) and returns as soon as it is enqueued.
+ *
+ * Error behaviour (all entry points):
+ *   - argument errors (bad sizes, unsupported combinations, NULL required pointers, misaligned
+ *     buffers) return FP4_EINVAL or FP4_EUNSUPPORTED synchronously, before anything is launched;
+ *     a format is never silently replaced by another one;
+ *   - a failed launch returns FP4_ECUDA; fp4_last_error() then describes it;
+ *   - data problems are never trapped on the device: non-finite inputs are counted in
+ *     fp4_counts.nonfinite and the outputs of the affected blocks are unspecified.
+ *
+ * Sources the operations follow (cited by page title and section):
+ *   [E]  "Sub-4-Bit Microscaling (NVFP4, MXFP4 & Walsh-Hadamard Rotation)" (Eluvix docs),
+ *        §1 E2M1, §2 MXFP4 vs NVFP4, §3 Walsh-Hadamard rotation.
+ *   [A]  "MXFP4 Quantization: Audit the 4.25-Bit Blocks", sections "Read the FP4 E2M1 value
+ *        lattice", "Read the shared E8M0 scale", "Encode one MXFP4 block step by step",
+ *        "Publish the MXFP4 audit receipt".
+ *   [X]  metrale `hardware::exec` module docs: the activation format picks the MMA kind; NVFP4
+ *        runs on the block-scaled FP4 MMA.
+ *   [P]  podcast "Adaptive Block-Scaled Data Types for FP4 Training" (segments on block scaling,
+ *        the Hadamard transform and stochastic rounding, and Four Over Six).
+ */
+#ifndef FP4MX_H
+#define FP4MX_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FP4_API __attribute__((visibility("default")))
+#else
+#define FP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp4_status {
+  FP4_OK = 0,
+  FP4_EINVAL = 1,        /* bad argument: size, NULL pointer, alignment, layout precondition */
+  FP4_EUNSUPPORTED = 2,  /* well-formed request for a combination this library does not run */
+  FP4_ECUDA = 3          /* a CUDA call or kernel launch failed */
+} fp4_status;
+
+typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
+
+/* MXFP4: 32 E2M1 elements share one E8M0 byte (value 2^(byte-127), 0xFF = NaN, never produced).
+ * NVFP4: 16 E2M1 elements share one E4M3 byte (positive, OCP E4M3FN: bias 7, max 448) under one
+ *        FP32 per-tensor global scale s_g.   [E] §2, [P] block-scaling segment. */
+typedef enum fp4_format { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_format;
+
+/* RNE: round to nearest on the E2M1 lattice {0,.5,1,1.5,2,3,4,6}, an exact tie takes the code with
+ * the even mantissa bit ([A] "Read the FP4 E2M1 value lattice").
+ * STOCHASTIC: round up to the next lattice point with probability (a-lo)/(hi-lo), decided by one
+ * 32-bit Philox4x32-10 word per element ([P] stochastic-rounding segment).  The word for flat
+ * row-major element index i is output word (i & 3) of Philox4x32-10 with key (seed low 32 bits,
+ * seed high 32 bits) and counter (i>>2 low 32, i>>2 high 32, 0, 0); the element rounds up iff
+ * word < ceil(p * 2^32).  Block scales are always chosen with RNE. */
+typedef enum fp4_round { FP4_RNE = 0, FP4_STOCHASTIC = 1 } fp4_round;
+
+/* MXFP4 shared-exponent rule.
+ * OCP_FLOOR : e = floor(log2 amax) - 2 clamped to [-127,127]; the block top may exceed 6 and
+ *             saturate ([A] "Read the shared E8M0 scale", worked example with max 13).
+ * NOSAT_CEIL: the smallest e with amax <= 6 * 2^e, clamped; never saturates but can leave the top
+ *             lattice steps 4 and 6 unused ([E] §2 "sawtooth cliff").
+ * An all-zero block uses e = 0 (byte 127) under both rules. */
+typedef enum fp4_mx_policy { FP4_MX_OCP_FLOOR = 0, FP4_MX_NOSAT_CEIL = 1 } fp4_mx_policy;
+
+/* Scale-byte layout.
+ * ROWMAJOR : scales[r * (cols/B) + j] is the scale of block j of row r.
+ * MMA_TILED: the layout the sm_100 block-scaled MMA reads from tensor memory.  Rows are grouped in
+ *            tiles of 128 and block columns in groups of 4; each (128 x 4) tile is 512 contiguous
+ *            bytes, tiles ordered block-column-group fastest:
+ *              off(r, j) = ((r/128) * (cols/B/4) + j/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + j%4
+ *            Requires rows % 128 == 0 and (cols/B) % 4 == 0.  fp4_block_gemm requires it. */
+typedef enum fp4_scale_layout { FP4_SCALES_ROWMAJOR = 0, FP4_SCALES_MMA_TILED = 1 } fp4_scale_layout;
+
+/* Encoding counters, tensor totals.  Lives in DEVICE memory; every quantize call zeroes it on its
+ * stream before counting.  underflow: nonzero source whose code is +-0.  saturation: normalised
+ * magnitude strictly above 6 (clamped to +-6).  nonfinite: Inf/NaN source elements.
+ * blocks_four: NVFP4 4/6 blocks that chose the max->4 scaling.  Counts come from the chosen
+ * encoding only.  [A] "Read the FP4 E2M1 value lattice", "Expose outlier and dead-zone damage". */
+typedef struct fp4_counts {
+  unsigned long long underflow;
+  unsigned long long saturation;
+  unsigned long long nonfinite;
+  unsigned long long blocks_four;
+} fp4_counts;
+
+/* Operation ids for fp4_workspace_size. */
+typedef enum fp4_op { FP4_OP_MX_QUANTIZE = 0, FP4_OP_NVFP4_QUANTIZE = 1, FP4_OP_FWHT_QUANTIZE = 2,
+                      FP4_OP_DEQUANTIZE = 3, FP4_OP_BLOCK_GEMM = 4 } fp4_op;
+
+/* ---------------------------------------------------------------------------------------------
+ * mx_quantize — MXFP4 quantisation of a row-major [rows, cols] tensor, blocks of 32 along rows.
+ * Follows [A] "Encode one MXFP4 block step by step": per block amax, shared exponent e (policy),
+ * y = x * 2^-e (exact), E2M1 encode (RNE or stochastic), saturate at 6, nibble pack.
+ *   x      : device, [rows, cols] of `dtype`, 32-byte aligned (FWHT input: 16-byte aligned).
+ *   block  : must be 32 (no block-size inference; anything else is FP4_EINVAL).
+ *   q      : device, [rows, cols/2] bytes, 8-byte aligned; element 2j in the low nibble of byte j, 2j+1 high
+ *            ([A] "Encode one MXFP4 block": values 0 and 1 share the first byte, low half first).
+ *   scales : device, rows*cols/32 E8M0 bytes in `layout`.
+ *   counts : device fp4_counts or NULL (no counting).
+ * Preconditions: rows >= 0, cols % 32 == 0 (an incomplete block is rejected), cols > 0 if rows > 0.
+ * Empty tensors (rows == 0) are accepted and launch nothing except zeroing `counts`. */
+FP4_API fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
+                       fp4_mx_policy policy, fp4_round round, unsigned long long seed,
+                       fp4_scale_layout layout, unsigned char* q, unsigned char* scales,
+                       fp4_counts* counts, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_quantize — NVFP4 two-level quantisation, blocks of 16 along rows.  [E] §2, [P] Four Over
+ * Six segment.  Global scale s_g = fl(amax_t / (6*M)) with M = 448 (M = 256 when four_six != 0,
+ * the reduced global range that keeps the max->4 candidate finite); s_g = 1 when amax_t == 0.
+ * For target T (6, and also 4 under four_six): inv_T = fl(1/fl(T*s_g)); block code =
+ * E4M3_RNE_satfinite(fl(amax_b * inv_T)) with decoded value d; elements y = fl(x * fl(1/fl(d*s_g)))
+ * are E2M1-encoded; a code of 0 encodes the whole block as signed zeros.  Under four_six each block
+ * keeps the candidate whose fp32 sum of squared dequantisation errors is strictly lower (ties
+ * keep 6).
+ *   global_in  : device float or NULL.  NULL: a first pass reduces amax_t over the tensor (two
+ *                passes over x).  Non-NULL: the caller fixes s_g = *global_in (one pass).
+ *   global_out : device float or NULL; receives the s_g used.
+ *   q, scales, counts : as in mx_quantize (E4M3 scale bytes).
+ *   workspace  : device, >= fp4_workspace_size(FP4_OP_NVFP4_QUANTIZE, rows, cols) bytes, 16-byte
+ *                aligned; required when global_in == NULL.  Clobbered.
+ * Preconditions: block == 16, cols % 16 == 0. */
+FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
+                          fp4_round round, int four_six, unsigned long long seed,
+                          fp4_scale_layout layout, const float* global_in, float* global_out,
+                          unsigned char* q, unsigned char* scales, fp4_counts* counts,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * fwht_quantize — normalised Walsh-Hadamard rotation of every row (length d), fused ahead of the
+ * quantiser.  [E] §3 "Orthogonal Walsh-Hadamard Outlier Rotation": H_d has entries +-1/sqrt(d)
+ * (Sylvester order, H[i][j] = (-1)^popcount(i&j)/sqrt(d)) and is applied by O(d log2 d) butterflies.
+ * The rotation is computed in fp32 in a fixed order: unnormalised radix-2 stages h = 1,2,4,...,d/2,
+ * each mapping (a,b) -> (a+b, a-b) for index pairs (i, i+h) with (i & h) == 0, then one multiply by
+ * c = fl(1/sqrt(d)).  The rotated fp32 values are then quantised exactly as nvfp4_quantize
+ * (format FP4_NVFP4, block 16; the global amax is taken over the rotated tensor) or as
+ * mx_quantize with FP4_MX_OCP_FLOOR (format FP4_MXFP4, block 32).  Stochastic rounding indexes
+ * Philox by the flat element index of the rotated [rows, d] tensor.
+ *   d           : power of two, 1024 <= d <= 16384.
+ *   rotated_out : device float [rows, d] or NULL; receives the rotated values (diagnostics).
+ *   other arguments as in nvfp4_quantize; four_six and global_in/out apply to FP4_NVFP4 only. */
+FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_format format,
+                         int block, fp4_round round, int four_six, unsigned long long seed,
+                         fp4_scale_layout layout, const float* global_in, float* global_out,
+                         float* rotated_out, unsigned char* q, unsigned char* scales,
+                         fp4_counts* counts, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * fp4_dequantize — x_hat = fl((v * d) * s_g) per element, v the E2M1 value of the nibble and d the
+ * decoded block scale (v*d is exact); MXFP4 has no s_g (x_hat = v * 2^e, exact).  bf16 output is
+ * the round-to-nearest-even of that fp32 value.  [A] "Encode one MXFP4 block step by step"
+ * (reconstruction = lattice value times scale), [X] block scales applied in FP32.
+ *   q, scales : device, as written by the quantisers (`layout` names the scale layout).
+ *   global    : device float, NVFP4 only (NULL for MXFP4).
+ *   out       : device [rows, cols] of out_dtype, 16-byte aligned. */
+FP4_API fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, fp4_format format,
+                          int block, fp4_scale_layout layout, const float* global, long rows,
+                          long cols, fp4_dtype out_dtype, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * fp4_block_gemm — W4A4 block-scaled GEMM C = alpha * A * B^T on the sm_100 tensor cores
+ * (tcgen05.mma kind::mxf4nvf4 with block scales, FP32 accumulation in tensor memory).
+ * [E] §2 (NVFP4 on the 5th-generation tensor core), [X] (NVFP4 activations take the block-scaled
+ * FP4 MMA).  C[m][n] = alpha * sum_kb dA[m][kb] * dB[n][kb] * sum_{k in kb} vA[m][k] * vB[n][k],
+ * alpha = (*Ag) * (*Bg) for NVFP4 and 1 for MXFP4; C is stored as bf16 (RNE), row-major with
+ * leading dimension ldc (elements).
+ *   Aq : device [M, K/2] packed E2M1, K-major (as written by the quantisers for a [M, K] tensor).
+ *   As : device scales of A in FP4_SCALES_MMA_TILED layout (E4M3 for NVFP4, E8M0 for MXFP4).
+ *   Bq, Bs : the same for B [N, K].
+ *   Ag, Bg : device floats (NVFP4 global scales); ignored (may be NULL) for MXFP4.
+ *   workspace : device, >= fp4_workspace_size(FP4_OP_BLOCK_GEMM, M, N) bytes, 16-byte aligned; the
+ *               kernel's status word (0 = ok, nonzero = a bounded pipeline wait gave up) is its
+ *               first 4 bytes; see fp4_gemm_status_word.
+ * Preconditions: M % 128 == 0, N % 256 == 0, K % 256 == 0, ldc >= N, ldc % 8 == 0, all pointers
+ * 16-byte aligned.  Other shapes return FP4_EUNSUPPORTED. */
+FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
+                          const unsigned char* Aq, const unsigned char* As, const float* Ag,
+                          const unsigned char* Bq, const unsigned char* Bs, const float* Bg,
+                          void* C, long ldc, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace `op` needs for the given sizes (rows/cols; M/N for the GEMM). */
+FP4_API size_t fp4_workspace_size(fp4_op op, long rows, long cols);
+
+/* Byte offset, inside fp4_block_gemm's workspace, of its 32-bit device status word. */
+FP4_API size_t fp4_gemm_status_word(void);
+
+/* Static description of a status code. */
+FP4_API const char* fp4_status_str(fp4_status s);
+
+/* Human-readable detail of the last non-OK status returned on the calling thread. */
+FP4_API const char* fp4_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4MX_H */

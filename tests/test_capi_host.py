@@ -1,0 +1,118 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every function that
+include/fp4mx.h declares, and rejects bad arguments synchronously (before any CUDA call), so
+these run on a machine without a device.  The pointers below are never dereferenced: every call
+fails validation first."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_scaled_fp4_amax_b200 as fp4
+from block_scaled_fp4_amax_b200 import build as fp4build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp4mx.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    fp4build.build()
+    return fp4.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^FP4_API\s+(?:const\s+)?[a-z0-9_]+\s*\*?\s*([a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert set(names) == set(fp4.EXPORTS), names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_workspace(L):
+    assert L.fp4_status_str(0) == b"FP4_OK"
+    assert b"EINVAL" in L.fp4_status_str(1)
+    assert L.fp4_workspace_size(fp4.OP_NVFP4_QUANTIZE, 8192, 8192) >= 4
+    assert L.fp4_workspace_size(fp4.OP_BLOCK_GEMM, 8192, 8192) >= 4
+    assert L.fp4_workspace_size(fp4.OP_MX_QUANTIZE, 8192, 8192) == 0
+    assert L.fp4_gemm_status_word() == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced
+
+
+def _mx(L, **kw):
+    a = dict(x=FAKE, dtype=1, rows=128, cols=256, block=32, policy=0, round=0, seed=0, layout=0,
+             q=FAKE, s=FAKE, c=None)
+    a.update(kw)
+    return L.mx_quantize(a["x"], a["dtype"], a["rows"], a["cols"], a["block"], a["policy"], a["round"],
+                         a["seed"], a["layout"], a["q"], a["s"], a["c"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(block=16), 1),                 # MXFP4 block must be 32: no block-size inference
+    (dict(block=24), 1),
+    (dict(cols=48), 1),                  # incomplete block
+    (dict(cols=0), 1),
+    (dict(rows=-1), 1),
+    (dict(dtype=7), 1),
+    (dict(policy=5), 1),
+    (dict(round=9), 1),
+    (dict(layout=4), 1),
+    (dict(layout=1, rows=100), 1),       # tiled scales need rows % 128 == 0
+    (dict(layout=1, cols=96), 1),        # ... and (cols/32) % 4 == 0
+    (dict(x=None), 1),
+    (dict(q=None), 1),
+    (dict(x=ctypes.c_void_p(0x10004)), 1),  # misaligned input
+])
+def test_mx_quantize_rejects(L, kw, status):
+    assert _mx(L, **kw) == status
+    assert L.fp4_last_error()
+
+
+def test_nvfp4_rejects(L):
+    # block 32 for NVFP4, no workspace without a global scale, MXFP4-only policy irrelevant
+    assert L.nvfp4_quantize(FAKE, 1, 128, 256, 32, 0, 0, 0, 0, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 0, 0, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == 1
+    assert L.nvfp4_quantize(FAKE, 1, 128, 200, 16, 0, 0, 0, 0, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 0, 0, 0, 0, None, None, FAKE, FAKE, None, FAKE, 8, None) == 1
+
+
+def test_fwht_rejects(L):
+    # d not a power of two / out of range, MXFP4 with four-over-six, block mismatch
+    assert L.fwht_quantize(FAKE, 1, 4, 3000, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 512, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 32768, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, 0, 32, 0, 1, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 2
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, 0, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, 5, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
+
+
+def test_dequant_rejects(L):
+    assert L.fp4_dequantize(FAKE, FAKE, 1, 32, 0, FAKE, 128, 256, 0, FAKE, None) == 1  # block mismatch
+    assert L.fp4_dequantize(FAKE, FAKE, 1, 16, 0, None, 128, 256, 0, FAKE, None) == 1  # NVFP4 needs s_g
+    assert L.fp4_dequantize(FAKE, FAKE, 0, 32, 0, None, 128, 80, 0, FAKE, None) == 1   # ragged block
+    assert L.fp4_dequantize(FAKE, FAKE, 0, 32, 0, None, 128, 256, 3, FAKE, None) == 1  # out dtype
+
+
+def test_gemm_rejects(L):
+    g = L.fp4_block_gemm
+    assert g(1, 100, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2  # M % 128
+    assert g(1, 128, 200, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2  # N % 256
+    assert g(1, 128, 256, 200, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2  # K % 256
+    assert g(1, 128, 256, 256, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 1  # no Ag
+    assert g(1, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 256, None) == 1  # ldc < N
+    assert g(1, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None, 0, None) == 1    # workspace
+    assert g(3, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 1  # format
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(fp4, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(fp4, "_lib", None)
+    with pytest.raises(ImportError):
+        fp4.lib()

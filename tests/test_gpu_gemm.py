@@ -1,0 +1,181 @@
+"""GPU parity: the tcgen05 block-scaled GEMM against the fp64 oracle.
+
+Bar: |C_gpu - C64| <= 1e-3 * sum_k |a_k b_k| per element, C64 the fp64 dot product of the exactly
+dequantised operands.  The bf16 output rounding alone can reach 2^-9 |C|, which exceeds that bound
+whenever |C| is a sizeable fraction of sum |a b| — small K, or same-sign data — so the small-shape
+cases add the bf16 rounding term 2^-8 |C64|; the full-size workloads (K = 8192 and 28672) are held
+to the bound alone.  Operands are quantised on the GPU (checked bit-exact
+against the oracle elsewhere) while the reference quantises independently on the CPU.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp4_amax_b200 as fp4
+import oracle as O
+from block_scaled_fp4_amax_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def npy(t):
+    return t.detach().cpu().numpy()
+
+
+def status_ok(ws):
+    torch.cuda.synchronize()
+    return int(ws[:4].view(torch.int32).item()) == 0
+
+
+def quant(x_cpu, fmt, cuda):
+    x = x_cpu.to(cuda)
+    if fmt == fp4.NVFP4:
+        q, s, g, _ = fp4.nvfp4_quantize(x, layout=fp4.MMA_TILED)
+        qo, so, go, _ = O.nvfp4_quantize(synth.as_f32_numpy(x_cpu))
+        return (q, s, g), (qo, so, go)
+    q, s, _ = fp4.mx_quantize(x, layout=fp4.MMA_TILED)
+    qo, so, _ = O.mx_quantize(synth.as_f32_numpy(x_cpu))
+    return (q, s, None), (qo, so, 1.0)
+
+
+def check(C, C64, S, extra_rel=2.0 ** -8):
+    err = np.abs(npy(C.float()).astype(np.float64) - C64)
+    bound = 1e-3 * S + extra_rel * np.abs(C64)
+    bad = err > bound
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside the bound; worst excess {float((err - bound).max())}"
+
+
+def gemm(fmt, A, B):
+    (Aq, As, Ag), (Bq, Bs, Bg) = A, B
+    C, ws = fp4.fp4_block_gemm(fmt, Aq, As, Bq, Bs, Ag, Bg)
+    assert status_ok(ws)
+    return C
+
+
+def packed_from_codes(codes):
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[:, 0::2] & 15) | ((codes[:, 1::2] & 15) << 4)
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
+def test_gemm_one_hot_structure(cuda, fmt):
+    """A[m, k] = 1 only at k = km(m); B[n, k] = 1 only at k = kn(n); every block scale distinct, so
+    C[m, n] = dA[m, km/B] * dB[n, km/B] when km(m) == kn(n), else 0 — an exact bf16 value.  This
+    pins the nibble order inside a byte, the K order inside the swizzled tile and the scale-tile
+    layout of both operands."""
+    M, N, K = 128, 256, 512
+    Bk = 16 if fmt == fp4.NVFP4 else 32
+    nb = K // Bk
+    km = (np.arange(M) * 7 + 3) % K
+    kn = (np.arange(N) * 5 + 1) % K
+    ca = np.zeros((M, K), np.uint8)
+    ca[np.arange(M), km] = 2  # code 2 = 1.0
+    cb = np.zeros((N, K), np.uint8)
+    cb[np.arange(N), kn] = 2
+    rng = np.random.default_rng(0)
+    if fmt == fp4.NVFP4:
+        sa = rng.integers(0x20, 0x50, size=(M, nb)).astype(np.uint8)   # E4M3 2^-3 .. 2^3
+        sb = rng.integers(0x20, 0x50, size=(N, nb)).astype(np.uint8)
+    else:
+        sa = rng.integers(120, 134, size=(M, nb)).astype(np.uint8)     # E8M0 2^-7 .. 2^6
+        sb = rng.integers(120, 134, size=(N, nb)).astype(np.uint8)
+    Aq = torch.from_numpy(packed_from_codes(ca)).to(cuda)
+    Bq = torch.from_numpy(packed_from_codes(cb)).to(cuda)
+    As = torch.from_numpy(O.scales_to_mma_tiled(sa)).to(cuda)
+    Bs = torch.from_numpy(O.scales_to_mma_tiled(sb)).to(cuda)
+    one = torch.ones(1, dtype=torch.float32, device=cuda)
+    C = gemm(fmt, (Aq, As, one), (Bq, Bs, one))
+    C64, S = O.gemm_f64(packed_from_codes(ca), sa, 1.0, packed_from_codes(cb), sb, 1.0, fmt)
+    got = npy(C.float()).astype(np.float64)
+    assert np.count_nonzero(C64) > 0
+    assert np.array_equal(got, C64)
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (256, 512, 1024), (384, 256, 2560)])
+def test_gemm_small_random(cuda, fmt, shape):
+    M, N, K = shape
+    A, Ao = quant(synth.gemm_operand(M, K, 1), fmt, cuda)
+    B, Bo = quant(synth.gemm_operand(N, K, 2), fmt, cuda)
+    C = gemm(fmt, A, B)
+    C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fmt)
+    check(C, C64, S)
+
+
+def test_gemm_positive_data_bf16_rounding(cuda):
+    """Same-sign operands (|C| ~ sum |ab|): the tolerance then includes bf16 output rounding."""
+    M, N, K = 128, 256, 1024
+    a = synth.normal_f32(M, K, 3).abs().to(torch.bfloat16)
+    b = synth.normal_f32(N, K, 4).abs().to(torch.bfloat16)
+    A, Ao = quant(a, fp4.NVFP4, cuda)
+    B, Bo = quant(b, fp4.NVFP4, cuda)
+    C = gemm(fp4.NVFP4, A, B)
+    C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fp4.NVFP4)
+    check(C, C64, S, extra_rel=2.0 ** -8)
+
+
+def test_gemm_nvfp4_config4_sampled(cuda):
+    """M = N = K = 8192 NVFP4 (A seed 1, B seed 2): 8 whole rows and 8 whole columns of C."""
+    M = N = K = 8192
+    a, b = synth.gemm_operand(M, K, 1), synth.gemm_operand(N, K, 2)
+    A, _ = quant_gpu_only(a, fp4.NVFP4, cuda)
+    B, _ = quant_gpu_only(b, fp4.NVFP4, cuda)
+    C = gemm(fp4.NVFP4, A, B)
+    rng = np.random.default_rng(42)
+    rows, cols = np.sort(rng.choice(M, 8, replace=False)), np.sort(rng.choice(N, 8, replace=False))
+    check_sampled(C, a, b, fp4.NVFP4, rows, cols)
+
+
+def test_gemm_mxfp4_config5_sampled(cuda):
+    """down_proj shape M = 4096, N = 8192, K = 28672, MXFP4 (E8M0 per 32): activations
+    bf16(silu(g) * u) (seed 3), weights N(0, 0.02) (seed 4).  8 rows and 8 columns of C."""
+    a, w = synth.swiglu_act(), synth.weight()
+    A, _ = quant_gpu_only(a, fp4.MXFP4, cuda)
+    B, _ = quant_gpu_only(w, fp4.MXFP4, cuda)
+    C = gemm(fp4.MXFP4, A, B)
+    rng = np.random.default_rng(43)
+    rows, cols = np.sort(rng.choice(4096, 8, replace=False)), np.sort(rng.choice(8192, 8, replace=False))
+    check_sampled(C, a, w, fp4.MXFP4, rows, cols)
+
+
+def quant_gpu_only(x_cpu, fmt, cuda):
+    x = x_cpu.to(cuda)
+    if fmt == fp4.NVFP4:
+        q, s, g, _ = fp4.nvfp4_quantize(x, layout=fp4.MMA_TILED)
+        return (q, s, g), None
+    q, s, _ = fp4.mx_quantize(x, layout=fp4.MMA_TILED)
+    return (q, s, None), None
+
+
+def check_sampled(C, a_cpu, b_cpu, fmt, rows, cols):
+    """Reference for whole sampled rows (all N) and whole sampled columns (all M)."""
+    def oq(x):
+        if fmt == fp4.NVFP4:
+            q, s, g, _ = O.nvfp4_quantize(synth.as_f32_numpy(x))
+            return q, s, g
+        q, s, _ = O.mx_quantize(synth.as_f32_numpy(x))
+        return q, s, 1.0
+
+    # the global scale of each operand comes from its full tensor
+    Aq, As, Ag = oq(a_cpu)
+    Bq, Bs, Bg = oq(b_cpu)
+    Cn = npy(C.float()).astype(np.float64)
+    C64, S = O.gemm_f64(Aq, As, Ag, Bq, Bs, Bg, fmt, rows=rows)
+    err = np.abs(Cn[rows] - C64)
+    assert np.all(err <= 1e-3 * S), float((err - 1e-3 * S).max())
+    C64, S = O.gemm_f64(Aq, As, Ag, Bq, Bs, Bg, fmt, cols=cols)
+    err = np.abs(Cn[:, cols] - C64)
+    assert np.all(err <= 1e-3 * S), float((err - 1e-3 * S).max())
+
+
+def test_gemm_ldc_and_status_word(cuda):
+    """A wider output buffer (ldc > N): columns beyond N stay untouched; the status word is 0."""
+    M, N, K = 128, 256, 256
+    A, Ao = quant(synth.gemm_operand(M, K, 5), fp4.NVFP4, cuda)
+    B, Bo = quant(synth.gemm_operand(N, K, 6), fp4.NVFP4, cuda)
+    big = torch.full((M, N + 64), 7.0, dtype=torch.bfloat16, device=cuda)
+    C, ws = fp4.fp4_block_gemm(fp4.NVFP4, A[0], A[1], B[0], B[1], A[2], B[2], out=big[:, :N])
+    assert status_ok(ws)
+    assert torch.all(big[:, N:] == 7.0)
+    C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fp4.NVFP4)
+    check(big[:, :N], C64, S)

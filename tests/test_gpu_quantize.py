@@ -1,0 +1,244 @@
+"""GPU parity: quantisers, Walsh-Hadamard rotation and dequantiser against the CPU oracle.
+
+Bar: packed nibbles, scale bytes, the global scale and all counters bit-exact (stochastic
+rounding included); rotated and dequantised values bit-exact (the stated bar is 1e-6 relative;
+both sides follow the same fp32 operation order, so they agree exactly).  Every call goes through
+the C ABI via the thin binding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp4_amax_b200 as fp4
+import oracle as O
+from block_scaled_fp4_amax_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def npy(t):
+    return t.detach().cpu().numpy()
+
+
+def counts_of(c):
+    v = [int(x) for x in c.cpu().tolist()]
+    return dict(underflow=v[0], saturation=v[1], nonfinite=v[2], blocks_four=v[3])
+
+
+def f32(t_cpu):
+    return synth.as_f32_numpy(t_cpu)
+
+
+def check_scales(gpu_scales, ora_scales, layout):
+    rows, nb = ora_scales.shape
+    want = O.scales_to_mma_tiled(ora_scales) if layout == fp4.MMA_TILED else ora_scales.ravel()
+    assert np.array_equal(npy(gpu_scales), want)
+
+
+def run_mx(x_cpu, cuda, policy=fp4.OCP_FLOOR, rnd=fp4.RNE, seed=0, layout=fp4.ROWMAJOR):
+    q, s, c = fp4.mx_quantize(x_cpu.to(cuda), policy=policy, round=rnd, seed=seed, layout=layout)
+    qo, so, co = O.mx_quantize(f32(x_cpu), policy=policy, round=rnd, seed=seed)
+    assert np.array_equal(npy(q), qo)
+    check_scales(s, so, layout)
+    assert counts_of(c) == co
+    return q, s, qo, so
+
+
+def run_nv(x_cpu, cuda, rnd=fp4.RNE, four_six=False, seed=0, layout=fp4.ROWMAJOR, global_in=None):
+    gin = None if global_in is None else torch.tensor([global_in], dtype=torch.float32, device=cuda)
+    q, s, g, c = fp4.nvfp4_quantize(x_cpu.to(cuda), round=rnd, four_six=four_six, seed=seed, layout=layout,
+                                    global_in=gin)
+    qo, so, go, co = O.nvfp4_quantize(f32(x_cpu), round=rnd, four_six=four_six, seed=seed, global_in=global_in)
+    assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    check_scales(s, so, layout)
+    assert counts_of(c) == co
+    return q, s, g, qo, so, go
+
+
+# ---------------------------------------------------------------------------------------------
+# The hardware conversions against the oracle's enumerated encoders
+
+def test_e2m1_encoder_exhaustive_band(cuda):
+    """Every fp32 with |y| in [2^-4, 8) (all mantissas, both signs) through the MXFP4 path with a
+    4.0 anchor per block (exponent 0, so y = x): nibbles and counters bit-exact."""
+    bits = np.arange(123 << 23, 130 << 23, dtype=np.uint32)
+    vals = bits.view(np.float32)
+    vals = np.concatenate([vals, -vals, np.float32([0.0, -0.0, 1e-30, -1e-30, 2.0 ** -149])])
+    n = len(vals)
+    nblk = -(-n // 31)
+    x = np.zeros((nblk, 32), dtype=np.float32)
+    x[:, 0] = 4.0
+    flat = np.zeros(nblk * 31, dtype=np.float32)
+    flat[:n] = vals
+    x[:, 1:] = flat.reshape(nblk, 31)
+    rows = nblk // 64 * 64
+    xt = torch.from_numpy(x[:rows].reshape(-1, 32 * 64).copy())
+    run_mx(xt, cuda)
+
+
+def test_e4m3_scale_encoder_midpoints(cuda):
+    """NVFP4 with s_g = fl(1/6): fl(6 s_g) == 1, so the scale code is the E4M3 encoding of the block
+    amax itself.  All E4M3 midpoints (ties) +-2 ulp, every code value, and a dense random set."""
+    sg = float(np.float32(1.0 / 6.0))
+    assert np.float32(6.0) * np.float32(sg) == np.float32(1.0)
+    vals = np.array([O.e4m3_value(c) for c in range(0x7F)])
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    near = np.concatenate([np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0)), mids])
+    u = np.concatenate([near, vals.astype(np.float32), np.float32([448.5, 464, 500, 1e6]),
+                        (2.0 ** np.random.default_rng(0).uniform(-11, 9, 200000)).astype(np.float32)])
+    n = (len(u) // 64 + 1) * 64
+    u = np.concatenate([u, np.full(n - len(u), 1.0, np.float32)])
+    x = np.zeros((n, 16), dtype=np.float32)
+    x[:, 0] = u
+    x[:, 1] = u * np.float32(0.3)
+    run_nv(torch.from_numpy(x.reshape(-1, 16 * 64).copy()), cuda, global_in=sg)
+
+
+# ---------------------------------------------------------------------------------------------
+# MXFP4
+
+@pytest.mark.parametrize("policy", [fp4.OCP_FLOOR, fp4.NOSAT_CEIL])
+@pytest.mark.parametrize("rnd", [fp4.RNE, fp4.STOCHASTIC])
+@pytest.mark.parametrize("layout", [fp4.ROWMAJOR, fp4.MMA_TILED])
+def test_mx_config1_fp32(cuda, policy, rnd, layout):
+    x = synth.mx_small()  # 256 x 512 fp32 N(0,1), seed 0
+    q, s, qo, so = run_mx(x, cuda, policy=policy, rnd=rnd, seed=11, layout=layout)
+    out = fp4.fp4_dequantize(q, s, fp4.MXFP4, layout=layout)
+    assert np.array_equal(npy(out), O.dequantize(qo, so, O.MXFP4))
+
+
+@pytest.mark.parametrize("rnd", [fp4.RNE, fp4.STOCHASTIC])
+def test_mx_bf16_scaled_and_ragged(cuda, rnd):
+    x = (synth.normal_f32(384, 1024, 21) * 37.0).to(torch.bfloat16)
+    run_mx(x, cuda, rnd=rnd, seed=5)
+    run_mx(synth.normal_bf16(3, 96, 22), cuda, rnd=rnd, seed=5)        # 3 rows, 3 blocks per row
+    run_mx(synth.normal_bf16(1, 32, 23), cuda, rnd=rnd)                 # a single block
+
+
+def test_mx_edge_values(cuda):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((128, 256)).astype(np.float32)
+    x[0] = 0.0                                     # all-zero blocks: exponent 0
+    x[1] = -0.0
+    x[2] = (2.0 ** -140) * np.sign(x[2])           # subnormal block maxima: exponent clamps to -127
+    x[3] = x[3] * 2.0 ** 120                        # |x| up to ~2^122
+    x[4, :32] = 6.1                                 # the sawtooth block
+    x[5] = np.float32(2.0 ** -126) * x[5]
+    xt = torch.from_numpy(x)
+    for pol in (fp4.OCP_FLOOR, fp4.NOSAT_CEIL):
+        run_mx(xt, cuda, policy=pol)
+
+
+def test_mx_empty_and_nonfinite_counts(cuda):
+    q, s, c = fp4.mx_quantize(torch.empty((0, 64), dtype=torch.float32, device=cuda))
+    assert q.numel() == 0 and counts_of(c)["nonfinite"] == 0
+    x = torch.randn(128, 256)
+    x[7, 3] = float("nan")
+    x[9, 100] = float("inf")
+    x[100, 0] = float("-inf")
+    _, _, c = fp4.mx_quantize(x.to(cuda))
+    assert counts_of(c)["nonfinite"] == 3
+
+
+# ---------------------------------------------------------------------------------------------
+# NVFP4
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rnd", [fp4.RNE, fp4.STOCHASTIC])
+@pytest.mark.parametrize("four_six", [False, True])
+def test_nvfp4_outliers_small(cuda, dtype, rnd, four_six):
+    x = synth.nv_outliers(384, 2048, seed=5)
+    x = x if dtype == torch.bfloat16 else x.float()
+    for layout in (fp4.ROWMAJOR, fp4.MMA_TILED):
+        q, s, g, qo, so, go = run_nv(x, cuda, rnd=rnd, four_six=four_six, seed=9, layout=layout)
+    out = fp4.fp4_dequantize(q, s, fp4.NVFP4, g, layout=fp4.MMA_TILED)
+    assert np.array_equal(npy(out), O.dequantize(qo, so, O.NVFP4, go))
+    outb = fp4.fp4_dequantize(q, s, fp4.NVFP4, g, layout=fp4.MMA_TILED, out_dtype=torch.bfloat16)
+    want = torch.from_numpy(O.dequantize(qo, so, O.NVFP4, go)).to(torch.bfloat16)
+    assert torch.equal(outb.cpu(), want)
+
+
+@pytest.mark.parametrize("four_six", [False, True])
+def test_nvfp4_caller_global_and_ragged(cuda, four_six):
+    x = synth.normal_bf16(5, 48, 31)
+    run_nv(x, cuda, four_six=four_six)
+    run_nv(x, cuda, four_six=four_six, global_in=0.001)
+    run_nv(synth.normal_bf16(256, 512, 32), cuda, four_six=four_six, global_in=1e-4)  # heavy saturation
+    run_nv(torch.zeros(64, 64), cuda, four_six=four_six)                               # amax 0 -> s_g = 1
+
+
+@pytest.mark.parametrize("four_six", [False, True])
+def test_nvfp4_config2_full(cuda, four_six):
+    """8192 x 8192 bf16 N(0,1) with 8 outlier columns x U(50,100), seed 5; plain and 4/6."""
+    x = synth.nv_outliers()
+    run_nv(x, cuda, four_six=four_six, layout=fp4.ROWMAJOR)
+
+
+# ---------------------------------------------------------------------------------------------
+# Walsh-Hadamard rotation fused with the quantisers
+
+@pytest.mark.parametrize("d", [1024, 2048, 4096, 8192, 16384])
+@pytest.mark.parametrize("fmt,rnd,four_six", [(fp4.NVFP4, fp4.RNE, False), (fp4.NVFP4, fp4.STOCHASTIC, False),
+                                              (fp4.NVFP4, fp4.RNE, True), (fp4.MXFP4, fp4.RNE, False),
+                                              (fp4.MXFP4, fp4.STOCHASTIC, False)])
+def test_fwht_small(cuda, d, fmt, rnd, four_six):
+    rows = 37  # ragged against the row slots per CTA
+    x = synth.fwht_laplace(rows, d, seed=6)
+    q, s, g, c, rot = fp4.fwht_quantize(x.to(cuda), fmt=fmt, round=rnd, four_six=four_six, seed=7, want_rotated=True)
+    y, qo, so, go, co = O.fwht_quantize(f32(x), fmt=fmt, round=rnd, four_six=four_six, seed=7)
+    assert np.array_equal(npy(rot), y)
+    if fmt == fp4.NVFP4:
+        assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+
+
+def test_fwht_fp32_input_and_tiled_scales(cuda):
+    x = synth.fwht_laplace(128, 8192, seed=12).float()
+    q, s, g, c, _ = fp4.fwht_quantize(x.to(cuda), layout=fp4.MMA_TILED)
+    y, qo, so, go, co = O.fwht_quantize(f32(x))
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), O.scales_to_mma_tiled(so))
+    assert counts_of(c) == co
+
+
+def test_fwht_caller_global(cuda):
+    x = synth.fwht_laplace(64, 8192, seed=13)
+    gin = torch.tensor([0.002], device=cuda)
+    q, s, g, c, _ = fp4.fwht_quantize(x.to(cuda), global_in=gin, round=fp4.STOCHASTIC, seed=3)
+    y, qo, so, go, co = O.fwht_quantize(f32(x), global_in=0.002, round=fp4.STOCHASTIC, seed=3)
+    assert np.array_equal(npy(q), qo) and np.array_equal(npy(s), so.ravel()) and counts_of(c) == co
+
+
+def test_fwht_config3_full(cuda):
+    """16384 tokens x d = 8192 bf16 Laplace(0,1), 8 channels spiked to 120, H_8192 + NVFP4 + SR
+    (Philox seed 7, flat element index), global amax of the rotated tensor: full comparison."""
+    x = synth.fwht_laplace()
+    q, s, g, c, _ = fp4.fwht_quantize(x.to(cuda), fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7)
+    y, qo, so, go, co = O.fwht_quantize(f32(x), fmt=O.NVFP4, round=O.STOCHASTIC, seed=7)
+    assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+    # the spikes are spread: 8 spikes contribute at most 8 * 120 / sqrt(8192) ~ 10.6 per value,
+    # plus the rotated Laplace noise; the rotated peak stays far below the 120 input spike
+    assert float(np.abs(y).max()) < 120.0 / 4
+
+
+# ---------------------------------------------------------------------------------------------
+# The GEMM workloads' quantisation (MXFP4 activations and weights at the down_proj shape)
+
+def test_mx_swiglu_activation_full(cuda):
+    a = synth.swiglu_act()  # 4096 x 28672 bf16
+    run_mx(a, cuda, layout=fp4.MMA_TILED)
+
+
+def test_mx_weight_rows_sampled(cuda):
+    w = synth.weight()  # 8192 x 28672 bf16 N(0, 0.02)
+    q, s, c = fp4.mx_quantize(w.to(cuda), layout=fp4.ROWMAJOR)
+    rows = np.random.default_rng(0).choice(8192, 256, replace=False)
+    qo, so, _ = O.mx_quantize(f32(w[torch.from_numpy(rows)]))
+    assert np.array_equal(npy(q)[rows], qo)
+    assert np.array_equal(npy(s).reshape(8192, -1)[rows], so)
