@@ -317,6 +317,48 @@ def secondary(args, dev, flush, td, pk):
                 "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
                 "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     del x3
+    fp4_peak = 4.0 * pk["bf16_tflops"]  # dense FP4 / BF16 nominal ratio 9 / 2.25 on the measured bf16 peak
+    # config 4: NVFP4 GEMM 8192^3
+    A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)
+    B = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 2).to(dev), layout=fp4.MMA_TILED)
+    C = torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev)
+    gws = torch.empty(256, dtype=torch.uint8, device=dev)
+    ms = timed(lambda: fp4.fp4_block_gemm(fp4.NVFP4, A[0], A[1], B[0], B[1], A[2], B[2], out=C, workspace=gws),
+               K, W, flush, td)
+    t = statistics.median(ms)
+    tf = 2 * 8192 ** 3 / (t * 1e-3) / 1e12
+    out.append({"workload": "NVFP4 block-scaled GEMM M=N=K=8192 (E4M3 per 16, fp32 accumulate, bf16 out)",
+                "ms": round(t, 4), "TFLOP/s": round(tf, 1), "frac_fp4_peak": round(tf / fp4_peak, 4),
+                "fp4_peak": fp4_peak, "peak_source": pk["source"] + " bf16 x 4 (nominal FP4/BF16 ratio)"})
+    del A, B, C
+    # config 5: MXFP4 down_proj, activations and weights quantised then GEMM, timed end to end
+    a = synth.swiglu_act().to(dev)
+    w = synth.weight().to(dev)
+    C = torch.empty((4096, 8192), dtype=torch.bfloat16, device=dev)
+    st = {}
+
+    def c5():
+        Aq = fp4.mx_quantize(a, layout=fp4.MMA_TILED)
+        Bq = fp4.mx_quantize(w, layout=fp4.MMA_TILED)
+        st["ab"] = (Aq, Bq)
+        fp4.fp4_block_gemm(fp4.MXFP4, Aq[0], Aq[1], Bq[0], Bq[1], out=C, workspace=gws)
+
+    ms = timed(c5, K, W, flush, td)
+    t_all = statistics.median(ms)
+    Aq, Bq = st["ab"]
+    ms = timed(lambda: fp4.fp4_block_gemm(fp4.MXFP4, Aq[0], Aq[1], Bq[0], Bq[1], out=C, workspace=gws), K, W, flush, td)
+    t_g = statistics.median(ms)
+    ms = timed(lambda: fp4.mx_quantize(w, layout=fp4.MMA_TILED), K, W, flush, td)
+    t_w = statistics.median(ms)
+    flop = 2 * 4096 * 8192 * 28672
+    qbytes = w.numel() * (2 + 0.5 + 1 / 32)
+    out.append({"workload": "MXFP4 down_proj 4096x8192x28672: quantise activations + weights, then GEMM",
+                "ms_end_to_end": round(t_all, 4), "gemm_ms": round(t_g, 4),
+                "gemm_TFLOP/s": round(flop / (t_g * 1e-3) / 1e12, 1),
+                "gemm_frac_fp4_peak": round(flop / (t_g * 1e-3) / 1e12 / fp4_peak, 4),
+                "weight_quantise_GB/s": round(qbytes / (t_w * 1e-3) / 1e9, 1),
+                "weight_quantise_frac_hbm": round(qbytes / (t_w * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                "end_to_end_TFLOP/s": round(flop / (t_all * 1e-3) / 1e12, 1)})
     return out
 
 

@@ -241,6 +241,120 @@ __device__ __forceinline__ float sr_round(float y, uint32_t r) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Block encoding helpers shared by the quantiser and the fused rotation (N = values per lane,
+// 1..16; packed words hold 8 nibbles each, value 0 in the lowest nibble).
+
+template <int N>
+__device__ __forceinline__ void e2m1_pack_n(const float* y, uint32_t* w) {
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k) w[k] = e2m1x8(y + 8 * k);
+  } else {
+    float t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) t[i] = (i < N) ? y[i] : 0.0f;
+    w[0] = e2m1x4(t);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void e2m1_unpack_n(const uint32_t* w, float* q) {
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k) e2m1_unpack<8>(w[k], q + 8 * k);
+  } else {
+    float o[4];
+    e2m1_unpack<4>(w[0], o);
+#pragma unroll
+    for (int i = 0; i < N; ++i) q[i] = o[i];
+  }
+}
+
+template <int N>
+__device__ __forceinline__ int zero_codes_n(const uint32_t* w) {
+  if constexpr (N >= 8) {
+    int z = 0;
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k) z += zero_nibbles(w[k]);
+    return z;
+  } else {
+    return zero_nibbles(w[0]) - (8 - N);  // the 8 - N padding nibbles encode 0.0
+  }
+}
+
+// N values scaled by R and E2M1-encoded (RNE or stochastic); saturations counted per value only
+// when the block maximum normalises above 6 (`top` = fl(amax * R), monotone in |x|).
+template <int N, bool SR>
+__device__ __forceinline__ void encode_n(const float* v, float R, float top, const uint32_t* rnd,
+                                         uint32_t* w, uint32_t& sat) {
+  float y[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
+  if (top > 6.0f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
+  }
+  if (SR) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = sr_round(y[i], rnd[i]);
+  }
+  e2m1_pack_n<N>(y, w);
+}
+
+// One NVFP4 candidate (target T through inv_t = fl(1/fl(T*s_g))): returns the E4M3 code, writes
+// the packed nibbles, the saturation count and the decoded scale d.
+template <int N, bool SR>
+__device__ __forceinline__ uint32_t nv_candidate_n(const float* v, float amax, float s_g, float inv_t,
+                                                   const uint32_t* rnd, uint32_t* w, uint32_t& sat,
+                                                   float& d) {
+  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
+  d = e4m3_value(sc);
+  sat = 0;
+  if (sc == 0) {
+    float y[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = copysignf(0.0f, v[i]);
+    e2m1_pack_n<N>(y, w);
+  } else {
+    const float R = __frcp_rn(__fmul_rn(d, s_g));
+    encode_n<N, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
+  }
+  return sc;
+}
+
+// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2).
+template <int N>
+__device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, float d, float s_g, float* sq) {
+  float q[N];
+  e2m1_unpack_n<N>(w, q);
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float xhat = __fmul_rn(__fmul_rn(q[i], d), s_g);
+    const float e = __fsub_rn(v[i], xhat);
+    sq[i] = __fmul_rn(e, e);
+  }
+}
+
+// fp32 sum of a block's squared errors in element order.  G = 1: the lane owns the block; G > 1:
+// every lane of the block adds the broadcast values of lanes 0..G-1 (each holding N values).
+template <int N, int G>
+__device__ __forceinline__ float block_sse_n(const float* sq, int lane) {
+  float acc = 0.0f;
+  if constexpr (G == 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) acc = __fadd_rn(acc, sq[i]);
+  } else {
+    const int base = lane & ~(G - 1);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc = __fadd_rn(acc, __shfl_sync(0xFFFFFFFFu, sq[i], base + g));
+    }
+  }
+  return acc;
+}
+
+// ---------------------------------------------------------------------------------------------
 // Scale-byte placement.  Row-major: the flat block index.  MMA tile layout: 128 x 4 tiles of
 // 512 bytes, block-column groups fastest (the layout tcgen05.cp 32x128b.warpx4 expects).
 __device__ __forceinline__ uint64_t scale_offset(uint64_t blk, uint32_t nb, bool tiled) {

@@ -128,22 +128,6 @@ __device__ __forceinline__ void load_row(const T* x, long long row, long long ro
   }
 }
 
-// Lattice value of each of N already-normalised values after E2M1 encoding (encode + decode).
-template <int N>
-__device__ __forceinline__ void e2m1_roundtrip(const float* y, float* q) {
-  if constexpr (N >= 8) {
-#pragma unroll
-    for (int c = 0; c < N / 8; ++c) e2m1_unpack<8>(e2m1x8(y + 8 * c), q + 8 * c);
-  } else {
-    float t[4], o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) t[i] = (i < N) ? y[i] : 0.0f;
-    e2m1_unpack<4>(e2m1x4(t), o);
-#pragma unroll
-    for (int i = 0; i < N; ++i) q[i] = o[i];
-  }
-}
-
 struct FwhtParams {
   const void* x;
   long long rows;
@@ -210,6 +194,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
   constexpr int GE = 1 << L;                     // elements per group
   constexpr int GL = (L >= LB) ? 1 : (1 << (LB - L));  // lanes per block
   constexpr int GA = GE < 4 ? 4 : GE;            // register array size for one group
+  constexpr int WN = GE >= 8 ? GE / 8 : 1;        // packed nibble words per group
   static_assert(L <= LB, "group larger than a block");
   extern __shared__ __align__(16) float smem[];
   const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
@@ -266,11 +251,12 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
       const float* g = v + (h << L);
       const int i0 = (t << L) | (h << HI);                      // index in row of g[0]
       const unsigned long long idx0 = (unsigned long long)prow * D + i0;
-      float amax = 0.0f;
+      uint32_t am = 0u;
 #pragma unroll
-      for (int i = 0; i < GE; ++i) amax = fmaxf(amax, fabsf(g[i]));
+      for (int i = 0; i < GE; ++i) am = max(am, __float_as_uint(g[i]) & 0x7FFFFFFFu);
 #pragma unroll
-      for (int o = 1; o < GL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      for (int o = 1; o < GL; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      const float amax = __uint_as_float(am);
       uint32_t rnd[GA];
       if (SR) {
         if constexpr (GE >= 4) {
@@ -281,101 +267,54 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
           for (int i = 0; i < GE; ++i) rnd[i] = ph.w[(idx0 + i) & 3];
         }
       }
-      float y[GA];
-      uint32_t sc, sat = 0, unf = 0, four = 0;
+      uint32_t w[WN], sc, sat = 0, four = 0;
       if (!NV) {
-        // MXFP4 OCP rule: e = floor(log2 amax) - 2, clamped, all-zero -> 0
-        const uint32_t bits = __float_as_uint(amax);
-        const int ef = (int)((bits >> 23) & 0xFFu);
-        int e = (amax == 0.0f) ? 0 : (ef == 0 ? -127 : ef - 129);
+        // MXFP4 OCP rule: e = floor(log2 amax) - 2, clamped to [-127, 127], all-zero -> 0
+        const int ef = (int)((am >> 23) & 0xFFu);
+        int e = (am == 0u) ? 0 : (ef == 0 ? -127 : ef - 129);
         e = e < -127 ? -127 : e;
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
-#pragma unroll
-        for (int i = 0; i < GE; ++i) {
-          float tt = __fmul_rn(g[i], inv);
-          sat += fabsf(tt) > 6.0f;
-          if (SR) { tt = sr_round(tt, rnd[i]); unf += (g[i] != 0.0f) & (tt == 0.0f); }
-          else unf += (g[i] != 0.0f) & (fabsf(tt) <= 0.25f);
-          y[i] = tt;
-        }
+        encode_n<GE, SR>(g, inv, __fmul_rn(amax, inv), rnd, w, sat);
         sc = (uint32_t)(e + 127);
       } else {
-        float yy[2][GA], sq[2][GA];
-        uint32_t scs[2], sats[2] = {0u, 0u}, unfs[2] = {0u, 0u};
-        const int ncand = FOUR_SIX ? 2 : 1;
+        float d6;
+        sc = nv_candidate_n<GE, SR>(g, amax, s_g, inv6, rnd, w, sat, d6);
+        if constexpr (FOUR_SIX) {
+          float d4, sq[GA];
+          uint32_t w4[WN], sat4;
+          const uint32_t sc4 = nv_candidate_n<GE, SR>(g, amax, s_g, inv4, rnd, w4, sat4, d4);
+          sq_errors_n<GE>(g, w, d6, s_g, sq);
+          const float sse6 = block_sse_n<GE, GL>(sq, lane);
+          sq_errors_n<GE>(g, w4, d4, s_g, sq);
+          const float sse4 = block_sse_n<GE, GL>(sq, lane);
+          if (sse4 < sse6) {
+            sc = sc4;
+            sat = sat4;
+            four = 1;
 #pragma unroll
-        for (int k = 0; k < ncand; ++k) {
-          const uint32_t code = e4m3_code(__fmul_rn(amax, k == 0 ? inv6 : inv4));
-          const float d = e4m3_value(code);
-          scs[k] = code;
-          const float R = code ? __frcp_rn(__fmul_rn(d, s_g)) : 0.0f;
-#pragma unroll
-          for (int i = 0; i < GE; ++i) {
-            float tt;
-            if (code == 0) {
-              tt = copysignf(0.0f, g[i]);
-              unfs[k] += g[i] != 0.0f;
-            } else {
-              tt = __fmul_rn(g[i], R);
-              sats[k] += fabsf(tt) > 6.0f;
-              if (SR) { tt = sr_round(tt, rnd[i]); unfs[k] += (g[i] != 0.0f) & (tt == 0.0f); }
-              else unfs[k] += (g[i] != 0.0f) & (fabsf(tt) <= 0.25f);
-            }
-            yy[k][i] = tt;
-          }
-          if (FOUR_SIX) {
-            // exact lattice values: |tt| rounds onto the lattice in the encoder; decode back
-            float qv[GA];
-            e2m1_roundtrip<GE>(yy[k], qv);
-#pragma unroll
-            for (int i = 0; i < GE; ++i) {
-              const float xhat = __fmul_rn(__fmul_rn(qv[i], d), s_g);
-              const float e = __fsub_rn(g[i], xhat);
-              sq[k][i] = __fmul_rn(e, e);
-            }
+            for (int k = 0; k < WN; ++k) w[k] = w4[k];
           }
         }
-        int pick = 0;
-        if (FOUR_SIX) {
-          float sse[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            // fp32 sum in element order: every lane of the block adds the broadcast squared
-            // errors of lanes 0..GL-1 of the block, so all of them hold the same sum
-            const int basel = lane & ~(GL - 1);
-            float acc = 0.0f;
-#pragma unroll
-            for (int gg = 0; gg < GL; ++gg) {
-#pragma unroll
-              for (int i = 0; i < GE; ++i) acc = __fadd_rn(acc, __shfl_sync(0xFFFFFFFFu, sq[k][i], basel + gg));
-            }
-            sse[k] = acc;
-          }
-          pick = (sse[1] < sse[0]) ? 1 : 0;
-          four = pick;
-        }
-#pragma unroll
-        for (int i = 0; i < GE; ++i) y[i] = pick ? yy[1][i] : yy[0][i];
-        sc = pick ? scs[1] : scs[0];
-        sat = pick ? sats[1] : sats[0];
-        unf = pick ? unfs[1] : unfs[0];
       }
       if (valid) {
+        if (am >= 0x7F800000u) {
 #pragma unroll
-        for (int i = 0; i < GE; ++i) cnt[2] += !isfinite(g[i]);
-        cnt[0] += unf;
+          for (int i = 0; i < GE; ++i) cnt[2] += !isfinite(g[i]);
+        }
+        int zx = 0;
+#pragma unroll
+        for (int i = 0; i < GE; ++i) zx += g[i] == 0.0f;
+        cnt[0] += (uint32_t)(zero_codes_n<GE>(w) - zx);
         cnt[1] += sat;
         uint8_t* qrow = p.q + prow * (D / 2);
         if constexpr (GE == 16) {
-          const uint32_t a = e2m1x8(y), b = e2m1x8(y + 8);
-          *reinterpret_cast<uint2*>(qrow + i0 / 2) = make_uint2(a, b);
+          *reinterpret_cast<uint2*>(qrow + i0 / 2) = make_uint2(w[0], w[WN - 1]);
         } else if constexpr (GE == 8) {
-          *reinterpret_cast<uint32_t*>(qrow + i0 / 2) = e2m1x8(y);
+          *reinterpret_cast<uint32_t*>(qrow + i0 / 2) = w[0];
         } else if constexpr (GE == 4) {
-          *reinterpret_cast<uint16_t*>(qrow + i0 / 2) = (uint16_t)e2m1x4(y);
+          *reinterpret_cast<uint16_t*>(qrow + i0 / 2) = (uint16_t)w[0];
         } else if constexpr (GE == 2) {
-          float y4[4] = {y[0], y[1], 0.0f, 0.0f};
-          qrow[i0 / 2] = (uint8_t)e2m1x4(y4);
+          qrow[i0 / 2] = (uint8_t)w[0];
         }
         if ((lane & (GL - 1)) == 0) {
           const unsigned long long blk = (unsigned long long)prow * nb + (i0 >> LB);
@@ -385,8 +324,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
       }
       if constexpr (GE == 1) {
         // one value per lane: pair nibbles across neighbouring lanes
-        float y4[4] = {y[0], 0.0f, 0.0f, 0.0f};
-        const uint32_t c1 = e2m1x4(y4) & 0xFu;
+        const uint32_t c1 = w[0] & 0xFu;
         const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, c1, 1);
         if (valid && !(lane & 1)) p.q[prow * (D / 2) + i0 / 2] = (uint8_t)(c1 | (other << 4));
       }

@@ -54,82 +54,6 @@ __device__ __forceinline__ NvScale nv_scales(const float* global_in, const uint3
   return s;
 }
 
-// E values scaled by `R` (a power of two for MXFP4) and E2M1-encoded (RNE or stochastic).
-// Returns the packed nibbles in w[E/8] (E = 8 or 16); adds saturations to `sat`.
-template <int E, bool SR>
-__device__ __forceinline__ void encode(const float* v, float R, float top, const uint32_t* rnd,
-                                       uint32_t* w, uint32_t& sat) {
-  float y[E];
-#pragma unroll
-  for (int i = 0; i < E; ++i) y[i] = __fmul_rn(v[i], R);
-  if (top > 6.0f) {  // some |y| > 6 only if the block maximum normalises above 6
-#pragma unroll
-    for (int i = 0; i < E; ++i) sat += fabsf(y[i]) > 6.0f;
-  }
-  if (SR) {
-#pragma unroll
-    for (int i = 0; i < E; ++i) y[i] = sr_round(y[i], rnd[i]);
-  }
-#pragma unroll
-  for (int k = 0; k < E / 8; ++k) w[k] = e2m1x8(y + 8 * k);
-}
-
-// One NVFP4 candidate (target T through inv_t): block scale code, packed nibbles, saturations.
-template <int E, bool SR>
-__device__ __forceinline__ uint32_t nv_candidate(const float* v, float amax, float s_g, float inv_t,
-                                                 const uint32_t* rnd, uint32_t* w, uint32_t& sat,
-                                                 float& d) {
-  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
-  d = e4m3_value(sc);
-  sat = 0;
-  if (sc == 0) {
-    float y[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) y[i] = copysignf(0.0f, v[i]);
-#pragma unroll
-    for (int k = 0; k < E / 8; ++k) w[k] = e2m1x8(y + 8 * k);
-  } else {
-    const float R = __frcp_rn(__fmul_rn(d, s_g));
-    encode<E, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
-  }
-  return sc;
-}
-
-// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2) of the lane's E values.
-template <int E>
-__device__ __forceinline__ void sq_errors(const float* v, const uint32_t* w, float d, float s_g, float* sq) {
-#pragma unroll
-  for (int k = 0; k < E / 8; ++k) {
-    float q[8];
-    e2m1_unpack<8>(w[k], q);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float xhat = __fmul_rn(__fmul_rn(q[i], d), s_g);
-      const float e = __fsub_rn(v[8 * k + i], xhat);
-      sq[8 * k + i] = __fmul_rn(e, e);
-    }
-  }
-}
-
-// fp32 sum of the block's squared errors in element order.  G = 1: the lane owns the block.
-// G > 1: every lane of the block adds the broadcast values of lanes 0..G-1 in order.
-template <int E, int G>
-__device__ __forceinline__ float block_sse(const float* sq, int lane) {
-  float acc = 0.0f;
-  if constexpr (G == 1) {
-#pragma unroll
-    for (int i = 0; i < E; ++i) acc = __fadd_rn(acc, sq[i]);
-  } else {
-    const int base = lane & ~(G - 1);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int i = 0; i < E; ++i) acc = __fadd_rn(acc, __shfl_sync(0xFFFFFFFFu, sq[i], base + g));
-    }
-  }
-  return acc;
-}
-
 struct QuantParams {
   const void* x;
   long long n_chunks;  // rows * cols / E
@@ -204,20 +128,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       if (!NV) {
         const int e = mx_exponent(am, p.policy);
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
-        encode<E, SR>(v, inv, __fmul_rn(amax, inv), rnd, w, sat);
+        encode_n<E, SR>(v, inv, __fmul_rn(amax, inv), rnd, w, sat);
         sc = (uint32_t)(e + 127);
       } else if (!FOUR_SIX) {
         float d;
-        sc = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d);
+        sc = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d);
       } else {
         float d6, d4, sq[E];
         uint32_t w4[W], sat4;
-        const uint32_t sc6 = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d6);
-        const uint32_t sc4 = nv_candidate<E, SR>(v, amax, ns.s_g, ns.inv4, rnd, w4, sat4, d4);
-        sq_errors<E>(v, w, d6, ns.s_g, sq);
-        const float sse6 = block_sse<E, G>(sq, lane);
-        sq_errors<E>(v, w4, d4, ns.s_g, sq);
-        const float sse4 = block_sse<E, G>(sq, lane);
+        const uint32_t sc6 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d6);
+        const uint32_t sc4 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv4, rnd, w4, sat4, d4);
+        sq_errors_n<E>(v, w, d6, ns.s_g, sq);
+        const float sse6 = block_sse_n<E, G>(sq, lane);
+        sq_errors_n<E>(v, w4, d4, ns.s_g, sq);
+        const float sse4 = block_sse_n<E, G>(sq, lane);
         sc = sc6;
         if (sse4 < sse6) {
           sc = sc4;
@@ -228,9 +152,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         }
       }
       if (valid) {
-        int zc = 0;
-#pragma unroll
-        for (int k = 0; k < W; ++k) zc += zero_nibbles(w[k]);
+        const int zc = zero_codes_n<E>(w);
         cnt[0] += (uint32_t)(zc - Vec32<T>::zeros(raw[u]));
         cnt[1] += sat;
         if (W == 2) {
