@@ -30,7 +30,8 @@ STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 
 # Every symbol include/fp4mx.h declares.
 EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
-           "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error")
+           "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error",
+           "nvfp4_quantize_noalloc")
 
 
 class Fp4Error(RuntimeError):
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
     L.fwht_quantize.argtypes = [P, I, LG, LG, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
     L.fp4_dequantize.argtypes = [P, P, I, I, I, P, LG, LG, I, P, P]
     L.fp4_block_gemm.argtypes = [I, I, I, I, P, P, P, P, P, P, P, LG, P, SZ, P]
+    L.nvfp4_quantize_noalloc.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P]
+    L.nvfp4_quantize_noalloc.restype = I
     L.fp4_workspace_size.argtypes = [I, LG, LG]
     L.fp4_workspace_size.restype = SZ
     L.fp4_gemm_status_word.argtypes = []
@@ -138,6 +141,22 @@ def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, se
     _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, round, int(bool(four_six)), seed,
                                 layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c), _ptr(ws),
                                 ws.numel(), _stream(stream)))
+    return q, s, g, c
+
+
+def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
+                           layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
+                           stream=None):
+    """nvfp4_quantize for callers that cannot hand the library a device workspace: the amax word
+    between the two passes lives in a fixed area of the library's own device memory.  Calls that
+    overlap on the GPU share that area and must be serialised.  Returns (q, scales, s_g, counts)."""
+    _need_cuda(x, global_in)
+    rows, cols = x.shape
+    q, s, c = _alloc_outputs(rows, cols, 16, x.device)
+    g = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, block, round, int(bool(four_six)),
+                                        seed, layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c),
+                                        _stream(stream)))
     return q, s, g, c
 
 

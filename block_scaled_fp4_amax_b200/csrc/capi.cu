@@ -64,6 +64,8 @@ fp4_status zero_counts(fp4_counts* counts, cudaStream_t s) {
 }  // namespace
 
 namespace fp4k {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;

@@ -9,6 +9,9 @@ namespace fp4k {
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Records the message fp4_last_error() returns on the calling thread.
+void set_last_error(const char* msg);
+
 struct QuantLaunch {
   const void* x;
   bool bf16;

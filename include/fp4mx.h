@@ -187,6 +187,28 @@ FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
                           const unsigned char* Bq, const unsigned char* Bs, const float* Bg,
                           void* C, long ldc, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_quantize_noalloc — nvfp4_quantize without a caller-supplied workspace, for callers that
+ * cannot allocate device memory: for example a plugin inside another runtime that receives only
+ * its input and output buffers, or a latency-critical loop that must not call cudaMalloc (which
+ * can synchronise the device).  The source pages have no counterpart; this is a library
+ * convenience.
+ *   Arguments, results and errors are those of nvfp4_quantize, minus `workspace`/`ws_bytes`.
+ *   Scratch: a fixed 256-byte array in this library's device memory (per GPU, kept until the
+ *   process exits).  A shape whose workspace need (fp4_workspace_size) exceeds it is rejected with
+ *   FP4_EUNSUPPORTED; today every shape needs one amax word and fits.
+ *   Allocation: none (no cudaMalloc, no cudaFree, no allocating library call).
+ *   First call on a device: looks up the array's device address with cudaGetSymbolAddress, with
+ *   that device current; make that first call before any stream capture.
+ *   Sharing: all calls on a device share the one array and it keeps the last call's contents; the
+ *   amax word is zeroed on `stream` at the start of each call.  Calls that overlap on the GPU (in
+ *   flight at the same time on different streams) race on it: serialise them. */
+FP4_API fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, long rows, long cols, int block,
+                                          fp4_round round, int four_six, unsigned long long seed,
+                                          fp4_scale_layout layout, const float* global_in, float* global_out,
+                                          unsigned char* q, unsigned char* scales, fp4_counts* counts,
+                                          void* stream);
+
 /* Bytes of device workspace `op` needs for the given sizes (rows/cols; M/N for the GEMM). */
 FP4_API size_t fp4_workspace_size(fp4_op op, long rows, long cols);
 
