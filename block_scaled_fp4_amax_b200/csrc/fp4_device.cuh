@@ -85,6 +85,18 @@ template <> struct Vec32<float> {
     for (int i = 0; i < 8; ++i) nz += (r.w[i] & 0x7FFFFFFFu) != 0u;
     return 8 - nz;
   }
+  // Largest magnitude bit pattern of the chunk; `any_zero` is set if some value is +-0.
+  __device__ __forceinline__ static uint32_t max_mag(const U8& r, bool& any_zero) {
+    uint32_t m = 0u, mn = 0xFFFFFFFFu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t a = r.w[i] & 0x7FFFFFFFu;
+      m = max(m, a);
+      mn = min(mn, a);
+    }
+    any_zero = mn == 0u;
+    return m;
+  }
 };
 template <> struct Vec32<__nv_bfloat16> {
   static constexpr int E = 16;
@@ -100,6 +112,19 @@ template <> struct Vec32<__nv_bfloat16> {
 #pragma unroll
     for (int i = 0; i < 8; ++i) nz += __popc(((r.w[i] & 0x7FFF7FFFu) + 0x7FFF7FFFu) & 0x80008000u);
     return 16 - nz;
+  }
+  // Largest magnitude as an fp32 bit pattern (16-bit lane-wise max of the bf16 magnitudes);
+  // `any_zero` is set if some value is +-0 (a zero half borrows: (m - 1) & ~m has its top bit).
+  __device__ __forceinline__ static uint32_t max_mag(const U8& r, bool& any_zero) {
+    uint32_t m = 0u, z = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t a = r.w[i] & 0x7FFF7FFFu;
+      asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(a));
+      z |= (a - 0x00010001u) & ~a;
+    }
+    any_zero = (z & 0x80008000u) != 0u;
+    return max(m & 0xFFFFu, m >> 16) << 16;
   }
 };
 
@@ -152,10 +177,8 @@ __device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
   return r;
 }
 
-// Decode the low E nibbles of `codes` back to fp32 (exact) through f16x2.
-template <int E>
-__device__ __forceinline__ void e2m1_unpack(uint32_t codes, float* v) {
-  uint32_t h[4];
+// The 8 nibbles of `codes` as four f16x2 words (byte b -> h[b], low nibble in the low half).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t* h) {
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
       "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
@@ -163,8 +186,45 @@ __device__ __forceinline__ void e2m1_unpack(uint32_t codes, float* v) {
       "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
       "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
       : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(codes));
+}
+
+// Decode the low E nibbles of `codes` back to fp32 (exact) through f16x2.
+template <int E>
+__device__ __forceinline__ void e2m1_unpack(uint32_t codes, float* v) {
+  uint32_t h[4];
+  e2m1x8_to_f16x2(codes, h);
 #pragma unroll
   for (int i = 0; i < E / 2; ++i) f16x2_to_f32(h[i], v[2 * i], v[2 * i + 1]);
+}
+
+// Two fp32 values in one 64-bit register (first value in the low half) and the sm_100 packed
+// fp32 arithmetic on such pairs: each half is an IEEE fp32 operation rounded to nearest even.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& lo, float& hi) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+  lo = __uint_as_float(a);
+  hi = __uint_as_float(b);
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 // E4M3 (E4M3FN) round to nearest even, saturating at 448; u >= 0.  Returns the code byte.
@@ -288,8 +348,14 @@ template <int N, bool SR>
 __device__ __forceinline__ void encode_n(const float* v, float R, float top, const uint32_t* rnd,
                                          uint32_t* w, uint32_t& sat) {
   float y[N];
+  if constexpr (N % 2 == 0) {
+    const f32x2 R2 = f2_pack(R, R);
 #pragma unroll
-  for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
+    for (int j = 0; j < N; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y[j], y[j + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
+  }
   if (top > 6.0f) {
 #pragma unroll
     for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
@@ -322,9 +388,38 @@ __device__ __forceinline__ uint32_t nv_candidate_n(const float* v, float amax, f
   return sc;
 }
 
-// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2).
+// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2), d the value of E4M3 `code`.
+// For pairs, v*d is formed in f16x2 straight from the nibble conversion: |v| <= 6 has two
+// significant bits and d four, so the product (at least 2^-10, at most 2688) is exact in f16.
 template <int N>
-__device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, float d, float s_g, float* sq) {
+__device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, uint32_t code, float d, float s_g,
+                                            float* sq) {
+  if constexpr (N % 2 == 0) {
+    uint32_t dh2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(dh2) : "h"((uint16_t)(code | (code << 8))));
+#pragma unroll
+    for (int k = 0; k < (N + 7) / 8; ++k) {
+      uint32_t h[4];
+      e2m1x8_to_f16x2(w[k], h);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = 8 * k + 2 * b;
+        if (j < N) {
+          uint32_t qd;
+          asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(qd) : "r"(h[b]), "r"(dh2));
+          float lo, hi;
+          f16x2_to_f32(qd, lo, hi);
+          // scalar __fmul_rn/__fsub_rn: never contracted into an FMA (packed f32x2 mul + sub
+          // pairs can be, which would round the error differently)
+          const float el = __fsub_rn(v[j], __fmul_rn(lo, s_g));
+          const float eh = __fsub_rn(v[j + 1], __fmul_rn(hi, s_g));
+          sq[j] = __fmul_rn(el, el);
+          sq[j + 1] = __fmul_rn(eh, eh);
+        }
+      }
+    }
+    return;
+  }
   float q[N];
   e2m1_unpack_n<N>(w, q);
 #pragma unroll

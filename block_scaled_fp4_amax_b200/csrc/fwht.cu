@@ -283,9 +283,9 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
           float d4, sq[GA];
           uint32_t w4[WN], sat4;
           const uint32_t sc4 = nv_candidate_n<GE, SR>(g, amax, s_g, inv4, rnd, w4, sat4, d4);
-          sq_errors_n<GE>(g, w, d6, s_g, sq);
+          sq_errors_n<GE>(g, w, sc, d6, s_g, sq);
           const float sse6 = block_sse_n<GE, GL>(sq, lane);
-          sq_errors_n<GE>(g, w4, d4, s_g, sq);
+          sq_errors_n<GE>(g, w4, sc4, d4, s_g, sq);
           const float sse4 = block_sse_n<GE, GL>(sq, lane);
           if (sse4 < sse6) {
             sc = sc4;

@@ -111,9 +111,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       const bool valid = c < p.n_chunks;
       float v[E];
       Vec32<T>::unpack(raw[u], v);
-      uint32_t am = 0u;
-#pragma unroll
-      for (int i = 0; i < E; ++i) am = max(am, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+      bool any_zero;
+      uint32_t am = Vec32<T>::max_mag(raw[u], any_zero);
 #pragma unroll
       for (int o = 1; o < G; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
       if (am >= 0x7F800000u && valid) {
@@ -138,9 +137,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         uint32_t w4[W], sat4;
         const uint32_t sc6 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d6);
         const uint32_t sc4 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv4, rnd, w4, sat4, d4);
-        sq_errors_n<E>(v, w, d6, ns.s_g, sq);
+        sq_errors_n<E>(v, w, sc6, d6, ns.s_g, sq);
         const float sse6 = block_sse_n<E, G>(sq, lane);
-        sq_errors_n<E>(v, w4, d4, ns.s_g, sq);
+        sq_errors_n<E>(v, w4, sc4, d4, ns.s_g, sq);
         const float sse4 = block_sse_n<E, G>(sq, lane);
         sc = sc6;
         if (sse4 < sse6) {
@@ -153,7 +152,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       }
       if (valid) {
         const int zc = zero_codes_n<E>(w);
-        cnt[0] += (uint32_t)(zc - Vec32<T>::zeros(raw[u]));
+        // a +-0 input always gives a zero code, so inputs are counted only when both occur
+        cnt[0] += (uint32_t)(zc - ((zc > 0 && any_zero) ? Vec32<T>::zeros(raw[u]) : 0));
         cnt[1] += sat;
         if (W == 2) {
           reinterpret_cast<uint2*>(p.q)[c] = make_uint2(w[0], w[W - 1]);
