@@ -6,14 +6,21 @@
 // kind with scale_vec::2X.  ("Sub-4-Bit Microscaling" §2: NVFP4 on the 5th-generation tensor
 // core; metrale `hardware::exec`: NVFP4 activations take the block-scaled FP4 MMA.)
 //
-// Structure: persistent CTAs (one per SM), 128 x 256 output tile, K consumed 256 values (128
-// bytes) per pipeline stage.  Six warps:
-//   warp 0     TMA producer: A/B tiles by 2-D tensor-map loads (128-byte swizzle), the scale
-//              tiles by 1-D bulk copies (they are contiguous in the MMA tile layout);
-//   warp 1     allocates tensor memory and issues, from one lane, tcgen05.cp (scales smem->TMEM)
-//              and tcgen05.mma; tcgen05.commit frees each smem stage and signals the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns a 32-lane quarter), scale
-//              by alpha, round to bf16, store.
+// Two kernels share the PTX helpers below.
+//
+// gemm_pair_kernel (M % 256 == 0): clusters of two CTAs on neighbouring SMs, each pair computing a
+// 256 x 256 tile with tcgen05 cta_group::2 (each SM holds half of A and half of B per stage), K
+// consumed 256 values per stage in a 5-6 stage ring.  Seven warps per CTA:
+//   warp 0     TMA producer (both CTAs): operand tiles by 2-D tensor maps with 128-byte swizzle,
+//              scale tiles by 3-D tensor maps; all loads complete on the leader's barrier;
+//   warp 6     (leader) copies each stage's scales smem -> TMEM (tcgen05.cp) into one of three
+//              TMEM scale buffers — issued from its own warp so the copies queue separately from
+//              the MMAs and overlap them;
+//   warp 1     (leader) issues tcgen05.mma kind::mxf4nvf4 and the commits that free smem stages,
+//              scale buffers and, per tile, hand the accumulator to the epilogue;
+//   warps 2-5  epilogue (both CTAs): tcgen05.ld the FP32 accumulator quarter this warp may access,
+//              scale by alpha, round to bf16, release the accumulator, store.
+// gemm_kernel (M % 256 == 128): the same pipeline on one SM with 128 x 256 tiles.
 // Every mbarrier wait is bounded in time; on expiry the kernel records the site in the caller's
 // status word, tells the other roles to stop, drains what it issued and frees tensor memory.
 #include <cuda.h>
@@ -344,6 +351,310 @@ constexpr int smem_bytes() {
 }
 
 // ---------------------------------------------------------------------------------------------
+// 2-SM variant: a cluster of two CTAs on neighbouring SMs computes a 256 x 256 output tile with
+// tcgen05 cta_group::2.  CTA r of the pair holds rows [128r, 128r+128) of the A tile and of the B
+// tile (the MMA splits M across the pair for A and D, N across the pair for B) plus the scales
+// for its A rows and for all 256 B rows.  Both CTAs' tensor-map loads complete on the leader's
+// (rank 0) barrier, which the leader arms for the pair's bytes; the leader alone issues
+// tcgen05.cp and tcgen05.mma, and its commits arrive on the barriers of both CTAs.  Each SM then
+// reads 32 KB of operands per 256-value K stage instead of 48 KB, and 5-6 stages fit.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_pair_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_pair_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(bar), "h"((uint16_t)3) : "memory");
+}
+__device__ __forceinline__ void tc_commit_local_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+template <bool NV>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                            uint32_t sfb, uint32_t accumulate) {
+  if constexpr (NV) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+  } else {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+  }
+}
+
+// M = 256 (the pair), N = 256
+__host__ __device__ constexpr uint32_t idesc_pair(bool nv, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((nv ? 0u : 1u) << 23) |
+         ((uint32_t)(256 >> 4) << 24) | (sfa_id << 29);
+}
+
+template <bool NV> struct PairCfg {
+  static constexpr int ATOMS = NV ? 4 : 2;
+  static constexpr int S = NV ? 5 : 6;
+  static constexpr int NB = 3;  // scale buffers in tensor memory
+  static constexpr int A_HALF = 128 * BKB, B_HALF = 128 * BKB;
+  static constexpr int SFA_BYTES = ATOMS * 512, SFB_BYTES = 2 * ATOMS * 512;
+  static constexpr int STAGE = A_HALF + B_HALF + SFA_BYTES + SFB_BYTES;
+  static constexpr int SMEM = 1024 + S * STAGE + 512;
+  static constexpr uint32_t SF_BUF = 12u * ATOMS;  // TMEM columns per scale buffer: SFA 4*ATOMS + SFB 8*ATOMS
+};
+constexpr int PAIR_THREADS = 224;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
+
+template <bool NV>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, Params p) {
+  using C = PairCfg<NV>;
+  constexpr int S = C::S, ATOMS = C::ATOMS, NB = C::NB;
+  constexpr uint32_t TX_PAIR = 2u * C::STAGE;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * C::A_HALF;
+  uint8_t* sSFA = sB + S * C::B_HALF;
+  uint8_t* sSFB = sSFA + S * C::SFA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::SFB_BYTES);
+  // bars: full[S] (leader), empty[S], sf_full[NB], sf_empty[NB], tmem_full, tmem_empty (leader), drain[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t sf_full0 = smem_u32(bars + 2 * S), sf_empty0 = smem_u32(bars + 2 * S + NB);
+  const uint32_t tmem_full = smem_u32(bars + 2 * S + 2 * NB), tmem_empty = smem_u32(bars + 2 * S + 2 * NB + 1);
+  const uint32_t drain0 = smem_u32(bars + 2 * S + 2 * NB + 2);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(sf_full0 + 8 * b, 1);
+      mbar_init(sf_empty0 + 8 * b, 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 8);  // 4 epilogue warps in each CTA of the pair
+    mbar_init(drain0, 1);
+    mbar_init(drain0 + 8, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers initialised and tensor memory allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int tiles_m = p.M / 256, tiles_n = p.N / 256;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kt_count = p.K / 256;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const uint32_t my_tiles = (uint32_t)((num_tiles - cid + ncl - 1) / ncl);
+  const uint32_t total = my_tiles * (uint32_t)kt_count;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
+      uint32_t g = 0;
+      bool ok = true, issued = false;
+      for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
+        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        for (int kt = 0; kt < kt_count; ++kt, ++g) {
+          const int s = g % S;
+          const uint32_t ph = (g / S) & 1;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0)) { ok = false; break; }
+          const uint32_t fb = map_rank(full0 + 8 * s, 0);  // the leader's barrier
+          if (leader) mbar_expect_tx(full0 + 8 * s, TX_PAIR);
+          tma_pair_2d(smem_u32(sA + s * C::A_HALF), &tmA, kt * BKB, tm * 256 + (int)rank * 128, fb);
+          tma_pair_2d(smem_u32(sB + s * C::B_HALF), &tmB, kt * BKB, tn * 256 + (int)rank * 128, fb);
+          tma_pair_3d(smem_u32(sSFA + s * C::SFA_BYTES), &tmSA, 0, kt * ATOMS, tm * 2 + (int)rank, fb);
+          tma_pair_3d(smem_u32(sSFB + s * C::SFB_BYTES), &tmSB, 0, kt * ATOMS, tn * 2, fb);
+          issued = true;
+        }
+      }
+      if (ok) {
+        // the last S releases: no tcgen05.commit arrival is still on its way to this CTA
+        for (int i = 0; i < S; ++i, ++g) {
+          const int s = g % S;
+          if (!mbar_wait(empty0 + 8 * s, ((g / S) & 1) ^ 1, abort_flag, p.status, 4)) break;
+        }
+      } else if (issued) {
+        // loads in flight complete on the leader's barrier, which this CTA cannot observe:
+        // give them a fixed, bounded time to land before shared memory is released
+        const unsigned long long t0 = now_ns();
+        while (now_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ scale copies (leader)
+    // Issued from their own warp so that they queue separately from the MMAs: iteration g's
+    // scales go to TMEM buffer g % NB once its stage has landed and the MMAs that last read
+    // the buffer have completed; a commit then tells the MMA warp the buffer is ready.
+    if (leader) {
+      bool ok = true;
+      uint32_t g = 0;
+      for (; g < total && ok; ++g) {
+        const int s = g % S, b = g % NB;
+        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 6)) { ok = false; break; }
+        if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 7)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t fa = smem_u32(sSFA + s * C::SFA_BYTES), fbs = smem_u32(sSFB + s * C::SFB_BYTES);
+          const uint32_t sfa = tmem + SFA_COL + b * C::SF_BUF, sfb = sfa + 4 * ATOMS;
+#pragma unroll
+          for (int a = 0; a < ATOMS; ++a) {
+            tc_cp_sf_pair(sfa + 4 * a, desc_sf(fa + a * 512));
+            tc_cp_sf_pair(sfb + 8 * a, desc_sf(fbs + a * 512));
+            tc_cp_sf_pair(sfb + 8 * a + 4, desc_sf(fbs + (ATOMS + a) * 512));
+          }
+          tc_commit_local_pair(sf_full0 + 8 * b);
+        }
+        __syncwarp();
+      }
+      if (ok) {
+        // the MMA warp's last releases of the scale buffers have landed
+        for (int i = 0; i < NB; ++i, ++g) {
+          const int b = g % NB;
+          if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8)) break;
+        }
+      } else if (lane == 0) {
+        tc_commit_local_pair(drain0 + 8);
+        const unsigned long long t0 = now_ns();
+        while (!mbar_try(drain0 + 8, 0) && now_ns() - t0 < kTimeoutNs) {
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader) {
+      bool ok = true;
+      uint32_t j = 0;
+      for (uint32_t g = 0; g < total && ok; ++g) {
+        const uint32_t kt = g % (uint32_t)kt_count;
+        const int s = g % S, b = g % NB;
+        j = g / (uint32_t)kt_count;
+        if (kt == 0) {
+          if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1)) { ok = false; break; }
+        }
+        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 2)) { ok = false; break; }
+        if (!mbar_wait(sf_full0 + 8 * b, (g / NB) & 1, abort_flag, p.status, 9)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + s * C::A_HALF), b0 = smem_u32(sB + s * C::B_HALF);
+          const uint32_t sfa = tmem + SFA_COL + b * C::SF_BUF, sfb = sfa + 4 * ATOMS;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int atom = NV ? t : (t >> 1);
+            const uint32_t sf_id = NV ? 0u : (uint32_t)((t & 1) * 2);
+            tc_mma_pair<NV>(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t),
+                            idesc_pair(NV, sf_id, sf_id), sfa + 4 * atom, sfb + 8 * atom,
+                            (kt > 0 || t > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(empty0 + 8 * s);                               // frees stage s in both CTAs
+          tc_commit_local_pair(sf_empty0 + 8 * b);                      // scale buffer b may be refilled
+          if (kt == (uint32_t)kt_count - 1) tc_commit_pair(tmem_full);  // accumulator ready in both CTAs
+        }
+        __syncwarp();
+      }
+      j = my_tiles;
+      if (ok) {
+        // both epilogues have released the last accumulator (all their arrivals have landed)
+        mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 5);
+      } else if (lane == 0) {
+        tc_commit_local_pair(drain0);
+        const unsigned long long t0 = now_ns();
+        while (!mbar_try(drain0, 0) && now_ns() - t0 < kTimeoutNs) {
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const float alpha = p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f;
+    const uint32_t empty_leader = map_rank(tmem_empty, 0);
+    uint32_t j = 0;
+    for (int tile = cid; tile < num_tiles; tile += ncl, ++j) {
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16);
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t r0[32], r1[32];
+        TC_LD32(taddr + c * 32, r0);
+        TC_LD32(taddr + (c + 1) * 32, r1);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          uint32_t b0, b1;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b0)
+              : "f"(__fmul_rn(__uint_as_float(r0[2 * i + 1]), alpha)), "f"(__fmul_rn(__uint_as_float(r0[2 * i]), alpha)));
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b1)
+              : "f"(__fmul_rn(__uint_as_float(r1[2 * i + 1]), alpha)), "f"(__fmul_rn(__uint_as_float(r1[2 * i]), alpha)));
+          pk[c * 16 + i] = b0;
+          pk[(c + 1) * 16 + i] = b1;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(empty_leader);  // accumulator read out in this warp's lanes
+      const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+      uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN);
+#pragma unroll
+      for (int v = 0; v < BN / 8; ++v) crow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Host side: tensor maps through the driver entry point (no link against libcuda).
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -371,14 +682,51 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint6
   return r == CUDA_SUCCESS;
 }
 
+// Scale tiles in the MMA tile layout viewed as a 3-D tensor of 32-bit words: 128 words (one
+// 512-byte 128x4 atom) x atoms per 128-row group x row groups.  A box of `atoms` atoms x
+// `groups` row groups lands in shared memory as consecutive atoms, group-major.
+static bool make_sf_map(CUtensorMap* m, const void* base, uint64_t atoms_row, uint64_t groups, uint32_t atoms,
+                        uint32_t box_groups) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, atoms_row, groups};
+  cuuint64_t strides[2] = {512, atoms_row * 512};
+  cuuint32_t box[3] = {128, atoms, box_groups};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace gemm
+
+static cudaError_t launch_gemm_pair(const GemmLaunch& L, const gemm::Params& p, cudaStream_t s) {
+  using namespace gemm;
+  const uint32_t atoms = L.nv ? 4 : 2;
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_map(&ta, L.Aq, (uint64_t)L.K / 2, (uint64_t)L.M, 128) ||
+      !make_map(&tb, L.Bq, (uint64_t)L.K / 2, (uint64_t)L.N, 128) ||
+      !make_sf_map(&tsa, L.As, (uint64_t)p.atoms_row, (uint64_t)L.M / 128, atoms, 1) ||
+      !make_sf_map(&tsb, L.Bs, (uint64_t)p.atoms_row, (uint64_t)L.N / 128, atoms, 2))
+    return cudaErrorInvalidValue;
+  const int tiles = (L.M / 256) * (L.N / 256);
+  const int pairs = num_sms() / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  if (L.nv) {
+    auto k = gemm_pair_kernel<true>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<true>::SMEM);
+    k<<<grid, PAIR_THREADS, PairCfg<true>::SMEM, s>>>(ta, tb, tsa, tsb, p);
+  } else {
+    auto k = gemm_pair_kernel<false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg<false>::SMEM);
+    k<<<grid, PAIR_THREADS, PairCfg<false>::SMEM, s>>>(ta, tb, tsa, tsb, p);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   using namespace gemm;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, L.Aq, (uint64_t)L.K / 2, (uint64_t)L.M, BM) ||
-      !make_map(&tb, L.Bq, (uint64_t)L.K / 2, (uint64_t)L.N, BN))
-    return cudaErrorInvalidValue;
   Params p;
   p.M = L.M; p.N = L.N; p.K = L.K; p.nv = L.nv ? 1 : 0;
   p.atoms = L.nv ? 4 : 2;
@@ -387,6 +735,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   p.C = reinterpret_cast<__nv_bfloat16_raw*>(L.C);
   p.ldc = L.ldc;
   p.status = L.status;
+  if (L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, L.Aq, (uint64_t)L.K / 2, (uint64_t)L.M, BM) ||
+      !make_map(&tb, L.Bq, (uint64_t)L.K / 2, (uint64_t)L.N, BN))
+    return cudaErrorInvalidValue;
   const int tiles = (L.M / BM) * (L.N / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   if (L.nv) {

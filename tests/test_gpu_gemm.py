@@ -58,12 +58,14 @@ def packed_from_codes(codes):
 
 
 @pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
-def test_gemm_one_hot_structure(cuda, fmt):
+@pytest.mark.parametrize("mn", [(128, 256), (256, 256), (512, 768)])  # 1-SM tiles; 2-SM pair tiles
+def test_gemm_one_hot_structure(cuda, fmt, mn):
     """A[m, k] = 1 only at k = km(m); B[n, k] = 1 only at k = kn(n); every block scale distinct, so
     C[m, n] = dA[m, km/B] * dB[n, km/B] when km(m) == kn(n), else 0 — an exact bf16 value.  This
     pins the nibble order inside a byte, the K order inside the swizzled tile and the scale-tile
     layout of both operands."""
-    M, N, K = 128, 256, 512
+    M, N = mn
+    K = 512
     Bk = 16 if fmt == fp4.NVFP4 else 32
     nb = K // Bk
     km = (np.arange(M) * 7 + 3) % K
