@@ -246,18 +246,31 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
 // ---------------------------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64 multiplies with the round
 // keys advanced by the Weyl increments.  Counter (blk lo, blk hi, 0, 0), key (seed lo, seed hi).
+// The round keys depend only on the seed (key + r * Weyl increment), so the host computes them once
+// and the kernels read them from their parameter block: a round is then two 32x32->64 multiplies
+// and two three-input XORs.
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+inline PhiloxKeys philox_keys(unsigned long long seed) {
+  PhiloxKeys K;
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = (uint32_t)seed + (uint32_t)r * 0x9E3779B9u;
+    K.k1[r] = (uint32_t)(seed >> 32) + (uint32_t)r * 0xBB67AE85u;
+  }
+  return K;
+}
+
 struct Philox4 { uint32_t w[4]; };
-__device__ __forceinline__ Philox4 philox4x32_10(uint64_t blk, uint64_t seed) {
+__device__ __forceinline__ Philox4 philox4x32_10(uint64_t blk, const PhiloxKeys& K) {
   uint32_t c0 = (uint32_t)blk, c1 = (uint32_t)(blk >> 32), c2 = 0u, c3 = 0u;
-  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
-    c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ K.k0[r];
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ K.k1[r];
+    c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
   }
   Philox4 o;
   o.w[0] = c0; o.w[1] = c1; o.w[2] = c2; o.w[3] = c3;
@@ -266,38 +279,44 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint64_t blk, uint64_t seed) {
 
 // Random words for E consecutive elements starting at flat index idx0 (idx0 % 4 == 0).
 template <int E>
-__device__ __forceinline__ void sr_words(uint64_t idx0, uint64_t seed, uint32_t* r) {
+__device__ __forceinline__ void sr_words(uint64_t idx0, const PhiloxKeys& K, uint32_t* r) {
 #pragma unroll
   for (int k = 0; k < E / 4; ++k) {
-    Philox4 p = philox4x32_10((idx0 >> 2) + k, seed);
+    Philox4 p = philox4x32_10((idx0 >> 2) + k, K);
 #pragma unroll
     for (int i = 0; i < 4; ++i) r[4 * k + i] = p.w[i];
   }
 }
 
-// Stochastic rounding of y onto the E2M1 lattice, returning the rounded lattice value (with the
-// sign of y).  For a = |y| <= 6: lo = largest lattice point <= a (steps of .5 below 2, 1 below 4,
-// 2 up to 6), p = (a - lo)/step; round up iff r < ceil(p * 2^32).  a - lo is exact (Sterbenz)
-// and the scaling by 2^32/step is a power of two, so the threshold is exact.  a > 6 clamps.
+__device__ __forceinline__ uint32_t f2u_ceil(float x) {  // x in [0, 2^32): ceil, exact
+  uint32_t u;
+  asm("cvt.rpi.u32.f32 %0, %1;" : "=r"(u) : "f"(x));
+  return u;
+}
+
+// Stochastic rounding of y onto the E2M1 lattice, returning the rounded lattice value with the
+// sign of y.  For a = |y| <= 6 with lo the largest lattice point <= a and p = (a - lo)/step, the
+// value rounds up iff r < ceil(p * 2^32); a > 6 clamps to 6.
+//   a in [1, 6]: the points of [2^e, 2^(e+1)) are 2^e * {1, 1.5} (and 4, 6 in [4, 8)), so lo keeps
+//     the top mantissa bit, and p * 2^32 is the remaining 22-bit mantissa field shifted left by 10
+//     (an exact integer); rounding up adds one unit of that top bit.
+//   a < 1: points 0, 0.5, 1; q = 2a and q - floor(q) are exact, and so is their product by 2^32;
+//     the threshold is its ceiling.
 __device__ __forceinline__ float sr_round(float y, uint32_t r) {
-  const float a = fabsf(y);
-  float lo, scale, step;
-  if (a < 2.0f) {
-    lo = __fmul_rn(floorf(__fmul_rn(a, 2.0f)), 0.5f); step = 0.5f; scale = 8589934592.0f;  // 2^33
-  } else if (a < 4.0f) {
-    lo = floorf(a); step = 1.0f; scale = 4294967296.0f;                                    // 2^32
+  const uint32_t bits = __float_as_uint(y);
+  const uint32_t ab = bits & 0x7FFFFFFFu;
+  uint32_t res;
+  if (ab >= 0x3F800000u) {
+    const uint32_t lo = ab & 0xFFC00000u;
+    const uint32_t t = (ab & 0x003FFFFFu) << 10;
+    res = (ab > 0x40C00000u) ? 0x40C00000u : (lo + ((r < t) ? 0x00400000u : 0u));
   } else {
-    lo = 4.0f; step = 2.0f; scale = 2147483648.0f;                                         // 2^31
+    const float q = __fmul_rn(__uint_as_float(ab), 2.0f);
+    const float fl = (q >= 1.0f) ? 1.0f : 0.0f;
+    const uint32_t th = f2u_ceil(__fmul_rn(__fsub_rn(q, fl), 4294967296.0f));
+    res = __float_as_uint(__fmul_rn(__fadd_rn(fl, (r < th) ? 1.0f : 0.0f), 0.5f));
   }
-  float v;
-  if (a > 6.0f) {
-    v = 6.0f;
-  } else {
-    const float t = ceilf(__fmul_rn(__fsub_rn(a, lo), scale));
-    const unsigned long long th = __float2ull_rn(t);
-    v = ((unsigned long long)r < th) ? __fadd_rn(lo, step) : lo;
-  }
-  return copysignf(v, y);
+  return __uint_as_float(res | (bits & 0x80000000u));
 }
 
 // ---------------------------------------------------------------------------------------------

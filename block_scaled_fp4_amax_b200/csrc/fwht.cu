@@ -41,14 +41,27 @@ __device__ __forceinline__ int swz(int i) {  // word offset of element i inside 
   return (row << 5) | ((((i >> 2) & 7) ^ (row & 7)) << 2) | (i & 3);
 }
 
+// One butterfly stage on local bit BIT: (v[p], v[p+h]) -> (v[p]+v[p+h], v[p]-v[p+h]).  For
+// BIT >= 1 the pairs (p, p+1) and (p+h, p+h+1) are processed together with the sm_100 packed
+// fp32 add/sub (each half an IEEE fp32 operation, so the result is identical to two scalar ones).
 template <int BIT>
 __device__ __forceinline__ void stage(float (&v)[32]) {
+  if constexpr (BIT == 0) {
 #pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    if (!(p & (1 << BIT))) {
-      const float a = v[p], b = v[p | (1 << BIT)];
+    for (int p = 0; p < 32; p += 2) {
+      const float a = v[p], b = v[p + 1];
       v[p] = __fadd_rn(a, b);
-      v[p | (1 << BIT)] = __fsub_rn(a, b);
+      v[p + 1] = __fsub_rn(a, b);
+    }
+  } else {
+    constexpr int H = 1 << BIT;
+#pragma unroll
+    for (int p = 0; p < 32; p += 2) {
+      if (!(p & H)) {
+        const f32x2 a = f2_pack(v[p], v[p + 1]), b = f2_pack(v[p + H], v[p + H + 1]);
+        f2_unpack(f2_add(a, b), v[p], v[p + 1]);
+        f2_unpack(f2_sub(a, b), v[p + H], v[p + H + 1]);
+      }
     }
   }
 }
@@ -62,18 +75,18 @@ __device__ __forceinline__ void stages(float (&v)[32]) {  // local bits LO..HI_-
 
 template <typename T>
 struct RowLoad {
-  static constexpr int NV = 32 * (int)sizeof(T) / 16;  // 16-byte chunks per thread
+  static constexpr int NV = 32 * (int)sizeof(T) / 32;  // 32-byte chunks per thread
 };
 
 // Round A + B + last-round rotation of one row into v[32] (last-round order: j = low | h << L).
 // `raw` holds this thread's round-A chunks.  Leaves the values unnormalised.
 template <typename T, int LOG_D>
-__device__ __forceinline__ void rotate_row(const uint4 (&raw)[RowLoad<T>::NV], float* srow, int t,
+__device__ __forceinline__ void rotate_row(const U8 (&raw)[RowLoad<T>::NV], float* srow, int t,
                                            float (&v)[32]) {
   using G = Geom<LOG_D>;
   // round A: index bits 0-4 local
 #pragma unroll
-  for (int c = 0; c < RowLoad<T>::NV; ++c) Vec<T>::unpack(raw[c], v + c * Vec<T>::E);
+  for (int c = 0; c < RowLoad<T>::NV; ++c) Vec32<T>::unpack(raw[c], v + c * Vec32<T>::E);
   stages<0, 5>(v);
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -116,15 +129,15 @@ __device__ __forceinline__ void rotate_row(const uint4 (&raw)[RowLoad<T>::NV], f
 
 template <typename T, int LOG_D>
 __device__ __forceinline__ void load_row(const T* x, long long row, long long rows, int t,
-                                         uint4 (&raw)[RowLoad<T>::NV]) {
+                                         U8 (&raw)[RowLoad<T>::NV]) {
   constexpr int D = 1 << LOG_D;
   if (row < rows) {
     const char* p = reinterpret_cast<const char*>(x + row * D + (long long)t * 32);
 #pragma unroll
-    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = ld16<false>(p + 16 * c);
+    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = ld32<false>(p + 32 * c);
   } else {
 #pragma unroll
-    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = 0; c < RowLoad<T>::NV; ++c) for (int i = 0; i < 8; ++i) raw[c].w[i] = 0u;
   }
 }
 
@@ -134,7 +147,7 @@ struct FwhtParams {
   float c;            // fl(1/sqrt(d))
   int tiled;
   int reverse;
-  unsigned long long seed;
+  PhiloxKeys keys;
   const float* global_in;
   uint32_t* amax_bits;
   float* global_out;
@@ -155,7 +168,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   const T* x = reinterpret_cast<const T*>(p.x);
   const long long step = (long long)gridDim.x * G::ROWS;
   float m = 0.0f;
-  uint4 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
   long long row = (long long)blockIdx.x * G::ROWS + slot;
   load_row<T, LOG_D>(x, row, p.rows, t, raw);
   for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = s_g;
   }
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};
-  uint4 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
   auto phys = [&](long long r) { return p.reverse ? (p.rows - 1 - r) : r; };
   long long row = (long long)blockIdx.x * G::ROWS + slot;
   load_row<T, LOG_D>(x, row < p.rows ? phys(row) : row, p.rows, t, raw);
@@ -260,9 +273,9 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
       uint32_t rnd[GA];
       if (SR) {
         if constexpr (GE >= 4) {
-          sr_words<GE>(idx0, p.seed, rnd);
+          sr_words<GE>(idx0, p.keys, rnd);
         } else {
-          const Philox4 ph = philox4x32_10(idx0 >> 2, p.seed);
+          const Philox4 ph = philox4x32_10(idx0 >> 2, p.keys);
 #pragma unroll
           for (int i = 0; i < GE; ++i) rnd[i] = ph.w[(idx0 + i) & 3];
         }
@@ -353,7 +366,7 @@ static FwhtParams make_params(const FwhtLaunch& L) {
   FwhtParams p;
   p.x = L.x; p.rows = L.rows;
   p.c = (float)(1.0 / sqrt((double)L.d));
-  p.tiled = L.tiled; p.reverse = 0; p.seed = L.seed;
+  p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed);
   p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
   p.six_m = L.four_six ? 1536.0f : 2688.0f;
   p.rotated_out = L.rotated_out; p.q = L.q; p.scales = L.scales; p.counts = L.counts;

@@ -61,7 +61,7 @@ struct QuantParams {
   int policy;          // MXFP4 exponent rule
   int tiled;           // scale layout
   int reverse;         // walk the tiles last-to-first (re-use the tail a previous pass left in L2)
-  unsigned long long seed;
+  PhiloxKeys keys;     // stochastic-rounding round keys (from the seed)
   const float* global_in;
   const uint32_t* amax_bits;
   float* global_out;
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       const float amax = __uint_as_float(am);
       const unsigned long long idx0 = (unsigned long long)c * E;
       uint32_t rnd[E];
-      if (SR) sr_words<E>(idx0, p.seed, rnd);
+      if (SR) sr_words<E>(idx0, p.keys, rnd);
       uint32_t w[W], sc, sat = 0, four = 0;
       if (!NV) {
         const int e = mx_exponent(am, p.policy);
@@ -294,7 +294,7 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   p.policy = L.policy;
   p.tiled = L.tiled;
   p.reverse = L.reverse;
-  p.seed = L.seed;
+  p.keys = philox_keys(L.seed);
   p.global_in = L.global_in;
   p.amax_bits = L.amax_bits;
   p.global_out = L.global_out;

@@ -100,7 +100,7 @@ typedef enum fp4_op { FP4_OP_MX_QUANTIZE = 0, FP4_OP_NVFP4_QUANTIZE = 1, FP4_OP_
  * mx_quantize — MXFP4 quantisation of a row-major [rows, cols] tensor, blocks of 32 along rows.
  * Follows [A] "Encode one MXFP4 block step by step": per block amax, shared exponent e (policy),
  * y = x * 2^-e (exact), E2M1 encode (RNE or stochastic), saturate at 6, nibble pack.
- *   x      : device, [rows, cols] of `dtype`, 32-byte aligned (FWHT input: 16-byte aligned).
+ *   x      : device, [rows, cols] of `dtype`, 32-byte aligned (the same for every quantiser).
  *   block  : must be 32 (no block-size inference; anything else is FP4_EINVAL).
  *   q      : device, [rows, cols/2] bytes, 8-byte aligned; element 2j in the low nibble of byte j, 2j+1 high
  *            ([A] "Encode one MXFP4 block": values 0 and 1 share the first byte, low half first).
