@@ -363,6 +363,32 @@ __device__ __forceinline__ int zero_codes_n(const uint32_t* w) {
 
 // N values scaled by R and E2M1-encoded (RNE or stochastic); saturations counted per value only
 // when the block maximum normalises above 6 (`top` = fl(amax * R), monotone in |x|).
+// `y` receives the scaled values fl(v * R) (before any stochastic rounding).
+template <int N, bool SR>
+__device__ __forceinline__ void encode_y_n(const float* v, float R, float top, const uint32_t* rnd,
+                                           float* y, uint32_t* w, uint32_t& sat) {
+  if constexpr (N % 2 == 0) {
+    const f32x2 R2 = f2_pack(R, R);
+#pragma unroll
+    for (int j = 0; j < N; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y[j], y[j + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
+  }
+  if (top > 6.0f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
+  }
+  if (SR) {
+    float t[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) t[i] = sr_round(y[i], rnd[i]);
+    e2m1_pack_n<N>(t, w);
+  } else {
+    e2m1_pack_n<N>(y, w);
+  }
+}
+
 template <int N, bool SR>
 __device__ __forceinline__ void encode_n(const float* v, float R, float top, const uint32_t* rnd,
                                          uint32_t* w, uint32_t& sat) {
@@ -386,40 +412,52 @@ __device__ __forceinline__ void encode_n(const float* v, float R, float top, con
   e2m1_pack_n<N>(y, w);
 }
 
-// One NVFP4 candidate (target T through inv_t = fl(1/fl(T*s_g))): returns the E4M3 code, writes
-// the packed nibbles, the saturation count and the decoded scale d.
-template <int N, bool SR>
-__device__ __forceinline__ uint32_t nv_candidate_n(const float* v, float amax, float s_g, float inv_t,
-                                                   const uint32_t* rnd, uint32_t* w, uint32_t& sat,
-                                                   float& d) {
-  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
-  d = e4m3_value(sc);
-  sat = 0;
-  if (sc == 0) {
-    float y[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) y[i] = copysignf(0.0f, v[i]);
-    e2m1_pack_n<N>(y, w);
-  } else {
-    const float R = __frcp_rn(__fmul_rn(d, s_g));
-    encode_n<N, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
+// NVFP4 per-code scale table: for every E4M3 code byte c, D = fl(value(c) * s_g) and
+// R = fl(1 / D) (all 256 bytes, so a caller-supplied negative or non-finite global scale indexes
+// inside it and behaves as the direct computation would).  Filled once per CTA into shared memory,
+// it replaces the per-block decode, multiply and reciprocal.  Entry 0 holds R = 0: a block whose
+// scale code is 0 has only finite values (a non-finite amax gives code 0x7E or 0x7F), so v * 0 is
+// the signed zero that block encodes to, and no branch is needed for it.
+constexpr int kScaleTab = 256;
+__device__ __forceinline__ void fill_scale_tab(float2* tab, float s_g) {
+  for (int c = threadIdx.x; c < kScaleTab; c += blockDim.x) {
+    const float D = __fmul_rn(e4m3_value((uint32_t)c), s_g);
+    tab[c] = make_float2(D, c == 0 ? 0.0f : __frcp_rn(D));
   }
+}
+
+// One NVFP4 candidate (target T through inv_t = fl(1/fl(T*s_g))): returns the E4M3 code and
+// writes the packed nibbles and the saturation count.
+template <int N, bool SR>
+__device__ __forceinline__ uint32_t nv_candidate_n(const float* v, float amax, float inv_t, const float2* tab,
+                                                   const uint32_t* rnd, uint32_t* w, uint32_t& sat) {
+  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
+  sat = 0;
+  const float R = tab[sc].y;  // 0 for code 0: every value encodes to its signed zero
+  encode_n<N, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
   return sc;
 }
 
-// Squared dequantisation errors fl((x - fl(fl(v*d)*s_g))^2), d the value of E4M3 `code`.
+// Squared dequantisation errors fl((x - fl(fl(q*d)*s_g))^2), d the value of E4M3 `code`.
+//
+// The packed words are decoded as `w ^ opaque0`, opaque0 a zero the kernel reads from its
+// parameters.  With CUDA 12.9 on sm_100a, `cvt.rn.f16x2.e2m1x2` applied to bytes 2 and 3 of a word
+// that was just assembled in registers from `cvt.rn.satfinite.e2m1x2.f32` results returned zeros in
+// some kernels (observed by comparing the decoded values with the stored nibbles).  A decode of a
+// word the compiler cannot trace back to those byte registers (one loaded from memory, or XORed
+// with a value only known at run time) is correct, so every in-register decode goes through it.
 // For pairs, v*d is formed in f16x2 straight from the nibble conversion: |v| <= 6 has two
 // significant bits and d four, so the product (at least 2^-10, at most 2688) is exact in f16.
 template <int N>
-__device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, uint32_t code, float d, float s_g,
-                                            float* sq) {
+__device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, uint32_t code, float s_g,
+                                            uint32_t opaque0, float* sq) {
   if constexpr (N % 2 == 0) {
     uint32_t dh2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(dh2) : "h"((uint16_t)(code | (code << 8))));
 #pragma unroll
     for (int k = 0; k < (N + 7) / 8; ++k) {
       uint32_t h[4];
-      e2m1x8_to_f16x2(w[k], h);
+      e2m1x8_to_f16x2(w[k] ^ opaque0, h);
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         const int j = 8 * k + 2 * b;
@@ -439,8 +477,12 @@ __device__ __forceinline__ void sq_errors_n(const float* v, const uint32_t* w, u
     }
     return;
   }
+  const float d = e4m3_value(code);
+  uint32_t wo[(N + 7) / 8];
+#pragma unroll
+  for (int k = 0; k < (N + 7) / 8; ++k) wo[k] = w[k] ^ opaque0;
   float q[N];
-  e2m1_unpack_n<N>(w, q);
+  e2m1_unpack_n<N>(wo, q);
 #pragma unroll
   for (int i = 0; i < N; ++i) {
     const float xhat = __fmul_rn(__fmul_rn(q[i], d), s_g);
@@ -466,6 +508,95 @@ __device__ __forceinline__ float block_sse_n(const float* sq, int lane) {
     }
   }
   return acc;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Four-over-six selection without the exact error sums in the common case.
+//
+// The selection rule compares S_T = fp32 sequential sum of fl(fl(v - fl(fl(q*d)*s_g))^2) for the
+// two candidates T = 6, 4.  A cheaper estimate of the same quantity is the scaled-domain residual
+//   A_T = fl(D^2) * sum (q_i - y_i)^2,   y_i = fl(v_i * R), R = fl(1/D), D = fl(d * s_g),
+// since (q_i - y_i) * D = -(e_i + theta_i v_i) with e_i = v_i - q_i d s_g and |theta_i| <= 3u
+// (u = 2^-24).  With Q = sum e_i^2 and P = sum |e_i||v_i| <= 4 amax sqrt(Q), first-order rounding
+// analysis gives |A_T - Q| <= 6uP + 22uQ and |S_T - Q| <= 2uP + 20uQ (16 terms, every operation
+// one rounding, no overflow, normal D), so |A_T - S_T| <= 32u amax sqrt(Q) + 42uQ.
+// The margin below is four times that (2^-17 = 128u on each term, sqrt(Q) <= 1.0001 sqrt(A_T) +
+// 2^-19 amax), plus 2^-35 amax^2 for the second-order terms and 2^-139 for subnormal squares.
+// When |A_4 - A_6| exceeds it, sign(A_4 - A_6) = sign(S_4 - S_6) and the estimate decides; the
+// caller computes S_T exactly otherwise.
+
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// sum over N values of (q_i - y_i)^2: q_i decoded from the packed nibbles (exact in f16), the
+// difference formed in fp32 from the f16 operand directly.  `opaque0` is a kernel-parameter zero
+// (see sq_errors_n).
+template <int N>
+__device__ __forceinline__ float resid_sq_n(const uint32_t* w, const float* y, uint32_t opaque0) {
+  static_assert(N % 2 == 0, "pairs");
+  f32x2 acc = 0ull;
+#pragma unroll
+  for (int k = 0; k < (N + 7) / 8; ++k) {
+    uint32_t h[4];
+    e2m1x8_to_f16x2(w[k] ^ opaque0, h);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = 8 * k + 2 * b;
+      if (j < N) {
+        float rl, rh;
+        asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
+            "sub.rn.f32.f16 %0, l, %3;\n\tsub.rn.f32.f16 %1, u, %4;\n\t}"
+            : "=f"(rl), "=f"(rh) : "r"(h[b]), "f"(y[j]), "f"(y[j + 1]));
+        const f32x2 r = f2_pack(rl, rh);
+        acc = f2_fma(r, r, acc);
+      }
+    }
+  }
+  float lo, hi;
+  f2_unpack(acc, lo, hi);
+  return lo + hi;
+}
+
+// One NVFP4 candidate as nv_candidate_n, plus D = fl(d * s_g) and the residual sum A (both 0
+// when the scale code is 0).
+template <int N, bool SR>
+__device__ __forceinline__ uint32_t nv_candidate_resid_n(const float* v, float amax, float inv_t, const float2* tab,
+                                                         const uint32_t* rnd, uint32_t opaque0, uint32_t* w,
+                                                         uint32_t& sat, float& D, float& A) {
+  const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
+  sat = 0;
+  const float2 DR = tab[sc];  // code 0: D = 0, R = 0, so y = +-0, the codes are zeros and A = 0
+  D = DR.x;
+  float y[N];
+  encode_y_n<N, SR>(v, DR.y, __fmul_rn(amax, DR.y), rnd, y, w, sat);
+  A = resid_sq_n<N>(w, y, opaque0);
+  return sc;
+}
+
+// Decide four-over-six from the estimates when the margin allows.  `am` is the block amax bit
+// pattern and A6/A4 the residual sums of the whole block.  Returns true when the exact sums are
+// needed; otherwise `four` holds the decision.
+__device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, uint32_t sc6, uint32_t sc4, float D6,
+                                                   float D4, float A6, float A4, bool& four) {
+  const float kDmin = __uint_as_float(0x21800000u);  // 2^-60
+  const float a6 = __fmul_rn(__fmul_rn(D6, D6), A6);
+  const float a4 = __fmul_rn(__fmul_rn(D4, D4), A4);
+  float r6, r4;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r6) : "f"(a6));
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r4) : "f"(a4));
+  const float m = 7.62939453e-06f * (amax * (r6 + r4) * 1.001f + a6 + a4) +  // 2^-17
+                  2.91038305e-11f * amax * amax +                             // 2^-35
+                  __uint_as_float(0x00000400u);                               // 2^-139
+  const float diff = a4 - a6;
+  // amax in [2^-50, 2^60), both codes nonzero, normal D, finite estimates (a NaN fails `<`)
+  const bool in_range = (am >= 0x26800000u) & (am < 0x5D800000u) & (sc6 != 0u) & (sc4 != 0u) & (D6 >= kDmin) &
+                        (D4 >= kDmin) & (a6 < INFINITY) & (a4 < INFINITY);
+  four = (am != 0u) & (diff < 0.0f);
+  // an all-zero block has equal (zero) sums and keeps 6 without the exact path
+  return (am != 0u) & !(in_range & (fabsf(diff) > m));
 }
 
 // ---------------------------------------------------------------------------------------------

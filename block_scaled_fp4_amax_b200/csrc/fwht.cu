@@ -148,6 +148,7 @@ struct FwhtParams {
   int tiled;
   int reverse;
   PhiloxKeys keys;
+  uint32_t zero;      // 0, read at run time: makes in-register nibble decodes opaque
   const float* global_in;
   uint32_t* amax_bits;
   float* global_out;
@@ -229,6 +230,8 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
     inv4 = __frcp_rn(__fmul_rn(4.0f, s_g));
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = s_g;
   }
+  __shared__ float2 tab[NV ? kScaleTab : 1];
+  if (NV) fill_scale_tab(tab, s_g);  // first read after the rotation's __syncthreads
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};
   U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
   auto phys = [&](long long r) { return p.reverse ? (p.rows - 1 - r) : r; };
@@ -290,23 +293,40 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
         encode_n<GE, SR>(g, inv, __fmul_rn(amax, inv), rnd, w, sat);
         sc = (uint32_t)(e + 127);
       } else {
-        float d6;
-        sc = nv_candidate_n<GE, SR>(g, amax, s_g, inv6, rnd, w, sat, d6);
         if constexpr (FOUR_SIX) {
-          float d4, sq[GA];
-          uint32_t w4[WN], sat4;
-          const uint32_t sc4 = nv_candidate_n<GE, SR>(g, amax, s_g, inv4, rnd, w4, sat4, d4);
-          sq_errors_n<GE>(g, w, sc, d6, s_g, sq);
-          const float sse6 = block_sse_n<GE, GL>(sq, lane);
-          sq_errors_n<GE>(g, w4, sc4, d4, s_g, sq);
-          const float sse4 = block_sse_n<GE, GL>(sq, lane);
-          if (sse4 < sse6) {
+          float sq[GA];
+          uint32_t w4[WN], sat4, sc4;
+          bool pick4 = false, undecided = true;
+          if constexpr (GE % 2 == 0) {
+            float D6, D4, A6, A4;
+            sc = nv_candidate_resid_n<GE, SR>(g, amax, inv6, tab, rnd, p.zero, w, sat, D6, A6);
+            sc4 = nv_candidate_resid_n<GE, SR>(g, amax, inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
+#pragma unroll
+            for (int o = 1; o < GL; o <<= 1) {  // butterfly: identical sums on every lane of the block
+              A6 += __shfl_xor_sync(0xFFFFFFFFu, A6, o);
+              A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
+            }
+            undecided = four_six_undecided(am, amax, sc, sc4, D6, D4, A6, A4, pick4);
+          } else {
+            sc = nv_candidate_n<GE, SR>(g, amax, inv6, tab, rnd, w, sat);
+            sc4 = nv_candidate_n<GE, SR>(g, amax, inv4, tab, rnd, w4, sat4);
+          }
+          if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform: the exact sums shuffle
+            sq_errors_n<GE>(g, w, sc, s_g, p.zero, sq);
+            const float sse6 = block_sse_n<GE, GL>(sq, lane);
+            sq_errors_n<GE>(g, w4, sc4, s_g, p.zero, sq);
+            const float sse4 = block_sse_n<GE, GL>(sq, lane);
+            pick4 = sse4 < sse6;
+          }
+          if (pick4) {
             sc = sc4;
             sat = sat4;
             four = 1;
 #pragma unroll
             for (int k = 0; k < WN; ++k) w[k] = w4[k];
           }
+        } else {
+          sc = nv_candidate_n<GE, SR>(g, amax, inv6, tab, rnd, w, sat);
         }
       }
       if (valid) {
@@ -366,7 +386,7 @@ static FwhtParams make_params(const FwhtLaunch& L) {
   FwhtParams p;
   p.x = L.x; p.rows = L.rows;
   p.c = (float)(1.0 / sqrt((double)L.d));
-  p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed);
+  p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed); p.zero = 0u;
   p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
   p.six_m = L.four_six ? 1536.0f : 2688.0f;
   p.rotated_out = L.rotated_out; p.q = L.q; p.scales = L.scales; p.counts = L.counts;

@@ -22,7 +22,8 @@
 namespace fp4k {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 4;      // 32-byte chunks in flight per lane
+constexpr int kUnroll46 = 2;    // four-over-six: compute-bound, so a smaller body is worth more
 
 // ---------------------------------------------------------------------------------------------
 // MXFP4 shared exponent from the amax bit pattern (exact): OCP floor(log2 amax) - 2, or the
@@ -62,6 +63,7 @@ struct QuantParams {
   int tiled;           // scale layout
   int reverse;         // walk the tiles last-to-first (re-use the tail a previous pass left in L2)
   PhiloxKeys keys;     // stochastic-rounding round keys (from the seed)
+  uint32_t zero;       // 0, read at run time: makes in-register nibble decodes opaque
   const float* global_in;
   const uint32_t* amax_bits;
   float* global_out;
@@ -71,22 +73,56 @@ struct QuantParams {
   unsigned long long* counts;
 };
 
+// Exact four-over-six choice for one chunk (the rare case the estimates cannot decide): reloads
+// the chunk's values (an L2 hit: the kernel read them moments ago) and compares the two fp32
+// sequential error sums.  Out of line so the unrolled main loop keeps a single copy of it; called
+// by the whole warp (the block sums shuffle when G > 1).
+template <typename T, int G>
+__device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, bool valid, uint32_t w6a, uint32_t w6b,
+                                                uint32_t w4a, uint32_t w4b, uint32_t sc6, uint32_t sc4, float s_g,
+                                                uint32_t zero) {
+  constexpr int E = Vec32<T>::E;
+  U8 raw;
+  if (valid) {  // plain 16-byte loads: ptxas 12.9 crashed on the 256-bit load asm in this function
+    const uint4 lo = __ldg(reinterpret_cast<const uint4*>(xb + c * 32));
+    const uint4 hi = __ldg(reinterpret_cast<const uint4*>(xb + c * 32 + 16));
+    raw.w[0] = lo.x; raw.w[1] = lo.y; raw.w[2] = lo.z; raw.w[3] = lo.w;
+    raw.w[4] = hi.x; raw.w[5] = hi.y; raw.w[6] = hi.z; raw.w[7] = hi.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) raw.w[i] = 0u;
+  }
+  float v[E], sq[E];
+  Vec32<T>::unpack(raw, v);
+  const int lane = threadIdx.x & 31;
+  const uint32_t w6[2] = {w6a, w6b}, w4[2] = {w4a, w4b};
+  sq_errors_n<E>(v, w6, sc6, s_g, zero, sq);
+  const float sse6 = block_sse_n<E, G>(sq, lane);
+  sq_errors_n<E>(v, w4, sc4, s_g, zero, sq);
+  const float sse4 = block_sse_n<E, G>(sq, lane);
+  return sse4 < sse6 ? 1u : 0u;
+}
+
 template <typename T, bool NV, bool SR, bool FOUR_SIX>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
   constexpr int E = Vec32<T>::E;  // 16 (bf16) or 8 (fp32)
   constexpr int B = NV ? 16 : 32;
   constexpr int G = B / E;
   constexpr int W = E / 8;        // packed words per chunk
+  constexpr int U = FOUR_SIX ? kUnroll46 : kUnroll;
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
-  const long long per_tile = 32LL * kUnroll;
+  const long long per_tile = 32LL * U;
   const long long ntiles = (p.n_chunks + per_tile - 1) / per_tile;
 
   NvScale ns{1.0f, 1.0f, 1.0f};
+  __shared__ float2 tab[NV ? kScaleTab : 1];
   if (NV) {
     ns = nv_scales(p.global_in, p.amax_bits, p.six_m);
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = ns.s_g;
+    fill_scale_tab(tab, ns.s_g);
+    __syncthreads();
   }
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};  // underflow, saturation, nonfinite, blocks_four
   const char* xb = reinterpret_cast<const char*>(p.x);
@@ -94,9 +130,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
   for (long long t = warp; t < ntiles; t += nwarps) {
     const long long tile = p.reverse ? (ntiles - 1 - t) : t;
     const long long c0 = tile * per_tile + lane;
-    U8 raw[kUnroll];
+    U8 raw[U];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const long long c = c0 + 32LL * u;
       if (c < p.n_chunks) {
         raw[u] = ld32<true>(xb + c * 32);
@@ -106,7 +142,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const long long c = c0 + 32LL * u;
       const bool valid = c < p.n_chunks;
       float v[E];
@@ -130,19 +166,23 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         encode_n<E, SR>(v, inv, __fmul_rn(amax, inv), rnd, w, sat);
         sc = (uint32_t)(e + 127);
       } else if (!FOUR_SIX) {
-        float d;
-        sc = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d);
+        sc = nv_candidate_n<E, SR>(v, amax, ns.inv6, tab, rnd, w, sat);
       } else {
-        float d6, d4, sq[E];
+        float D6, D4, A6, A4;
         uint32_t w4[W], sat4;
-        const uint32_t sc6 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv6, rnd, w, sat, d6);
-        const uint32_t sc4 = nv_candidate_n<E, SR>(v, amax, ns.s_g, ns.inv4, rnd, w4, sat4, d4);
-        sq_errors_n<E>(v, w, sc6, d6, ns.s_g, sq);
-        const float sse6 = block_sse_n<E, G>(sq, lane);
-        sq_errors_n<E>(v, w4, sc4, d4, ns.s_g, sq);
-        const float sse4 = block_sse_n<E, G>(sq, lane);
+        const uint32_t sc6 = nv_candidate_resid_n<E, SR>(v, amax, ns.inv6, tab, rnd, p.zero, w, sat, D6, A6);
+        const uint32_t sc4 = nv_candidate_resid_n<E, SR>(v, amax, ns.inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) {  // butterfly: every lane of the block gets the same sums
+          A6 += __shfl_xor_sync(0xFFFFFFFFu, A6, o);
+          A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
+        }
+        bool pick4;
+        const bool undecided = four_six_undecided(am, amax, sc6, sc4, D6, D4, A6, A4, pick4);
+        if (__any_sync(0xFFFFFFFFu, undecided))  // warp-uniform call: the exact sums shuffle
+          pick4 = four_six_exact<T, G>(xb, c, valid, w[0], w[W - 1], w4[0], w4[W - 1], sc6, sc4, ns.s_g, p.zero) != 0u;
         sc = sc6;
-        if (sse4 < sse6) {
+        if (pick4) {
           sc = sc4;
           sat = sat4;
           four = 1;
@@ -270,10 +310,22 @@ static int grid_for(long long work_items, int per_cta) {
   return (int)(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
+// One wave of resident CTAs (the kernel loops over tiles), so no CTA waits in a tail wave.
 template <typename T, bool NV, bool SR, bool FS>
 static cudaError_t launch_q(const QuantParams& p, cudaStream_t s) {
-  const long long tiles = (p.n_chunks + 32LL * kUnroll - 1) / (32LL * kUnroll);
-  const int grid = grid_for(tiles * 32, kThreads);
+  static int per_sm = 0;  // resident CTAs per SM for this instantiation (same on every sm_100 device)
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<T, NV, SR, FS>, kThreads, 0) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  constexpr int U = FS ? kUnroll46 : kUnroll;
+  const long long tiles = (p.n_chunks + 32LL * U - 1) / (32LL * U);
+  const long long want = (tiles * 32 + kThreads - 1) / kThreads;
+  const long long cap = (long long)num_sms() * per_sm;
+  const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
   quantize_kernel<T, NV, SR, FS><<<grid, kThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
@@ -295,6 +347,7 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   p.tiled = L.tiled;
   p.reverse = L.reverse;
   p.keys = philox_keys(L.seed);
+  p.zero = 0u;
   p.global_in = L.global_in;
   p.amax_bits = L.amax_bits;
   p.global_out = L.global_out;

@@ -11,6 +11,8 @@ Workloads (shapes are parameters so the same recipe serves small parity cases):
   gemm_normal   bf16 N(0,1)                                  seeds 1, 2  (8192 x 8192 each)
   swiglu_act    bf16 silu(g) * u, g, u ~ N(0,1)              seed 3      (4096 x 28672)
   weight        bf16 N(0, 0.02)                              seed 4      (8192 x 28672)
+  lattice_steps k / 8 for integers k uniform in [-48, 48]       (parity cases: exact ties between
+                                                                 the two four-over-six candidates)
 """
 from __future__ import annotations
 
@@ -78,6 +80,15 @@ def swiglu_act(rows: int = 4096, cols: int = 28672, seed: int = 3) -> torch.Tens
 
 def weight(rows: int = 8192, cols: int = 28672, seed: int = 4, std: float = 0.02) -> torch.Tensor:
     return normal_bf16(rows, cols, seed, std)
+
+
+def lattice_steps(rows: int, cols: int, seed: int, denom: int = 8, kmax: int = 48) -> torch.Tensor:
+    """bf16 values k / denom, k uniform on [-kmax, kmax] (exact in bf16).  Such blocks sit on or
+    near both four-over-six grids at once, so many of them have equal or nearly equal block
+    errors under the two candidates."""
+    rng = np.random.default_rng(seed)
+    k = rng.integers(-kmax, kmax + 1, size=(rows, cols))
+    return _to_bf16((k / denom).astype(np.float32))
 
 
 def as_f32_numpy(t: torch.Tensor) -> np.ndarray:

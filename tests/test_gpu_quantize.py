@@ -168,6 +168,19 @@ def test_nvfp4_caller_global_and_ragged(cuda, four_six):
     run_nv(torch.zeros(64, 64), cuda, four_six=four_six)                               # amax 0 -> s_g = 1
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rnd", [fp4.RNE, fp4.STOCHASTIC])
+def test_nvfp4_four_six_near_ties(cuda, dtype, rnd):
+    """Blocks of k/8 values: about 2% have candidate error sums too close for the cheap estimate
+    to separate, and about 1% would be decided wrongly by it, so this fails unless the exact
+    fp32 sums are taken whenever the estimate is inside its error margin."""
+    x = synth.lattice_steps(512, 1024, 41)
+    x = x if dtype == torch.bfloat16 else x.float()
+    run_nv(x, cuda, rnd=rnd, four_six=True, seed=3)
+    run_nv(x, cuda, rnd=rnd, four_six=True, seed=3, global_in=1.0 / 256)
+    run_nv(x, cuda, rnd=rnd, four_six=True, seed=3, global_in=0.0037)
+
+
 @pytest.mark.parametrize("four_six", [False, True])
 def test_nvfp4_config2_full(cuda, four_six):
     """8192 x 8192 bf16 N(0,1) with 8 outlier columns x U(50,100), seed 5; plain and 4/6."""
