@@ -114,16 +114,16 @@ template <> struct Vec32<__nv_bfloat16> {
     return 16 - nz;
   }
   // Largest magnitude as an fp32 bit pattern (16-bit lane-wise max of the bf16 magnitudes);
-  // `any_zero` is set if some value is +-0 (a zero half borrows: (m - 1) & ~m has its top bit).
+  // `any_zero` is set if some value is +-0 (lane-wise minimum magnitude 0).
   __device__ __forceinline__ static uint32_t max_mag(const U8& r, bool& any_zero) {
-    uint32_t m = 0u, z = 0u;
+    uint32_t m = 0u, mn = 0x7FFF7FFFu;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t a = r.w[i] & 0x7FFF7FFFu;
       asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(a));
-      z |= (a - 0x00010001u) & ~a;
+      asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(a));
     }
-    any_zero = (z & 0x80008000u) != 0u;
+    any_zero = ((mn & 0xFFFFu) == 0u) | ((mn >> 16) == 0u);
     return max(m & 0xFFFFu, m >> 16) << 16;
   }
 };
@@ -361,10 +361,11 @@ __device__ __forceinline__ int zero_codes_n(const uint32_t* w) {
   }
 }
 
-// N values scaled by R and E2M1-encoded (RNE or stochastic); saturations counted per value only
-// when the block maximum normalises above 6 (`top` = fl(amax * R), monotone in |x|).
-// `y` receives the scaled values fl(v * R) (before any stochastic rounding).
-template <int N, bool SR>
+// N values scaled by R and E2M1-encoded (RNE or stochastic); with CNT, saturations are counted per
+// value only when the block maximum normalises above 6 (`top` = fl(amax * R), monotone in |x|);
+// without it the caller counts them (sat_count_bf16x16).  `y` receives the scaled values
+// fl(v * R) (before any stochastic rounding).
+template <int N, bool SR, bool CNT = true>
 __device__ __forceinline__ void encode_y_n(const float* v, float R, float top, const uint32_t* rnd,
                                            float* y, uint32_t* w, uint32_t& sat) {
   if constexpr (N % 2 == 0) {
@@ -375,7 +376,7 @@ __device__ __forceinline__ void encode_y_n(const float* v, float R, float top, c
 #pragma unroll
     for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
   }
-  if (top > 6.0f) {
+  if (CNT && top > 6.0f) {
 #pragma unroll
     for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
   }
@@ -389,27 +390,35 @@ __device__ __forceinline__ void encode_y_n(const float* v, float R, float top, c
   }
 }
 
-template <int N, bool SR>
+template <int N, bool SR, bool CNT = true>
 __device__ __forceinline__ void encode_n(const float* v, float R, float top, const uint32_t* rnd,
                                          uint32_t* w, uint32_t& sat) {
   float y[N];
-  if constexpr (N % 2 == 0) {
-    const f32x2 R2 = f2_pack(R, R);
+  encode_y_n<N, SR, CNT>(v, R, top, rnd, y, w, sat);
+}
+
+// Saturation count of 16 bf16 values (8 packed words) under the scale pair (D, R = fl(1/D)):
+// the number of values with fl(|v| * R) > 6.  The predicate is monotone in |v|, so it holds
+// exactly for |v| >= t, t the smallest bf16 magnitude that satisfies it.  6D and the real
+// threshold (6 + 2^-22) / R differ by about 2^-22 relative while one bf16 step is at least 2^-8,
+// so t is one of the three bf16 values from b0 = bf16_rd(fl(6 * D)) up, and two predicate tests
+// pick it.  The count is then 8 bf16x2 compares accumulated in bf16x2 (exact small integers).
+// Only meaningful when the block maximum saturates (fl(amax * R) > 6, so D is positive and finite).
+__device__ __forceinline__ uint32_t sat_count_bf16x16(const uint32_t* w, float D, float R) {
+  const uint32_t xb = __float_as_uint(__fmul_rn(6.0f, D)) & 0xFFFF0000u;
+  const uint32_t tb = (__fmul_rn(__uint_as_float(xb), R) > 6.0f)             ? xb
+                      : (__fmul_rn(__uint_as_float(xb + 0x10000u), R) > 6.0f) ? xb + 0x10000u
+                                                                              : xb + 0x20000u;
+  const uint32_t t2 = (tb >> 16) | (tb & 0xFFFF0000u);
+  uint32_t acc;
+  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(acc) : "r"(w[0] & 0x7FFF7FFFu), "r"(t2));
 #pragma unroll
-    for (int j = 0; j < N; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y[j], y[j + 1]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
+  for (int i = 1; i < 8; ++i) {
+    uint32_t s;
+    asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(s) : "r"(w[i] & 0x7FFF7FFFu), "r"(t2));
+    asm("add.rn.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(s));
   }
-  if (top > 6.0f) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
-  }
-  if (SR) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) y[i] = sr_round(y[i], rnd[i]);
-  }
-  e2m1_pack_n<N>(y, w);
+  return (uint32_t)(__uint_as_float(acc << 16) + __uint_as_float(acc & 0xFFFF0000u));
 }
 
 // NVFP4 per-code scale table: for every E4M3 code byte c, D = fl(value(c) * s_g) and
@@ -428,13 +437,15 @@ __device__ __forceinline__ void fill_scale_tab(float2* tab, float s_g) {
 
 // One NVFP4 candidate (target T through inv_t = fl(1/fl(T*s_g))): returns the E4M3 code and
 // writes the packed nibbles and the saturation count.
-template <int N, bool SR>
+template <int N, bool SR, bool CNT = true>
 __device__ __forceinline__ uint32_t nv_candidate_n(const float* v, float amax, float inv_t, const float2* tab,
-                                                   const uint32_t* rnd, uint32_t* w, uint32_t& sat) {
+                                                   const uint32_t* rnd, uint32_t* w, uint32_t& sat,
+                                                   float2* DR_out = nullptr) {
   const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
   sat = 0;
-  const float R = tab[sc].y;  // 0 for code 0: every value encodes to its signed zero
-  encode_n<N, SR>(v, R, __fmul_rn(amax, R), rnd, w, sat);
+  const float2 DR = tab[sc];  // R = 0 for code 0: every value encodes to its signed zero
+  encode_n<N, SR, CNT>(v, DR.y, __fmul_rn(amax, DR.y), rnd, w, sat);
+  if (DR_out) *DR_out = DR;
   return sc;
 }
 
@@ -521,7 +532,8 @@ __device__ __forceinline__ float block_sse_n(const float* sq, int lane) {
 // analysis gives |A_T - Q| <= 6uP + 22uQ and |S_T - Q| <= 2uP + 20uQ (16 terms, every operation
 // one rounding, no overflow, normal D), so |A_T - S_T| <= 32u amax sqrt(Q) + 42uQ.
 // The margin below is four times that (2^-17 = 128u on each term, sqrt(Q) <= 1.0001 sqrt(A_T) +
-// 2^-19 amax), plus 2^-35 amax^2 for the second-order terms and 2^-139 for subnormal squares.
+// 2^-19 amax), plus 2^-35 amax^2 for the second-order terms and 2^-139 for subnormal squares;
+// amax sqrt(A) <= (amax^2 + A) / 2 then gives the square-root-free form used below.
 // When |A_4 - A_6| exceeds it, sign(A_4 - A_6) = sign(S_4 - S_6) and the estimate decides; the
 // caller computes S_T exactly otherwise.
 
@@ -537,7 +549,7 @@ __device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
 template <int N>
 __device__ __forceinline__ float resid_sq_n(const uint32_t* w, const float* y, uint32_t opaque0) {
   static_assert(N % 2 == 0, "pairs");
-  f32x2 acc = 0ull;
+  float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
   for (int k = 0; k < (N + 7) / 8; ++k) {
     uint32_t h[4];
@@ -550,28 +562,27 @@ __device__ __forceinline__ float resid_sq_n(const uint32_t* w, const float* y, u
         asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
             "sub.rn.f32.f16 %0, l, %3;\n\tsub.rn.f32.f16 %1, u, %4;\n\t}"
             : "=f"(rl), "=f"(rh) : "r"(h[b]), "f"(y[j]), "f"(y[j + 1]));
-        const f32x2 r = f2_pack(rl, rh);
-        acc = f2_fma(r, r, acc);
+        acc0 = fmaf(rl, rl, acc0);
+        acc1 = fmaf(rh, rh, acc1);
       }
     }
   }
-  float lo, hi;
-  f2_unpack(acc, lo, hi);
-  return lo + hi;
+  return acc0 + acc1;
 }
 
 // One NVFP4 candidate as nv_candidate_n, plus D = fl(d * s_g) and the residual sum A (both 0
 // when the scale code is 0).
-template <int N, bool SR>
+template <int N, bool SR, bool CNT = true>
 __device__ __forceinline__ uint32_t nv_candidate_resid_n(const float* v, float amax, float inv_t, const float2* tab,
                                                          const uint32_t* rnd, uint32_t opaque0, uint32_t* w,
-                                                         uint32_t& sat, float& D, float& A) {
+                                                         uint32_t& sat, float& D, float& A, float* R_out = nullptr) {
   const uint32_t sc = e4m3_code(__fmul_rn(amax, inv_t));
   sat = 0;
   const float2 DR = tab[sc];  // code 0: D = 0, R = 0, so y = +-0, the codes are zeros and A = 0
   D = DR.x;
+  if (R_out) *R_out = DR.y;
   float y[N];
-  encode_y_n<N, SR>(v, DR.y, __fmul_rn(amax, DR.y), rnd, y, w, sat);
+  encode_y_n<N, SR, CNT>(v, DR.y, __fmul_rn(amax, DR.y), rnd, y, w, sat);
   A = resid_sq_n<N>(w, y, opaque0);
   return sc;
 }
@@ -579,21 +590,18 @@ __device__ __forceinline__ uint32_t nv_candidate_resid_n(const float* v, float a
 // Decide four-over-six from the estimates when the margin allows.  `am` is the block amax bit
 // pattern and A6/A4 the residual sums of the whole block.  Returns true when the exact sums are
 // needed; otherwise `four` holds the decision.
-__device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, uint32_t sc6, uint32_t sc4, float D6,
-                                                   float D4, float A6, float A4, bool& four) {
-  const float kDmin = __uint_as_float(0x21800000u);  // 2^-60
+__device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, float D6, float D4, float A6,
+                                                   float A4, bool& four) {
   const float a6 = __fmul_rn(__fmul_rn(D6, D6), A6);
   const float a4 = __fmul_rn(__fmul_rn(D4, D4), A4);
-  float r6, r4;
-  asm("sqrt.approx.f32 %0, %1;" : "=f"(r6) : "f"(a6));
-  asm("sqrt.approx.f32 %0, %1;" : "=f"(r4) : "f"(a4));
-  const float m = 7.62939453e-06f * (amax * (r6 + r4) * 1.001f + a6 + a4) +  // 2^-17
-                  2.91038305e-11f * amax * amax +                             // 2^-35
-                  __uint_as_float(0x00000400u);                               // 2^-139
+  const float sa = a6 + a4;
+  // amax (sqrt a6 + sqrt a4) <= amax^2 + (a6 + a4) / 2, so this is at least the margin above
+  const float m = 7.62939453e-06f * (1.02f * amax * amax + 2.0f * sa) + __uint_as_float(0x00000400u);  // 2^-17, 2^-139
   const float diff = a4 - a6;
-  // amax in [2^-50, 2^60), both codes nonzero, normal D, finite estimates (a NaN fails `<`)
-  const bool in_range = (am >= 0x26800000u) & (am < 0x5D800000u) & (sc6 != 0u) & (sc4 != 0u) & (D6 >= kDmin) &
-                        (D4 >= kDmin) & (a6 < INFINITY) & (a4 < INFINITY);
+  // amax in [2^-50, 2^60); D4 >= D6 (monotone rounding of amax/(T s_g)) and D6 >= 2^-60 (so both
+  // codes are nonzero and D is normal); finite estimates (a NaN fails `<`)
+  const bool in_range = (am >= 0x26800000u) & (am < 0x5D800000u) & (D6 >= __uint_as_float(0x21800000u)) &
+                        (sa < INFINITY);
   four = (am != 0u) & (diff < 0.0f);
   // an all-zero block has equal (zero) sums and keeps 6 without the exact path
   return (am != 0u) & !(in_range & (fabsf(diff) > m));

@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
               A6 += __shfl_xor_sync(0xFFFFFFFFu, A6, o);
               A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
             }
-            undecided = four_six_undecided(am, amax, sc, sc4, D6, D4, A6, A4, pick4);
+            undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
           } else {
             sc = nv_candidate_n<GE, SR>(g, amax, inv6, tab, rnd, w, sat);
             sc4 = nv_candidate_n<GE, SR>(g, amax, inv4, tab, rnd, w4, sat4);

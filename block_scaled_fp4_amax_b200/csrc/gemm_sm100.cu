@@ -10,16 +10,16 @@
 //
 // gemm_pair_kernel (M % 256 == 0): clusters of two CTAs on neighbouring SMs, each pair computing a
 // 256 x 256 tile with tcgen05 cta_group::2 (each SM holds half of A and half of B per stage), K
-// consumed 256 values per stage in a 5-6 stage ring.  Seven warps per CTA:
+// consumed 256 values per stage in a 5-6 stage ring.  Twelve warps per CTA:
 //   warp 0     TMA producer (both CTAs): operand tiles by 2-D tensor maps with 128-byte swizzle,
 //              scale tiles by 3-D tensor maps; all loads complete on the leader's barrier;
-//   warp 6     (leader) copies each stage's scales smem -> TMEM (tcgen05.cp) into one of three
-//              TMEM scale buffers — issued from its own warp so the copies queue separately from
-//              the MMAs and overlap them;
+//   warps 2-3  (leader) copy each stage's scales smem -> TMEM (tcgen05.cp) into one of three
+//              TMEM scale buffers, half of the scale atoms each — issued from their own warps so
+//              the copies queue separately from the MMAs and overlap them;
 //   warp 1     (leader) issues tcgen05.mma kind::mxf4nvf4 and the commits that free smem stages,
 //              scale buffers and, per tile, hand the accumulator to the epilogue;
-//   warps 2-5  epilogue (both CTAs): tcgen05.ld the FP32 accumulator quarter this warp may access,
-//              scale by alpha, round to bf16, release the accumulator, store.
+//   warps 4-11 epilogue (both CTAs): each tcgen05.lds a 32-row x 128-column part of the FP32
+//              accumulator, releases it, then scales by alpha, rounds to bf16 and stores.
 // gemm_kernel (M % 256 == 128): the same pipeline on one SM with 128 x 256 tiles.
 // Every mbarrier wait is bounded in time; on expiry the kernel records the site in the caller's
 // status word, tells the other roles to stop, drains what it issued and frees tensor memory.
@@ -130,6 +130,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdes
                  "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
                  ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
   }
+}
+
+// Two fp32 accumulator words scaled by alpha and rounded to bf16 (RNE), the first in the low half.
+__device__ __forceinline__ uint32_t bf16x2_scaled(uint32_t lo, uint32_t hi, float alpha) {
+  uint32_t b;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+      : "=r"(b)
+      : "f"(__fmul_rn(__uint_as_float(hi), alpha)), "f"(__fmul_rn(__uint_as_float(lo), alpha)));
+  return b;
 }
 
 #define TC_LD32(taddr, r)                                                                                   \
@@ -425,7 +434,10 @@ template <bool NV> struct PairCfg {
   static constexpr int SMEM = 1024 + S * STAGE + 512;
   static constexpr uint32_t SF_BUF = 12u * ATOMS;  // TMEM columns per scale buffer: SFA 4*ATOMS + SFB 8*ATOMS
 };
-constexpr int PAIR_THREADS = 224;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6 scale copies
+// warp 0 TMA, 1 MMA, 2-3 scale copies, 4-11 epilogue (two warps per tensor-memory lane quadrant,
+// one per 128-column half of the accumulator)
+constexpr int PAIR_THREADS = 384;
+constexpr int PAIR_CP_WARPS = 2;
 
 template <bool NV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
@@ -433,6 +445,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, Params p) {
   using C = PairCfg<NV>;
   constexpr int S = C::S, ATOMS = C::ATOMS, NB = C::NB;
+  static_assert(SFA_COL + NB * (int)C::SF_BUF <= TMEM_COLS, "scale buffers exceed the tensor-memory allocation");
   constexpr uint32_t TX_PAIR = 2u * C::STAGE;
 
   extern __shared__ uint8_t smem_raw[];
@@ -442,8 +455,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint8_t* sSFA = sB + S * C::B_HALF;
   uint8_t* sSFB = sSFA + S * C::SFA_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::SFB_BYTES);
-  // bars: full[S] (leader), empty[S], sf_full[NB], sf_empty[NB], tmem_full, tmem_empty (leader), drain[2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 4);
+  // bars: full[S] (leader), empty[S], sf_full[NB], sf_empty[NB], tmem_full, tmem_empty (leader),
+  // drain[1 + PAIR_CP_WARPS] (MMA warp, each scale-copy warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 3 + PAIR_CP_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -460,13 +474,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < NB; ++b) {
-      mbar_init(sf_full0 + 8 * b, 1);
+      mbar_init(sf_full0 + 8 * b, PAIR_CP_WARPS);  // one commit per scale-copy warp
       mbar_init(sf_empty0 + 8 * b, 1);
     }
     mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 8);  // 4 epilogue warps in each CTA of the pair
-    mbar_init(drain0, 1);
-    mbar_init(drain0 + 8, 1);
+    mbar_init(tmem_empty, 16);  // 8 epilogue warps in each CTA of the pair
+    for (int i = 0; i <= PAIR_CP_WARPS; ++i) mbar_init(drain0 + 8 * i, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -523,11 +536,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       }
     }
-  } else if (warp == 6) {
+  } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------------ scale copies (leader)
-    // Issued from their own warp so that they queue separately from the MMAs: iteration g's
-    // scales go to TMEM buffer g % NB once its stage has landed and the MMAs that last read
-    // the buffer have completed; a commit then tells the MMA warp the buffer is ready.
+    // Issued from their own warps so that they queue separately from the MMAs, and split over two
+    // warps (each a contiguous half of the stage's scale atoms, all three copies of an atom):
+    // tcgen05.cp issue from one thread was the limit with NVFP4's 12 copies per stage.  Iteration
+    // g's scales go to TMEM buffer g % NB once its stage has landed and the MMAs that last read
+    // the buffer have completed; each warp's commit then counts towards the buffer being ready.
+    const int ci = warp - 2;
+    constexpr int PER = ATOMS / PAIR_CP_WARPS;
+    static_assert(ATOMS % PAIR_CP_WARPS == 0, "whole atoms per copy warp");
     if (leader) {
       bool ok = true;
       uint32_t g = 0;
@@ -540,7 +558,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const uint32_t fa = smem_u32(sSFA + s * C::SFA_BYTES), fbs = smem_u32(sSFB + s * C::SFB_BYTES);
           const uint32_t sfa = tmem + SFA_COL + b * C::SF_BUF, sfb = sfa + 4 * ATOMS;
 #pragma unroll
-          for (int a = 0; a < ATOMS; ++a) {
+          for (int i = 0; i < PER; ++i) {
+            const int a = ci * PER + i;
             tc_cp_sf_pair(sfa + 4 * a, desc_sf(fa + a * 512));
             tc_cp_sf_pair(sfb + 8 * a, desc_sf(fbs + a * 512));
             tc_cp_sf_pair(sfb + 8 * a + 4, desc_sf(fbs + (ATOMS + a) * 512));
@@ -556,9 +575,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8)) break;
         }
       } else if (lane == 0) {
-        tc_commit_local_pair(drain0 + 8);
+        const uint32_t dr = drain0 + 8 * (1 + ci);
+        tc_commit_local_pair(dr);
         const unsigned long long t0 = now_ns();
-        while (!mbar_try(drain0 + 8, 0) && now_ns() - t0 < kTimeoutNs) {
+        while (!mbar_try(dr, 0) && now_ns() - t0 < kTimeoutNs) {
         }
       }
       __syncwarp();
@@ -608,8 +628,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       __syncwarp();
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
-    const int q = warp & 3;
+    // ------------------------------------------------------------------ epilogue (warps 4..11, both CTAs)
+    // Warp w reads tensor-memory lanes 32 (w % 4).. (its rows) and accumulator columns
+    // 128 (w >= 8).. : four 32-column loads, one wait, then the accumulator is released to the MMA
+    // warp before the conversion and the stores, so the next tile's MMAs wait only for the loads.
+    const int q = warp & 3, half = warp >= 8 ? 1 : 0;
     const float alpha = p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f;
     const uint32_t empty_leader = map_rank(tmem_empty, 0);
     uint32_t j = 0;
@@ -617,32 +640,28 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int tm = tile % tiles_m, tn = tile / tiles_m;
       if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16);
-      uint32_t pk[BN / 2];
-#pragma unroll
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t r0[32], r1[32];
-        TC_LD32(taddr + c * 32, r0);
-        TC_LD32(taddr + (c + 1) * 32, r1);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          uint32_t b0, b1;
-          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b0)
-              : "f"(__fmul_rn(__uint_as_float(r0[2 * i + 1]), alpha)), "f"(__fmul_rn(__uint_as_float(r0[2 * i]), alpha)));
-          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b1)
-              : "f"(__fmul_rn(__uint_as_float(r1[2 * i + 1]), alpha)), "f"(__fmul_rn(__uint_as_float(r1[2 * i]), alpha)));
-          pk[c * 16 + i] = b0;
-          pk[(c + 1) * 16 + i] = b1;
-        }
-      }
+      const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      TC_LD32(taddr, r0);
+      TC_LD32(taddr + 32, r1);
+      TC_LD32(taddr + 64, r2);
+      TC_LD32(taddr + 96, r3);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(empty_leader);  // accumulator read out in this warp's lanes
-      const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
-      uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN);
+      if (lane == 0) mbar_arrive_cluster(empty_leader);  // this warp's part of the accumulator is read
+      uint32_t pk[64];
 #pragma unroll
-      for (int v = 0; v < BN / 8; ++v) crow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = bf16x2_scaled(r0[2 * i], r0[2 * i + 1], alpha);
+        pk[16 + i] = bf16x2_scaled(r1[2 * i], r1[2 * i + 1], alpha);
+        pk[32 + i] = bf16x2_scaled(r2[2 * i], r2[2 * i + 1], alpha);
+        pk[48 + i] = bf16x2_scaled(r3[2 * i], r3[2 * i + 1], alpha);
+      }
+      const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+      uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN + half * 128);
+#pragma unroll
+      for (int v = 0; v < 16; ++v) crow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
   }
 

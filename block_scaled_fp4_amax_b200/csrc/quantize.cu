@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
   constexpr int G = B / E;
   constexpr int W = E / 8;        // packed words per chunk
   constexpr int U = FOUR_SIX ? kUnroll46 : kUnroll;
+  constexpr bool kBF = E == 16;   // bf16 input: saturations counted with bf16x2 compares
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
@@ -163,22 +164,42 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
       if (!NV) {
         const int e = mx_exponent(am, p.policy);
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
-        encode_n<E, SR>(v, inv, __fmul_rn(amax, inv), rnd, w, sat);
+        const float top = __fmul_rn(amax, inv);
+        encode_n<E, SR, !kBF>(v, inv, top, rnd, w, sat);
+        if constexpr (kBF) {  // D = 2^e exactly (2^-127 is the subnormal 0x00400000)
+          const float D = __uint_as_float(e > -127 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
+          const uint32_t n = sat_count_bf16x16(raw[u].w, D, inv);
+          sat = top > 6.0f ? n : 0u;
+        }
         sc = (uint32_t)(e + 127);
       } else if (!FOUR_SIX) {
-        sc = nv_candidate_n<E, SR>(v, amax, ns.inv6, tab, rnd, w, sat);
+        float2 DR;
+        sc = nv_candidate_n<E, SR, !kBF>(v, amax, ns.inv6, tab, rnd, w, sat, &DR);
+        if constexpr (kBF) {
+          const uint32_t n = sat_count_bf16x16(raw[u].w, DR.x, DR.y);
+          sat = __fmul_rn(amax, DR.y) > 6.0f ? n : 0u;
+        }
       } else {
-        float D6, D4, A6, A4;
+        float D6, D4, A6, A4, R6, R4;
         uint32_t w4[W], sat4;
-        const uint32_t sc6 = nv_candidate_resid_n<E, SR>(v, amax, ns.inv6, tab, rnd, p.zero, w, sat, D6, A6);
-        const uint32_t sc4 = nv_candidate_resid_n<E, SR>(v, amax, ns.inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
+        const uint32_t sc6 =
+            nv_candidate_resid_n<E, SR, !kBF>(v, amax, ns.inv6, tab, rnd, p.zero, w, sat, D6, A6, &R6);
+        const uint32_t sc4 =
+            nv_candidate_resid_n<E, SR, !kBF>(v, amax, ns.inv4, tab, rnd, p.zero, w4, sat4, D4, A4, &R4);
+        if constexpr (kBF) {
+          // target 6: about half the blocks saturate their maximum, so count without a branch;
+          // target 4 normalises the maximum to about 4 and saturates only with a clamped scale
+          const uint32_t n = sat_count_bf16x16(raw[u].w, D6, R6);
+          sat = __fmul_rn(amax, R6) > 6.0f ? n : 0u;
+          if (__fmul_rn(amax, R4) > 6.0f) sat4 = sat_count_bf16x16(raw[u].w, D4, R4);
+        }
 #pragma unroll
         for (int o = 1; o < G; o <<= 1) {  // butterfly: every lane of the block gets the same sums
           A6 += __shfl_xor_sync(0xFFFFFFFFu, A6, o);
           A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
         }
         bool pick4;
-        const bool undecided = four_six_undecided(am, amax, sc6, sc4, D6, D4, A6, A4, pick4);
+        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
         if (__any_sync(0xFFFFFFFFu, undecided))  // warp-uniform call: the exact sums shuffle
           pick4 = four_six_exact<T, G>(xb, c, valid, w[0], w[W - 1], w4[0], w4[W - 1], sc6, sc4, ns.s_g, p.zero) != 0u;
         sc = sc6;

@@ -130,6 +130,44 @@ def test_mx_edge_values(cuda):
         run_mx(xt, cuda, policy=pol)
 
 
+def _bf16_steps_around(center, n, rng):
+    """n bf16 values on consecutive bf16 steps centred on bf16(center), random signs (float32)."""
+    b = np.array([center], dtype=np.float32).view(np.uint32)[0] >> 16
+    bits = (b + np.arange(-(n // 2), n - n // 2)).astype(np.uint32) << 16
+    vals = bits.view(np.float32).copy()
+    return vals * rng.choice(np.array([-1.0, 1.0], dtype=np.float32), n)
+
+
+def test_saturation_count_bf16_near_threshold(cuda):
+    """Blocks whose maximum saturates, every other value on consecutive bf16 steps around the
+    saturation threshold 6*d (NVFP4, caller global scale 1, so the block scale is d) or 6*2^e
+    (MXFP4): the saturation counters must equal the oracle's per-element count."""
+    rng = np.random.default_rng(11)
+    ds = [(1 + m / 8) * 2.0 ** k for k in range(-6, 7) for m in range(8)]
+    nv = []
+    for _ in range(4096):
+        d = ds[rng.integers(len(ds))]
+        blk = np.empty(16, dtype=np.float32)
+        blk[0] = 6 * d * 1.03           # maps to scale d, normalises above 6
+        blk[1:] = _bf16_steps_around(6 * d, 15, rng)
+        nv.append(rng.permutation(blk))
+    x = torch.from_numpy(np.concatenate(nv).reshape(-1, 512)).to(torch.bfloat16)
+    for fs in (False, True):
+        run_nv(x, cuda, four_six=fs, global_in=1.0)
+    mx = []
+    for _ in range(2048):
+        e = int(rng.integers(-20, 21))
+        blk = np.empty(32, dtype=np.float32)
+        blk[0] = 7 * 2.0 ** e           # floor(log2) = e + 2: shared exponent e, normalises to 7
+        blk[1:] = _bf16_steps_around(6 * 2.0 ** e, 31, rng)
+        mx.append(rng.permutation(blk))
+    x = torch.from_numpy(np.concatenate(mx).reshape(-1, 512)).to(torch.bfloat16)
+    _, _, c = fp4.mx_quantize(x.to(cuda))
+    _, _, co = O.mx_quantize(f32(x))
+    assert counts_of(c) == co and co["saturation"] > 0
+    run_mx(x, cuda)
+
+
 def test_mx_empty_and_nonfinite_counts(cuda):
     q, s, c = fp4.mx_quantize(torch.empty((0, 64), dtype=torch.float32, device=cuda))
     assert q.numel() == 0 and counts_of(c)["nonfinite"] == 0
