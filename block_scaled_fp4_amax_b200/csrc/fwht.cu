@@ -198,21 +198,47 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   }
 }
 
-// Pass 2: rotate again, normalise, quantise from registers.
-template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX>
-__global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams p) {
+// Last-round order -> 32 consecutive values per thread, through the (free) row buffer: the thread
+// writes its 2^NH groups of 2^L consecutive values and reads back elements [32 t, 32 t + 32), so
+// that every quantisation block lies inside one thread.  Both the writes (consecutive 16-byte
+// chunks across a warp) and the reads (one swizzled 128-byte row per thread) are conflict-free.
+template <int LOG_D>
+__device__ __forceinline__ void to_consecutive(float* srow, int t, float (&v)[32]) {
   using G = Geom<LOG_D>;
-  constexpr int L = G::L, NH = G::NH, HI = G::HI, D = G::D;
+  constexpr int L = G::L, NH = G::NH, HI = G::HI;
+#pragma unroll
+  for (int h = 0; h < (1 << NH); ++h) {
+    const int i0 = (t << L) | (h << HI);
+    if constexpr (L >= 2) {
+#pragma unroll
+      for (int q = 0; q < (1 << L) / 4; ++q) {
+        const float* f = v + (h << L) + 4 * q;
+        *reinterpret_cast<float4*>(srow + swz(i0 + 4 * q)) = make_float4(f[0], f[1], f[2], f[3]);
+      }
+    } else if constexpr (L == 1) {
+      *reinterpret_cast<float2*>(srow + swz(i0)) = make_float2(v[h << 1], v[(h << 1) + 1]);
+    } else {
+      srow[swz(i0)] = v[h];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 f = *reinterpret_cast<const float4*>(srow + swz((t << 5) + 4 * q));
+    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+  }
+  __syncthreads();  // row buffer free for the next row
+}
+
+// Pass 2: rotate again, normalise, quantise from registers (whole blocks per thread).
+template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX>
+__global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 : 1) fwht_quant_kernel(FwhtParams p) {
+  using G = Geom<LOG_D>;
+  constexpr int D = G::D;
   constexpr int B = NV ? 16 : 32;
-  constexpr int LB = NV ? 4 : 5;                 // log2 block
-  constexpr int GE = 1 << L;                     // elements per group
-  constexpr int GL = (L >= LB) ? 1 : (1 << (LB - L));  // lanes per block
-  constexpr int GA = GE < 4 ? 4 : GE;            // register array size for one group
-  constexpr int WN = GE >= 8 ? GE / 8 : 1;        // packed nibble words per group
-  static_assert(L <= LB, "group larger than a block");
+  constexpr int W = B / 8;  // packed nibble words per block
   extern __shared__ __align__(16) float smem[];
   const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
-  const int lane = threadIdx.x & 31;
   float* srow = smem + slot * D;
   const T* x = reinterpret_cast<const T*>(p.x);
   const long long step = (long long)gridDim.x * G::ROWS;
@@ -242,124 +268,92 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_quant_kernel(FwhtParams
     load_row<T, LOG_D>(x, rn < p.rows ? phys(rn) : rn, p.rows, t, nxt);
     float v[32];
     rotate_row<T, LOG_D>(raw, srow, t, v);
-    const bool valid = row < p.rows;
+    to_consecutive<LOG_D>(srow, t, v);
+    const bool valid = row < p.rows;  // uniform over the row's warps
     const long long prow = valid ? phys(row) : 0;
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], p.c);
     if (valid && p.rotated_out) {
+      float4* dst = reinterpret_cast<float4*>(p.rotated_out + prow * D + (t << 5));
 #pragma unroll
-      for (int h = 0; h < (1 << NH); ++h) {
-        float* dst = p.rotated_out + prow * D + ((t << L) | (h << HI));
-        if constexpr (L >= 2) {
-#pragma unroll
-          for (int q = 0; q < GE / 4; ++q)
-            reinterpret_cast<float4*>(dst)[q] = make_float4(v[(h << L) + 4 * q], v[(h << L) + 4 * q + 1],
-                                                            v[(h << L) + 4 * q + 2], v[(h << L) + 4 * q + 3]);
-        } else if constexpr (L == 1) {
-          *reinterpret_cast<float2*>(dst) = make_float2(v[h << 1], v[(h << 1) + 1]);
-        } else {
-          *dst = v[h];
-        }
-      }
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
 #pragma unroll
-    for (int h = 0; h < (1 << NH); ++h) {
-      const float* g = v + (h << L);
-      const int i0 = (t << L) | (h << HI);                      // index in row of g[0]
+    for (int b = 0; b < 32 / B; ++b) {
+      const float* g = v + b * B;
+      const int i0 = (t << 5) + b * B;  // index in row of g[0]
       const unsigned long long idx0 = (unsigned long long)prow * D + i0;
-      uint32_t am = 0u;
+      uint32_t am = 0u, mn = 0xFFFFFFFFu;
 #pragma unroll
-      for (int i = 0; i < GE; ++i) am = max(am, __float_as_uint(g[i]) & 0x7FFFFFFFu);
-#pragma unroll
-      for (int o = 1; o < GL; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-      const float amax = __uint_as_float(am);
-      uint32_t rnd[GA];
-      if (SR) {
-        if constexpr (GE >= 4) {
-          sr_words<GE>(idx0, p.keys, rnd);
-        } else {
-          const Philox4 ph = philox4x32_10(idx0 >> 2, p.keys);
-#pragma unroll
-          for (int i = 0; i < GE; ++i) rnd[i] = ph.w[(idx0 + i) & 3];
-        }
+      for (int i = 0; i < B; ++i) {
+        const uint32_t a = __float_as_uint(g[i]) & 0x7FFFFFFFu;
+        am = max(am, a);
+        mn = min(mn, a);
       }
-      uint32_t w[WN], sc, sat = 0, four = 0;
+      const float amax = __uint_as_float(am);
+      uint32_t w[W], sc, sat = 0, four = 0;
       if (!NV) {
         // MXFP4 OCP rule: e = floor(log2 amax) - 2, clamped to [-127, 127], all-zero -> 0
         const int ef = (int)((am >> 23) & 0xFFu);
         int e = (am == 0u) ? 0 : (ef == 0 ? -127 : ef - 129);
         e = e < -127 ? -127 : e;
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
-        encode_n<GE, SR>(g, inv, __fmul_rn(amax, inv), rnd, w, sat);
-        sc = (uint32_t)(e + 127);
-      } else {
-        if constexpr (FOUR_SIX) {
-          float sq[GA];
-          uint32_t w4[WN], sat4, sc4;
-          bool pick4 = false, undecided = true;
-          if constexpr (GE % 2 == 0) {
-            float D6, D4, A6, A4;
-            sc = nv_candidate_resid_n<GE, SR>(g, amax, inv6, tab, rnd, p.zero, w, sat, D6, A6);
-            sc4 = nv_candidate_resid_n<GE, SR>(g, amax, inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
+        const float top = __fmul_rn(amax, inv);
 #pragma unroll
-            for (int o = 1; o < GL; o <<= 1) {  // butterfly: identical sums on every lane of the block
-              A6 += __shfl_xor_sync(0xFFFFFFFFu, A6, o);
-              A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
-            }
-            undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
-          } else {
-            sc = nv_candidate_n<GE, SR>(g, amax, inv6, tab, rnd, w, sat);
-            sc4 = nv_candidate_n<GE, SR>(g, amax, inv4, tab, rnd, w4, sat4);
-          }
-          if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform: the exact sums shuffle
-            sq_errors_n<GE>(g, w, sc, s_g, p.zero, sq);
-            const float sse6 = block_sse_n<GE, GL>(sq, lane);
-            sq_errors_n<GE>(g, w4, sc4, s_g, p.zero, sq);
-            const float sse4 = block_sse_n<GE, GL>(sq, lane);
-            pick4 = sse4 < sse6;
-          }
-          if (pick4) {
-            sc = sc4;
-            sat = sat4;
-            four = 1;
-#pragma unroll
-            for (int k = 0; k < WN; ++k) w[k] = w4[k];
-          }
-        } else {
-          sc = nv_candidate_n<GE, SR>(g, amax, inv6, tab, rnd, w, sat);
+        for (int hf = 0; hf < B / 16; ++hf) {  // two 16-value halves under the block's one scale
+          uint32_t rnd[16];
+          if (SR) sr_words<16>(idx0 + 16 * hf, p.keys, rnd);
+          encode_n<16, SR>(g + 16 * hf, inv, top, rnd, w + 2 * hf, sat);
         }
+        sc = (uint32_t)(e + 127);
+      } else if constexpr (FOUR_SIX) {
+        uint32_t rnd[B];
+        if (SR) sr_words<B>(idx0, p.keys, rnd);
+        uint32_t w4[W], sat4;
+        float D6, D4, A6, A4;
+        sc = nv_candidate_resid_n<B, SR>(g, amax, inv6, tab, rnd, p.zero, w, sat, D6, A6);
+        const uint32_t sc4 = nv_candidate_resid_n<B, SR>(g, amax, inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
+        bool pick4;
+        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
+        if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform branch
+          float sq[B];
+          sq_errors_n<B>(g, w, sc, s_g, p.zero, sq);
+          const float sse6 = block_sse_n<B, 1>(sq, 0);
+          sq_errors_n<B>(g, w4, sc4, s_g, p.zero, sq);
+          const float sse4 = block_sse_n<B, 1>(sq, 0);
+          pick4 = sse4 < sse6;
+        }
+        if (pick4) {
+          sc = sc4;
+          sat = sat4;
+          four = 1;
+#pragma unroll
+          for (int k = 0; k < W; ++k) w[k] = w4[k];
+        }
+      } else {
+        uint32_t rnd[B];
+        if (SR) sr_words<B>(idx0, p.keys, rnd);
+        sc = nv_candidate_n<B, SR>(g, amax, inv6, tab, rnd, w, sat);
       }
       if (valid) {
         if (am >= 0x7F800000u) {
 #pragma unroll
-          for (int i = 0; i < GE; ++i) cnt[2] += !isfinite(g[i]);
+          for (int i = 0; i < B; ++i) cnt[2] += !isfinite(g[i]);
         }
-        int zx = 0;
+        const int zc = zero_codes_n<B>(w);
+        int zx = 0;  // a +-0 input always gives a zero code: count inputs only when both occur
+        if (zc > 0 && mn == 0u) {
 #pragma unroll
-        for (int i = 0; i < GE; ++i) zx += g[i] == 0.0f;
-        cnt[0] += (uint32_t)(zero_codes_n<GE>(w) - zx);
+          for (int i = 0; i < B; ++i) zx += g[i] == 0.0f;
+        }
+        cnt[0] += (uint32_t)(zc - zx);
         cnt[1] += sat;
-        uint8_t* qrow = p.q + prow * (D / 2);
-        if constexpr (GE == 16) {
-          *reinterpret_cast<uint2*>(qrow + i0 / 2) = make_uint2(w[0], w[WN - 1]);
-        } else if constexpr (GE == 8) {
-          *reinterpret_cast<uint32_t*>(qrow + i0 / 2) = w[0];
-        } else if constexpr (GE == 4) {
-          *reinterpret_cast<uint16_t*>(qrow + i0 / 2) = (uint16_t)w[0];
-        } else if constexpr (GE == 2) {
-          qrow[i0 / 2] = (uint8_t)w[0];
-        }
-        if ((lane & (GL - 1)) == 0) {
-          const unsigned long long blk = (unsigned long long)prow * nb + (i0 >> LB);
-          p.scales[scale_offset(blk, nb, p.tiled)] = (uint8_t)sc;
-          cnt[3] += four;
-        }
-      }
-      if constexpr (GE == 1) {
-        // one value per lane: pair nibbles across neighbouring lanes
-        const uint32_t c1 = w[0] & 0xFu;
-        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, c1, 1);
-        if (valid && !(lane & 1)) p.q[prow * (D / 2) + i0 / 2] = (uint8_t)(c1 | (other << 4));
+        uint2* q2 = reinterpret_cast<uint2*>(p.q + prow * (D / 2) + i0 / 2);
+#pragma unroll
+        for (int k = 0; k < W; k += 2) q2[k / 2] = make_uint2(w[k], w[k + 1]);
+        const unsigned long long blk = (unsigned long long)prow * nb + (unsigned)(i0 / B);
+        p.scales[scale_offset(blk, nb, p.tiled)] = (uint8_t)sc;
+        cnt[3] += four;
       }
     }
 #pragma unroll
