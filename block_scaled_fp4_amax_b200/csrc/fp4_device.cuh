@@ -294,29 +294,41 @@ __device__ __forceinline__ uint32_t f2u_ceil(float x) {  // x in [0, 2^32): ceil
   return u;
 }
 
-// Stochastic rounding of y onto the E2M1 lattice, returning the rounded lattice value with the
-// sign of y.  For a = |y| <= 6 with lo the largest lattice point <= a and p = (a - lo)/step, the
-// value rounds up iff r < ceil(p * 2^32); a > 6 clamps to 6.
-//   a in [1, 6]: the points of [2^e, 2^(e+1)) are 2^e * {1, 1.5} (and 4, 6 in [4, 8)), so lo keeps
-//     the top mantissa bit, and p * 2^32 is the remaining 22-bit mantissa field shifted left by 10
-//     (an exact integer); rounding up adds one unit of that top bit.
-//   a < 1: points 0, 0.5, 1; q = 2a and q - floor(q) are exact, and so is their product by 2^32;
-//     the threshold is its ceiling.
-__device__ __forceinline__ float sr_round(float y, uint32_t r) {
+// Stochastic rounding of y onto the E2M1 lattice, returned directly as its 4-bit code (sign in
+// bit 3).  For a = |y| <= 6 with lo the largest lattice point <= a and p = (a - lo)/step, the value
+// rounds up iff r < ceil(p * 2^32); a > 6 (and Inf/NaN) gives 6.  The lattice is consecutive in
+// code order, so the result is code(lo) + up, capped at 7:
+//   a in [1, 8): the points of [2^e, 2^(e+1)) are 2^e * {1, 1.5}, so code(lo) = 2 + 2e + (top
+//     mantissa bit) = (bits >> 22) - 252, and p * 2^32 is the remaining 22-bit mantissa field
+//     shifted left by 10 (an exact integer);
+//   a < 1: points 0, 0.5, 1 (codes 0, 1, 2); T = a * 2^33 is exact, code(lo) = [T >= 2^32] and
+//     p * 2^32 = T - [T >= 2^32] * 2^32 (exact), whose ceiling is the threshold.
+__device__ __forceinline__ uint32_t sr_code(float y, uint32_t r) {
   const uint32_t bits = __float_as_uint(y);
   const uint32_t ab = bits & 0x7FFFFFFFu;
-  uint32_t res;
-  if (ab >= 0x3F800000u) {
-    const uint32_t lo = ab & 0xFFC00000u;
-    const uint32_t t = (ab & 0x003FFFFFu) << 10;
-    res = (ab > 0x40C00000u) ? 0x40C00000u : (lo + ((r < t) ? 0x00400000u : 0u));
-  } else {
-    const float q = __fmul_rn(__uint_as_float(ab), 2.0f);
-    const float fl = (q >= 1.0f) ? 1.0f : 0.0f;
-    const uint32_t th = f2u_ceil(__fmul_rn(__fsub_rn(q, fl), 4294967296.0f));
-    res = __float_as_uint(__fmul_rn(__fadd_rn(fl, (r < th) ? 1.0f : 0.0f), 0.5f));
+  const float T = __fmul_rn(__uint_as_float(ab), 8589934592.0f);  // 2^33
+  const bool half = T >= 4294967296.0f;                           // a >= 0.5
+  const uint32_t th_small = f2u_ceil(half ? __fsub_rn(T, 4294967296.0f) : T);
+  const bool ge1 = ab >= 0x3F800000u;
+  const uint32_t th = ge1 ? (ab & 0x003FFFFFu) << 10 : th_small;
+  const uint32_t lo = ge1 ? (ab >> 22) - 252u : (half ? 1u : 0u);
+  const uint32_t code = min(lo + (r < th ? 1u : 0u), 7u);
+  return code | ((bits >> 28) & 8u);
+}
+
+// N stochastically rounded codes packed 8 per word, value 0 in the lowest nibble.
+template <int N>
+__device__ __forceinline__ void sr_pack_n(const float* y, const uint32_t* rnd, uint32_t* w) {
+#pragma unroll
+  for (int k = 0; k < (N + 7) / 8; ++k) {
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      const int j = 8 * k + i;
+      acc = (acc << 4) | (j < N ? sr_code(y[j], rnd[j]) : 0u);
+    }
+    w[k] = acc;
   }
-  return __uint_as_float(res | (bits & 0x80000000u));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -381,10 +393,7 @@ __device__ __forceinline__ void encode_y_n(const float* v, float R, float top, c
     for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
   }
   if (SR) {
-    float t[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) t[i] = sr_round(y[i], rnd[i]);
-    e2m1_pack_n<N>(t, w);
+    sr_pack_n<N>(y, rnd, w);
   } else {
     e2m1_pack_n<N>(y, w);
   }
