@@ -134,12 +134,16 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   if (!global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = zero_counts(counts, s)) != FP4_OK) return st;
+  if (counts && !aligned(counts, 8)) return fail(FP4_EINVAL, "counts must be 8-byte aligned");
+  // with an amax pass (and a non-empty tensor) that pass zeroes the counters; otherwise a memset does
+  const bool amax_pass = !global_in && (long long)rows * cols > 0;
+  if (!amax_pass && (st = zero_counts(counts, s)) != FP4_OK) return st;
   uint32_t* amax = static_cast<uint32_t*>(workspace);
   cudaError_t e;
-  if (!global_in) {
+  if (amax_pass) {
     if ((e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s)) != cudaSuccess) return cuda_fail(e, "zeroing amax");
-    if ((e = fp4k::launch_amax(x, dtype == FP4_BF16, (long long)rows * cols, amax, s)) != cudaSuccess)
+    if ((e = fp4k::launch_amax(x, dtype == FP4_BF16, (long long)rows * cols, amax,
+                               reinterpret_cast<unsigned long long*>(counts), s)) != cudaSuccess)
       return cuda_fail(e, "nvfp4 amax launch");
   }
   fp4k::QuantLaunch L{};
@@ -167,7 +171,10 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   if (rotated_out && !aligned(rotated_out, 16)) return fail(FP4_EINVAL, "rotated_out must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = zero_counts(counts, s)) != FP4_OK) return st;
+  if (counts && !aligned(counts, 8)) return fail(FP4_EINVAL, "counts must be 8-byte aligned");
+  // with an amax pass (and a non-empty tensor) that pass zeroes the counters; otherwise a memset does
+  const bool amax_pass = nv && !global_in && rows > 0;
+  if (!amax_pass && (st = zero_counts(counts, s)) != FP4_OK) return st;
   fp4k::FwhtLaunch L{};
   L.x = x; L.bf16 = dtype == FP4_BF16; L.rows = rows; L.d = (int)d; L.nv = nv;
   L.sr = round == FP4_STOCHASTIC; L.four_six = nv && four_six; L.seed = seed;
@@ -178,7 +185,7 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_
   L.rotated_out = rotated_out;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e;
-  if (nv && !global_in) {
+  if (amax_pass) {
     if ((e = cudaMemsetAsync(L.amax_bits, 0, sizeof(uint32_t), s)) != cudaSuccess) return cuda_fail(e, "zeroing amax");
     if ((e = fp4k::launch_fwht_amax(L, s)) != cudaSuccess) return cuda_fail(e, "fwht amax launch");
   }

@@ -163,6 +163,8 @@ struct FwhtParams {
 template <typename T, int LOG_D>
 __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams p) {
   using G = Geom<LOG_D>;
+  // the counters the following quantise pass accumulates into start at zero (stream order)
+  if (p.counts && blockIdx.x == 0 && threadIdx.x < 4) p.counts[threadIdx.x] = 0ull;
   extern __shared__ __align__(16) float smem[];
   const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
   float* srow = smem + slot * G::D;

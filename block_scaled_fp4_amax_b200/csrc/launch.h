@@ -72,7 +72,9 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
-cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits, cudaStream_t s);
+// Tensor amax into *amax_bits (zeroed by the caller); also zeroes `counts` (4 words) if non-null.
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
+                        unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s);

@@ -238,7 +238,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
 // their L2 lines so the second pass, walking the tiles in reverse, starts on resident data.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long n_chunks,
-                                                        uint32_t* amax_bits) {
+                                                        uint32_t* amax_bits, unsigned long long* counts) {
+  // the counters the following quantise pass accumulates into start at zero (stream order)
+  if (counts && blockIdx.x == 0 && threadIdx.x < 4) counts[threadIdx.x] = 0ull;
   constexpr int E = Vec32<T>::E;
   const char* xb = reinterpret_cast<const char*>(x);
   const long long tid = (long long)blockIdx.x * kThreads + threadIdx.x;
@@ -381,12 +383,13 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
                 : dispatch_q<float>(p, L.nv, L.sr, L.four_six, s);
 }
 
-cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits, cudaStream_t s) {
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
+                        unsigned long long* counts, cudaStream_t s) {
   const long long chunks = n_elems / (bf16 ? 16 : 8);
   if (chunks == 0) return cudaSuccess;
   const int grid = grid_for(chunks / 4 + 1, kThreads);
-  if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits);
-  else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits);
+  if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
+  else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
   return cudaGetLastError();
 }
 
