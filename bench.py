@@ -116,13 +116,16 @@ class Clocks:
 
 
 def dist():
+    """One process per GPU (torchrun env); NCCL on GPUs, gloo where there is no GPU (host tests)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
         import datetime
         import torch.distributed as td
         local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        td.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return td, td.get_rank(), ws, local
     return None, 0, 1, 0
 
@@ -135,9 +138,15 @@ def barrier(td):
 def max_over_ranks(td, v):
     if td is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if td.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     td.all_reduce(t, op=td.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, bytes_per_rank_step, ms_step_max):
+    """Whole-job GB/s: the bytes all ranks processed in a step over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_step_max * 1e-3) / 1e9
 
 
 def timed(fn, K, W, flush, td, events_per_step=True):
@@ -219,7 +228,7 @@ def run_ours(args, td, rank, world, local):
     clk = clocks.stop(t0, t1)
     ms_step = max_over_ranks(td, sum(ms) / len(ms))
     bytes_step = 2 * NV_BYTES_2PASS * n
-    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    value = job_throughput(world, bytes_step, ms_step)
 
     # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g
     g = step.g[1].clone()
@@ -250,7 +259,7 @@ def run_ours(args, td, rank, world, local):
 
     ems = timed(e2e_step, max(3, args.steps // 10), args.warmup, flush, td)
     e_ms = max_over_ranks(td, sum(ems) / len(ems))
-    e2e = {"value": round(world * bytes_step / (e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    e2e = {"value": round(job_throughput(world, bytes_step, e_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": int(host_in.numel() * 2),
            "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_q + host_s + host_g)),
            "ms_per_step": round(e_ms, 4)}

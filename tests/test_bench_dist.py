@@ -1,0 +1,65 @@
+"""Host-side checks of bench.py's multi-process path (world size 2, gloo on CPU).
+
+Every rank runs its own replica of the workload; the bench times a step as the maximum over ranks
+and reports the bytes of all ranks over that time.  These tests run the same helpers in two gloo
+processes, and check that the reference arm does no work on ranks other than 0."""
+import multiprocessing as mp
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    td, r, w, _ = bench.dist()
+    try:
+        bench.barrier(td)
+        step_ms = 1.0 + 0.5 * rank                 # rank 1 is the slow one
+        m = bench.max_over_ranks(td, step_ms)
+        q.put((r, w, m, bench.job_throughput(w, 1e9, m)))
+    finally:
+        td.destroy_process_group()
+
+
+def test_two_gloo_ranks_time_the_step_as_the_slowest_rank():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o[0] for o in out] == [0, 1] and all(o[1] == world for o in out)
+    assert all(o[2] == pytest.approx(1.5) for o in out)          # max over ranks, seen by every rank
+    assert all(o[3] == pytest.approx(2 * 1e9 / 1.5e-3 / 1e9) for o in out)  # both ranks' bytes / slowest time
+
+
+def test_job_throughput_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.job_throughput(1, 4.5625 * 2 ** 26, 0.1) == pytest.approx(4.5625 * 2 ** 26 / 1e-4 / 1e9)
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
