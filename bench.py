@@ -375,7 +375,9 @@ def secondary(args, dev, flush, td, pk):
 def run_reference(args, rank):
     """The oracle (plain C, single thread) on a bounded sample of the headline workload."""
     import oracle as O
-    rows = 512
+    # about 2 s of single-threaded oracle work per 512 rows (plain + 4/6): size the per-step sample
+    # so that the whole run stays near two minutes whatever --steps is
+    rows = max(16, min(512, 30720 // max(1, args.steps)))
     x = synth.as_f32_numpy(synth.nv_outliers()[:rows])
     for _ in range(args.warmup):
         O.nvfp4_quantize(x[:64], four_six=False)
