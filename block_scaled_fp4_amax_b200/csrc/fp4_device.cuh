@@ -406,6 +406,28 @@ __device__ __forceinline__ void encode_n(const float* v, float R, float top, con
   encode_y_n<N, SR, CNT>(v, R, top, rnd, y, w, sat);
 }
 
+// Count of the 16 bf16 values (8 packed words) whose magnitude is at least the bf16 magnitude
+// pattern t (both halves of t2), by bf16x2 compares accumulated in bf16x2 (exact small integers).
+__device__ __forceinline__ uint32_t count_ge_bf16x16(const uint32_t* w, uint32_t t2) {
+  uint32_t acc;
+  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(acc) : "r"(w[0] & 0x7FFF7FFFu), "r"(t2));
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    uint32_t s;
+    asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(s) : "r"(w[i] & 0x7FFF7FFFu), "r"(t2));
+    asm("add.rn.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(s));
+  }
+  return (uint32_t)(__uint_as_float(acc << 16) + __uint_as_float(acc & 0xFFFF0000u));
+}
+
+// MXFP4 saturation count of 16 bf16 values under the shared exponent e (scale 2^e, normal 6 * 2^e):
+// scaling by 2^-e is exact, so |v| * 2^-e > 6 iff |v| > 6 * 2^e, i.e. |v| is at least the bf16
+// value one step above 6 * 2^e = 1.5 * 2^(e+2) (bf16 pattern ((e + 129) << 7) | 0x40).
+__device__ __forceinline__ uint32_t mx_sat_count_bf16x16(const uint32_t* w, int e) {
+  const uint32_t t = (((uint32_t)(e + 129)) << 7 | 0x40u) + 1u;
+  return count_ge_bf16x16(w, t | (t << 16));
+}
+
 // Saturation count of 16 bf16 values (8 packed words) under the scale pair (D, R = fl(1/D)):
 // the number of values with fl(|v| * R) > 6.  The predicate is monotone in |v|, so it holds
 // exactly for |v| >= t, t the smallest bf16 magnitude that satisfies it.  6D and the real
@@ -418,16 +440,7 @@ __device__ __forceinline__ uint32_t sat_count_bf16x16(const uint32_t* w, float D
   const uint32_t tb = (__fmul_rn(__uint_as_float(xb), R) > 6.0f)             ? xb
                       : (__fmul_rn(__uint_as_float(xb + 0x10000u), R) > 6.0f) ? xb + 0x10000u
                                                                               : xb + 0x20000u;
-  const uint32_t t2 = (tb >> 16) | (tb & 0xFFFF0000u);
-  uint32_t acc;
-  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(acc) : "r"(w[0] & 0x7FFF7FFFu), "r"(t2));
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    uint32_t s;
-    asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(s) : "r"(w[i] & 0x7FFF7FFFu), "r"(t2));
-    asm("add.rn.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(s));
-  }
-  return (uint32_t)(__uint_as_float(acc << 16) + __uint_as_float(acc & 0xFFFF0000u));
+  return count_ge_bf16x16(w, (tb >> 16) | (tb & 0xFFFF0000u));
 }
 
 // NVFP4 per-code scale table: for every E4M3 code byte c, D = fl(value(c) * s_g) and
@@ -619,11 +632,46 @@ __device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, floa
 // ---------------------------------------------------------------------------------------------
 // Scale-byte placement.  Row-major: the flat block index.  MMA tile layout: 128 x 4 tiles of
 // 512 bytes, block-column groups fastest (the layout tcgen05.cp 32x128b.warpx4 expects).
+__device__ __forceinline__ uint64_t scale_offset_rj(uint64_t r, uint32_t j, uint32_t nb) {
+  return ((r >> 7) * (nb >> 2) + (j >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (j & 3u);
+}
+// For a blocks-per-row count known at compile time (the compiler divides by a constant).
 __device__ __forceinline__ uint64_t scale_offset(uint64_t blk, uint32_t nb, bool tiled) {
   if (!tiled) return blk;
-  const uint32_t r = (uint32_t)(blk / nb), j = (uint32_t)(blk - (uint64_t)r * nb);
-  return ((uint64_t)(r >> 7) * (nb >> 2) + (j >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u +
-         (j & 3u);
+  const uint64_t r = blk / nb;
+  return scale_offset_rj(r, (uint32_t)(blk - r * nb), nb);
+}
+
+// Unsigned 32-bit division by an invariant divisor through a precomputed multiplier (Granlund and
+// Montgomery, "Division by Invariant Integers using Multiplication", PLDI 1994, section 4): with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1, every n < 2^32 has
+// n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0), t the high word of m * n.
+struct DivU32 {
+  uint32_t d, m, s1, s2;
+};
+inline DivU32 make_divu32(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (1ull << l) < d) ++l;
+  DivU32 v;
+  v.d = d;
+  v.m = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+  v.s1 = l < 1 ? l : 1;
+  v.s2 = l > 1 ? l - 1 : 0;
+  return v;
+}
+__device__ __forceinline__ uint32_t div_u32(uint32_t n, const DivU32& v) {
+  const uint32_t t = __umulhi(v.m, n);
+  return (t + ((n - t) >> v.s1)) >> v.s2;
+}
+// For a run-time blocks-per-row count: the 32-bit path by multiplier, 64-bit division beyond it.
+__device__ __forceinline__ uint64_t scale_offset(uint64_t blk, const DivU32& nb, bool tiled) {
+  if (!tiled) return blk;
+  if (blk < (1ull << 32)) {
+    const uint32_t r = div_u32((uint32_t)blk, nb);
+    return scale_offset_rj(r, (uint32_t)blk - r * nb.d, nb.d);
+  }
+  const uint64_t r = blk / nb.d;
+  return scale_offset_rj(r, (uint32_t)(blk - r * nb.d), nb.d);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -58,7 +58,7 @@ __device__ __forceinline__ NvScale nv_scales(const float* global_in, const uint3
 struct QuantParams {
   const void* x;
   long long n_chunks;  // rows * cols / E
-  uint32_t nb;         // blocks per row
+  DivU32 nb;           // blocks per row (with its division multiplier)
   int policy;          // MXFP4 exponent rule
   int tiled;           // scale layout
   int reverse;         // walk the tiles last-to-first (re-use the tail a previous pass left in L2)
@@ -166,10 +166,17 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
         const float top = __fmul_rn(amax, inv);
         encode_n<E, SR, !kBF>(v, inv, top, rnd, w, sat);
-        if constexpr (kBF) {  // D = 2^e exactly (2^-127 is the subnormal 0x00400000)
-          const float D = __uint_as_float(e > -127 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
-          const uint32_t n = sat_count_bf16x16(raw[u].w, D, inv);
-          sat = top > 6.0f ? n : 0u;
+        if constexpr (kBF) {
+          // 6 * 2^e is a normal bf16 for e in [-127, 126]; a non-finite block (e = 126 or 127 from
+          // an Inf/NaN maximum) keeps the general count, as does e = 127
+          if (e <= 125 && am < 0x7F800000u) {
+            const uint32_t n = mx_sat_count_bf16x16(raw[u].w, e);
+            sat = top > 6.0f ? n : 0u;
+          } else {
+            const float D = __uint_as_float(e > -127 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
+            const uint32_t n = sat_count_bf16x16(raw[u].w, D, inv);
+            sat = top > 6.0f ? n : 0u;
+          }
         }
         sc = (uint32_t)(e + 127);
       } else if (!FOUR_SIX) {
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long
 template <bool NV, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, const uint8_t* scales,
                                                            const float* global, long long n_groups,
-                                                           uint32_t nb, int tiled, void* out) {
+                                                           DivU32 nb, int tiled, void* out) {
   constexpr int B = NV ? 16 : 32;
   const float s_g = NV ? *global : 1.0f;
   const long long stride = (long long)gridDim.x * kThreads;
@@ -365,7 +372,7 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   const int E = L.bf16 ? 16 : 8;
   p.x = L.x;
   p.n_chunks = (long long)(L.rows * L.cols / E);
-  p.nb = (uint32_t)(L.cols / (L.nv ? 16 : 32));
+  p.nb = make_divu32((uint32_t)(L.cols / (L.nv ? 16 : 32)));
   p.policy = L.policy;
   p.tiled = L.tiled;
   p.reverse = L.reverse;
@@ -396,7 +403,7 @@ cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* a
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s) {
   const long long groups = L.rows * L.cols / 16;
   if (groups == 0) return cudaSuccess;
-  const uint32_t nb = (uint32_t)(L.cols / (L.nv ? 16 : 32));
+  const DivU32 nb = make_divu32((uint32_t)(L.cols / (L.nv ? 16 : 32)));
   const int grid = grid_for(groups, kThreads);
   if (L.nv) {
     if (L.out_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(L.q, L.scales, L.global, groups, nb, L.tiled, L.out);
