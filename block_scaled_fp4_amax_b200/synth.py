@@ -13,6 +13,7 @@ Workloads (shapes are parameters so the same recipe serves small parity cases):
   weight        bf16 N(0, 0.02)                              seed 4      (8192 x 28672)
   lattice_steps k / 8 for integers k uniform in [-48, 48]       (parity cases: exact ties between
                                                                  the two four-over-six candidates)
+  rht_signs     d fair sign bits, packed in uint32 words         (randomised rotation)
 """
 from __future__ import annotations
 
@@ -89,6 +90,13 @@ def lattice_steps(rows: int, cols: int, seed: int, denom: int = 8, kmax: int = 4
     rng = np.random.default_rng(seed)
     k = rng.integers(-kmax, kmax + 1, size=(rows, cols))
     return _to_bf16((k / denom).astype(np.float32))
+
+
+def rht_signs(d: int, seed: int) -> np.ndarray:
+    """Sign vector of the randomised rotation: d independent fair bits, packed 32 per uint32 word
+    (bit i % 32 of word i // 32 set = channel i negated)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 2 ** 32, size=d // 32, dtype=np.uint64).astype(np.uint32)
 
 
 def as_f32_numpy(t: torch.Tensor) -> np.ndarray:

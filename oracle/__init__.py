@@ -94,6 +94,8 @@ def lib():
         L.ora_fwht_norm_const.argtypes = [ctypes.c_long]
         L.ora_fwht_rows.restype = None
         L.ora_fwht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
+        L.ora_rht_rows.restype = None
+        L.ora_rht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P, P]
         _lib = L
     return _lib
 
@@ -218,19 +220,25 @@ def dequantize_f64(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
     return out
 
 
-def fwht(x) -> np.ndarray:
-    """Normalised Walsh-Hadamard rotation of every row (fixed butterfly order, fp32)."""
+def fwht(x, signs=None) -> np.ndarray:
+    """Normalised Walsh-Hadamard rotation of every row (fixed butterfly order, fp32).  With `signs`
+    (uint32 [d/32], bit i negates channel i first) it is the randomised rotation c * H * D."""
     x = _f32(x)
     rows, d = x.shape
     y = np.zeros_like(x)
-    lib().ora_fwht_rows(_p(x), rows, d, _p(y))
+    if signs is None:
+        lib().ora_fwht_rows(_p(x), rows, d, _p(y))
+    else:
+        sg = np.ascontiguousarray(signs, dtype=np.uint32)
+        assert sg.size == d // 32
+        lib().ora_rht_rows(_p(x), rows, d, sg.ctypes.data_as(ctypes.c_void_p), _p(y))
     return y
 
 
 def fwht_quantize(x, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
-                  global_in=None):
-    """Rotation followed by the quantiser of `fmt` on the rotated fp32 tensor."""
-    y = fwht(x)
+                  global_in=None, signs=None):
+    """Rotation (randomised with `signs`) followed by the quantiser of `fmt` on the rotated fp32 tensor."""
+    y = fwht(x, signs)
     if fmt == NVFP4:
         q, s, sg, c = nvfp4_quantize(y, round=round, four_six=four_six, seed=seed, global_in=global_in)
         return y, q, s, sg, c

@@ -389,11 +389,19 @@ void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, lon
 
 float ora_fwht_norm_const(long d) { return (float)(1.0L / sqrtl((long double)d)); }
 
-void ora_fwht_rows(const float* x, long rows, long d, float* y) {
+/* Randomised rotation ([P], the random Hadamard transform segment: a Hadamard transform with random
+ * signs).  Reading: Q = c * H * D, D = diag(s) with s_i = -1 where bit i of the caller's sign vector
+ * is set (bit i % 32 of word i / 32) and +1 otherwise; the signs multiply the input before the
+ * butterflies (negation is exact), so with no bits set this is the plain rotation.  Q is
+ * orthogonal (H * H = d * I), and its inverse is c * D * H.                                     */
+void ora_rht_rows(const float* x, long rows, long d, const uint32_t* signs, float* y) {
   float c = ora_fwht_norm_const(d);
   for (long r = 0; r < rows; ++r) {
     float* v = y + r * d;
-    memcpy(v, x + r * d, (size_t)d * sizeof(float));
+    for (long i = 0; i < d; ++i) {
+      const int neg = signs ? (int)((signs[i / 32] >> (i % 32)) & 1u) : 0;
+      v[i] = neg ? -x[r * d + i] : x[r * d + i];
+    }
     for (long h = 1; h < d; h *= 2) {
       for (long i = 0; i < d; ++i) {
         if (i & h) continue;
@@ -405,3 +413,5 @@ void ora_fwht_rows(const float* x, long rows, long d, float* y) {
     for (long i = 0; i < d; ++i) v[i] = v[i] * c;
   }
 }
+
+void ora_fwht_rows(const float* x, long rows, long d, float* y) { ora_rht_rows(x, rows, d, 0, y); }

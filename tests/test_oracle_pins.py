@@ -361,6 +361,50 @@ def test_fwht_parseval():
     assert np.max(np.abs(n1 / n0 - 1)) < 1e-6
 
 
+def _sign_vector(bits_words, d):
+    """+-1 per channel from the packed sign bits (bit i % 32 of word i // 32 set -> -1)."""
+    w = np.asarray(bits_words, dtype=np.uint32)
+    b = (w[np.arange(d) // 32] >> (np.arange(d) % 32).astype(np.uint32)) & 1
+    return np.where(b == 1, -1.0, 1.0)
+
+
+def test_rht_without_signs_is_the_plain_rotation():
+    x = O._f32(np.random.default_rng(12).standard_normal((3, 2048)))
+    assert np.array_equal(O.fwht(x, np.zeros(64, dtype=np.uint32)), O.fwht(x))
+
+
+def test_rht_inverse_is_exact_on_small_integers():
+    """Q = c H D with Q^-1 = c D H: rotating with the signs, then rotating back without them and
+    negating the signed channels, returns small-integer inputs exactly (d = 4^k makes c a power of
+    two).  A rotation that applied the signs after the butterflies would not invert this way."""
+    from block_scaled_fp4_amax_b200 import synth
+    rng = np.random.default_rng(13)
+    for d in (1024, 4096):
+        sg = synth.rht_signs(d, 21)
+        s = _sign_vector(sg, d)
+        x = rng.integers(-8, 9, size=(2, d)).astype(np.float32)
+        y = O.fwht(x, sg)
+        back = (s * O.fwht(y).astype(np.float64)).astype(np.float32)
+        assert np.array_equal(back, x)
+        assert not np.array_equal(y, O.fwht(x))      # the signs change the rotation
+
+
+def test_rht_matches_explicit_matrix():
+    """c H D x in fp64 from scipy's Hadamard matrix and the decoded signs, within the butterflies'
+    fp32 rounding."""
+    from scipy.linalg import hadamard
+    from block_scaled_fp4_amax_b200 import synth
+    d = 1024
+    sg = synth.rht_signs(d, 22)
+    s = _sign_vector(sg, d)
+    x = O._f32(np.random.default_rng(14).standard_normal((3, d)))
+    Q = hadamard(d).astype(np.float64) * s[None, :] / math.sqrt(d)
+    ref = x.astype(np.float64) @ Q.T
+    got = O.fwht(x, sg).astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < math.log2(d) * 2.0 ** -23
+    assert np.allclose(Q @ Q.T, np.eye(d), atol=1e-12)   # orthogonal
+
+
 # ---------------------------------------------------------------------------------------------
 # Dequantisation and the GEMM reference
 
