@@ -325,6 +325,17 @@ def secondary(args, dev, flush, td, pk):
     out.append({"workload": "FWHT d=8192 + NVFP4 + stochastic rounding, 16384x8192 bf16, two passes",
                 "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
                 "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    # the same with the randomised rotation c*H*D (seeded sign bits, one 32-bit word per 32 channels)
+    sg = torch.from_numpy(synth.rht_signs(8192, 33).view(np.int32)).to(dev)
+
+    def c3r():
+        fp4.fwht_quantize(x3, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7, workspace=ws, signs=sg)
+
+    ms = timed(c3r, K, W, flush, td)
+    t = statistics.median(ms)
+    out.append({"workload": "randomised FWHT (c*H*D) d=8192 + NVFP4 + stochastic rounding, 16384x8192 bf16",
+                "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
+                "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     del x3
     fp4_peak = 4.0 * pk["bf16_tflops"]  # dense FP4 / BF16 nominal ratio 9 / 2.25 on the measured bf16 peak
     # config 4: NVFP4 GEMM 8192^3

@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
     P, I, LG, ULL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_ulonglong, ctypes.c_size_t
     L.mx_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P]
     L.nvfp4_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P, SZ, P]
-    L.fwht_quantize.argtypes = [P, I, LG, LG, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
+    L.fwht_quantize.argtypes = [P, I, LG, LG, P, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
     L.fp4_dequantize.argtypes = [P, P, I, I, I, P, LG, LG, I, P, P]
     L.fp4_block_gemm.argtypes = [I, I, I, I, P, P, P, P, P, P, P, LG, P, SZ, P]
     L.nvfp4_quantize_noalloc.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P]
@@ -162,17 +162,21 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = F
 
 def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
                   layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, want_rotated: bool = False,
-                  block: int | None = None, stream=None, workspace: torch.Tensor | None = None):
-    """Walsh-Hadamard rotation of each row fused with the quantiser of `fmt`.
+                  block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
+                  signs: torch.Tensor | None = None):
+    """Walsh-Hadamard rotation of each row fused with the quantiser of `fmt`; with `signs` (device
+    int32/uint32 [d/32], bit i negates channel i first) the randomised rotation c*H*D.
     Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
-    _need_cuda(x, global_in)
+    _need_cuda(x, global_in, signs)
     rows, d = x.shape
     B = block if block is not None else (16 if fmt == NVFP4 else 32)
     q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, x.device)
     g = torch.empty(1, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
     rot = torch.empty((rows, d), dtype=torch.float32, device=x.device) if want_rotated else None
     ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, x.device, rows, d)
-    _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, fmt, B, round, int(bool(four_six)), seed,
+    if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
+        raise ValueError("signs must hold d/32 32-bit words")
+    _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, _ptr(signs), fmt, B, round, int(bool(four_six)), seed,
                                layout, _ptr(global_in), _ptr(g), _ptr(rot), _ptr(q), _ptr(s), _ptr(c),
                                _ptr(ws), ws.numel(), _stream(stream)))
     return q, s, g, c, rot

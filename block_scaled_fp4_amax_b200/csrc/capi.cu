@@ -156,7 +156,8 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "nvfp4_quantize launch");
 }
 
-fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_format format,
+fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, const unsigned int* signs,
+                         fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,
                          fp4_scale_layout layout, const float* global_in, float* global_out,
                          float* rotated_out, unsigned char* q, unsigned char* scales,
@@ -170,6 +171,7 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_
   if (nv && !global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   if (rotated_out && !aligned(rotated_out, 16)) return fail(FP4_EINVAL, "rotated_out must be 16-byte aligned");
+  if (signs && !aligned(signs, 4)) return fail(FP4_EINVAL, "signs must be 4-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (counts && !aligned(counts, 8)) return fail(FP4_EINVAL, "counts must be 8-byte aligned");
   // with an amax pass (and a non-empty tensor) that pass zeroes the counters; otherwise a memset does
@@ -183,6 +185,7 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_
   L.amax_bits = static_cast<uint32_t*>(workspace);
   L.global_out = nv ? global_out : nullptr;
   L.rotated_out = rotated_out;
+  L.signs = signs;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e;
   if (amax_pass) {

@@ -79,14 +79,19 @@ struct RowLoad {
 };
 
 // Round A + B + last-round rotation of one row into v[32] (last-round order: j = low | h << L).
-// `raw` holds this thread's round-A chunks.  Leaves the values unnormalised.
+// `raw` holds this thread's round-A chunks, elements [32 t, 32 t + 32); bit j of `sgn` negates
+// element 32 t + j first (randomised rotation; 0 = plain).  Leaves the values unnormalised.
 template <typename T, int LOG_D>
 __device__ __forceinline__ void rotate_row(const U8 (&raw)[RowLoad<T>::NV], float* srow, int t,
-                                           float (&v)[32]) {
+                                           uint32_t sgn, float (&v)[32]) {
   using G = Geom<LOG_D>;
   // round A: index bits 0-4 local
 #pragma unroll
   for (int c = 0; c < RowLoad<T>::NV; ++c) Vec32<T>::unpack(raw[c], v + c * Vec32<T>::E);
+  if (sgn) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(__float_as_uint(v[j]) ^ ((sgn << (31 - j)) & 0x80000000u));
+  }
   stages<0, 5>(v);
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -154,6 +159,7 @@ struct FwhtParams {
   float* global_out;
   float six_m;
   float* rotated_out;
+  const uint32_t* signs;
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;
@@ -169,6 +175,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
   float* srow = smem + slot * G::D;
   const T* x = reinterpret_cast<const T*>(p.x);
+  const uint32_t sgn = p.signs ? p.signs[t] : 0u;
   const long long step = (long long)gridDim.x * G::ROWS;
   float m = 0.0f;
   U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
     load_row<T, LOG_D>(x, row + step, p.rows, t, nxt);
     float v[32];
-    rotate_row<T, LOG_D>(raw, srow, t, v);
+    rotate_row<T, LOG_D>(raw, srow, t, sgn, v);
     if (row < p.rows) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
@@ -243,6 +250,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
   const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
   float* srow = smem + slot * D;
   const T* x = reinterpret_cast<const T*>(p.x);
+  const uint32_t sgn = p.signs ? p.signs[t] : 0u;
   const long long step = (long long)gridDim.x * G::ROWS;
   const uint32_t nb = D / B;
 
@@ -269,7 +277,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
     const long long rn = row + step;
     load_row<T, LOG_D>(x, rn < p.rows ? phys(rn) : rn, p.rows, t, nxt);
     float v[32];
-    rotate_row<T, LOG_D>(raw, srow, t, v);
+    rotate_row<T, LOG_D>(raw, srow, t, sgn, v);
     to_consecutive<LOG_D>(srow, t, v);
     const bool valid = row < p.rows;  // uniform over the row's warps
     const long long prow = valid ? phys(row) : 0;
@@ -385,7 +393,7 @@ static FwhtParams make_params(const FwhtLaunch& L) {
   p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed); p.zero = 0u;
   p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
   p.six_m = L.four_six ? 1536.0f : 2688.0f;
-  p.rotated_out = L.rotated_out; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
+  p.rotated_out = L.rotated_out; p.signs = L.signs; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
   return p;
 }
 

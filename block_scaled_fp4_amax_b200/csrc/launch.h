@@ -56,6 +56,7 @@ struct FwhtLaunch {
   uint32_t* amax_bits;   // workspace word (pass 1 output / pass 2 input)
   float* global_out;
   float* rotated_out;
+  const uint32_t* signs;  // randomised rotation: bit i negates channel i (nullptr: plain rotation)
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;

@@ -145,10 +145,16 @@ FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, lon
  * (format FP4_NVFP4, block 16; the global amax is taken over the rotated tensor) or as
  * mx_quantize with FP4_MX_OCP_FLOOR (format FP4_MXFP4, block 32).  Stochastic rounding indexes
  * Philox by the flat element index of the rotated [rows, d] tensor.
+ * With `signs` the rotation is randomised ([P], random Hadamard transform): Q = c * H * D, where
+ * D = diag(+-1) negates channel i (before the butterflies) when bit i % 32 of signs[i / 32] is set.
+ * Q is orthogonal, so rotating both GEMM operands along K with the same signs leaves A * B^T
+ * unchanged up to quantisation.
  *   d           : power of two, 1024 <= d <= 16384.
+ *   signs       : device uint32 [d / 32], 4-byte aligned, or NULL (plain rotation); caller-owned.
  *   rotated_out : device float [rows, d] or NULL; receives the rotated values (diagnostics).
  *   other arguments as in nvfp4_quantize; four_six and global_in/out apply to FP4_NVFP4 only. */
-FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, fp4_format format,
+FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d,
+                         const unsigned int* signs, fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,
                          fp4_scale_layout layout, const float* global_in, float* global_out,
                          float* rotated_out, unsigned char* q, unsigned char* scales,

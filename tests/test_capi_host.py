@@ -85,12 +85,12 @@ def test_nvfp4_rejects(L):
 
 def test_fwht_rejects(L):
     # d not a power of two / out of range, MXFP4 with four-over-six, block mismatch
-    assert L.fwht_quantize(FAKE, 1, 4, 3000, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
-    assert L.fwht_quantize(FAKE, 1, 4, 512, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
-    assert L.fwht_quantize(FAKE, 1, 4, 32768, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
-    assert L.fwht_quantize(FAKE, 1, 4, 8192, 0, 32, 0, 1, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 2
-    assert L.fwht_quantize(FAKE, 1, 4, 8192, 0, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
-    assert L.fwht_quantize(FAKE, 1, 4, 8192, 5, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 3000, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 512, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 32768, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 0, 32, 0, 1, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 2
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 0, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 5, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
 
 
 def test_dequant_rejects(L):

@@ -278,6 +278,73 @@ def test_fwht_config3_full(cuda):
     assert float(np.abs(y).max()) < 120.0 / 4
 
 
+# Randomised rotation (signs D before the butterflies: Q = c H D)
+
+def _signs_dev(d, seed, cuda):
+    return torch.from_numpy(synth.rht_signs(d, seed).view(np.int32)).to(cuda)
+
+
+@pytest.mark.parametrize("d", [1024, 8192, 16384])
+@pytest.mark.parametrize("fmt,rnd,four_six", [(fp4.NVFP4, fp4.RNE, False), (fp4.NVFP4, fp4.STOCHASTIC, False),
+                                              (fp4.NVFP4, fp4.RNE, True), (fp4.MXFP4, fp4.STOCHASTIC, False)])
+def test_rht_small(cuda, d, fmt, rnd, four_six):
+    rows = 37
+    x = synth.fwht_laplace(rows, d, seed=6)
+    sg = synth.rht_signs(d, 31)
+    q, s, g, c, rot = fp4.fwht_quantize(x.to(cuda), fmt=fmt, round=rnd, four_six=four_six, seed=7, want_rotated=True,
+                                        signs=_signs_dev(d, 31, cuda))
+    y, qo, so, go, co = O.fwht_quantize(f32(x), fmt=fmt, round=rnd, four_six=four_six, seed=7, signs=sg)
+    assert np.array_equal(npy(rot), y)
+    if fmt == fp4.NVFP4:
+        assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+
+
+def test_rht_config3_full(cuda):
+    """The full fused-rotation workload (16384 x 8192 bf16, NVFP4, stochastic rounding, seed 7)
+    with a randomised rotation: bit-exact against the oracle."""
+    x = synth.fwht_laplace()
+    sg = synth.rht_signs(8192, 32)
+    q, s, g, c, _ = fp4.fwht_quantize(x.to(cuda), fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7,
+                                      signs=_signs_dev(8192, 32, cuda))
+    y, qo, so, go, co = O.fwht_quantize(f32(x), fmt=O.NVFP4, round=O.STOCHASTIC, seed=7, signs=sg)
+    assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+
+
+def test_rht_gemm_end_to_end(cuda):
+    """(X Q^T)(W Q^T)^T = X W^T for the orthogonal Q = c H D.
+    - The GPU's rotated fp32 operands reproduce X W^T in fp64 to fp32 rounding (orthogonality end
+      to end through the kernel).
+    - Rotating both operands along K with the same signs, quantising to MXFP4 and multiplying on the
+      tensor cores approximates X W^T.  With outlier channels in X, the power-of-two 32-value scales
+      lose less to the rotated operands than to the raw ones (NVFP4's 16-value E4M3 scales already
+      isolate an outlier channel, so the rotation is not expected to help there)."""
+    M, N, K = 256, 256, 4096
+    X = synth.nv_outliers(M, K, seed=41).float()
+    W = synth.normal_bf16(N, K, 42).float()
+    ref = X.double() @ W.double().T
+    sd = _signs_dev(K, 43, cuda)
+    err = lambda C: float(torch.linalg.norm(C - ref) / torch.linalg.norm(ref))
+
+    qa, sa, _, _, ya = fp4.fwht_quantize(X.to(cuda), fmt=fp4.MXFP4, layout=fp4.MMA_TILED, signs=sd, want_rotated=True)
+    qb, sb, _, _, yb = fp4.fwht_quantize(W.to(cuda), fmt=fp4.MXFP4, layout=fp4.MMA_TILED, signs=sd, want_rotated=True)
+    assert err(ya.double().cpu() @ yb.double().cpu().T) < 1e-5
+    C_rht, ws = fp4.fp4_block_gemm(fp4.MXFP4, qa, sa, qb, sb)
+    assert int(ws[:4].view(torch.int32).item()) == 0
+
+    pa, ra, _ = fp4.mx_quantize(X.to(cuda), layout=fp4.MMA_TILED)
+    pb, rb, _ = fp4.mx_quantize(W.to(cuda), layout=fp4.MMA_TILED)
+    C_plain, _ = fp4.fp4_block_gemm(fp4.MXFP4, pa, ra, pb, rb)
+    e_rht, e_plain = err(C_rht.double().cpu()), err(C_plain.double().cpu())
+    assert e_rht < 0.25 and e_plain < 0.25   # two FP4 operands: ~0.15-0.2 normwise
+    assert e_rht < e_plain
+
+
 # ---------------------------------------------------------------------------------------------
 # The GEMM workloads' quantisation (MXFP4 activations and weights at the down_proj shape)
 
