@@ -337,6 +337,20 @@ def secondary(args, dev, flush, td, pk):
                 "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
                 "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     del x3
+    # SwiGLU fused ahead of the rotation: g, u bf16 [16384, 8192] read in both passes
+    gg, uu = (t_.to(dev) for t_ in synth.swiglu_inputs(16384, 8192, seed=3))
+
+    def c3s():
+        fp4.swiglu_fwht_quantize(gg, uu, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7, workspace=ws)
+
+    ms = timed(c3s, K, W, flush, td)
+    t = statistics.median(ms)
+    bs = (2 * 2 * 2 + 0.5 + 1 / 16) * gg.numel()
+    out.append({"workload": "SiLU(g)*u -> FWHT d=8192 -> NVFP4 + stochastic rounding, 16384x8192 bf16 g and u",
+                "ms": round(t, 4), "GB/s": round(bs / (t * 1e-3) / 1e9, 1),
+                "frac_hbm": round(bs / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    del gg, uu
+    
     fp4_peak = 4.0 * pk["bf16_tflops"]  # dense FP4 / BF16 nominal ratio 9 / 2.25 on the measured bf16 peak
     # config 4: NVFP4 GEMM 8192^3
     A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)

@@ -29,7 +29,7 @@ OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEM
 STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 
 # Every symbol include/fp4mx.h declares.
-EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
+EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
            "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error",
            "nvfp4_quantize_noalloc")
 
@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
     L.mx_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P]
     L.nvfp4_quantize.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P, SZ, P]
     L.fwht_quantize.argtypes = [P, I, LG, LG, P, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
+    L.swiglu_fwht_quantize.argtypes = [P, P, I, LG, LG, P, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
     L.fp4_dequantize.argtypes = [P, P, I, I, I, P, LG, LG, I, P, P]
     L.fp4_block_gemm.argtypes = [I, I, I, I, P, P, P, P, P, P, P, LG, P, SZ, P]
     L.nvfp4_quantize_noalloc.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P]
@@ -67,7 +68,8 @@ def lib() -> ctypes.CDLL:
     L.fp4_status_str.restype = ctypes.c_char_p
     L.fp4_last_error.argtypes = []
     L.fp4_last_error.restype = ctypes.c_char_p
-    for name in ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "fp4_dequantize", "fp4_block_gemm"):
+    for name in ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize",
+                 "fp4_block_gemm"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -180,6 +182,30 @@ def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six:
                                layout, _ptr(global_in), _ptr(g), _ptr(rot), _ptr(q), _ptr(s), _ptr(c),
                                _ptr(ws), ws.numel(), _stream(stream)))
     return q, s, g, c, rot
+
+
+def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, round: int = RNE,
+                         four_six: bool = False, seed: int = 0, layout: int = ROWMAJOR,
+                         global_in: torch.Tensor | None = None, want_rotated: bool = False,
+                         block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
+                         signs: torch.Tensor | None = None):
+    """fl(SiLU(g) * u) in fp32 (never stored), rotated (randomised with `signs`) and quantised to `fmt`.
+    g, u: bf16 [rows, d].  Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
+    _need_cuda(g, u, global_in, signs)
+    if g.shape != u.shape:
+        raise ValueError("g and u must have the same shape")
+    rows, d = g.shape
+    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, g.device)
+    gs = torch.empty(1, dtype=torch.float32, device=g.device) if fmt == NVFP4 else None
+    rot = torch.empty((rows, d), dtype=torch.float32, device=g.device) if want_rotated else None
+    ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, g.device, rows, d)
+    if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
+        raise ValueError("signs must hold d/32 32-bit words")
+    _check(lib().swiglu_fwht_quantize(_ptr(g), _ptr(u), _dtype_code(g), rows, d, _ptr(signs), fmt, B, round,
+                                      int(bool(four_six)), seed, layout, _ptr(global_in), _ptr(gs), _ptr(rot),
+                                      _ptr(q), _ptr(s), _ptr(c), _ptr(ws), ws.numel(), _stream(stream)))
+    return q, s, gs, c, rot
 
 
 def fp4_dequantize(q: torch.Tensor, scales: torch.Tensor, fmt: int, global_scale: torch.Tensor | None = None,

@@ -156,8 +156,8 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "nvfp4_quantize launch");
 }
 
-fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, const unsigned int* signs,
-                         fp4_format format,
+static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dtype, long rows, long d,
+                                     const unsigned int* signs, fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,
                          fp4_scale_layout layout, const float* global_in, float* global_out,
                          float* rotated_out, unsigned char* q, unsigned char* scales,
@@ -186,6 +186,7 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, cons
   L.global_out = nv ? global_out : nullptr;
   L.rotated_out = rotated_out;
   L.signs = signs;
+  L.u = u;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e;
   if (amax_pass) {
@@ -194,6 +195,27 @@ fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, cons
   }
   e = fp4k::launch_fwht_quantize(L, s);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fwht_quantize launch");
+}
+
+fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d, const unsigned int* signs,
+                         fp4_format format, int block, fp4_round round, int four_six, unsigned long long seed,
+                         fp4_scale_layout layout, const float* global_in, float* global_out,
+                         float* rotated_out, unsigned char* q, unsigned char* scales,
+                         fp4_counts* counts, void* workspace, size_t ws_bytes, void* stream) {
+  return fwht_quantize_impl(x, nullptr, dtype, rows, d, signs, format, block, round, four_six, seed, layout,
+                            global_in, global_out, rotated_out, q, scales, counts, workspace, ws_bytes, stream);
+}
+
+fp4_status swiglu_fwht_quantize(const void* g, const void* u, fp4_dtype dtype, long rows, long d,
+                                const unsigned int* signs, fp4_format format, int block, fp4_round round, int four_six, unsigned long long seed,
+                                fp4_scale_layout layout, const float* global_in, float* global_out,
+                                float* rotated_out, unsigned char* q, unsigned char* scales,
+                                fp4_counts* counts, void* workspace, size_t ws_bytes, void* stream) {
+  if (dtype != FP4_BF16) return fail(FP4_EUNSUPPORTED, "swiglu_fwht_quantize takes bf16 g and u");
+  if (rows > 0 && !u) return fail(FP4_EINVAL, "NULL u");
+  if (u && !aligned(u, 32)) return fail(FP4_EINVAL, "u must be 32-byte aligned");
+  return fwht_quantize_impl(g, u, dtype, rows, d, signs, format, block, round, four_six, seed, layout, global_in,
+                            global_out, rotated_out, q, scales, counts, workspace, ws_bytes, stream);
 }
 
 fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, fp4_format format,

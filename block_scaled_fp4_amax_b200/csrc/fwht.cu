@@ -73,6 +73,36 @@ __device__ __forceinline__ void stages(float (&v)[32]) {  // local bits LO..HI_-
   }
 }
 
+// SwiGLU activation fl(SiLU(g) * u) with a written-out exponential, every step one explicitly rounded
+// fp32 operation: Cody and Waite's argument reduction ("Software Manual for the Elementary
+// Functions", 1980) x = n ln2 + r, n = rint(x log2 e), ln2 split into a 12-significant-bit head
+// (n * head exact) and a tail; the degree-6 Taylor polynomial of e^r in Horner form; an exact scaling
+// by 2^n.  SiLU(g) = g * fl(1 / fl(1 + e^-g)) with a correctly rounded reciprocal.
+__device__ __forceinline__ float pow2_exact(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+__device__ __forceinline__ float exp_cw(float x) {
+  if (x != x) return x;
+  if (x > 88.5f) return __int_as_float(0x7F800000);
+  if (x < -103.0f) return 0.0f;
+  const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));
+  float r = __fsub_rn(x, __fmul_rn(n, 0x1.62ep-1f));
+  r = __fsub_rn(r, __fmul_rn(n, 0x1.0bfbe8p-15f));
+  float q = 0x1.6c16c2p-10f;
+  q = __fadd_rn(__fmul_rn(q, r), 0x1.111112p-7f);
+  q = __fadd_rn(__fmul_rn(q, r), 0x1.555556p-5f);
+  q = __fadd_rn(__fmul_rn(q, r), 0x1.555556p-3f);
+  q = __fadd_rn(__fmul_rn(q, r), 0.5f);
+  q = __fadd_rn(__fmul_rn(q, r), 1.0f);
+  q = __fadd_rn(__fmul_rn(q, r), 1.0f);
+  const int k = (int)n;
+  if (k > 127) return __fmul_rn(__fmul_rn(q, pow2_exact(127)), pow2_exact(k - 127));
+  if (k >= -126) return __fmul_rn(q, pow2_exact(k));
+  return __fmul_rn(__fmul_rn(q, pow2_exact(k + 64)), pow2_exact(-64));
+}
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const float e = exp_cw(-g);
+  return __fmul_rn(__fmul_rn(g, __frcp_rn(__fadd_rn(1.0f, e))), u);
+}
+
 template <typename T>
 struct RowLoad {
   static constexpr int NV = 32 * (int)sizeof(T) / 32;  // 32-byte chunks per thread
@@ -81,13 +111,22 @@ struct RowLoad {
 // Round A + B + last-round rotation of one row into v[32] (last-round order: j = low | h << L).
 // `raw` holds this thread's round-A chunks, elements [32 t, 32 t + 32); bit j of `sgn` negates
 // element 32 t + j first (randomised rotation; 0 = plain).  Leaves the values unnormalised.
-template <typename T, int LOG_D>
-__device__ __forceinline__ void rotate_row(const U8 (&raw)[RowLoad<T>::NV], float* srow, int t,
+template <typename T, int LOG_D, bool GATED = false>
+__device__ __forceinline__ void rotate_row(const U8 (&raw)[RowLoad<T>::NV], const U8* rawu, float* srow, int t,
                                            uint32_t sgn, float (&v)[32]) {
   using G = Geom<LOG_D>;
   // round A: index bits 0-4 local
 #pragma unroll
   for (int c = 0; c < RowLoad<T>::NV; ++c) Vec32<T>::unpack(raw[c], v + c * Vec32<T>::E);
+  if constexpr (GATED) {  // raw holds g, rawu holds u: the rotated input is fl(SiLU(g) * u)
+#pragma unroll
+    for (int c = 0; c < RowLoad<T>::NV; ++c) {
+      float w[Vec32<T>::E];
+      Vec32<T>::unpack(rawu[c], w);
+#pragma unroll
+      for (int i = 0; i < Vec32<T>::E; ++i) v[c * Vec32<T>::E + i] = silu_mul(v[c * Vec32<T>::E + i], w[i]);
+    }
+  }
   if (sgn) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(__float_as_uint(v[j]) ^ ((sgn << (31 - j)) & 0x80000000u));
@@ -160,13 +199,14 @@ struct FwhtParams {
   float six_m;
   float* rotated_out;
   const uint32_t* signs;
+  const void* u;      // SwiGLU path: x holds g, u holds the up projection (same layout)
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;
 };
 
 // Pass 1 (NVFP4 without a caller scale): amax of the rotated tensor.
-template <typename T, int LOG_D>
+template <typename T, int LOG_D, bool GATED>
 __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams p) {
   using G = Geom<LOG_D>;
   // the counters the following quantise pass accumulates into start at zero (stream order)
@@ -178,19 +218,26 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   const uint32_t sgn = p.signs ? p.signs[t] : 0u;
   const long long step = (long long)gridDim.x * G::ROWS;
   float m = 0.0f;
-  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV], rawu[GATED ? RowLoad<T>::NV : 1];
   long long row = (long long)blockIdx.x * G::ROWS + slot;
-  load_row<T, LOG_D>(x, row, p.rows, t, raw);
+  if (!GATED) load_row<T, LOG_D>(x, row, p.rows, t, raw);
   for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
-    load_row<T, LOG_D>(x, row + step, p.rows, t, nxt);
+    if constexpr (GATED) {  // two inputs per row: loaded for the current row, no prefetch
+      load_row<T, LOG_D>(x, row, p.rows, t, raw);
+      load_row<T, LOG_D>(reinterpret_cast<const T*>(p.u), row, p.rows, t, rawu);
+    } else {
+      load_row<T, LOG_D>(x, row + step, p.rows, t, nxt);
+    }
     float v[32];
-    rotate_row<T, LOG_D>(raw, srow, t, sgn, v);
+    rotate_row<T, LOG_D, GATED>(raw, rawu, srow, t, sgn, v);
     if (row < p.rows) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
     }
+    if (!GATED) {
 #pragma unroll
-    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+      for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+    }
     row += step;
   }
   // |fl(c*u)| is monotone in |u|: scale the maximum once.
@@ -240,7 +287,7 @@ __device__ __forceinline__ void to_consecutive(float* srow, int t, float (&v)[32
 }
 
 // Pass 2: rotate again, normalise, quantise from registers (whole blocks per thread).
-template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX>
+template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX, bool GATED>
 __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 : 1) fwht_quant_kernel(FwhtParams p) {
   using G = Geom<LOG_D>;
   constexpr int D = G::D;
@@ -269,15 +316,21 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
   __shared__ float2 tab[NV ? kScaleTab : 1];
   if (NV) fill_scale_tab(tab, s_g);  // first read after the rotation's __syncthreads
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};
-  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV];
+  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV], rawu[GATED ? RowLoad<T>::NV : 1];
   auto phys = [&](long long r) { return p.reverse ? (p.rows - 1 - r) : r; };
   long long row = (long long)blockIdx.x * G::ROWS + slot;
-  load_row<T, LOG_D>(x, row < p.rows ? phys(row) : row, p.rows, t, raw);
+  if (!GATED) load_row<T, LOG_D>(x, row < p.rows ? phys(row) : row, p.rows, t, raw);
   for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
-    const long long rn = row + step;
-    load_row<T, LOG_D>(x, rn < p.rows ? phys(rn) : rn, p.rows, t, nxt);
+    if constexpr (GATED) {  // two inputs per row: loaded for the current row, no prefetch
+      const long long pr = row < p.rows ? phys(row) : row;
+      load_row<T, LOG_D>(x, pr, p.rows, t, raw);
+      load_row<T, LOG_D>(reinterpret_cast<const T*>(p.u), pr, p.rows, t, rawu);
+    } else {
+      const long long rn = row + step;
+      load_row<T, LOG_D>(x, rn < p.rows ? phys(rn) : rn, p.rows, t, nxt);
+    }
     float v[32];
-    rotate_row<T, LOG_D>(raw, srow, t, sgn, v);
+    rotate_row<T, LOG_D, GATED>(raw, rawu, srow, t, sgn, v);
     to_consecutive<LOG_D>(srow, t, v);
     const bool valid = row < p.rows;  // uniform over the row's warps
     const long long prow = valid ? phys(row) : 0;
@@ -366,20 +419,23 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
         cnt[3] += four;
       }
     }
+    if (!GATED) {
 #pragma unroll
-    for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+      for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+    }
     row += step;
   }
   if (p.counts) flush_counts<4>(cnt, p.counts);
 }
 
 // ---------------------------------------------------------------------------------------------
-template <typename T, int LOG_D>
-static int fwht_grid(long long rows) {
+// One wave of resident CTAs of `kernel` (each loops over rows).
+template <int LOG_D, typename K>
+static int fwht_grid(K kernel, long long rows) {
   using G = Geom<LOG_D>;
   const int smem = G::ROWS * G::D * 4;
   int per_sm = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwht_amax_kernel<T, LOG_D>, G::CTA, smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, G::CTA, smem);
   if (per_sm < 1) per_sm = 1;
   const long long want = (rows + G::ROWS - 1) / G::ROWS;
   const long long cap = (long long)num_sms() * per_sm;
@@ -393,71 +449,77 @@ static FwhtParams make_params(const FwhtLaunch& L) {
   p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed); p.zero = 0u;
   p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
   p.six_m = L.four_six ? 1536.0f : 2688.0f;
-  p.rotated_out = L.rotated_out; p.signs = L.signs; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
+  p.rotated_out = L.rotated_out; p.signs = L.signs; p.u = L.u; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
   return p;
 }
 
-template <typename T, int LOG_D>
+template <typename T, int LOG_D, bool GATED>
 static cudaError_t amax_d(const FwhtParams& p, cudaStream_t s) {
   using G = Geom<LOG_D>;
   const int smem = G::ROWS * G::D * 4;
-  cudaFuncSetAttribute(fwht_amax_kernel<T, LOG_D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  fwht_amax_kernel<T, LOG_D><<<fwht_grid<T, LOG_D>(p.rows), G::CTA, smem, s>>>(p);
+  auto k = fwht_amax_kernel<T, LOG_D, GATED>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  k<<<fwht_grid<LOG_D>(k, p.rows), G::CTA, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-template <typename T, int LOG_D, bool NV, bool SR, bool FS>
+template <typename T, int LOG_D, bool NV, bool SR, bool FS, bool GATED>
 static cudaError_t quant_d(const FwhtParams& p, cudaStream_t s) {
   using G = Geom<LOG_D>;
   const int smem = G::ROWS * G::D * 4;
-  auto k = fwht_quant_kernel<T, LOG_D, NV, SR, FS>;
+  auto k = fwht_quant_kernel<T, LOG_D, NV, SR, FS, GATED>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  k<<<fwht_grid<T, LOG_D>(p.rows), G::CTA, smem, s>>>(p);
+  k<<<fwht_grid<LOG_D>(k, p.rows), G::CTA, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-template <typename T, int LOG_D>
+template <typename T, int LOG_D, bool GATED>
 static cudaError_t quant_sel(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
-  if (!L.nv) return L.sr ? quant_d<T, LOG_D, false, true, false>(p, s) : quant_d<T, LOG_D, false, false, false>(p, s);
-  if (L.four_six) return L.sr ? quant_d<T, LOG_D, true, true, true>(p, s) : quant_d<T, LOG_D, true, false, true>(p, s);
-  return L.sr ? quant_d<T, LOG_D, true, true, false>(p, s) : quant_d<T, LOG_D, true, false, false>(p, s);
+  if (!L.nv)
+    return L.sr ? quant_d<T, LOG_D, false, true, false, GATED>(p, s) : quant_d<T, LOG_D, false, false, false, GATED>(p, s);
+  if (L.four_six)
+    return L.sr ? quant_d<T, LOG_D, true, true, true, GATED>(p, s) : quant_d<T, LOG_D, true, false, true, GATED>(p, s);
+  return L.sr ? quant_d<T, LOG_D, true, true, false, GATED>(p, s) : quant_d<T, LOG_D, true, false, false, GATED>(p, s);
 }
 
-template <typename T>
+template <typename T, bool GATED>
 static cudaError_t dispatch_amax(const FwhtParams& p, int d, cudaStream_t s) {
   switch (d) {
-    case 1024: return amax_d<T, 10>(p, s);
-    case 2048: return amax_d<T, 11>(p, s);
-    case 4096: return amax_d<T, 12>(p, s);
-    case 8192: return amax_d<T, 13>(p, s);
-    case 16384: return amax_d<T, 14>(p, s);
+    case 1024: return amax_d<T, 10, GATED>(p, s);
+    case 2048: return amax_d<T, 11, GATED>(p, s);
+    case 4096: return amax_d<T, 12, GATED>(p, s);
+    case 8192: return amax_d<T, 13, GATED>(p, s);
+    case 16384: return amax_d<T, 14, GATED>(p, s);
   }
   return cudaErrorInvalidValue;
 }
 
-template <typename T>
+template <typename T, bool GATED>
 static cudaError_t dispatch_quant(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
   switch (L.d) {
-    case 1024: return quant_sel<T, 10>(p, L, s);
-    case 2048: return quant_sel<T, 11>(p, L, s);
-    case 4096: return quant_sel<T, 12>(p, L, s);
-    case 8192: return quant_sel<T, 13>(p, L, s);
-    case 16384: return quant_sel<T, 14>(p, L, s);
+    case 1024: return quant_sel<T, 10, GATED>(p, L, s);
+    case 2048: return quant_sel<T, 11, GATED>(p, L, s);
+    case 4096: return quant_sel<T, 12, GATED>(p, L, s);
+    case 8192: return quant_sel<T, 13, GATED>(p, L, s);
+    case 16384: return quant_sel<T, 14, GATED>(p, L, s);
   }
   return cudaErrorInvalidValue;
 }
 
+// The SwiGLU (gated) path is built for bf16 inputs only.
 cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s) {
   if (L.rows == 0) return cudaSuccess;
   FwhtParams p = make_params(L);
-  return L.bf16 ? dispatch_amax<__nv_bfloat16>(p, L.d, s) : dispatch_amax<float>(p, L.d, s);
+  if (L.u) return L.bf16 ? dispatch_amax<__nv_bfloat16, true>(p, L.d, s) : cudaErrorInvalidValue;
+  return L.bf16 ? dispatch_amax<__nv_bfloat16, false>(p, L.d, s) : dispatch_amax<float, false>(p, L.d, s);
 }
 
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s) {
   if (L.rows == 0) return cudaSuccess;
   FwhtParams p = make_params(L);
   p.reverse = (L.nv && !L.global_in) ? 1 : 0;
-  return L.bf16 ? dispatch_quant<__nv_bfloat16>(p, L, s) : dispatch_quant<float>(p, L, s);
+  if (L.u) return L.bf16 ? dispatch_quant<__nv_bfloat16, true>(p, L, s) : cudaErrorInvalidValue;
+  return L.bf16 ? dispatch_quant<__nv_bfloat16, false>(p, L, s) : dispatch_quant<float, false>(p, L, s);
 }
 
 }  // namespace fp4k

@@ -57,6 +57,7 @@ struct FwhtLaunch {
   float* global_out;
   float* rotated_out;
   const uint32_t* signs;  // randomised rotation: bit i negates channel i (nullptr: plain rotation)
+  const void* u;          // SwiGLU path (bf16): x is g, u the up projection; nullptr otherwise
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;

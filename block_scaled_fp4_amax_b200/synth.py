@@ -14,6 +14,7 @@ Workloads (shapes are parameters so the same recipe serves small parity cases):
   lattice_steps k / 8 for integers k uniform in [-48, 48]       (parity cases: exact ties between
                                                                  the two four-over-six candidates)
   rht_signs     d fair sign bits, packed in uint32 words         (randomised rotation)
+  swiglu_inputs bf16 g, u ~ N(0,1), streams (3,0) and (3,1)       (fused SwiGLU -> rotation path)
 """
 from __future__ import annotations
 
@@ -77,6 +78,14 @@ def swiglu_act(rows: int = 4096, cols: int = 28672, seed: int = 3) -> torch.Tens
     u = np.random.default_rng([seed, 1]).standard_normal((rows, cols), dtype=np.float32)
     a = g / (np.float32(1.0) + np.exp(-g)) * u
     return _to_bf16(a)
+
+
+def swiglu_inputs(rows: int, cols: int, seed: int = 3) -> tuple[torch.Tensor, torch.Tensor]:
+    """The two bf16 inputs g, u ~ N(0,1) of the fused SwiGLU path, from the same two streams as
+    swiglu_act (each rounded to bf16; the activation itself is formed by the path under test)."""
+    g = np.random.default_rng([seed, 0]).standard_normal((rows, cols), dtype=np.float32)
+    u = np.random.default_rng([seed, 1]).standard_normal((rows, cols), dtype=np.float32)
+    return _to_bf16(g), _to_bf16(u)
 
 
 def weight(rows: int = 8192, cols: int = 28672, seed: int = 4, std: float = 0.02) -> torch.Tensor:

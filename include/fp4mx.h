@@ -161,6 +161,25 @@ FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long
                          fp4_counts* counts, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * swiglu_fwht_quantize — the SwiGLU activation fused ahead of the (optionally randomised) rotation and
+ * the quantiser.  [E] §3 places the rotation in the SwiGLU epilogue; here the activation
+ * a = fl(SiLU(g) * u) is formed in fp32 from the two bf16 inputs and rotated without being stored, so
+ * it is never rounded to bf16.  SiLU(g) = g * fl(1 / fl(1 + e^-g)); the exponential follows Cody and
+ * Waite's argument reduction (x = n ln2 + r, n = rint(x log2 e), ln2 = 0x1.62ep-1 + 0x1.0bfbe8p-15)
+ * with the degree-6 Taylor polynomial of e^r in Horner form and an exact scaling by 2^n; e^x = +Inf
+ * above 88.5 and +0 below -103.  Every step is one fp32 rounding, so the activation is reproducible
+ * bit for bit.  Everything after the activation is fwht_quantize.
+ *   g, u  : device bf16 [rows, d] each, row-major, 32-byte aligned (dtype must be FP4_BF16, else
+ *           FP4_EUNSUPPORTED).
+ *   other arguments as in fwht_quantize. */
+FP4_API fp4_status swiglu_fwht_quantize(const void* g, const void* u, fp4_dtype dtype, long rows, long d,
+                                const unsigned int* signs, fp4_format format, int block, fp4_round round,
+                                int four_six, unsigned long long seed, fp4_scale_layout layout,
+                                const float* global_in, float* global_out, float* rotated_out,
+                                unsigned char* q, unsigned char* scales, fp4_counts* counts,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * fp4_dequantize — x_hat = fl((v * d) * s_g) per element, v the E2M1 value of the nibble and d the
  * decoded block scale (v*d is exact); MXFP4 has no s_g (x_hat = v * 2^e, exact).  bf16 output is
  * the round-to-nearest-even of that fp32 value.  [A] "Encode one MXFP4 block step by step"

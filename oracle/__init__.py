@@ -96,6 +96,10 @@ def lib():
         L.ora_fwht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
         L.ora_rht_rows.restype = None
         L.ora_rht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P, P]
+        L.ora_exp_cw.restype = ctypes.c_float
+        L.ora_exp_cw.argtypes = [ctypes.c_float]
+        L.ora_silu_mul_rows.restype = None
+        L.ora_silu_mul_rows.argtypes = [P, P, ctypes.c_long, P]
         _lib = L
     return _lib
 
@@ -233,6 +237,28 @@ def fwht(x, signs=None) -> np.ndarray:
         assert sg.size == d // 32
         lib().ora_rht_rows(_p(x), rows, d, sg.ctypes.data_as(ctypes.c_void_p), _p(y))
     return y
+
+
+def exp_cw(x: float) -> float:
+    """The written-out fp32 exponential used by the SwiGLU activation (Cody-Waite reduction,
+    degree-6 Taylor polynomial)."""
+    return float(lib().ora_exp_cw(float(np.float32(x))))
+
+
+def silu_mul(g, u) -> np.ndarray:
+    """a = fl(SiLU(g) * u) elementwise in fp32, SiLU(g) = g * fl(1 / fl(1 + exp(-g)))."""
+    g, u = _f32(g), _f32(u)
+    assert g.shape == u.shape
+    a = np.zeros_like(g)
+    lib().ora_silu_mul_rows(_p(g), _p(u), g.size, _p(a))
+    return a
+
+
+def swiglu_fwht_quantize(g, u, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
+                         global_in=None, signs=None):
+    """SiLU(g) * u in fp32 (no storage rounding), then the rotation and quantiser of fwht_quantize."""
+    return fwht_quantize(silu_mul(g, u), fmt=fmt, round=round, four_six=four_six, seed=seed,
+                         global_in=global_in, signs=signs)
 
 
 def fwht_quantize(x, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,

@@ -381,6 +381,61 @@ void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, lon
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* SwiGLU activation a = SiLU(g) * u in fp32, for the fused SiLU -> rotation -> quantiser path
+ * ([E] §3 places the rotation in the SwiGLU epilogue).  The exponential is written out so that a
+ * second implementation can reproduce it bit for bit: Cody and Waite's argument reduction (W. J.
+ * Cody and W. Waite, "Software Manual for the Elementary Functions", 1980) x = n ln2 + r with
+ * n = rint(x log2(e)) and ln2 split into an 11-bit head and a tail, then the degree-6 Taylor
+ * polynomial of e^r in Horner form (|r| <= 0.35: truncation below 2^-24 relative), then an exact
+ * scaling by 2^n.  Every operation is one fp32 rounding, in the order written.
+ *   exp: x > 88.5 -> +Inf, x < -103 -> +0; otherwise the steps above.
+ *   SiLU(g) = g * fl(1 / fl(1 + exp(-g)))  (one correctly rounded reciprocal)
+ *   a = fl(SiLU(g) * u)                                                                          */
+static float ora_pow2(int k) { /* 2^k for k in [-126, 127], exact */
+  uint32_t b = (uint32_t)(k + 127) << 23;
+  float f;
+  memcpy(&f, &b, 4);
+  return f;
+}
+
+/* p * 2^n, p in [0.7, 1.42], n in [-149, 128]: one rounding at most (only a subnormal result rounds) */
+static float ora_scale_pow2(float p, int n) {
+  if (n > 127) return (p * ora_pow2(127)) * ora_pow2(n - 127);
+  if (n >= -126) return p * ora_pow2(n);
+  return (p * ora_pow2(n + 64)) * ora_pow2(-64);
+}
+
+/* ln2 head: 12 significant bits, so n * head is exact for |n| <= 4096; tail = fl(ln2 - head) */
+float ora_exp_cw(float x) {
+  if (x != x) return x;
+  if (x > 88.5f) return INFINITY;
+  if (x < -103.0f) return 0.0f;
+  const float log2e = 0x1.715476p+0f, ln2_hi = 0x1.62ep-1f, ln2_lo = 0x1.0bfbe8p-15f;
+  float t = x * log2e;
+  float n = rintf(t);
+  float r = x - n * ln2_hi;
+  r = r - n * ln2_lo;
+  float p = 0x1.6c16c2p-10f;   /* fl(1/720) */
+  p = p * r + 0x1.111112p-7f;  /* fl(1/120) */
+  p = p * r + 0x1.555556p-5f;  /* fl(1/24) */
+  p = p * r + 0x1.555556p-3f;  /* fl(1/6) */
+  p = p * r + 0.5f;
+  p = p * r + 1.0f;
+  p = p * r + 1.0f;
+  return ora_scale_pow2(p, (int)n);
+}
+
+float ora_silu_mul(float g, float u) {
+  float e = ora_exp_cw(-g);
+  float s = g * (1.0f / (1.0f + e));
+  return s * u;
+}
+
+void ora_silu_mul_rows(const float* g, const float* u, long n, float* a) {
+  for (long i = 0; i < n; ++i) a[i] = ora_silu_mul(g[i], u[i]);
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Normalised Walsh-Hadamard rotation of each row ([E] §3: H_d with entries +-1/sqrt(d), applied by
  * O(d log2 d) add/subtract butterflies).  Reading: natural (Sylvester) order; fp32; the
  * unnormalised stages run in the fixed order h = 1, 2, 4, ..., d/2, each mapping

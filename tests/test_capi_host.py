@@ -93,6 +93,18 @@ def test_fwht_rejects(L):
     assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 5, 16, 0, 0, 0, 0, None, None, None, FAKE, FAKE, None, None, 0, None) == 1
 
 
+def test_swiglu_fwht_rejects(L):
+    # fp32 inputs (bf16 only), a NULL or misaligned up projection, and the rotation's own checks
+    assert L.swiglu_fwht_quantize(FAKE, FAKE, 0, 4, 8192, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None,
+                                  FAKE, 256, None) == 2
+    assert L.swiglu_fwht_quantize(FAKE, None, 1, 4, 8192, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None,
+                                  FAKE, 256, None) == 1
+    assert L.swiglu_fwht_quantize(FAKE, ctypes.c_void_p(0x10010), 1, 4, 8192, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE,
+                                  None, FAKE, 256, None) == 1
+    assert L.swiglu_fwht_quantize(FAKE, FAKE, 1, 4, 3000, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None,
+                                  FAKE, 256, None) == 1
+
+
 def test_dequant_rejects(L):
     assert L.fp4_dequantize(FAKE, FAKE, 1, 32, 0, FAKE, 128, 256, 0, FAKE, None) == 1  # block mismatch
     assert L.fp4_dequantize(FAKE, FAKE, 1, 16, 0, None, 128, 256, 0, FAKE, None) == 1  # NVFP4 needs s_g

@@ -345,6 +345,40 @@ def test_rht_gemm_end_to_end(cuda):
     assert e_rht < e_plain
 
 
+# SwiGLU activation fused ahead of the rotation: a = fl(SiLU(g) * u) formed in fp32, never stored
+
+@pytest.mark.parametrize("d", [1024, 8192, 16384])
+@pytest.mark.parametrize("fmt,rnd,four_six,rht", [(fp4.NVFP4, fp4.RNE, False, False), (fp4.NVFP4, fp4.STOCHASTIC, False, True),
+                                                  (fp4.NVFP4, fp4.RNE, True, False), (fp4.MXFP4, fp4.RNE, False, True)])
+def test_swiglu_fwht_small(cuda, d, fmt, rnd, four_six, rht):
+    rows = 37
+    g, u = synth.swiglu_inputs(rows, d, seed=3)
+    sg = synth.rht_signs(d, 34) if rht else None
+    q, s, gs, c, rot = fp4.swiglu_fwht_quantize(g.to(cuda), u.to(cuda), fmt=fmt, round=rnd, four_six=four_six,
+                                                seed=7, want_rotated=True,
+                                                signs=_signs_dev(d, 34, cuda) if rht else None)
+    y, qo, so, go, co = O.swiglu_fwht_quantize(f32(g), f32(u), fmt=fmt, round=rnd, four_six=four_six, seed=7,
+                                               signs=sg)
+    assert np.array_equal(npy(rot), y)       # the activation and the rotation, bit for bit
+    if fmt == fp4.NVFP4:
+        assert np.float32(npy(gs)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+
+
+def test_swiglu_fwht_full(cuda):
+    """16384 x 8192 bf16 g, u (seed 3 streams): SiLU(g) * u -> H_8192 -> NVFP4 with stochastic
+    rounding (seed 7), the global amax over the rotated activation: full comparison."""
+    g, u = synth.swiglu_inputs(16384, 8192, seed=3)
+    q, s, gs, c, _ = fp4.swiglu_fwht_quantize(g.to(cuda), u.to(cuda), round=fp4.STOCHASTIC, seed=7)
+    y, qo, so, go, co = O.swiglu_fwht_quantize(f32(g), f32(u), round=O.STOCHASTIC, seed=7)
+    assert np.float32(npy(gs)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co
+
+
 # ---------------------------------------------------------------------------------------------
 # The GEMM workloads' quantisation (MXFP4 activations and weights at the down_proj shape)
 

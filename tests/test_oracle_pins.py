@@ -405,6 +405,43 @@ def test_rht_matches_explicit_matrix():
     assert np.allclose(Q @ Q.T, np.eye(d), atol=1e-12)   # orthogonal
 
 
+def test_exp_cw_against_the_exponential():
+    """The written-out exponential of the SwiGLU path: within 4 units of 2^-24 (relative) of e^x over
+    the normal range, exact at 0, and the stated saturation at both ends."""
+    xs = np.linspace(-87.0, 88.0, 20001, dtype=np.float32)
+    rel = max(abs(O.exp_cw(x) - math.exp(float(x))) / math.exp(float(x)) for x in xs)
+    assert rel < 4 * 2.0 ** -24
+    assert O.exp_cw(0.0) == 1.0 and O.exp_cw(-0.0) == 1.0
+    assert O.exp_cw(88.6) == math.inf and O.exp_cw(-103.5) == 0.0
+    assert math.isnan(O.exp_cw(float("nan")))
+    # monotone across the reduction boundaries (n changes every ln2)
+    ys = [O.exp_cw(x) for x in np.linspace(-5.0, 5.0, 4001, dtype=np.float32)]
+    assert all(b >= a for a, b in zip(ys, ys[1:]))
+
+
+def test_silu_mul_against_fp64():
+    rng = np.random.default_rng(15)
+    g = rng.standard_normal(20000).astype(np.float32) * 4
+    u = rng.standard_normal(20000).astype(np.float32)
+    a = O.silu_mul(g, u).astype(np.float64)
+    g64, u64 = g.astype(np.float64), u.astype(np.float64)
+    ref = g64 / (1.0 + np.exp(-g64)) * u64
+    ok = np.abs(ref) > 1e-30
+    assert np.max(np.abs(a[ok] - ref[ok]) / np.abs(ref[ok])) < 8 * 2.0 ** -24
+    z = O.silu_mul(np.zeros(3, np.float32), np.float32([1, -2, 3]))
+    assert np.array_equal(z, np.zeros(3, np.float32))
+    big = O.silu_mul(np.float32([40.0]), np.float32([3.0]))   # SiLU(g) = g once e^-g vanishes
+    assert big[0] == np.float32(120.0)
+
+
+def test_swiglu_rotation_composes_the_parts():
+    from block_scaled_fp4_amax_b200 import synth
+    g, u = (synth.as_f32_numpy(t) for t in synth.swiglu_inputs(4, 1024, 3))
+    y, q, s, sg, c = O.swiglu_fwht_quantize(g, u, seed=7)
+    y2 = O.fwht(O.silu_mul(g, u))
+    assert np.array_equal(y, y2)
+
+
 # ---------------------------------------------------------------------------------------------
 # Dequantisation and the GEMM reference
 
