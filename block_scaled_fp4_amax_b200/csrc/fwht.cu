@@ -429,7 +429,9 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
 }
 
 // ---------------------------------------------------------------------------------------------
-// One wave of resident CTAs of `kernel` (each loops over rows).
+// CTAs to launch: the resident count of the amax pass (the lighter kernel), also for the quantise
+// pass, whose CTAs then run as about one and a half waves over rows of equal cost; that measured
+// slightly faster than one wave of the quantise pass's own resident count (uneven row tails).
 template <int LOG_D, typename K>
 static int fwht_grid(K kernel, long long rows) {
   using G = Geom<LOG_D>;
@@ -469,7 +471,8 @@ static cudaError_t quant_d(const FwhtParams& p, cudaStream_t s) {
   const int smem = G::ROWS * G::D * 4;
   auto k = fwht_quant_kernel<T, LOG_D, NV, SR, FS, GATED>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  k<<<fwht_grid<LOG_D>(k, p.rows), G::CTA, smem, s>>>(p);
+  cudaFuncSetAttribute(fwht_amax_kernel<T, LOG_D, GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  k<<<fwht_grid<LOG_D>(fwht_amax_kernel<T, LOG_D, GATED>, p.rows), G::CTA, smem, s>>>(p);
   return cudaGetLastError();
 }
 
