@@ -1,6 +1,6 @@
 // fp4_device.cuh — device-side building blocks shared by the quantise / rotate / dequantise
-// kernels of libfp4mx: 16-byte vector loads, the sm_100 FP4/FP8 conversion instructions,
-// Philox4x32-10 and the E2M1 rounding rules.
+// kernels of libfp4mx: 256-bit lane loads, the sm_100 FP4/FP8 conversion instructions,
+// Philox4x32-10, the E2M1 rounding rules and the block encoders.
 //
 // Every floating-point step that decides a code is an explicitly rounded fp32 intrinsic
 // (__fmul_rn, __fadd_rn, __fsub_rn, __frcp_rn, __fdiv_rn) so the compiler cannot contract or
@@ -14,38 +14,7 @@
 namespace fp4k {
 
 // ---------------------------------------------------------------------------------------------
-// Loads.  16 bytes per lane, read-only path.  `Stream` loads are marked evict-first (data that
-// will not be read again); the default keeps the line in L2 for a following pass.
-template <bool Stream>
-__device__ __forceinline__ uint4 ld16(const void* p) {
-  if (Stream) return __ldcs(reinterpret_cast<const uint4*>(p));
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
-// Element type traits: E values per 16-byte chunk, unpacked to fp32 (exact).
-template <typename T> struct Vec;
-template <> struct Vec<float> {
-  static constexpr int E = 4;
-  __device__ __forceinline__ static void unpack(const uint4& r, float* v) {
-    v[0] = __uint_as_float(r.x); v[1] = __uint_as_float(r.y);
-    v[2] = __uint_as_float(r.z); v[3] = __uint_as_float(r.w);
-  }
-};
-template <> struct Vec<__nv_bfloat16> {
-  static constexpr int E = 8;
-  __device__ __forceinline__ static void unpack(const uint4& r, float* v) {
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-};
-
+// Loads.
 // 32 bytes per lane (sm_100 256-bit load): a warp reads 1 KiB of contiguous memory per
 // instruction.  `Stream` marks the lines evict-first in L2 (last use); otherwise they are kept
 // for a following pass.
@@ -158,10 +127,6 @@ __device__ __forceinline__ uint32_t e2m1x4(const float* y) {
       : "=r"(out)
       : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]));
   return out;
-}
-template <int E>
-__device__ __forceinline__ uint32_t e2m1_pack(const float* y) {
-  if constexpr (E == 8) return e2m1x8(y); else return e2m1x4(y);
 }
 
 // Two f16 halves of a 32-bit word to fp32 (exact), without type punning.
@@ -559,11 +524,6 @@ __device__ __forceinline__ float block_sse_n(const float* sq, int lane) {
 // When |A_4 - A_6| exceeds it, sign(A_4 - A_6) = sign(S_4 - S_6) and the estimate decides; the
 // caller computes S_T exactly otherwise.
 
-__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 
 // sum over N values of (q_i - y_i)^2: q_i decoded from the packed nibbles (exact in f16), the
 // difference formed in fp32 from the f16 operand directly.  `opaque0` is a kernel-parameter zero

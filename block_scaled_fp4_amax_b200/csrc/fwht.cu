@@ -13,11 +13,17 @@
 //   round B : the thread gathers the 32 values that differ in index bits 5-9, stages h=32..512;
 //   last    : the thread gathers the values that differ in the remaining high bits together with
 //             2^L consecutive values (index bits 0..L-1, L = 5 - #high bits) and runs the last
-//             stages, multiplies by c and quantises straight from registers.  A 16-value NVFP4
-//             block then spans 2^(4-L) adjacent lanes (amax = xor-shuffle), a Philox call covers
-//             whole 4-value groups (L >= 2), and the packed nibbles are contiguous across lanes.
+//             stages;
+//   quantise: the values go back through the row buffer so that each thread holds 32 consecutive
+//             rotated values (two NVFP4 blocks or one MXFP4 block), multiplies by c and quantises
+//             whole blocks from registers.
 // Shared memory holds one fp32 row per row slot; 16-byte chunks are XOR-swizzled by the low
 // three bits of their 32-value row so that every round's accesses are bank-conflict free.
+//
+// Two optional inputs change what is rotated, not how:
+//   signs : the randomised rotation c * H * D ([P], random Hadamard transform): bit j of a
+//           thread's sign word negates its round-A value j before the butterflies;
+//   u     : the SwiGLU path (bf16): x holds g, and the rotated input is fl(SiLU(g) * u).
 #include "fp4_device.cuh"
 #include "launch.h"
 
