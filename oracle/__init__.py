@@ -81,6 +81,9 @@ def lib():
         L.ora_mx_quantize.restype = None
         L.ora_mx_quantize.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_uint64, P, P, P]
+        L.ora_mx_quantize_at.restype = None
+        L.ora_mx_quantize_at.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_uint64, ctypes.c_uint64, P, P, P]
         L.ora_nvfp4_global_scale.restype = ctypes.c_float
         L.ora_nvfp4_global_scale.argtypes = [ctypes.c_float, ctypes.c_int]
         L.ora_nvfp4_quantize.restype = None
@@ -186,6 +189,20 @@ def mx_quantize(x, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0):
     s = np.zeros((rows, cols // 32), dtype=np.uint8)
     c = _Counts()
     lib().ora_mx_quantize(_p(x), rows, cols, int(policy), int(round), int(seed), _p(q), _p(s), ctypes.byref(c))
+    return q, s, c.as_dict()
+
+
+def mx_quantize_rows_at(x, idx_base: int, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0):
+    """mx_quantize of rows that start at flat element index `idx_base` of a larger tensor (the
+    random words of stochastic rounding follow the flat index)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    assert cols % 32 == 0
+    q = np.zeros((rows, cols // 2), dtype=np.uint8)
+    s = np.zeros((rows, cols // 32), dtype=np.uint8)
+    c = _Counts()
+    lib().ora_mx_quantize_at(_p(x), rows, cols, int(policy), int(round), int(seed), int(idx_base), _p(q), _p(s),
+                             ctypes.byref(c))
     return q, s, c.as_dict()
 
 

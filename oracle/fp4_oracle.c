@@ -218,8 +218,10 @@ static void pack_pairs(const uint8_t* codes, int n, uint8_t* out) {
 }
 
 /* x: [rows, cols] fp32 row-major; q: [rows, cols/2]; scales: [rows, cols/32] row-major bytes. */
-void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
-                     uint8_t* q, uint8_t* scales, ora_counts* cnt) {
+/* idx_base: flat element index of x[0] in the tensor the rows belong to (the random words of
+ * stochastic rounding are indexed by it; 0 for a whole tensor). */
+void ora_mx_quantize_at(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
+                        uint64_t idx_base, uint8_t* q, uint8_t* scales, ora_counts* cnt) {
   const int B = 32;
   long nb = cols / B;
   uint8_t codes[32];
@@ -228,10 +230,15 @@ void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round
       const float* xb = x + r * cols + j * B;
       int e = ora_mx_exponent(block_amax(xb, B), policy);
       scales[r * nb + j] = (uint8_t)(e + 127);
-      ora_mx_encode_block(xb, B, e, round, seed, (uint64_t)(r * cols + j * B), codes, cnt);
+      ora_mx_encode_block(xb, B, e, round, seed, idx_base + (uint64_t)(r * cols + j * B), codes, cnt);
       pack_pairs(codes, B, q + r * (cols / 2) + j * (B / 2));
     }
   }
+}
+
+void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
+                     uint8_t* q, uint8_t* scales, ora_counts* cnt) {
+  ora_mx_quantize_at(x, rows, cols, policy, round, seed, 0, q, scales, cnt);
 }
 
 /* ------------------------------------------------------------------------------------------ */

@@ -379,6 +379,50 @@ def test_swiglu_fwht_full(cuda):
     assert counts_of(c) == co
 
 
+# Past 2^31 elements: 64-bit chunk, block, scale and Philox indices
+
+def test_quantise_beyond_2p31_elements(cuda):
+    """65537 x 32768 bf16 = 2,147,516,416 elements; the last row lies wholly past element 2^31.  The
+    tensor is a seeded 128-row base repeated with a per-row factor (built on the device); sampled rows
+    around the 2^31 boundary are compared with the oracle on the same bits."""
+    rows, cols = 65537, 32768
+    base = synth.normal_bf16(128, cols, 51).to(cuda)
+    fac = torch.from_numpy(np.random.default_rng(52).uniform(0.5, 2.0, rows).astype(np.float32)).to(cuda)
+    x = torch.empty((rows, cols), dtype=torch.bfloat16, device=cuda)
+    for r0 in range(0, rows, 8192):   # chunks keep the temporaries small
+        r1 = min(rows, r0 + 8192)
+        idx = torch.arange(r0, r1, device=cuda) % 128
+        x[r0:r1] = (base[idx].float() * fac[r0:r1, None]).to(torch.bfloat16)
+    assert x.numel() > 2 ** 31
+    sample = [0, 1, 65535, 65536]      # row 65536 starts at element 2^31 exactly
+
+    q, s, c = fp4.mx_quantize(x, round=fp4.STOCHASTIC, seed=11)
+    # stochastic rounding indexes Philox by the flat element index: the oracle quantises each
+    # sampled row at its true flat offset
+    for r in sample:
+        xr = f32(x[r:r + 1].cpu())
+        qo, so, _ = O.mx_quantize_rows_at(xr, r * cols, round=O.STOCHASTIC, seed=11)
+        assert np.array_equal(npy(q[r:r + 1]), qo)
+        assert np.array_equal(npy(s.view(rows, cols // 32)[r:r + 1]), so)
+
+    g = torch.tensor([0.004], dtype=torch.float32, device=cuda)
+    q, s, gg, c = fp4.nvfp4_quantize(x, global_in=g)
+    for r in sample:
+        xr = f32(x[r:r + 1].cpu())
+        qo, so, _, _ = O.nvfp4_quantize(xr, global_in=0.004)
+        assert np.array_equal(npy(q[r:r + 1]), qo)
+        assert np.array_equal(npy(s.view(rows, cols // 16)[r:r + 1]), so)
+    out = fp4.fp4_dequantize(q, s, fp4.NVFP4, gg, out_dtype=torch.bfloat16)
+    for r in sample:
+        want = O.dequantize(npy(q[r:r + 1]), npy(s.view(rows, cols // 16)[r:r + 1]), O.NVFP4, np.float32(0.004))
+        assert torch.equal(out[r:r + 1].cpu(), torch.from_numpy(want).to(torch.bfloat16))
+    # the two-pass call: the tensor amax over all 2.1 G values sets the global scale
+    _, _, g2, _ = fp4.nvfp4_quantize(x)
+    amax = float(x.abs().max().float().item())
+    assert np.float32(npy(g2)[0]) == np.float32(np.float32(amax) / np.float32(2688.0))
+    del x, q, s, out
+
+
 # ---------------------------------------------------------------------------------------------
 # The GEMM workloads' quantisation (MXFP4 activations and weights at the down_proj shape)
 

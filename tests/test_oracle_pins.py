@@ -368,6 +368,17 @@ def _sign_vector(bits_words, d):
     return np.where(b == 1, -1.0, 1.0)
 
 
+def test_mx_rows_at_offset_match_the_whole_tensor():
+    """Stochastic rounding follows the flat element index: quantising one row at its flat offset
+    reproduces that row of the whole-tensor call (used for sampled rows of very large tensors)."""
+    from block_scaled_fp4_amax_b200 import synth
+    x = synth.as_f32_numpy(synth.mx_small())
+    q0, s0, _ = O.mx_quantize(x, round=O.STOCHASTIC, seed=3)
+    for r in (0, 5, 255):
+        q1, s1, _ = O.mx_quantize_rows_at(x[r:r + 1], r * x.shape[1], round=O.STOCHASTIC, seed=3)
+        assert np.array_equal(q0[r:r + 1], q1) and np.array_equal(s0[r:r + 1], s1)
+
+
 def test_rht_without_signs_is_the_plain_rotation():
     x = O._f32(np.random.default_rng(12).standard_normal((3, 2048)))
     assert np.array_equal(O.fwht(x, np.zeros(64, dtype=np.uint32)), O.fwht(x))
