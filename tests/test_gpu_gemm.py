@@ -181,3 +181,25 @@ def test_gemm_ldc_and_status_word(cuda):
     assert torch.all(big[:, N:] == 7.0)
     C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fp4.NVFP4)
     check(big[:, :N], C64, S)
+
+
+def test_gemm_output_beyond_2p31_elements(cuda):
+    """M = 65792, N = 32768, K = 256 NVFP4: 2,155,872,256 bf16 outputs, rows from 65536 on lying
+    wholly past element 2^31 of C.  Sampled rows on both sides of the boundary against the fp64
+    product of the exactly dequantised operands (1e-3 sum|ab| plus the bf16 rounding term)."""
+    M, N, K = 65792, 32768, 256
+    a = synth.gemm_operand(M, K, 61)
+    b = synth.gemm_operand(N, K, 62)
+    qa, sa, ga, _ = fp4.nvfp4_quantize(a.to(cuda), layout=fp4.MMA_TILED)
+    qb, sb, gb, _ = fp4.nvfp4_quantize(b.to(cuda), layout=fp4.MMA_TILED)
+    C, ws = fp4.fp4_block_gemm(fp4.NVFP4, qa, sa, qb, sb, ga, gb)
+    assert status_ok(ws) and C.numel() > 2 ** 31
+    rows = [0, 65535, 65536, M - 1]
+    qo, so, go, _ = O.nvfp4_quantize(synth.as_f32_numpy(a))        # whole A: its own global scale
+    A64 = O.dequantize(qo[rows], so[rows], O.NVFP4, go).astype(np.float64)
+    qbo, sbo, gbo, _ = O.nvfp4_quantize(synth.as_f32_numpy(b))
+    B64 = O.dequantize(qbo, sbo, O.NVFP4, gbo).astype(np.float64)
+    C64 = A64 @ B64.T
+    S = np.abs(A64) @ np.abs(B64).T
+    check(C[rows], C64, S)
+    del C
