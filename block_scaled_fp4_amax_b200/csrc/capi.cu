@@ -152,6 +152,7 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   L.tiled = layout == FP4_SCALES_MMA_TILED; L.reverse = global_in ? 0 : 1;
   L.global_in = global_in; L.amax_bits = amax; L.global_out = global_out;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
+  L.pdl = amax_pass;
   e = fp4k::launch_quantize(L, s);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "nvfp4_quantize launch");
 }
@@ -187,6 +188,7 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   L.rotated_out = rotated_out;
   L.signs = signs;
   L.u = u;
+  L.pdl = amax_pass;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e;
   if (amax_pass) {

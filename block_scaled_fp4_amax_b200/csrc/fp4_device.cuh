@@ -14,6 +14,15 @@
 namespace fp4k {
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch (sm_90 and later).  A kernel launched with programmatic stream
+// serialisation may be scheduled while its predecessor on the stream still runs.  grid_dep_wait()
+// blocks until that predecessor has completed and its memory is visible (a no-op after an
+// ordinary launch); grid_dep_trigger() lets the dependent grid be scheduled once every CTA of this
+// grid has started, so its CTAs take SMs as this grid's CTAs retire instead of after a launch gap.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
 // Loads.
 // 32 bytes per lane (sm_100 256-bit load): a warp reads 1 KiB of contiguous memory per
 // instruction.  `Stream` marks the lines evict-first in L2 (last use); otherwise they are kept

@@ -215,6 +215,7 @@ struct FwhtParams {
 template <typename T, int LOG_D, bool GATED>
 __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams p) {
   using G = Geom<LOG_D>;
+  grid_dep_trigger();  // the quantise pass may take SMs as this grid's CTAs retire
   // the counters the following quantise pass accumulates into start at zero (stream order)
   if (p.counts && blockIdx.x == 0 && threadIdx.x < 4) p.counts[threadIdx.x] = 0ull;
   extern __shared__ __align__(16) float smem[];
@@ -306,6 +307,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
   const uint32_t sgn = p.signs ? p.signs[t] : 0u;
   const long long step = (long long)gridDim.x * G::ROWS;
   const uint32_t nb = D / B;
+  grid_dep_wait();  // after the amax pass (programmatic launch): its results are visible from here
 
   float s_g = 1.0f, inv6 = 1.0f, inv4 = 1.0f;
   if (NV) {
@@ -472,23 +474,24 @@ static cudaError_t amax_d(const FwhtParams& p, cudaStream_t s) {
 }
 
 template <typename T, int LOG_D, bool NV, bool SR, bool FS, bool GATED>
-static cudaError_t quant_d(const FwhtParams& p, cudaStream_t s) {
+static cudaError_t quant_d(const FwhtParams& p, bool pdl, cudaStream_t s) {
   using G = Geom<LOG_D>;
   const int smem = G::ROWS * G::D * 4;
   auto k = fwht_quant_kernel<T, LOG_D, NV, SR, FS, GATED>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   cudaFuncSetAttribute(fwht_amax_kernel<T, LOG_D, GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  k<<<fwht_grid<LOG_D>(fwht_amax_kernel<T, LOG_D, GATED>, p.rows), G::CTA, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(fwht_grid<LOG_D>(fwht_amax_kernel<T, LOG_D, GATED>, p.rows)), dim3(G::CTA), smem, s,
+                    pdl, p);
 }
 
 template <typename T, int LOG_D, bool GATED>
 static cudaError_t quant_sel(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
+  const bool d = L.pdl;
   if (!L.nv)
-    return L.sr ? quant_d<T, LOG_D, false, true, false, GATED>(p, s) : quant_d<T, LOG_D, false, false, false, GATED>(p, s);
+    return L.sr ? quant_d<T, LOG_D, false, true, false, GATED>(p, d, s) : quant_d<T, LOG_D, false, false, false, GATED>(p, d, s);
   if (L.four_six)
-    return L.sr ? quant_d<T, LOG_D, true, true, true, GATED>(p, s) : quant_d<T, LOG_D, true, false, true, GATED>(p, s);
-  return L.sr ? quant_d<T, LOG_D, true, true, false, GATED>(p, s) : quant_d<T, LOG_D, true, false, false, GATED>(p, s);
+    return L.sr ? quant_d<T, LOG_D, true, true, true, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, true, GATED>(p, d, s);
+  return L.sr ? quant_d<T, LOG_D, true, true, false, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, false, GATED>(p, d, s);
 }
 
 template <typename T, bool GATED>

@@ -3,9 +3,27 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <utility>
 #include <stdint.h>
 
 namespace fp4k {
+
+// Launch `kernel` with an optional programmatic-dependent-launch attribute (see grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 int num_sms();  // SM count of the current device (cached per device)
 
@@ -29,6 +47,7 @@ struct QuantLaunch {
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;  // 4 counters or NULL
+  bool pdl;       // launched right after the amax pass: programmatic dependent launch
 };
 
 struct DequantLaunch {
@@ -58,6 +77,7 @@ struct FwhtLaunch {
   float* rotated_out;
   const uint32_t* signs;  // randomised rotation: bit i negates channel i (nullptr: plain rotation)
   const void* u;          // SwiGLU path (bf16): x is g, u the up projection; nullptr otherwise
+  bool pdl;               // quantise pass right after the amax pass: programmatic dependent launch
   uint8_t* q;
   uint8_t* scales;
   unsigned long long* counts;
@@ -75,6 +95,7 @@ struct GemmLaunch {
 
 cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
 // Tensor amax into *amax_bits (zeroed by the caller); also zeroes `counts` (4 words) if non-null.
+// Lets the following quantise pass, launched with QuantLaunch::pdl, be scheduled as it retires.
 cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
                         unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
   const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
   const long long per_tile = 32LL * U;
   const long long ntiles = (p.n_chunks + per_tile - 1) / per_tile;
+  grid_dep_wait();  // after the amax pass (programmatic launch): its results are visible from here
 
   NvScale ns{1.0f, 1.0f, 1.0f};
   __shared__ float2 tab[NV ? kScaleTab : 1];
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long n_chunks,
                                                         uint32_t* amax_bits, unsigned long long* counts) {
+  grid_dep_trigger();  // the quantise pass may take SMs as this grid's CTAs retire
   // the counters the following quantise pass accumulates into start at zero (stream order)
   if (counts && blockIdx.x == 0 && threadIdx.x < 4) counts[threadIdx.x] = 0ull;
   constexpr int E = Vec32<T>::E;
@@ -342,7 +344,7 @@ static int grid_for(long long work_items, int per_cta) {
 
 // One wave of resident CTAs (the kernel loops over tiles), so no CTA waits in a tail wave.
 template <typename T, bool NV, bool SR, bool FS>
-static cudaError_t launch_q(const QuantParams& p, cudaStream_t s) {
+static cudaError_t launch_q(const QuantParams& p, bool pdl, cudaStream_t s) {
   static int per_sm = 0;  // resident CTAs per SM for this instantiation (same on every sm_100 device)
   if (per_sm == 0) {
     int n = 0;
@@ -356,15 +358,14 @@ static cudaError_t launch_q(const QuantParams& p, cudaStream_t s) {
   const long long want = (tiles * 32 + kThreads - 1) / kThreads;
   const long long cap = (long long)num_sms() * per_sm;
   const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
-  quantize_kernel<T, NV, SR, FS><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(quantize_kernel<T, NV, SR, FS>, dim3(grid), dim3(kThreads), 0, s, pdl, p);
 }
 
 template <typename T>
-static cudaError_t dispatch_q(const QuantParams& p, bool nv, bool sr, bool fs, cudaStream_t s) {
-  if (!nv) return sr ? launch_q<T, false, true, false>(p, s) : launch_q<T, false, false, false>(p, s);
-  if (fs) return sr ? launch_q<T, true, true, true>(p, s) : launch_q<T, true, false, true>(p, s);
-  return sr ? launch_q<T, true, true, false>(p, s) : launch_q<T, true, false, false>(p, s);
+static cudaError_t dispatch_q(const QuantParams& p, bool nv, bool sr, bool fs, bool pdl, cudaStream_t s) {
+  if (!nv) return sr ? launch_q<T, false, true, false>(p, pdl, s) : launch_q<T, false, false, false>(p, pdl, s);
+  if (fs) return sr ? launch_q<T, true, true, true>(p, pdl, s) : launch_q<T, true, false, true>(p, pdl, s);
+  return sr ? launch_q<T, true, true, false>(p, pdl, s) : launch_q<T, true, false, false>(p, pdl, s);
 }
 
 cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
@@ -386,8 +387,8 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   p.scales = L.scales;
   p.counts = L.counts;
   if (p.n_chunks == 0) return cudaSuccess;
-  return L.bf16 ? dispatch_q<__nv_bfloat16>(p, L.nv, L.sr, L.four_six, s)
-                : dispatch_q<float>(p, L.nv, L.sr, L.four_six, s);
+  return L.bf16 ? dispatch_q<__nv_bfloat16>(p, L.nv, L.sr, L.four_six, L.pdl, s)
+                : dispatch_q<float>(p, L.nv, L.sr, L.four_six, L.pdl, s);
 }
 
 cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
