@@ -26,7 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp4_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, IF4 = 0, 1, 2
 RNE, STOCHASTIC = 0, 1
 OCP_FLOOR, NOSAT_CEIL = 0, 1
 
@@ -63,6 +63,10 @@ def lib():
         L.ora_e2m1_encode_rne.argtypes = [ctypes.c_float]
         L.ora_e2m1_encode_sr.restype = ctypes.c_int
         L.ora_e2m1_encode_sr.argtypes = [ctypes.c_float, ctypes.c_uint32]
+        L.ora_int4_value.restype = ctypes.c_double
+        L.ora_int4_value.argtypes = [ctypes.c_int]
+        L.ora_int4_encode_rne.restype = ctypes.c_int
+        L.ora_int4_encode_rne.argtypes = [ctypes.c_float]
         L.ora_e4m3_value.restype = ctypes.c_double
         L.ora_e4m3_value.argtypes = [ctypes.c_int]
         L.ora_e4m3_encode_rne_satfinite.restype = ctypes.c_int
@@ -129,6 +133,16 @@ def e2m1_encode_rne(y: float) -> int:
 
 def e2m1_encode_sr(y: float, r: int) -> int:
     return lib().ora_e2m1_encode_sr(float(y), int(r))
+
+
+def int4_value(code: int) -> float:
+    """Value of a sign-magnitude INT4 nibble of IF4 (-7..7, bit 3 the sign)."""
+    return lib().ora_int4_value(int(code))
+
+
+def int4_encode_rne(y: float) -> int:
+    """IF4's INT4 nibble for a value already divided by the integer step."""
+    return lib().ora_int4_encode_rne(float(y))
 
 
 def e4m3_value(code: int) -> float:
@@ -206,8 +220,11 @@ def mx_quantize_rows_at(x, idx_base: int, policy: int = OCP_FLOOR, round: int = 
     return q, s, c.as_dict()
 
 
-def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, global_in=None):
-    """NVFP4 quantise. Returns (q, scales [rows, cols/16], s_g, counts)."""
+def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, global_in=None, if4: bool = False):
+    """NVFP4 quantise (with `if4`, IF4: each block E2M1 or INT4, the choice in scale bit 7).
+    Returns (q, scales [rows, cols/16], s_g, counts)."""
+    assert not (four_six and if4)
+    mode = 2 if if4 else int(bool(four_six))
     x = _f32(x)
     rows, cols = x.shape
     assert cols % 16 == 0
@@ -216,13 +233,14 @@ def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, g
     gin = None if global_in is None else np.array([global_in], dtype=np.float32)
     gout = np.zeros(1, dtype=np.float32)
     c = _Counts()
-    lib().ora_nvfp4_quantize(_p(x), rows, cols, int(round), int(bool(four_six)), int(seed),
+    lib().ora_nvfp4_quantize(_p(x), rows, cols, int(round), mode, int(seed),
                              None if gin is None else _p(gin), _p(gout), _p(q), _p(s), ctypes.byref(c))
     return q, s, float(gout[0]), c.as_dict()
 
 
 def dequantize(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
-    """fp32 reconstruction fl(fl(v*d)*s_g) (NVFP4) / v*2^e (MXFP4)."""
+    """fp32 reconstruction fl(fl(v*d)*s_g) (NVFP4) / v*2^e (MXFP4); IF4 blocks flagged INT4 in
+    scale bit 7 give fl(fl(k*d)*fl(s_g*fl(6/7)))."""
     q = np.ascontiguousarray(q, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     rows, half = q.shape

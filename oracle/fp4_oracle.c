@@ -297,9 +297,78 @@ static float nv_candidate(const float* x, int n, float amax_b, float s_g, float 
   return sse;
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* IF4 ([P] IF4 segment): each 16-block takes the NVFP4 block scale (block amax over 6, cast to
+ * E4M3), is encoded twice, as E2M1 and as a signed integer scaled by 7/6 (the block maximum lands
+ * on 7 instead of 6, so an integer step is 6/7 of the E2M1 unit), and keeps the encoding with the
+ * lower squared error.  The choice goes into the scale byte's sign bit, which NVFP4 never uses
+ * (0 = E2M1, 1 = INT4).  Readings where the segment is silent:
+ *   - the INT4 nibble is sign-magnitude like E2M1: bit 3 is the sign of y, bits 0-2 hold |k| <= 7,
+ *     so the integer lattice is -7..7 and -0 is encodable;
+ *   - the step is formed in fp32 as s7 = fl(s_g * fl(6/7)) per tensor, D7 = fl(d * s7),
+ *     R7 = fl(1 / D7); y = fl(x * R7); k = nearest integer to y, ties to even, |k| clamped to 7;
+ *     the reconstruction is fl(fl(k * d) * s7) (k * d is exact), the INT4 analogue of
+ *     fl(fl(v * d) * s_g);
+ *   - INT4 is kept iff its fp32 sequential error sum is strictly lower (a tie or a NaN keeps E2M1),
+ *     and a block whose scale code is 0 keeps E2M1 (both reconstructions are zero);
+ *   - the global scale is plain NVFP4's (M = 448); round to nearest only;
+ *   - counters of an INT4 block: saturation |y| > 7, underflow x != 0 with k = 0.               */
+
+double ora_int4_value(int code) {
+  int mag = code & 7;
+  return (code & 8) ? -(double)mag : (double)mag;
+}
+
+/* Nearest of the integers 0..7 to |y| (ties to the even one), by enumerating the lattice; a
+ * magnitude above 7, Inf included, clamps to 7.  The sign bit follows signbit(y).             */
+int ora_int4_encode_rne(float y) {
+  double a = fabs((double)y);
+  int best = 7;
+  if (!(a > 7.0)) {
+    double bestd = INFINITY;
+    best = 0;
+    for (int k = 0; k < 8; ++k) {
+      double d = fabs(a - (double)k);
+      if (d < bestd || (d == bestd && (k & 1) == 0 && (best & 1) == 1)) {
+        best = k;
+        bestd = d;
+      }
+    }
+  }
+  return (signbit(y) ? 8 : 0) | best;
+}
+
+/* The INT4 candidate of one block with E4M3 scale code sc (nonzero): codes, counters and the
+ * fp32 sequential sum of squared errors.                                                       */
+static float if4_int_candidate(const float* x, int n, int sc, float s_g, uint8_t* codes, ora_counts* c) {
+  float six_sevenths = 6.0f / 7.0f;
+  float s7 = s_g * six_sevenths;
+  float d = (float)ora_e4m3_value(sc);
+  float D7 = d * s7;
+  float R7 = 1.0f / D7;
+  memset(c, 0, sizeof(*c));
+  for (int i = 0; i < n; ++i) {
+    float y = x[i] * R7;
+    int code = ora_int4_encode_rne(y);
+    if (isfinite(y) && fabsf(y) > 7.0f) c->saturation += 1;
+    if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
+    codes[i] = (uint8_t)code;
+  }
+  float sse = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float kd = (float)(ora_int4_value(codes[i]) * (double)d); /* exact: <= 7 significant bits */
+    float xhat = kd * s7;
+    float err = x[i] - xhat;
+    float sq = err * err;
+    sse = sse + sq;
+  }
+  return sse;
+}
+
 /* x: [rows, cols] fp32; q: [rows, cols/2]; scales: [rows, cols/16] row-major E4M3 bytes.
+ * mode: 0 plain NVFP4, 1 four over six, 2 IF4.
  * global_in: NULL -> s_g from the tensor amax; else s_g = *global_in.                          */
-void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int four_six, uint64_t seed,
+void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mode, uint64_t seed,
                         const float* global_in, float* global_out, uint8_t* q, uint8_t* scales,
                         ora_counts* cnt) {
   const int B = 16;
@@ -313,7 +382,7 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int fou
       float a = fabsf(x[i]);
       if (a > amax_t) amax_t = a;
     }
-    s_g = ora_nvfp4_global_scale(amax_t, four_six);
+    s_g = ora_nvfp4_global_scale(amax_t, mode == 1);
   }
   if (global_out) *global_out = s_g;
   uint8_t c6[16], c4[16];
@@ -330,11 +399,19 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int fou
       const uint8_t* pick = c6;
       int sc = sc6;
       ora_counts k = k6;
-      if (four_six) {
+      if (mode == 1) {
         float sse4 = nv_candidate(xb, B, amax_b, s_g, 4.0f, round, seed, idx0, c4, &sc4, &k4);
         if (sse4 < sse6) {
           pick = c4;
           sc = sc4;
+          k = k4;
+          cnt->blocks_four += 1;
+        }
+      } else if (mode == 2 && sc6 != 0) {
+        float sse7 = if4_int_candidate(xb, B, sc6, s_g, c4, &k4);
+        if (sse7 < sse6) {
+          pick = c4;
+          sc = sc6 | 0x80;
           k = k4;
           cnt->blocks_four += 1;
         }
@@ -350,11 +427,15 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int fou
 /* ------------------------------------------------------------------------------------------ */
 /* Dequantisation ([A] "Encode one MXFP4 block step by step": reconstruction = lattice value times
  * the block scale; [X]: block scales applied in FP32).  x_hat = fl(fl(v*d) * s_g) for NVFP4, where
- * v*d is exact, and x_hat = v * 2^(byte-127) for MXFP4 (exact).  Row-major scales.            */
+ * v*d is exact, and x_hat = v * 2^(byte-127) for MXFP4 (exact).  format 2 is IF4: a scale byte
+ * with bit 7 set holds an INT4 block, x_hat = fl(fl(k*d) * s7) with d from the low 7 bits and
+ * s7 = fl(s_g * fl(6/7)); otherwise the NVFP4 rule.  Row-major scales.                         */
 void ora_dequantize(const uint8_t* q, const uint8_t* scales, int format, long rows, long cols,
                     float s_g, float* out) {
   int B = (format == 0) ? 32 : 16;
   long nb = cols / B;
+  float six_sevenths = 6.0f / 7.0f;
+  float s7 = s_g * six_sevenths;
   for (long r = 0; r < rows; ++r) {
     for (long k = 0; k < cols; ++k) {
       uint8_t byte = q[r * (cols / 2) + k / 2];
@@ -363,6 +444,9 @@ void ora_dequantize(const uint8_t* q, const uint8_t* scales, int format, long ro
       double v = ora_e2m1_value(code);
       if (format == 0) {
         out[r * cols + k] = (float)ldexp(v, (int)sb - 127);
+      } else if (format == 2 && (sb & 0x80)) {
+        float kd = (float)(ora_int4_value(code) * ora_e4m3_value(sb & 0x7F));
+        out[r * cols + k] = kd * s7;
       } else {
         float vd = (float)(v * ora_e4m3_value(sb));
         out[r * cols + k] = vd * s_g;

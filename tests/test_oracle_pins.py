@@ -311,6 +311,121 @@ def test_four_over_six_picks_lower_error_candidate_brute_force():
 
 
 # ---------------------------------------------------------------------------------------------
+# IF4 (E2M1 or INT4 per block, the choice in the scale byte's sign bit)
+
+IF4_ROW = [int(v) for v in golden_rows("if4.txt")[0]]
+
+
+def _if4_step(sg):
+    """fp32 INT4 step of a block with E4M3 scale 1: fl(1 * fl(s_g * fl(num/den)))."""
+    n, dd = IF4_ROW[5], IF4_ROW[6]
+    return np.float32(np.float32(sg) * (np.float32(n) / np.float32(dd)))
+
+
+def test_int4_encoder_is_rint_clipped_with_sign_bit():
+    """Lattice enumeration against numpy's round-half-even, clipped to the 7 the stretch allows."""
+    assert IF4_ROW[1] == 7 and IF4_ROW[2] == 6
+    rng = np.random.default_rng(11)
+    ys = np.concatenate([rng.uniform(-10, 10, 4000), np.arange(-9, 9.5, 0.5), [0.0, -0.0, 7.4999, -7.5001,
+                                                                                np.inf, -np.inf, 1e30]])
+    for y in ys.astype(np.float32):
+        k = int(np.clip(np.rint(np.abs(np.float64(y))), 0, IF4_ROW[1]))
+        want = (8 if np.signbit(y) else 0) | k
+        assert O.int4_encode_rne(float(y)) == want, y
+    for c in range(16):
+        v = O.int4_value(c)
+        assert abs(v) == (c & 7) and (math.copysign(1.0, v) < 0) == bool(c & 8)
+
+
+def test_if4_block_on_the_int4_lattice_is_exact_and_flagged():
+    """x_i = k_i * step: the INT4 branch reconstructs exactly, E2M1 cannot (6/7 is off its
+    lattice), so the block takes INT4, the flag (scale bit 7) is set and the nibbles are k."""
+    step = _if4_step(1.0)
+    k = np.array([-7, -6, -5, -4, -3, -2, -1, 0, 1, 2, 3, 4, 5, 6, 7, 3])
+    assert k.size == IF4_ROW[0]
+    x = (k.astype(np.float32) * step).astype(np.float32)[None, :]
+    q, s, sg, c = O.nvfp4_quantize(x, global_in=1.0, if4=True)
+    assert s[0, 0] >> 7 == IF4_ROW[4] and O.e4m3_value(int(s[0, 0]) & 0x7F) == 1.0
+    assert c["blocks_four"] == 1 and c["saturation"] == 0 and c["underflow"] == 0
+    codes = np.stack([q & 15, q >> 4], -1).ravel()
+    assert [int(O.int4_value(int(v))) for v in codes] == k.tolist()
+    assert np.array_equal(O.dequantize(q, s, O.IF4, sg), x)
+    # mixed-pair alignment: an INT4 unit over an E2M1 unit of the same scale is 6/7; two INT4
+    # operands multiply to 36/49 of the E2M1 product
+    assert abs(float(step) - IF4_ROW[5] / IF4_ROW[6]) < 2 ** -24
+    assert abs(float(step) ** 2 - IF4_ROW[7] / IF4_ROW[8]) < 2 ** -22
+
+
+def test_if4_block_on_the_e2m1_lattice_keeps_fp4():
+    """Zero E2M1 error cannot be beaten strictly, and an all-zero block is a tie: both keep E2M1
+    with the plain NVFP4 bytes and the flag clear."""
+    x = np.array([[6, 4, 3, 2, 1.5, 1, 0.5, 0, -6, -4, -3, -2, -1.5, -1, -0.5, 3],
+                  [0] * 16], dtype=np.float32)
+    q, s, sg, c = O.nvfp4_quantize(x, global_in=1.0, if4=True)
+    q0, s0, _, _ = O.nvfp4_quantize(x, global_in=1.0)
+    assert c["blocks_four"] == 0 and (s >> 7 == IF4_ROW[3]).all()
+    assert np.array_equal(q, q0) and np.array_equal(s, s0)
+    assert np.array_equal(O.dequantize(q, s, O.IF4, sg), x)
+
+
+def test_if4_saturation_and_clamped_scale():
+    """With a small caller global scale the block scale clamps at 448 and elements beyond 7 steps
+    saturate to +-7.  s_g = 2^-10 makes the step exactly 0.375 (fl(448 * fl(6/7)) = 384)."""
+    sg = 2.0 ** -10
+    step = np.float32(np.float32(448.0) * _if4_step(sg))
+    assert step == np.float32(0.375)
+    k = np.array([1, -2, 3, -4, 5, -6, 6, 5, -4, 3, -2, 1, 2, 4, 10, -12])
+    x = (k * 0.375).astype(np.float32)[None, :]
+    q, s, _, c = O.nvfp4_quantize(x, global_in=sg, if4=True)
+    assert s[0, 0] == (0x80 | 0x7E)  # INT4 flag over E4M3 448
+    assert c["saturation"] == 2 and c["underflow"] == 0 and c["blocks_four"] == 1
+    codes = np.stack([q & 15, q >> 4], -1).ravel()
+    assert [int(O.int4_value(int(v))) for v in codes] == np.clip(k, -7, 7).tolist()
+
+
+def test_if4_never_worse_than_nvfp4_and_keeps_its_fp4_blocks():
+    """Per block the IF4 error (fp64, from the reconstruction) is at most plain NVFP4's; blocks
+    that keep E2M1 carry exactly the NVFP4 nibbles and scale; INT4 blocks err by at most half a
+    step per unsaturated element; a flat distribution picks INT4 more often than a heavy-tailed
+    one, and a rotated Gaussian about as often as a plain one."""
+    rng = np.random.default_rng(12)
+    frac = {}
+    for name, x in [("uniform", rng.uniform(-1, 1, (32, 512))), ("gauss", rng.standard_normal((32, 512))),
+                    ("laplace", rng.laplace(size=(32, 512)))]:
+        x = O._f32(x)
+        q, s, sg, c = O.nvfp4_quantize(x, if4=True)
+        q0, s0, sg0, _ = O.nvfp4_quantize(x)
+        assert sg == sg0
+        flag = (s >> 7).astype(bool)
+        frac[name] = flag.mean()
+        assert c["blocks_four"] == flag.sum()
+        keep = np.repeat(~flag, 8, axis=1)
+        assert np.array_equal(q[keep], q0[keep]) and np.array_equal(s[~flag], s0[~flag])
+        assert np.array_equal(s[flag] & 0x7F, s0[flag])
+        xh = O.dequantize(q, s, O.IF4, sg).astype(np.float64)
+        xh0 = O.dequantize(q0, s0, O.NVFP4, sg0).astype(np.float64)
+        e = ((x - xh) ** 2).reshape(32, -1, 16).sum(-1)
+        e0 = ((x - xh0) ** 2).reshape(32, -1, 16).sum(-1)
+        assert (e <= e0 * (1 + 1e-5) + 1e-30).all()
+        d = np.array([O.e4m3_value(int(b) & 0x7F) for b in s.ravel()]).reshape(s.shape)
+        step = np.repeat(d * float(_if4_step(sg)), 16, axis=1)
+        fl16 = np.repeat(flag, 16, axis=1)
+        inside = fl16 & (np.abs(x) <= 7 * step)
+        assert (np.abs(x - xh)[inside] <= 0.5 * step[inside] * (1 + 2 ** -20)).all()
+    assert frac["uniform"] > frac["gauss"] > frac["laplace"] > 0
+    xr = O.fwht(O._f32(rng.standard_normal((32, 512))))
+    _, s, _, _ = O.nvfp4_quantize(xr, if4=True)
+    assert abs((s >> 7).mean() - frac["gauss"]) < 0.1
+
+
+def test_if4_nonfinite_blocks_keep_fp4():
+    x = O._f32(np.random.default_rng(13).uniform(-1, 1, (1, 48)))
+    x[0, 3], x[0, 20], x[0, 40] = np.inf, np.nan, -np.inf
+    q, s, _, c = O.nvfp4_quantize(x, global_in=1.0, if4=True)
+    assert c["nonfinite"] == 3 and (s >> 7 == 0).all()
+
+
+# ---------------------------------------------------------------------------------------------
 # Walsh-Hadamard rotation
 
 def test_fwht_norm_constant():
