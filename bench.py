@@ -350,7 +350,26 @@ def secondary(args, dev, flush, td, pk):
                 "ms": round(t, 4), "GB/s": round(bs / (t * 1e-3) / 1e9, 1),
                 "frac_hbm": round(bs / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     del gg, uu
-    
+    # IF4 (E2M1 or INT4 per block) on the headline tensor: two passes, and the quantise pass alone
+    xi = synth.nv_outliers().to(dev)
+    gi = torch.empty(1, dtype=torch.float32, device=dev)
+    fp4.nvfp4_quantize(xi, if4=True, workspace=ws)
+
+    def cif4():
+        fp4.nvfp4_quantize(xi, if4=True, workspace=ws)
+
+    ms = timed(cif4, K, W, flush, td)
+    t = statistics.median(ms)
+    gi.copy_(fp4.nvfp4_quantize(xi, workspace=ws)[2])
+    ms1 = timed(lambda: fp4.nvfp4_quantize(xi, if4=True, global_in=gi), K, W, flush, td)
+    t1 = statistics.median(ms1)
+    out.append({"workload": "IF4 quantisation (E2M1 or INT4 per 16-block) 8192x8192 bf16 outliers, two passes",
+                "ms": round(t, 4), "GB/s": round(NV_BYTES_2PASS * xi.numel() / (t * 1e-3) / 1e9, 1),
+                "quantise_pass_ms": round(t1, 4),
+                "quantise_pass_GB/s": round(NV_BYTES_1PASS * xi.numel() / (t1 * 1e-3) / 1e9, 1),
+                "quantise_pass_frac_hbm": round(NV_BYTES_1PASS * xi.numel() / (t1 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    del xi
+
     fp4_peak = 4.0 * pk["bf16_tflops"]  # dense FP4 / BF16 nominal ratio 9 / 2.25 on the measured bf16 peak
     # config 4: NVFP4 GEMM 8192^3
     A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)
@@ -425,20 +444,20 @@ def run_reference(args, rank):
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-CASES = ("nv", "nv46", "nv_amax", "mx", "fwht", "gemm_nv", "gemm_mx", "dequant")
+CASES = ("nv", "nv46", "nv_amax", "if4", "mx", "fwht", "gemm_nv", "gemm_mx", "dequant")
 
 
 def run_case(name, reps):
     """Run one kernel on its full-size workload `reps` times (for profiler captures)."""
     dev = torch.device("cuda", 0)
-    if name in ("nv", "nv46", "nv_amax"):
+    if name in ("nv", "nv46", "nv_amax", "if4"):
         x = synth.nv_outliers().to(dev)
         g = torch.tensor([0.02], device=dev)
         for _ in range(reps):
             if name == "nv_amax":
                 fp4.nvfp4_quantize(x)
             else:
-                fp4.nvfp4_quantize(x, four_six=(name == "nv46"), global_in=g)
+                fp4.nvfp4_quantize(x, four_six=(name == "nv46"), if4=(name == "if4"), global_in=g)
     elif name == "mx":
         a = synth.swiglu_act().to(dev)
         for _ in range(reps):

@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libfp4mx.so")
 
 # enums of include/fp4mx.h
 F32, BF16 = 0, 1
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, IF4 = 0, 1, 2          # fp4_format
+NV_PLAIN, NV_FOUR_SIX, NV_IF4 = 0, 1, 2  # fp4_nv_mode
 RNE, STOCHASTIC = 0, 1
 OCP_FLOOR, NOSAT_CEIL = 0, 1
 ROWMAJOR, MMA_TILED = 0, 1
@@ -131,16 +132,23 @@ def mx_quantize(x: torch.Tensor, policy: int = OCP_FLOOR, round: int = RNE, seed
     return q, s, c
 
 
+def _nv_mode(four_six: bool, if4: bool) -> int:
+    if four_six and if4:
+        raise ValueError("four_six and if4 are exclusive block modes")
+    return NV_IF4 if if4 else (NV_FOUR_SIX if four_six else NV_PLAIN)
+
+
 def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
                    layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
-                   stream=None, workspace: torch.Tensor | None = None):
-    """NVFP4: returns (q, scales, s_g float32[1] on device, counts)."""
+                   stream=None, workspace: torch.Tensor | None = None, if4: bool = False):
+    """NVFP4 (with `if4`, IF4: E2M1 or INT4 per block, flagged in scale bit 7): returns
+    (q, scales, s_g float32[1] on device, counts)."""
     _need_cuda(x, global_in)
     rows, cols = x.shape
     q, s, c = _alloc_outputs(rows, cols, 16, x.device)
     g = torch.empty(1, dtype=torch.float32, device=x.device)
     ws = workspace if workspace is not None else _workspace(OP_NVFP4_QUANTIZE, x.device, rows, cols)
-    _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, round, int(bool(four_six)), seed,
+    _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, round, _nv_mode(four_six, if4), seed,
                                 layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c), _ptr(ws),
                                 ws.numel(), _stream(stream)))
     return q, s, g, c
@@ -148,7 +156,7 @@ def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, se
 
 def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
                            layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
-                           stream=None):
+                           stream=None, if4: bool = False):
     """nvfp4_quantize for callers that cannot hand the library a device workspace: the amax word
     between the two passes lives in a fixed area of the library's own device memory.  Calls that
     overlap on the GPU share that area and must be serialised.  Returns (q, scales, s_g, counts)."""
@@ -156,7 +164,7 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = F
     rows, cols = x.shape
     q, s, c = _alloc_outputs(rows, cols, 16, x.device)
     g = torch.empty(1, dtype=torch.float32, device=x.device)
-    _check(lib().nvfp4_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, block, round, int(bool(four_six)),
+    _check(lib().nvfp4_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, block, round, _nv_mode(four_six, if4),
                                         seed, layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c),
                                         _stream(stream)))
     return q, s, g, c
@@ -171,7 +179,7 @@ def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six:
     Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
     _need_cuda(x, global_in, signs)
     rows, d = x.shape
-    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    B = block if block is not None else (32 if fmt == MXFP4 else 16)
     q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, x.device)
     g = torch.empty(1, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
     rot = torch.empty((rows, d), dtype=torch.float32, device=x.device) if want_rotated else None
@@ -195,7 +203,7 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
     if g.shape != u.shape:
         raise ValueError("g and u must have the same shape")
     rows, d = g.shape
-    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    B = block if block is not None else (32 if fmt == MXFP4 else 16)
     q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, g.device)
     gs = torch.empty(1, dtype=torch.float32, device=g.device) if fmt == NVFP4 else None
     rot = torch.empty((rows, d), dtype=torch.float32, device=g.device) if want_rotated else None
@@ -214,7 +222,7 @@ def fp4_dequantize(q: torch.Tensor, scales: torch.Tensor, fmt: int, global_scale
     """x_hat [rows, 2*q.shape[1]] in out_dtype."""
     _need_cuda(q, scales, global_scale)
     rows, half = q.shape
-    B = block if block is not None else (16 if fmt == NVFP4 else 32)
+    B = block if block is not None else (32 if fmt == MXFP4 else 16)
     out = torch.empty((rows, 2 * half), dtype=out_dtype, device=q.device)
     _check(lib().fp4_dequantize(_ptr(q), _ptr(scales), fmt, B, layout, _ptr(global_scale), rows, 2 * half,
                                 _dtype_code(out), _ptr(out), _stream(stream)))

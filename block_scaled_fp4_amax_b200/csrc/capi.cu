@@ -117,7 +117,7 @@ fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int
   if ((st = zero_counts(counts, s)) != FP4_OK) return st;
   fp4k::QuantLaunch L{};
   L.x = x; L.bf16 = dtype == FP4_BF16; L.rows = rows; L.cols = cols; L.nv = false;
-  L.policy = policy; L.sr = round == FP4_STOCHASTIC; L.four_six = false; L.seed = seed;
+  L.policy = policy; L.sr = round == FP4_STOCHASTIC; L.mode = 0; L.seed = seed;
   L.tiled = layout == FP4_SCALES_MMA_TILED; L.reverse = 0;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e = fp4k::launch_quantize(L, s);
@@ -125,12 +125,15 @@ fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int
 }
 
 fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
-                          fp4_round round, int four_six, unsigned long long seed,
+                          fp4_round round, int mode, unsigned long long seed,
                           fp4_scale_layout layout, const float* global_in, float* global_out,
                           unsigned char* q, unsigned char* scales, fp4_counts* counts,
                           void* workspace, size_t ws_bytes, void* stream) {
   fp4_status st = check_quant_common(x, dtype, rows, cols, block, 16, round, layout, q, scales);
   if (st != FP4_OK) return st;
+  if (mode != FP4_NV_PLAIN && mode != FP4_NV_FOUR_SIX && mode != FP4_NV_IF4)
+    return fail(FP4_EINVAL, "NVFP4 block mode %d unknown", mode);
+  if (mode == FP4_NV_IF4 && round != FP4_RNE) return fail(FP4_EUNSUPPORTED, "IF4 is defined with round to nearest only");
   if (!global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -148,7 +151,7 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   }
   fp4k::QuantLaunch L{};
   L.x = x; L.bf16 = dtype == FP4_BF16; L.rows = rows; L.cols = cols; L.nv = true;
-  L.policy = 0; L.sr = round == FP4_STOCHASTIC; L.four_six = four_six != 0; L.seed = seed;
+  L.policy = 0; L.sr = round == FP4_STOCHASTIC; L.mode = mode; L.seed = seed;
   L.tiled = layout == FP4_SCALES_MMA_TILED; L.reverse = global_in ? 0 : 1;
   L.global_in = global_in; L.amax_bits = amax; L.global_out = global_out;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
@@ -168,7 +171,10 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   if (d < 1024 || d > 16384 || (d & (d - 1))) return fail(FP4_EINVAL, "d = %ld must be a power of two in [1024, 16384]", d);
   fp4_status st = check_quant_common(x, dtype, rows, d, block, nv ? 16 : 32, round, layout, q, scales);
   if (st != FP4_OK) return st;
+  if (four_six != FP4_NV_PLAIN && four_six != FP4_NV_FOUR_SIX && four_six != FP4_NV_IF4)
+    return fail(FP4_EINVAL, "NVFP4 block mode %d unknown", four_six);
   if (!nv && four_six) return fail(FP4_EUNSUPPORTED, "four-over-six is defined for NVFP4 only");
+  if (four_six == FP4_NV_IF4) return fail(FP4_EUNSUPPORTED, "the rotation path has no IF4 mode");
   if (nv && !global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   if (rotated_out && !aligned(rotated_out, 16)) return fail(FP4_EINVAL, "rotated_out must be 16-byte aligned");
@@ -180,7 +186,7 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   if (!amax_pass && (st = zero_counts(counts, s)) != FP4_OK) return st;
   fp4k::FwhtLaunch L{};
   L.x = x; L.bf16 = dtype == FP4_BF16; L.rows = rows; L.d = (int)d; L.nv = nv;
-  L.sr = round == FP4_STOCHASTIC; L.four_six = nv && four_six; L.seed = seed;
+  L.sr = round == FP4_STOCHASTIC; L.four_six = nv && four_six == FP4_NV_FOUR_SIX; L.seed = seed;
   L.tiled = layout == FP4_SCALES_MMA_TILED;
   L.global_in = nv ? global_in : nullptr;
   L.amax_bits = static_cast<uint32_t*>(workspace);
@@ -223,8 +229,9 @@ fp4_status swiglu_fwht_quantize(const void* g, const void* u, fp4_dtype dtype, l
 fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, fp4_format format,
                           int block, fp4_scale_layout layout, const float* global, long rows,
                           long cols, fp4_dtype out_dtype, void* out, void* stream) {
-  if (format != FP4_MXFP4 && format != FP4_NVFP4) return fail(FP4_EINVAL, "format %d unknown", (int)format);
-  const bool nv = format == FP4_NVFP4;
+  if (format != FP4_MXFP4 && format != FP4_NVFP4 && format != FP4_IF4)
+    return fail(FP4_EINVAL, "format %d unknown", (int)format);
+  const bool nv = format != FP4_MXFP4;
   const int B = nv ? 16 : 32;
   if (block != B) return fail(FP4_EINVAL, "block %d does not match the format's block size %d", block, B);
   if (out_dtype != FP4_F32 && out_dtype != FP4_BF16) return fail(FP4_EINVAL, "out dtype %d unknown", (int)out_dtype);
@@ -235,9 +242,9 @@ fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, f
     return fail(FP4_EINVAL, "MMA-tiled scales need rows %% 128 == 0 and (cols/block) %% 4 == 0");
   if (rows == 0) return FP4_OK;
   if (!q || !scales || !out) return fail(FP4_EINVAL, "NULL q, scales or out");
-  if (nv && !global) return fail(FP4_EINVAL, "NVFP4 dequantisation needs the global scale");
+  if (nv && !global) return fail(FP4_EINVAL, "NVFP4 and IF4 dequantisation need the global scale");
   if (!aligned(q, 8) || !aligned(out, 16)) return fail(FP4_EINVAL, "q must be 8-byte and out 16-byte aligned");
-  fp4k::DequantLaunch L{q, scales, nv, layout == FP4_SCALES_MMA_TILED, nv ? global : nullptr,
+  fp4k::DequantLaunch L{q, scales, (int)format, layout == FP4_SCALES_MMA_TILED, nv ? global : nullptr,
                         rows, cols, out_dtype == FP4_BF16, out};
   cudaError_t e = fp4k::launch_dequant(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_dequantize launch");
@@ -247,6 +254,8 @@ fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K, const unsigned
                           const unsigned char* As, const float* Ag, const unsigned char* Bq,
                           const unsigned char* Bs, const float* Bg, void* C, long ldc,
                           void* workspace, size_t ws_bytes, void* stream) {
+  if (format == FP4_IF4)
+    return fail(FP4_EUNSUPPORTED, "IF4 operands have no tensor-core path (the block-scaled MMA reads E2M1 only)");
   if (format != FP4_MXFP4 && format != FP4_NVFP4) return fail(FP4_EINVAL, "format %d unknown", (int)format);
   const bool nv = format == FP4_NVFP4;
   if (M <= 0 || N <= 0 || K <= 0) return fail(FP4_EINVAL, "bad GEMM shape %d x %d x %d", M, N, K);

@@ -34,7 +34,7 @@ fp4_status noalloc_fail(fp4_status s, const char* msg) {
 }  // namespace
 
 extern "C" fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, long rows, long cols, int block,
-                                             fp4_round round, int four_six, unsigned long long seed,
+                                             fp4_round round, int mode, unsigned long long seed,
                                              fp4_scale_layout layout, const float* global_in, float* global_out,
                                              unsigned char* q, unsigned char* scales, fp4_counts* counts,
                                              void* stream) {
@@ -67,6 +67,6 @@ extern "C" fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, lon
   }
   // nvfp4_quantize zeroes the amax word on `stream` before its first pass, so the contents left by
   // the previous call do not leak into this one.
-  return nvfp4_quantize(x, dtype, rows, cols, block, round, four_six, seed, layout, global_in, global_out, q, scales,
+  return nvfp4_quantize(x, dtype, rows, cols, block, round, mode, seed, layout, global_in, global_out, q, scales,
                         counts, scratch, kNoallocScratchBytes, stream);
 }

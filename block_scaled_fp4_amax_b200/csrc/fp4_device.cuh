@@ -362,7 +362,7 @@ __device__ __forceinline__ void encode_y_n(const float* v, float R, float top, c
 #pragma unroll
     for (int i = 0; i < N; ++i) y[i] = __fmul_rn(v[i], R);
   }
-  if (CNT && top > 6.0f) {
+  if (CNT && !(top <= 6.0f)) {  // a NaN top (a NaN in the block) still counts its infinities
 #pragma unroll
     for (int i = 0; i < N; ++i) sat += fabsf(y[i]) > 6.0f;
   }
@@ -403,17 +403,18 @@ __device__ __forceinline__ uint32_t mx_sat_count_bf16x16(const uint32_t* w, int 
 }
 
 // Saturation count of 16 bf16 values (8 packed words) under the scale pair (D, R = fl(1/D)):
-// the number of values with fl(|v| * R) > 6.  The predicate is monotone in |v|, so it holds
-// exactly for |v| >= t, t the smallest bf16 magnitude that satisfies it.  6D and the real
-// threshold (6 + 2^-22) / R differ by about 2^-22 relative while one bf16 step is at least 2^-8,
-// so t is one of the three bf16 values from b0 = bf16_rd(fl(6 * D)) up, and two predicate tests
-// pick it.  The count is then 8 bf16x2 compares accumulated in bf16x2 (exact small integers).
-// Only meaningful when the block maximum saturates (fl(amax * R) > 6, so D is positive and finite).
-__device__ __forceinline__ uint32_t sat_count_bf16x16(const uint32_t* w, float D, float R) {
-  const uint32_t xb = __float_as_uint(__fmul_rn(6.0f, D)) & 0xFFFF0000u;
-  const uint32_t tb = (__fmul_rn(__uint_as_float(xb), R) > 6.0f)             ? xb
-                      : (__fmul_rn(__uint_as_float(xb + 0x10000u), R) > 6.0f) ? xb + 0x10000u
-                                                                              : xb + 0x20000u;
+// the number of values with fl(|v| * R) > lim (6 for E2M1, 7 for IF4's INT4).  The predicate is
+// monotone in |v|, so it holds exactly for |v| >= t, t the smallest bf16 magnitude that satisfies
+// it.  lim * D and the real threshold (lim + 2^-22) / R differ by about 2^-22 relative while one
+// bf16 step is at least 2^-8, so t is one of the three bf16 values from b0 = bf16_rd(fl(lim * D))
+// up, and two predicate tests pick it.  The count is then 8 bf16x2 compares accumulated in bf16x2
+// (exact small integers).  Only meaningful when the block maximum saturates (fl(amax * R) > lim,
+// so D is positive and finite).
+__device__ __forceinline__ uint32_t sat_count_bf16x16(const uint32_t* w, float D, float R, float lim = 6.0f) {
+  const uint32_t xb = __float_as_uint(__fmul_rn(lim, D)) & 0xFFFF0000u;
+  const uint32_t tb = (__fmul_rn(__uint_as_float(xb), R) > lim)             ? xb
+                      : (__fmul_rn(__uint_as_float(xb + 0x10000u), R) > lim) ? xb + 0x10000u
+                                                                             : xb + 0x20000u;
   return count_ge_bf16x16(w, (tb >> 16) | (tb & 0xFFFF0000u));
 }
 
@@ -515,6 +516,70 @@ __device__ __forceinline__ float block_sse_n(const float* sq, int lane) {
     }
   }
   return acc;
+}
+
+// ---------------------------------------------------------------------------------------------
+// IF4 ("Adaptive Block-Scaled Data Types" podcast, IF4 segment): every 16-block is encoded as
+// plain NVFP4 E2M1 and as sign-magnitude INT4 on the step D7 = fl(d * s7), s7 = fl(s_g * fl(6/7))
+// (the block maximum lands on 7 instead of 6).  INT4 is kept iff its fp32 sequential error sum is
+// strictly lower, and the choice is bit 7 of the E4M3 scale byte.
+constexpr float kSixSevenths = 0x1.b6db6ep-1f;  // fl(6/7)
+
+// Per-code INT4 step table: for every E4M3 byte c, D7 = fl(value(c) * s7) and R7 = fl(1 / D7)
+// when that is a finite nonzero number, else 0 (code 0 included).  A block whose R7 is 0 keeps
+// E2M1: its INT4 candidate has no usable step.
+__device__ __forceinline__ void fill_int4_tab(float2* tab, float s7) {
+  for (int c = threadIdx.x; c < kScaleTab; c += blockDim.x) {
+    const float D7 = __fmul_rn(e4m3_value((uint32_t)c), s7);
+    const float R7 = __frcp_rn(D7);
+    tab[c] = make_float2(D7, (fabsf(R7) < INFINITY && R7 != 0.0f) ? R7 : 0.0f);
+  }
+}
+
+// Sum over the 8 nibble positions i of (bits of 2^23) << 4i, modulo 2^32: what packing the raw
+// bit patterns of fl(a + 2^23) adds on top of the integers a.
+__host__ __device__ constexpr uint32_t int4_pack_fold() {
+  uint32_t f = 0u;
+  for (int i = 0; i < 8; ++i) f += 0x4B000000u << (4 * i);
+  return f;
+}
+
+// INT4 candidate of N values (N % 8 == 0) with step reciprocal R7, E4M3 scale value d and
+// s7: the packed sign-magnitude nibbles and the squared errors fl((x - fl(fl(k*d)*s7))^2).
+//   |k| = nearest integer to min(|fl(x * R7)|, 7), ties to even: adding 2^23 rounds a value in
+//   [0, 7] to an integer in the low mantissa bits (one ulp is 1 there), so the bit patterns pack
+//   with one shift-add per value and a constant correction (int4_pack_fold).
+//   The sign bits are those of the E2M1 candidate's nibbles (`w_e2m1`): both are the sign of
+//   fl(x * R), and R, R7 have the sign of s_g.
+//   x_hat has the sign of x (or is zero), so |x - x_hat| = |x| - |x_hat| exactly; |k| * d is exact
+//   (at most 7 significant bits).
+template <int N>
+__device__ __forceinline__ void int4_candidate_n(const float* v, float R7, float d, float s7,
+                                                 const uint32_t* w_e2m1, uint32_t* w7, float* sq) {
+  static_assert(N % 8 == 0, "whole packed words");
+  const f32x2 R2 = f2_pack(R7, R7), M2 = f2_pack(0x1p23f, 0x1p23f), d2 = f2_pack(d, d);
+#pragma unroll
+  for (int k = 0; k < N / 8; ++k) {
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const int j = 8 * k + i;
+      float y0, y1;
+      f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y0, y1);
+      const f32x2 t = f2_add(f2_pack(fminf(fabsf(y0), 7.0f), fminf(fabsf(y1), 7.0f)), M2);
+      float t0, t1;
+      f2_unpack(t, t0, t1);
+      acc += __float_as_uint(t0) << (4 * i);
+      acc += __float_as_uint(t1) << (4 * i + 4);
+      float kd0, kd1;
+      f2_unpack(f2_mul(f2_sub(t, M2), d2), kd0, kd1);
+      const float e0 = __fsub_rn(fabsf(v[j]), __fmul_rn(kd0, s7));
+      const float e1 = __fsub_rn(fabsf(v[j + 1]), __fmul_rn(kd1, s7));
+      sq[j] = __fmul_rn(e0, e0);
+      sq[j + 1] = __fmul_rn(e1, e1);
+    }
+    w7[k] = (acc - int4_pack_fold()) | (w_e2m1[k] & 0x88888888u);
+  }
 }
 
 // ---------------------------------------------------------------------------------------------

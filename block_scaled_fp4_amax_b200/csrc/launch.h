@@ -37,7 +37,7 @@ struct QuantLaunch {
   bool nv;        // NVFP4 (block 16, E4M3) vs MXFP4 (block 32, E8M0)
   int policy;     // MXFP4 exponent rule
   bool sr;        // stochastic rounding
-  bool four_six;  // NVFP4 4/6
+  int mode;       // NVFP4 block mode: 0 plain, 1 four-over-six, 2 IF4
   unsigned long long seed;
   int tiled;      // scale layout
   int reverse;    // walk tiles last-to-first
@@ -53,7 +53,7 @@ struct QuantLaunch {
 struct DequantLaunch {
   const uint8_t* q;
   const uint8_t* scales;
-  bool nv;
+  int format;     // 0 MXFP4, 1 NVFP4, 2 IF4
   int tiled;
   const float* global;
   long long rows, cols;

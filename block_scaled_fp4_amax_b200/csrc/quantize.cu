@@ -23,15 +23,20 @@ namespace fp4k {
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;      // 32-byte chunks in flight per lane
-constexpr int kUnroll46 = 2;    // four-over-six: compute-bound, so a smaller body is worth more
+constexpr int kUnroll46 = 2;    // four-over-six and IF4: compute-bound, so a smaller body is worth more
+
+// NVFP4 block modes: plain, four-over-six, IF4 (E2M1 or INT4 per block)
+constexpr int kPlain = 0, kFourSix = 1, kIF4 = 2;
 
 // ---------------------------------------------------------------------------------------------
 // MXFP4 shared exponent from the amax bit pattern (exact): OCP floor(log2 amax) - 2, or the
-// smallest e with amax <= 6 * 2^e; clamped to [-127, 127]; an all-zero block takes e = 0.
+// smallest e with amax <= 6 * 2^e; clamped to [-127, 127]; an all-zero block takes e = 0.  A
+// non-finite maximum (Inf or NaN: exponent field 255) counts as 2^128, e = 126 under both rules.
 __device__ __forceinline__ int mx_exponent(uint32_t bits, int policy) {
   const int ef = (int)((bits >> 23) & 0xFFu);
   if (bits == 0u) return 0;
   if (ef == 0) return -127;  // subnormal maximum: below 2^-126, clamps
+  if (ef == 255) return 126;
   const int E = ef - 127;
   const int e = (policy == 0) ? E - 2 : (((bits & 0x7FFFFFu) <= 0x400000u) ? E - 2 : E - 1);
   return e < -127 ? -127 : e;
@@ -103,13 +108,15 @@ __device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, boo
   return sse4 < sse6 ? 1u : 0u;
 }
 
-template <typename T, bool NV, bool SR, bool FOUR_SIX>
+template <typename T, bool NV, bool SR, int MODE>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
+  constexpr bool FOUR_SIX = MODE == kFourSix;
+  constexpr bool IF4 = MODE == kIF4;
   constexpr int E = Vec32<T>::E;  // 16 (bf16) or 8 (fp32)
   constexpr int B = NV ? 16 : 32;
   constexpr int G = B / E;
   constexpr int W = E / 8;        // packed words per chunk
-  constexpr int U = FOUR_SIX ? kUnroll46 : kUnroll;
+  constexpr int U = MODE != kPlain ? kUnroll46 : kUnroll;
   constexpr bool kBF = E == 16;   // bf16 input: saturations counted with bf16x2 compares
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
@@ -120,10 +127,16 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
 
   NvScale ns{1.0f, 1.0f, 1.0f};
   __shared__ float2 tab[NV ? kScaleTab : 1];
+  __shared__ float2 tab7[IF4 ? kScaleTab : 1];
+  float s7 = 0.0f;
   if (NV) {
     ns = nv_scales(p.global_in, p.amax_bits, p.six_m);
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = ns.s_g;
     fill_scale_tab(tab, ns.s_g);
+    if (IF4) {
+      s7 = __fmul_rn(ns.s_g, kSixSevenths);
+      fill_int4_tab(tab7, s7);
+    }
     __syncthreads();
   }
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};  // underflow, saturation, nonfinite, blocks_four
@@ -174,9 +187,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
             const uint32_t n = mx_sat_count_bf16x16(raw[u].w, e);
             sat = top > 6.0f ? n : 0u;
           } else {
+            // a NaN top (a NaN in the block, e = 126) still counts the block's infinities
             const float D = __uint_as_float(e > -127 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
             const uint32_t n = sat_count_bf16x16(raw[u].w, D, inv);
-            sat = top > 6.0f ? n : 0u;
+            sat = !(top <= 6.0f) ? n : 0u;
           }
         }
         sc = (uint32_t)(e + 127);
@@ -186,6 +200,31 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         if constexpr (kBF) {
           const uint32_t n = sat_count_bf16x16(raw[u].w, DR.x, DR.y);
           sat = __fmul_rn(amax, DR.y) > 6.0f ? n : 0u;
+        }
+        if constexpr (IF4) {
+          // both candidates' exact error sums (fp32, element order), INT4 kept iff strictly lower
+          float sq[E];
+          sq_errors_n<E>(v, w, sc, ns.s_g, p.zero, sq);
+          const float sse6 = block_sse_n<E, G>(sq, lane);
+          const float2 DR7 = tab7[sc];
+          uint32_t w7[W];
+          int4_candidate_n<E>(v, DR7.y, e4m3_value(sc), s7, w, w7, sq);
+          const float sse7 = block_sse_n<E, G>(sq, lane);
+          if (DR7.y != 0.0f && sse7 < sse6) {
+            sc |= 0x80u;
+            four = 1;
+            sat = 0;
+            if (__fmul_rn(amax, DR7.y) > 7.0f) {
+              if constexpr (kBF) {
+                sat = sat_count_bf16x16(raw[u].w, DR7.x, DR7.y, 7.0f);
+              } else {
+#pragma unroll
+                for (int i = 0; i < E; ++i) sat += fabsf(__fmul_rn(v[i], DR7.y)) > 7.0f;
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < W; ++k) w[k] = w7[k];
+          }
         }
       } else {
         float D6, D4, A6, A4, R6, R4;
@@ -289,29 +328,44 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long
 
 // ---------------------------------------------------------------------------------------------
 // Dequantiser: each lane expands 8 packed bytes (16 values).  x_hat = fl(fl(v*d)*s_g) (NVFP4) or
-// v * 2^(byte-127) (MXFP4, exact).  bf16 output is the RNE cast of the fp32 value.
-template <bool NV, bool OUT_BF16>
+// v * 2^(byte-127) (MXFP4, exact); IF4 blocks whose scale byte has bit 7 set hold INT4 nibbles,
+// x_hat = fl(fl(k*d)*s7) with d from the low 7 bits and s7 = fl(s_g * fl(6/7)).  bf16 output is
+// the RNE cast of the fp32 value.
+template <int FMT, bool OUT_BF16>  // FMT: 0 MXFP4, 1 NVFP4, 2 IF4
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, const uint8_t* scales,
                                                            const float* global, long long n_groups,
                                                            DivU32 nb, int tiled, void* out) {
+  constexpr bool NV = FMT != 0;
   constexpr int B = NV ? 16 : 32;
   const float s_g = NV ? *global : 1.0f;
+  const float s7 = FMT == 2 ? __fmul_rn(s_g, kSixSevenths) : 0.0f;
   const long long stride = (long long)gridDim.x * kThreads;
   for (long long g = (long long)blockIdx.x * kThreads + threadIdx.x; g < n_groups; g += stride) {
     const uint2 w = *reinterpret_cast<const uint2*>(q + g * 8);
     const unsigned long long blk = (unsigned long long)(g * 16) / B;
     const uint8_t sb = scales[scale_offset(blk, nb, tiled)];
+    const bool int4 = FMT == 2 && (sb & 0x80u);
     float d;
-    if (NV) d = e4m3_value(sb);
+    if (NV) d = e4m3_value(FMT == 2 ? (sb & 0x7Fu) : sb);
     else d = __uint_as_float((uint32_t)sb << 23);  // 2^(sb-127); sb = 0 -> 0 (handled below)
     float v[16];
-    e2m1_unpack<8>(w.x, v);
-    e2m1_unpack<8>(w.y, v + 8);
+    if (int4) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t c = ((i < 8 ? w.x : w.y) >> (4 * (i & 7))) & 15u;
+        const float m = (float)(c & 7u);
+        v[i] = (c & 8u) ? -m : m;
+      }
+    } else {
+      e2m1_unpack<8>(w.x, v);
+      e2m1_unpack<8>(w.y, v + 8);
+    }
+    const float sf = int4 ? s7 : s_g;
     float o[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       if (NV) {
-        o[i] = __fmul_rn(__fmul_rn(v[i], d), s_g);
+        o[i] = __fmul_rn(__fmul_rn(v[i], d), sf);
       } else if (sb != 0) {
         o[i] = __fmul_rn(v[i], d);
       } else {
@@ -343,29 +397,31 @@ static int grid_for(long long work_items, int per_cta) {
 }
 
 // One wave of resident CTAs (the kernel loops over tiles), so no CTA waits in a tail wave.
-template <typename T, bool NV, bool SR, bool FS>
+template <typename T, bool NV, bool SR, int MODE>
 static cudaError_t launch_q(const QuantParams& p, bool pdl, cudaStream_t s) {
   static int per_sm = 0;  // resident CTAs per SM for this instantiation (same on every sm_100 device)
   if (per_sm == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<T, NV, SR, FS>, kThreads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quantize_kernel<T, NV, SR, MODE>, kThreads, 0) != cudaSuccess ||
         n < 1)
       n = 1;
     per_sm = n;
   }
-  constexpr int U = FS ? kUnroll46 : kUnroll;
+  constexpr int U = MODE != kPlain ? kUnroll46 : kUnroll;
   const long long tiles = (p.n_chunks + 32LL * U - 1) / (32LL * U);
   const long long want = (tiles * 32 + kThreads - 1) / kThreads;
   const long long cap = (long long)num_sms() * per_sm;
   const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
-  return launch_pdl(quantize_kernel<T, NV, SR, FS>, dim3(grid), dim3(kThreads), 0, s, pdl, p);
+  return launch_pdl(quantize_kernel<T, NV, SR, MODE>, dim3(grid), dim3(kThreads), 0, s, pdl, p);
 }
 
 template <typename T>
-static cudaError_t dispatch_q(const QuantParams& p, bool nv, bool sr, bool fs, bool pdl, cudaStream_t s) {
-  if (!nv) return sr ? launch_q<T, false, true, false>(p, pdl, s) : launch_q<T, false, false, false>(p, pdl, s);
-  if (fs) return sr ? launch_q<T, true, true, true>(p, pdl, s) : launch_q<T, true, false, true>(p, pdl, s);
-  return sr ? launch_q<T, true, true, false>(p, pdl, s) : launch_q<T, true, false, false>(p, pdl, s);
+static cudaError_t dispatch_q(const QuantParams& p, bool nv, bool sr, int mode, bool pdl, cudaStream_t s) {
+  if (!nv) return sr ? launch_q<T, false, true, kPlain>(p, pdl, s) : launch_q<T, false, false, kPlain>(p, pdl, s);
+  if (mode == kIF4) return launch_q<T, true, false, kIF4>(p, pdl, s);  // round to nearest only
+  if (mode == kFourSix)
+    return sr ? launch_q<T, true, true, kFourSix>(p, pdl, s) : launch_q<T, true, false, kFourSix>(p, pdl, s);
+  return sr ? launch_q<T, true, true, kPlain>(p, pdl, s) : launch_q<T, true, false, kPlain>(p, pdl, s);
 }
 
 cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
@@ -382,13 +438,13 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   p.global_in = L.global_in;
   p.amax_bits = L.amax_bits;
   p.global_out = L.global_out;
-  p.six_m = L.four_six ? 1536.0f : 2688.0f;
+  p.six_m = L.mode == kFourSix ? 1536.0f : 2688.0f;
   p.q = L.q;
   p.scales = L.scales;
   p.counts = L.counts;
   if (p.n_chunks == 0) return cudaSuccess;
-  return L.bf16 ? dispatch_q<__nv_bfloat16>(p, L.nv, L.sr, L.four_six, L.pdl, s)
-                : dispatch_q<float>(p, L.nv, L.sr, L.four_six, L.pdl, s);
+  return L.bf16 ? dispatch_q<__nv_bfloat16>(p, L.nv, L.sr, L.mode, L.pdl, s)
+                : dispatch_q<float>(p, L.nv, L.sr, L.mode, L.pdl, s);
 }
 
 cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
@@ -404,14 +460,16 @@ cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* a
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s) {
   const long long groups = L.rows * L.cols / 16;
   if (groups == 0) return cudaSuccess;
-  const DivU32 nb = make_divu32((uint32_t)(L.cols / (L.nv ? 16 : 32)));
+  const DivU32 nb = make_divu32((uint32_t)(L.cols / (L.format != 0 ? 16 : 32)));
   const int grid = grid_for(groups, kThreads);
-  if (L.nv) {
-    if (L.out_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(L.q, L.scales, L.global, groups, nb, L.tiled, L.out);
-    else dequant_kernel<true, false><<<grid, kThreads, 0, s>>>(L.q, L.scales, L.global, groups, nb, L.tiled, L.out);
+  const float* gl = L.format != 0 ? L.global : nullptr;
+  auto go = [&](auto kernel) { kernel<<<grid, kThreads, 0, s>>>(L.q, L.scales, gl, groups, nb, L.tiled, L.out); };
+  if (L.format == 2) {
+    if (L.out_bf16) go(dequant_kernel<2, true>); else go(dequant_kernel<2, false>);
+  } else if (L.format == 1) {
+    if (L.out_bf16) go(dequant_kernel<1, true>); else go(dequant_kernel<1, false>);
   } else {
-    if (L.out_bf16) dequant_kernel<false, true><<<grid, kThreads, 0, s>>>(L.q, L.scales, nullptr, groups, nb, L.tiled, L.out);
-    else dequant_kernel<false, false><<<grid, kThreads, 0, s>>>(L.q, L.scales, nullptr, groups, nb, L.tiled, L.out);
+    if (L.out_bf16) go(dequant_kernel<0, true>); else go(dequant_kernel<0, false>);
   }
   return cudaGetLastError();
 }

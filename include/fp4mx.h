@@ -51,8 +51,21 @@ typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
 
 /* MXFP4: 32 E2M1 elements share one E8M0 byte (value 2^(byte-127), 0xFF = NaN, never produced).
  * NVFP4: 16 E2M1 elements share one E4M3 byte (positive, OCP E4M3FN: bias 7, max 448) under one
- *        FP32 per-tensor global scale s_g.   [E] §2, [P] block-scaling segment. */
-typedef enum fp4_format { FP4_MXFP4 = 0, FP4_NVFP4 = 1 } fp4_format;
+ *        FP32 per-tensor global scale s_g.   [E] §2, [P] block-scaling segment.
+ * IF4:   NVFP4 whose blocks may instead hold INT4: a scale byte with bit 7 set (the sign bit NVFP4
+ *        never uses) marks a block of sign-magnitude integers k in -7..7 (bit 3 the sign, bits 0-2
+ *        |k|) with value k * d * s7, d the E4M3 value of the low 7 bits, s7 = fl(s_g * fl(6/7)).
+ *        Written by nvfp4_quantize with FP4_NV_IF4; read by fp4_dequantize.  [P] IF4 segment. */
+typedef enum fp4_format { FP4_MXFP4 = 0, FP4_NVFP4 = 1, FP4_IF4 = 2 } fp4_format;
+
+/* NVFP4 block mode (the `mode` argument of the NVFP4 quantisers).
+ * PLAIN   : every block scales its maximum to 6.
+ * FOUR_SIX: each block also tries a maximum of 4 and keeps the lower-error one ([P] Four Over
+ *           Six segment); the global scale uses M = 256.
+ * IF4     : each block also tries INT4 on the step 6/7 of the E2M1 unit and keeps the lower-error
+ *           one, flagged in scale bit 7 (format FP4_IF4; [P] IF4 segment); M = 448, round to
+ *           nearest only. */
+typedef enum fp4_nv_mode { FP4_NV_PLAIN = 0, FP4_NV_FOUR_SIX = 1, FP4_NV_IF4 = 2 } fp4_nv_mode;
 
 /* RNE: round to nearest on the E2M1 lattice {0,.5,1,1.5,2,3,4,6}, an exact tie takes the code with
  * the even mantissa bit ([A] "Read the FP4 E2M1 value lattice").
@@ -82,8 +95,9 @@ typedef enum fp4_scale_layout { FP4_SCALES_ROWMAJOR = 0, FP4_SCALES_MMA_TILED = 
 
 /* Encoding counters, tensor totals.  Lives in DEVICE memory; every quantize call zeroes it on its
  * stream before counting.  underflow: nonzero source whose code is +-0.  saturation: normalised
- * magnitude strictly above 6 (clamped to +-6).  nonfinite: Inf/NaN source elements.
- * blocks_four: NVFP4 4/6 blocks that chose the max->4 scaling.  Counts come from the chosen
+ * magnitude strictly above 6 (clamped to +-6), an infinite one included.  nonfinite: Inf/NaN source elements.
+ * blocks_four: blocks that took the alternative candidate: the max->4 scaling under FOUR_SIX,
+ * INT4 under IF4 (whose saturation bound is 7 integer steps).  Counts come from the chosen
  * encoding only.  [A] "Read the FP4 E2M1 value lattice", "Expose outlier and dead-zone damage". */
 typedef struct fp4_counts {
   unsigned long long underflow;
@@ -115,13 +129,20 @@ FP4_API fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long c
 
 /* ---------------------------------------------------------------------------------------------
  * nvfp4_quantize — NVFP4 two-level quantisation, blocks of 16 along rows.  [E] §2, [P] Four Over
- * Six segment.  Global scale s_g = fl(amax_t / (6*M)) with M = 448 (M = 256 when four_six != 0,
- * the reduced global range that keeps the max->4 candidate finite); s_g = 1 when amax_t == 0.
- * For target T (6, and also 4 under four_six): inv_T = fl(1/fl(T*s_g)); block code =
+ * Six and IF4 segments.  Global scale s_g = fl(amax_t / (6*M)) with M = 448 (M = 256 under
+ * FP4_NV_FOUR_SIX, the reduced global range that keeps the max->4 candidate finite); s_g = 1 when
+ * amax_t == 0.  For target T (6, and also 4 under FOUR_SIX): inv_T = fl(1/fl(T*s_g)); block code =
  * E4M3_RNE_satfinite(fl(amax_b * inv_T)) with decoded value d; elements y = fl(x * fl(1/fl(d*s_g)))
- * are E2M1-encoded; a code of 0 encodes the whole block as signed zeros.  Under four_six each block
+ * are E2M1-encoded; a code of 0 encodes the whole block as signed zeros.  Under FOUR_SIX each block
  * keeps the candidate whose fp32 sum of squared dequantisation errors is strictly lower (ties
- * keep 6).
+ * keep 6).  Under FP4_NV_IF4 the T = 6 block also gets an INT4 candidate: D7 = fl(d * s7),
+ * s7 = fl(s_g * fl(6/7)), R7 = fl(1/D7); |k| = nearest integer (ties to even) to
+ * min(|fl(x * R7)|, 7), the sign that of fl(x * R7); reconstruction fl(fl(k*d) * s7).  It is kept,
+ * with scale bit 7 set, iff R7 is a finite nonzero number and its fp32 sequential error sum is
+ * strictly below the E2M1 one (ties and NaN keep E2M1).  IF4 assumes s_g > 0: a caller-supplied
+ * negative global scale gives in-bounds but unspecified bytes.
+ *   mode       : fp4_nv_mode (0, 1 or 2; other values are FP4_EINVAL); FP4_NV_IF4 with
+ *                FP4_STOCHASTIC is FP4_EUNSUPPORTED.
  *   global_in  : device float or NULL.  NULL: a first pass reduces amax_t over the tensor (two
  *                passes over x).  Non-NULL: the caller fixes s_g = *global_in (one pass).
  *   global_out : device float or NULL; receives the s_g used.
@@ -130,7 +151,7 @@ FP4_API fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long c
  *                aligned; required when global_in == NULL.  Clobbered.
  * Preconditions: block == 16, cols % 16 == 0. */
 FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
-                          fp4_round round, int four_six, unsigned long long seed,
+                          fp4_round round, int mode, unsigned long long seed,
                           fp4_scale_layout layout, const float* global_in, float* global_out,
                           unsigned char* q, unsigned char* scales, fp4_counts* counts,
                           void* workspace, size_t ws_bytes, void* stream);
@@ -152,7 +173,8 @@ FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, lon
  *   d           : power of two, 1024 <= d <= 16384.
  *   signs       : device uint32 [d / 32], 4-byte aligned, or NULL (plain rotation); caller-owned.
  *   rotated_out : device float [rows, d] or NULL; receives the rotated values (diagnostics).
- *   other arguments as in nvfp4_quantize; four_six and global_in/out apply to FP4_NVFP4 only. */
+ *   other arguments as in nvfp4_quantize; four_six (FP4_NV_PLAIN or FP4_NV_FOUR_SIX; FP4_NV_IF4
+ *   is FP4_EUNSUPPORTED here) and global_in/out apply to FP4_NVFP4 only. */
 FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d,
                          const unsigned int* signs, fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,
@@ -181,11 +203,13 @@ FP4_API fp4_status swiglu_fwht_quantize(const void* g, const void* u, fp4_dtype 
 
 /* ---------------------------------------------------------------------------------------------
  * fp4_dequantize — x_hat = fl((v * d) * s_g) per element, v the E2M1 value of the nibble and d the
- * decoded block scale (v*d is exact); MXFP4 has no s_g (x_hat = v * 2^e, exact).  bf16 output is
+ * decoded block scale (v*d is exact); MXFP4 has no s_g (x_hat = v * 2^e, exact).  FP4_IF4 (block
+ * 16): a block whose scale byte has bit 7 set is INT4, x_hat = fl((k * d) * s7) with d the E4M3
+ * value of the low 7 bits and s7 = fl(s_g * fl(6/7)); other blocks follow NVFP4.  bf16 output is
  * the round-to-nearest-even of that fp32 value.  [A] "Encode one MXFP4 block step by step"
- * (reconstruction = lattice value times scale), [X] block scales applied in FP32.
+ * (reconstruction = lattice value times scale), [X] block scales applied in FP32, [P] IF4 segment.
  *   q, scales : device, as written by the quantisers (`layout` names the scale layout).
- *   global    : device float, NVFP4 only (NULL for MXFP4).
+ *   global    : device float, NVFP4 and IF4 only (NULL for MXFP4).
  *   out       : device [rows, cols] of out_dtype, 16-byte aligned. */
 FP4_API fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, fp4_format format,
                           int block, fp4_scale_layout layout, const float* global, long rows,
@@ -206,7 +230,8 @@ FP4_API fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* s
  *               kernel's status word (0 = ok, nonzero = a bounded pipeline wait gave up) is its
  *               first 4 bytes; see fp4_gemm_status_word.
  * Preconditions: M % 128 == 0, N % 256 == 0, K % 256 == 0, ldc >= N, ldc % 8 == 0, all pointers
- * 16-byte aligned.  Other shapes return FP4_EUNSUPPORTED. */
+ * 16-byte aligned.  Other shapes return FP4_EUNSUPPORTED, as does FP4_IF4 (the block-scaled MMA
+ * reads E2M1 only; dequantise IF4 operands first). */
 FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
                           const unsigned char* Aq, const unsigned char* As, const float* Ag,
                           const unsigned char* Bq, const unsigned char* Bs, const float* Bg,
@@ -229,7 +254,7 @@ FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
  *   amax word is zeroed on `stream` at the start of each call.  Calls that overlap on the GPU (in
  *   flight at the same time on different streams) race on it: serialise them. */
 FP4_API fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, long rows, long cols, int block,
-                                          fp4_round round, int four_six, unsigned long long seed,
+                                          fp4_round round, int mode, unsigned long long seed,
                                           fp4_scale_layout layout, const float* global_in, float* global_out,
                                           unsigned char* q, unsigned char* scales, fp4_counts* counts,
                                           void* stream);

@@ -54,8 +54,10 @@ static int e2m1_nearest_mag(double a) {
 
 /* RNE encode of a normalised value y.  Magnitudes strictly above 6 clamp to 6 ([A]: "the lab
  * clamps them to signed 6").  The sign bit always follows signbit(y), so a negative value that
- * rounds to zero encodes -0 (0x8).  Returns the 4-bit code. */
+ * rounds to zero encodes -0 (0x8).  E2M1 has no NaN ([E] §1); reading: a NaN encodes as +6 (0x7),
+ * its sign carrying no meaning.  Returns the 4-bit code. */
 int ora_e2m1_encode_rne(float y) {
+  if (isnan(y)) return 7;
   double a = fabs((double)y);
   int mag = (a > 6.0) ? 7 : e2m1_nearest_mag(a);
   return (signbit(y) ? 8 : 0) | mag;
@@ -102,6 +104,7 @@ uint32_t ora_sr_word(uint64_t seed, uint64_t idx) {
  * lattice magnitudes (lo = a when a is a lattice point); p = (a-lo)/(hi-lo) is exact; the value
  * rounds up iff r < ceil(p * 2^32).  a > 6 clamps to 6 (saturation, as for RNE).             */
 int ora_e2m1_encode_sr(float y, uint32_t r) {
+  if (isnan(y)) return 7; /* as for RNE */
   double a = fabs((double)y);
   int sign = signbit(y) ? 8 : 0;
   if (a > 6.0) return sign | 7;
@@ -129,8 +132,10 @@ double ora_e4m3_value(int code) {
 }
 
 /* Round-to-nearest-even onto the positive E4M3 lattice, saturating to 448 (the "satfinite"
- * reading: a magnitude above 448 becomes 448, never NaN).  u >= 0.  Ties take the even code.   */
+ * reading: a magnitude above 448, Inf included, becomes 448).  u >= 0.  Ties take the even code.
+ * A NaN u (a block holding a NaN) gives E4M3's NaN byte 0x7F, so the block decodes to NaN.   */
 int ora_e4m3_encode_rne_satfinite(float u) {
+  if (isnan(u)) return 0x7F;
   double a = (double)u;
   if (!(a <= 448.0)) return 0x7E;
   int best = 0;
@@ -169,8 +174,11 @@ static int floor_log2(double a) { /* a > 0 finite: exact via frexp (a = f * 2^x,
   return x - 1;
 }
 
+/* A non-finite block maximum (a block holding Inf or NaN) counts as 2^128, just above every
+ * float: e = 126 under both rules (reading; the pages leave non-finite input open).          */
 int ora_mx_exponent(float amax, int policy) {
   if (amax == 0.0f) return 0;
+  if (!isfinite(amax)) return 126;
   double a = (double)amax;
   int e;
   if (policy == 0) {
@@ -195,17 +203,20 @@ void ora_mx_encode_block(const float* x, int n, int e, int round, uint64_t seed,
     if (!isfinite(x[i])) cnt->nonfinite += 1;
     float y = x[i] * inv_scale;
     int c = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
-    if (isfinite(y) && fabsf(y) > 6.0f) cnt->saturation += 1;
+    if (fabsf(y) > 6.0f) cnt->saturation += 1; /* Inf included, NaN not */
     if (x[i] != 0.0f && (c & 7) == 0) cnt->underflow += 1;
     codes[i] = (uint8_t)c;
   }
 }
 
+/* Largest magnitude of n values; a NaN anywhere makes it NaN (the IEEE maximum that propagates
+ * NaN, as torch.amax does).                                                                    */
 static float block_amax(const float* x, int n) {
   float m = 0.0f;
   for (int i = 0; i < n; ++i) {
     float a = fabsf(x[i]);
-    if (a > m) m = a;
+    if (isnan(a) || a > m) m = a;
+    if (isnan(m)) break;
   }
   return m;
 }
@@ -281,7 +292,7 @@ static float nv_candidate(const float* x, int n, float amax_b, float s_g, float 
     for (int i = 0; i < n; ++i) {
       float y = x[i] * R;
       int code = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
-      if (isfinite(y) && fabsf(y) > 6.0f) c->saturation += 1;
+      if (fabsf(y) > 6.0f) c->saturation += 1; /* Inf included, NaN not */
       if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
       codes[i] = (uint8_t)code;
     }
@@ -320,8 +331,10 @@ double ora_int4_value(int code) {
 }
 
 /* Nearest of the integers 0..7 to |y| (ties to the even one), by enumerating the lattice; a
- * magnitude above 7, Inf included, clamps to 7.  The sign bit follows signbit(y).             */
+ * magnitude above 7, Inf included, clamps to 7.  The sign bit follows signbit(y); a NaN gives +7
+ * (as E2M1 gives +6).                                                                          */
 int ora_int4_encode_rne(float y) {
+  if (isnan(y)) return 7;
   double a = fabs((double)y);
   int best = 7;
   if (!(a > 7.0)) {
@@ -350,7 +363,7 @@ static float if4_int_candidate(const float* x, int n, int sc, float s_g, uint8_t
   for (int i = 0; i < n; ++i) {
     float y = x[i] * R7;
     int code = ora_int4_encode_rne(y);
-    if (isfinite(y) && fabsf(y) > 7.0f) c->saturation += 1;
+    if (fabsf(y) > 7.0f) c->saturation += 1; /* Inf included, NaN not */
     if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
     codes[i] = (uint8_t)code;
   }
@@ -377,10 +390,11 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mod
   if (global_in) {
     s_g = *global_in;
   } else {
-    float amax_t = 0.0f;
+    float amax_t = 0.0f; /* NaN-propagating maximum, as block_amax */
     for (long i = 0; i < rows * cols; ++i) {
       float a = fabsf(x[i]);
-      if (a > amax_t) amax_t = a;
+      if (isnan(a) || a > amax_t) amax_t = a;
+      if (isnan(amax_t)) break;
     }
     s_g = ora_nvfp4_global_scale(amax_t, mode == 1);
   }

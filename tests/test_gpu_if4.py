@@ -1,0 +1,96 @@
+"""GPU parity of IF4 (podcast "Adaptive Block-Scaled Data Types for FP4 Training", IF4 segment):
+per 16-block E2M1 or sign-magnitude INT4, the choice in the scale byte's bit 7.
+
+Bar: nibbles, scale bytes (flag included), the global scale and all counters bit-exact; the
+dequantised values bit-exact.  The choice compares exact fp32 error sums on both sides, so the
+near-tie inputs below only pass if the kernel takes every fp32 step in the oracle's order.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp4_amax_b200 as fp4
+import oracle as O
+from block_scaled_fp4_amax_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def npy(t):
+    return t.detach().cpu().numpy()
+
+
+def counts_of(c):
+    v = [int(x) for x in c.cpu().tolist()]
+    return dict(underflow=v[0], saturation=v[1], nonfinite=v[2], blocks_four=v[3])
+
+
+def run_if4(x_cpu, cuda, layout=fp4.ROWMAJOR, global_in=None, dequant=True):
+    gin = None if global_in is None else torch.tensor([global_in], dtype=torch.float32, device=cuda)
+    q, s, g, c = fp4.nvfp4_quantize(x_cpu.to(cuda), if4=True, layout=layout, global_in=gin)
+    x = synth.as_f32_numpy(x_cpu)
+    qo, so, go, co = O.nvfp4_quantize(x, if4=True, global_in=global_in)
+    assert np.array_equal(np.float32(npy(g)[0]), np.float32(go), equal_nan=True)
+    assert np.array_equal(npy(q), qo)
+    want_s = O.scales_to_mma_tiled(so) if layout == fp4.MMA_TILED else so.ravel()
+    assert np.array_equal(npy(s), want_s)
+    assert counts_of(c) == co
+    if dequant:
+        ref = O.dequantize(qo, so, O.IF4, go)
+        out = fp4.fp4_dequantize(q, s, fp4.IF4, g, layout=layout)
+        assert np.array_equal(npy(out), ref, equal_nan=True)
+        outb = fp4.fp4_dequantize(q, s, fp4.IF4, g, layout=layout, out_dtype=torch.bfloat16)
+        want = torch.from_numpy(ref).to(torch.bfloat16)
+        assert np.array_equal(npy(outb.float()), npy(want.float()), equal_nan=True)
+    return co
+
+
+def int4_lattice(rows, cols, seed):
+    """Values k * fl(6/7) (the INT4 step of scale 1 under s_g = 1), k uniform in -7..7, one |k| = 7
+    per block so each block's scale is exactly 1."""
+    rng = np.random.default_rng(seed)
+    k = rng.integers(-7, 8, size=(rows, cols))
+    k[:, ::16] = np.where(rng.random((rows, cols // 16)) < 0.5, -7, 7)
+    step = np.float32(6.0) / np.float32(7.0)
+    return torch.from_numpy((k.astype(np.float32) * step).astype(np.float32))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("layout", [fp4.ROWMAJOR, fp4.MMA_TILED])
+def test_if4_outliers_small(cuda, dtype, layout):
+    x = synth.nv_outliers(384, 2048, seed=5)
+    co = run_if4(x if dtype == torch.bfloat16 else x.float(), cuda, layout=layout)
+    assert 0 < co["blocks_four"] < 384 * 2048 // 16
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_if4_near_ties_and_distributions(cuda, dtype):
+    cast = (lambda t: t.to(torch.bfloat16)) if dtype == torch.bfloat16 else (lambda t: t.float())
+    rng = np.random.default_rng(21)
+    run_if4(cast(synth.lattice_steps(512, 1024, 41)), cuda)
+    run_if4(cast(synth.lattice_steps(256, 1024, 42, denom=7, kmax=49)), cuda, global_in=1.0 / 256)
+    run_if4(cast(torch.from_numpy(rng.uniform(-1, 1, (256, 1024)).astype(np.float32))), cuda)
+    run_if4(cast(torch.from_numpy(rng.laplace(size=(256, 1024)).astype(np.float32))), cuda)
+    co = run_if4(int4_lattice(128, 1024, 22).float(), cuda, global_in=1.0)
+    assert co["blocks_four"] > 0.9 * 128 * 1024 // 16
+
+
+def test_if4_edges(cuda):
+    run_if4(synth.normal_bf16(5, 48, 31), cuda)                              # ragged: 5 rows, 3 blocks
+    run_if4(synth.normal_bf16(5, 48, 31), cuda, global_in=0.001)
+    run_if4(synth.normal_bf16(256, 512, 32), cuda, global_in=1e-4)           # clamped scales, saturation
+    run_if4(synth.normal_bf16(64, 256, 33), cuda, global_in=1e-30)           # tiny step, still normal
+    run_if4(torch.zeros(64, 64), cuda)                                       # amax 0 -> s_g = 1, all ties
+    x = synth.normal_f32(64, 256, 34)
+    x[3, 5], x[10, 100], x[63, 255] = float("inf"), float("nan"), float("-inf")
+    co = run_if4(x, cuda, global_in=0.01)                                    # non-finite blocks keep E2M1
+    assert co["nonfinite"] == 3 and co["blocks_four"] > 0
+    co = run_if4(x, cuda)                                                    # NaN global scale
+    assert co["blocks_four"] == 0
+    x = synth.normal_f32(64, 256, 35) * 1e-38                               # subnormal inputs
+    run_if4(x, cuda)
+
+
+def test_if4_full_outliers(cuda):
+    """8192 x 8192 bf16 N(0,1) with 8 outlier columns x U(50,100), seed 5, two-pass global scale."""
+    run_if4(synth.nv_outliers(), cuda, dequant=False)

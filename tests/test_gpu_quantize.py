@@ -49,7 +49,7 @@ def run_nv(x_cpu, cuda, rnd=fp4.RNE, four_six=False, seed=0, layout=fp4.ROWMAJOR
     q, s, g, c = fp4.nvfp4_quantize(x_cpu.to(cuda), round=rnd, four_six=four_six, seed=seed, layout=layout,
                                     global_in=gin)
     qo, so, go, co = O.nvfp4_quantize(f32(x_cpu), round=rnd, four_six=four_six, seed=seed, global_in=global_in)
-    assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(np.float32(npy(g)[0]), np.float32(go), equal_nan=True)
     assert np.array_equal(npy(q), qo)
     check_scales(s, so, layout)
     assert counts_of(c) == co
@@ -177,6 +177,32 @@ def test_mx_empty_and_nonfinite_counts(cuda):
     x[100, 0] = float("-inf")
     _, _, c = fp4.mx_quantize(x.to(cuda))
     assert counts_of(c)["nonfinite"] == 3
+
+
+def nonfinite_input(dtype, seed):
+    """N(0,1) with NaN of both signs, +-Inf, and a block holding both, at fixed positions."""
+    x = synth.normal_f32(128, 256, seed)
+    b = x.view(torch.int32)
+    b[7, 3], b[7, 40], b[9, 100], b[100, 0] = 0x7FC00000, -0x400000, 0x7F800000, -0x800000
+    b[64, 16], b[64, 17], b[127, 255] = 0x7FC00000, -0x800000, 0x7F800000
+    return x.to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rnd", [fp4.RNE, fp4.STOCHASTIC])
+def test_nonfinite_inputs_parity(cuda, dtype, rnd):
+    """Blocks holding Inf or NaN: an Inf saturates to +-6 under a saturated scale (E4M3 448, E8M0
+    2^126), a NaN maximum gives the NaN scale byte 0x7F (NVFP4) and +6 codes, and a NaN anywhere
+    makes the two-pass global scale NaN.  Codes, scales and counters bit-exact."""
+    x = nonfinite_input(dtype, 36)
+    for policy in (fp4.OCP_FLOOR, fp4.NOSAT_CEIL):
+        run_mx(x, cuda, policy=policy, rnd=rnd, seed=4)
+    for four_six in (False, True):
+        run_nv(x, cuda, rnd=rnd, four_six=four_six, seed=4, global_in=0.01)
+        q, s, g, qo, so, go = run_nv(x, cuda, rnd=rnd, four_six=four_six, seed=4)
+        assert np.isnan(go)
+        out = fp4.fp4_dequantize(q, s, fp4.NVFP4, g)
+        assert np.array_equal(npy(out), O.dequantize(qo, so, O.NVFP4, go), equal_nan=True)
 
 
 # ---------------------------------------------------------------------------------------------

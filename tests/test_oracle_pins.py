@@ -311,6 +311,34 @@ def test_four_over_six_picks_lower_error_candidate_brute_force():
 
 
 # ---------------------------------------------------------------------------------------------
+# Non-finite inputs (the pages leave them open; these are the readings the library follows)
+
+def test_nonfinite_readings():
+    """NaN propagates through the block and tensor maxima as in torch.amax; an E4M3 scale of a NaN
+    maximum is the NaN byte torch's float8_e4m3fn cast gives (0x7F); Inf saturates to 448 (0x7E);
+    E2M1 and INT4 have no NaN and encode one as their largest positive code."""
+    nan_e4m3 = torch.tensor([float("nan")]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+    assert O.e4m3_encode(float("nan")) == (nan_e4m3 & 0x7F) == 0x7F
+    assert O.e4m3_encode(float("inf")) == 0x7E
+    assert O.e2m1_encode_rne(float("nan")) == 7 and O.e2m1_encode_sr(float("nan"), 0) == 7
+    assert O.e2m1_encode_rne(float("-inf")) == 15 and O.int4_encode_rne(float("nan")) == 7
+    assert O.mx_exponent(float("inf")) == 126 and O.mx_exponent(float("nan"), O.NOSAT_CEIL) == 126
+    x = O._f32(np.random.default_rng(14).standard_normal((4, 64)))
+    x[1, 5] = np.nan
+    x[2, 40] = -np.inf
+    assert torch.isnan(torch.from_numpy(x).abs().amax())
+    q, s, sg, c = O.nvfp4_quantize(x)
+    assert np.isnan(sg) and (s == 0x7F).all() and c["nonfinite"] == 2
+    q, s, sg, c = O.nvfp4_quantize(x, global_in=0.01)
+    blk = torch.from_numpy(x).abs().reshape(4, 4, 16).amax(-1).numpy()
+    assert (s[np.isnan(blk)] == 0x7F).all() and (s[np.isinf(blk)] == 0x7E).all()
+    codes = np.stack([q & 15, q >> 4], -1).reshape(4, 64)
+    assert (codes[1, :16] == 7).all() and codes[2, 40] == 15
+    q, s, c = O.mx_quantize(x)
+    assert s[1, 0] == s[2, 1] == 126 + 127 and c["nonfinite"] == 2
+
+
+# ---------------------------------------------------------------------------------------------
 # IF4 (E2M1 or INT4 per block, the choice in the scale byte's sign bit)
 
 IF4_ROW = [int(v) for v in golden_rows("if4.txt")[0]]
