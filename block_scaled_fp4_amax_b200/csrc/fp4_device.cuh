@@ -582,6 +582,37 @@ __device__ __forceinline__ void int4_candidate_n(const float* v, float R7, float
   }
 }
 
+// The INT4 candidate for the estimate path: the packed nibbles of int4_candidate_n and the
+// residual sum sum (k - y)^2 = sum (|y| - |k|)^2 (k has the sign of y), formed with FMAs into
+// two partial sums (an estimate; if4_undecided allows for its rounding).
+template <int N>
+__device__ __forceinline__ float int4_encode_resid_n(const float* v, float R7, const uint32_t* w_e2m1, uint32_t* w7) {
+  static_assert(N % 8 == 0, "whole packed words");
+  const f32x2 R2 = f2_pack(R7, R7), M2 = f2_pack(0x1p23f, 0x1p23f);
+  float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+  for (int k = 0; k < N / 8; ++k) {
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const int j = 8 * k + i;
+      float y0, y1;
+      f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y0, y1);
+      const f32x2 t = f2_add(f2_pack(fminf(fabsf(y0), 7.0f), fminf(fabsf(y1), 7.0f)), M2);
+      float t0, t1, m0, m1;
+      f2_unpack(t, t0, t1);
+      acc += __float_as_uint(t0) << (4 * i);
+      acc += __float_as_uint(t1) << (4 * i + 4);
+      f2_unpack(f2_sub(t, M2), m0, m1);
+      const float r0 = fabsf(y0) - m0, r1 = fabsf(y1) - m1;
+      acc0 = fmaf(r0, r0, acc0);
+      acc1 = fmaf(r1, r1, acc1);
+    }
+    w7[k] = (acc - int4_pack_fold()) | (w_e2m1[k] & 0x88888888u);
+  }
+  return acc0 + acc1;
+}
+
 // ---------------------------------------------------------------------------------------------
 // Four-over-six selection without the exact error sums in the common case.
 //
@@ -661,6 +692,26 @@ __device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, floa
   four = (am != 0u) & (diff < 0.0f);
   // an all-zero block has equal (zero) sums and keeps 6 without the exact path
   return (am != 0u) & !(in_range & (fabsf(diff) > m));
+}
+
+// IF4: the same test for the E2M1 candidate (D, A) against the INT4 one (D7, A7).  The INT4
+// reconstruction fl(fl(k*d)*s7), its step D7 = fl(d*s7) and y = fl(v*fl(1/D7)) take the rounded
+// steps of the E2M1 ones (k*d exact, then one product with a per-tensor factor), so the bound
+// holds as derived; D7 <= D, so the range test is on D7.  `eligible` is false when the INT4 step
+// has no finite nonzero reciprocal: such a block keeps E2M1 without the exact path.  Returns true
+// when the exact sums are needed; otherwise `int4` holds the decision.
+__device__ __forceinline__ bool if4_undecided(uint32_t am, float amax, float D, float D7, float A, float A7,
+                                              bool eligible, bool& int4) {
+  const float a6 = __fmul_rn(__fmul_rn(D, D), A);
+  const float a7 = __fmul_rn(__fmul_rn(D7, D7), A7);
+  const float sa = a6 + a7;
+  const float m = 7.62939453e-06f * (1.02f * amax * amax + 2.0f * sa) + __uint_as_float(0x00000400u);  // 2^-17, 2^-139
+  const float diff = a7 - a6;
+  const bool in_range = (am >= 0x26800000u) & (am < 0x5D800000u) & (D7 >= __uint_as_float(0x21800000u)) &
+                        (sa < INFINITY);
+  const bool live = eligible & (am != 0u);
+  int4 = live & (diff < 0.0f);
+  return live & !(in_range & (fabsf(diff) > m));
 }
 
 // ---------------------------------------------------------------------------------------------

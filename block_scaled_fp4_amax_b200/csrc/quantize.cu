@@ -78,17 +78,11 @@ struct QuantParams {
   unsigned long long* counts;
 };
 
-// Exact four-over-six choice for one chunk (the rare case the estimates cannot decide): reloads
-// the chunk's values (an L2 hit: the kernel read them moments ago) and compares the two fp32
-// sequential error sums.  Out of line so the unrolled main loop keeps a single copy of it; called
-// by the whole warp (the block sums shuffle when G > 1).
-template <typename T, int G>
-__device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, bool valid, uint32_t w6a, uint32_t w6b,
-                                                uint32_t w4a, uint32_t w4b, uint32_t sc6, uint32_t sc4, float s_g,
-                                                uint32_t zero) {
-  constexpr int E = Vec32<T>::E;
+// Reload one chunk's values for an exact decision (an L2 hit: the kernel read them moments ago).
+template <typename T>
+__device__ __forceinline__ void reload_chunk(const char* xb, long long c, bool valid, float* v) {
   U8 raw;
-  if (valid) {  // plain 16-byte loads: ptxas 12.9 crashed on the 256-bit load asm in this function
+  if (valid) {  // plain 16-byte loads: ptxas 12.9 crashed on the 256-bit load asm in these functions
     const uint4 lo = __ldg(reinterpret_cast<const uint4*>(xb + c * 32));
     const uint4 hi = __ldg(reinterpret_cast<const uint4*>(xb + c * 32 + 16));
     raw.w[0] = lo.x; raw.w[1] = lo.y; raw.w[2] = lo.z; raw.w[3] = lo.w;
@@ -97,8 +91,19 @@ __device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, boo
 #pragma unroll
     for (int i = 0; i < 8; ++i) raw.w[i] = 0u;
   }
-  float v[E], sq[E];
   Vec32<T>::unpack(raw, v);
+}
+
+// Exact four-over-six choice for one chunk (the rare case the estimates cannot decide): compares
+// the two fp32 sequential error sums.  Out of line so the unrolled main loop keeps a single copy
+// of it; called by the whole warp (the block sums shuffle when G > 1).
+template <typename T, int G>
+__device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, bool valid, uint32_t w6a, uint32_t w6b,
+                                                uint32_t w4a, uint32_t w4b, uint32_t sc6, uint32_t sc4, float s_g,
+                                                uint32_t zero) {
+  constexpr int E = Vec32<T>::E;
+  float v[E], sq[E];
+  reload_chunk<T>(xb, c, valid, v);
   const int lane = threadIdx.x & 31;
   const uint32_t w6[2] = {w6a, w6b}, w4[2] = {w4a, w4b};
   sq_errors_n<E>(v, w6, sc6, s_g, zero, sq);
@@ -106,6 +111,25 @@ __device__ __noinline__ uint32_t four_six_exact(const char* xb, long long c, boo
   sq_errors_n<E>(v, w4, sc4, s_g, zero, sq);
   const float sse4 = block_sse_n<E, G>(sq, lane);
   return sse4 < sse6 ? 1u : 0u;
+}
+
+// Exact IF4 choice for one chunk, as four_six_exact: the E2M1 error sum against the INT4 one
+// (the INT4 candidate is rebuilt from the values; `wa`/`wb` are the E2M1 words, whose sign bits
+// it takes).  Returns 1 when INT4 is strictly lower.
+template <typename T, int G>
+__device__ __noinline__ uint32_t if4_exact(const char* xb, long long c, bool valid, uint32_t wa, uint32_t wb,
+                                           uint32_t sc, float s_g, float R7, float s7, uint32_t zero) {
+  constexpr int E = Vec32<T>::E;
+  float v[E], sq[E];
+  reload_chunk<T>(xb, c, valid, v);
+  const int lane = threadIdx.x & 31;
+  const uint32_t w[2] = {wa, wb};
+  uint32_t w7[2];
+  sq_errors_n<E>(v, w, sc, s_g, zero, sq);
+  const float sse6 = block_sse_n<E, G>(sq, lane);
+  int4_candidate_n<E>(v, R7, e4m3_value(sc), s7, w, w7, sq);
+  const float sse7 = block_sse_n<E, G>(sq, lane);
+  return sse7 < sse6 ? 1u : 0u;
 }
 
 template <typename T, bool NV, bool SR, int MODE>
@@ -194,37 +218,51 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
           }
         }
         sc = (uint32_t)(e + 127);
+      } else if (IF4) {
+        // E2M1 and INT4 candidates with their scaled-domain residual estimates; the exact fp32
+        // error sums only where the estimates are too close to call (INT4 kept iff strictly lower)
+        float D, A, R;
+        sc = nv_candidate_resid_n<E, false, !kBF>(v, amax, ns.inv6, tab, rnd, p.zero, w, sat, D, A, &R);
+        if constexpr (kBF) {
+          const uint32_t n = sat_count_bf16x16(raw[u].w, D, R);
+          sat = __fmul_rn(amax, R) > 6.0f ? n : 0u;
+        }
+        const float2 DR7 = tab7[sc];
+        uint32_t w7[W];
+        float A7 = int4_encode_resid_n<E>(v, DR7.y, w, w7);
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) {
+          A += __shfl_xor_sync(0xFFFFFFFFu, A, o);
+          A7 += __shfl_xor_sync(0xFFFFFFFFu, A7, o);
+        }
+        const bool eligible = DR7.y != 0.0f;
+        bool pick;
+        const bool undecided = if4_undecided(am, amax, D, DR7.x, A, A7, eligible, pick);
+        if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform call: the exact sums shuffle
+          const uint32_t lower = if4_exact<T, G>(xb, c, valid, w[0], w[W - 1], sc, ns.s_g, DR7.y, s7, p.zero);
+          pick = eligible && lower != 0u;
+        }
+        if (pick) {
+          sc |= 0x80u;
+          four = 1;
+          sat = 0;
+          if (__fmul_rn(amax, DR7.y) > 7.0f) {
+            if constexpr (kBF) {
+              sat = sat_count_bf16x16(raw[u].w, DR7.x, DR7.y, 7.0f);
+            } else {
+#pragma unroll
+              for (int i = 0; i < E; ++i) sat += fabsf(__fmul_rn(v[i], DR7.y)) > 7.0f;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < W; ++k) w[k] = w7[k];
+        }
       } else if (!FOUR_SIX) {
         float2 DR;
         sc = nv_candidate_n<E, SR, !kBF>(v, amax, ns.inv6, tab, rnd, w, sat, &DR);
         if constexpr (kBF) {
           const uint32_t n = sat_count_bf16x16(raw[u].w, DR.x, DR.y);
           sat = __fmul_rn(amax, DR.y) > 6.0f ? n : 0u;
-        }
-        if constexpr (IF4) {
-          // both candidates' exact error sums (fp32, element order), INT4 kept iff strictly lower
-          float sq[E];
-          sq_errors_n<E>(v, w, sc, ns.s_g, p.zero, sq);
-          const float sse6 = block_sse_n<E, G>(sq, lane);
-          const float2 DR7 = tab7[sc];
-          uint32_t w7[W];
-          int4_candidate_n<E>(v, DR7.y, e4m3_value(sc), s7, w, w7, sq);
-          const float sse7 = block_sse_n<E, G>(sq, lane);
-          if (DR7.y != 0.0f && sse7 < sse6) {
-            sc |= 0x80u;
-            four = 1;
-            sat = 0;
-            if (__fmul_rn(amax, DR7.y) > 7.0f) {
-              if constexpr (kBF) {
-                sat = sat_count_bf16x16(raw[u].w, DR7.x, DR7.y, 7.0f);
-              } else {
-#pragma unroll
-                for (int i = 0; i < E; ++i) sat += fabsf(__fmul_rn(v[i], DR7.y)) > 7.0f;
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < W; ++k) w[k] = w7[k];
-          }
         }
       } else {
         float D6, D4, A6, A4, R6, R4;
