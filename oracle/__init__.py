@@ -97,6 +97,8 @@ def lib():
         L.ora_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
         L.ora_dequantize_f64.restype = None
         L.ora_dequantize_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
+        L.ora_e2m1_to_e4m3.restype = None
+        L.ora_e2m1_to_e4m3.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
         L.ora_fwht_norm_const.restype = ctypes.c_float
         L.ora_fwht_norm_const.argtypes = [ctypes.c_long]
         L.ora_fwht_rows.restype = None
@@ -256,6 +258,15 @@ def dequantize_f64(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
     rows, half = q.shape
     out = np.zeros((rows, half * 2), dtype=np.float64)
     lib().ora_dequantize_f64(_p(q), _p(scales), int(fmt), rows, half * 2, float(s_g), _p(out))
+    return out
+
+
+def e2m1_to_e4m3(q) -> np.ndarray:
+    """E4M3 byte of value * 2^-6 for every nibble of q [rows, cols/2] -> uint8 [rows, cols]."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    rows, half = q.shape
+    out = np.zeros((rows, 2 * half), dtype=np.uint8)
+    lib().ora_e2m1_to_e4m3(_p(q), rows, 2 * half, _p(out))
     return out
 
 

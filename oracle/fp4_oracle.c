@@ -469,6 +469,23 @@ void ora_dequantize(const uint8_t* q, const uint8_t* scales, int format, long ro
   }
 }
 
+/* E2M1 nibbles to E4M3 bytes ([X]: devices without the FP4 MMA run the operands on the FP8 MMA
+ * after an exact conversion whose 2^6 folds into the scale).  Definition: the E4M3 encoding of
+ * value(n) * 2^-6 (exact: at most 2 significant bits, magnitude in [2^-7, 6 * 2^-6]), with the
+ * nibble's sign bit, so -0 maps to 0x80.  q: [rows, cols/2] packed as the quantisers write;
+ * out: [rows, cols], one byte per element.                                                      */
+void ora_e2m1_to_e4m3(const uint8_t* q, long rows, long cols, uint8_t* out) {
+  for (long r = 0; r < rows; ++r) {
+    for (long k = 0; k < cols; ++k) {
+      uint8_t byte = q[r * (cols / 2) + k / 2];
+      int code = (k & 1) ? (byte >> 4) : (byte & 15);
+      double mag = fabs(ora_e2m1_value(code));
+      int e = ora_e4m3_encode_rne_satfinite((float)ldexp(mag, -6));
+      out[r * cols + k] = (uint8_t)((code & 8 ? 0x80 : 0) | e);
+    }
+  }
+}
+
 /* Exact fp64 dequantisation (for the GEMM reference): v * d * s_g with no rounding.            */
 void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, long rows, long cols,
                         float s_g, double* out) {

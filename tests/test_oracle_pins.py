@@ -42,6 +42,21 @@ def test_e2m1_to_e4m3_identity_all_codes():
             assert got == want and math.copysign(1, got) == math.copysign(1, want), (c, hex(b))
 
 
+def test_e2m1_to_e4m3_expansion_equals_the_printed_identity():
+    """The oracle's expansion (an E4M3 encode of value * 2^-6 per nibble) against the page's bit
+    identity applied to every possible packed byte, low nibble first."""
+    rows = {r[0]: r[1] for r in golden_rows("e2m1_to_e4m3.txt")}
+    ms, mm, sh = int(rows["mask_sign"], 16) & 0xFF, int(rows["mask_mag"], 16) & 0xFF, int(rows["shift"])
+    q = np.arange(256, dtype=np.uint8).reshape(8, 32)
+    got = O.e2m1_to_e4m3(q)
+    for r in range(8):
+        for j in range(32):
+            byte = int(q[r, j])
+            for h, n in enumerate((byte & 15, byte >> 4)):
+                b = n << 4
+                assert got[r, 2 * j + h] == ((b & ms) | ((b & mm) >> sh)), (byte, h)
+
+
 def test_e2m1_rne_worked_values_and_ties():
     # exact points stay; ties go to the even mantissa code; >6 saturates; -tiny keeps its sign
     cases = {1.5: 3, 2.5: 4, 0.15: 0, 6.5: 7, 0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 3.5: 6, 5.0: 6,
