@@ -421,6 +421,22 @@ def secondary(args, dev, flush, td, pk):
                 "weight_quantise_GB/s": round(qbytes / (t_w * 1e-3) / 1e9, 1),
                 "weight_quantise_frac_hbm": round(qbytes / (t_w * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                 "end_to_end_TFLOP/s": round(flop / (t_all * 1e-3) / 1e12, 1)})
+    # the same GEMM on the FP8 tensor-core route: E4M3 expansions of the MXFP4 operands, then
+    # kind::mxf8f6f4 (the 1-SM kernel); against the dense FP8 peak, the measured bf16 peak x 2
+    A8 = fp4.fp4_to_e4m3(Aq[0])
+    B8 = fp4.fp4_to_e4m3(Bq[0])
+    ms = timed(lambda: (fp4.fp4_to_e4m3(Aq[0], out=A8), fp4.fp4_to_e4m3(Bq[0], out=B8)), K, W, flush, td)
+    t_x = statistics.median(ms)
+    ms = timed(lambda: fp4.fp4_block_gemm_e4m3(A8, Aq[1], B8, Bq[1], out=C, workspace=gws), K, W, flush, td)
+    t_8 = statistics.median(ms)
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    xbytes = (Aq[0].numel() + Bq[0].numel()) * 3  # read the nibbles, write twice as many bytes
+    out.append({"workload": "MXFP4 down_proj 4096x8192x28672 on the FP8 route: E4M3 expansion, kind::mxf8f6f4 GEMM",
+                "expand_ms": round(t_x, 4), "expand_GB/s": round(xbytes / (t_x * 1e-3) / 1e9, 1),
+                "expand_frac_hbm": round(xbytes / (t_x * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                "gemm_ms": round(t_8, 4), "gemm_TFLOP/s": round(flop / (t_8 * 1e-3) / 1e12, 1),
+                "gemm_frac_fp8_peak": round(flop / (t_8 * 1e-3) / 1e12 / fp8_peak, 4), "fp8_peak": fp8_peak,
+                "peak_source": pk["source"] + " bf16 x 2 (nominal FP8/BF16 ratio)"})
     return out
 
 
@@ -453,7 +469,7 @@ def run_reference(args, rank):
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-CASES = ("nv", "nv46", "nv_amax", "if4", "mx", "fwht", "gemm_nv", "gemm_mx", "dequant")
+CASES = ("nv", "nv46", "nv_amax", "if4", "mx", "fwht", "gemm_nv", "gemm_mx", "gemm_e4m3", "dequant")
 
 
 def run_case(name, reps):
@@ -480,6 +496,12 @@ def run_case(name, reps):
         q, s, g, _ = fp4.nvfp4_quantize(x)
         for _ in range(reps):
             fp4.fp4_dequantize(q, s, fp4.NVFP4, g, out_dtype=torch.bfloat16)
+    elif name == "gemm_e4m3":
+        A = fp4.mx_quantize(synth.swiglu_act().to(dev), layout=fp4.MMA_TILED)
+        B = fp4.mx_quantize(synth.weight().to(dev), layout=fp4.MMA_TILED)
+        A8, B8 = fp4.fp4_to_e4m3(A[0]), fp4.fp4_to_e4m3(B[0])
+        for _ in range(reps):
+            fp4.fp4_block_gemm_e4m3(A8, A[1], B8, B[1])
     elif name in ("gemm_nv", "gemm_mx"):
         if name == "gemm_nv":
             A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)

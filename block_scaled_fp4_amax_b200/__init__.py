@@ -32,7 +32,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 # Every symbol include/fp4mx.h declares.
 EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
            "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error",
-           "nvfp4_quantize_noalloc")
+           "nvfp4_quantize_noalloc", "fp4_to_e4m3", "fp4_block_gemm_e4m3")
 
 
 class Fp4Error(RuntimeError):
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
     L.swiglu_fwht_quantize.argtypes = [P, P, I, LG, LG, P, I, I, I, I, ULL, I, P, P, P, P, P, P, P, SZ, P]
     L.fp4_dequantize.argtypes = [P, P, I, I, I, P, LG, LG, I, P, P]
     L.fp4_block_gemm.argtypes = [I, I, I, I, P, P, P, P, P, P, P, LG, P, SZ, P]
+    L.fp4_to_e4m3.argtypes = [P, LG, LG, P, P]
+    L.fp4_block_gemm_e4m3.argtypes = [I, I, I, P, P, P, P, P, LG, P, SZ, P]
     L.nvfp4_quantize_noalloc.argtypes = [P, I, LG, LG, I, I, I, ULL, I, P, P, P, P, P, P]
     L.nvfp4_quantize_noalloc.restype = I
     L.fp4_workspace_size.argtypes = [I, LG, LG]
@@ -70,7 +72,7 @@ def lib() -> ctypes.CDLL:
     L.fp4_last_error.argtypes = []
     L.fp4_last_error.restype = ctypes.c_char_p
     for name in ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize",
-                 "fp4_block_gemm"):
+                 "fp4_block_gemm", "fp4_to_e4m3", "fp4_block_gemm_e4m3"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -243,4 +245,29 @@ def fp4_block_gemm(fmt: int, Aq: torch.Tensor, As: torch.Tensor, Bq: torch.Tenso
     ws = workspace if workspace is not None else _workspace(OP_BLOCK_GEMM, Aq.device, M, N)
     _check(lib().fp4_block_gemm(fmt, M, N, K, _ptr(Aq), _ptr(As), _ptr(Ag), _ptr(Bq), _ptr(Bs), _ptr(Bg),
                                 _ptr(C), C.stride(0), _ptr(ws), ws.numel(), _stream(stream)))
+    return C, ws
+
+
+def fp4_to_e4m3(q: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """E4M3 bytes (value * 2^-6 of every nibble) of packed E2M1 q [rows, cols/2] -> uint8 [rows, cols]."""
+    _need_cuda(q)
+    rows, half = q.shape
+    o = out if out is not None else torch.empty((rows, 2 * half), dtype=torch.uint8, device=q.device)
+    _check(lib().fp4_to_e4m3(_ptr(q), rows, 2 * half, _ptr(o), _stream(stream)))
+    return o
+
+
+def fp4_block_gemm_e4m3(A8: torch.Tensor, As: torch.Tensor, B8: torch.Tensor, Bs: torch.Tensor,
+                        out: torch.Tensor | None = None, stream=None, workspace: torch.Tensor | None = None):
+    """MXFP4 GEMM on the FP8 tensor-core path from E4M3 expansions (fp4_to_e4m3) and MMA-tiled E8M0
+    scales.  Returns (C bf16 [M, N], workspace); workspace[0:4] holds the kernel status word."""
+    _need_cuda(A8, As, B8, Bs)
+    M, K = A8.shape
+    N = B8.shape[0]
+    if B8.shape[1] != K:
+        raise ValueError("A and B disagree on K")
+    C = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A8.device)
+    ws = workspace if workspace is not None else _workspace(OP_BLOCK_GEMM, A8.device, M, N)
+    _check(lib().fp4_block_gemm_e4m3(M, N, K, _ptr(A8), _ptr(As), _ptr(B8), _ptr(Bs), _ptr(C), C.stride(0),
+                                     _ptr(ws), ws.numel(), _stream(stream)))
     return C, ws

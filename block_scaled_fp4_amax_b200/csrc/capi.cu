@@ -272,9 +272,41 @@ fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K, const unsigned
   uint32_t* status = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return cuda_fail(e, "zeroing gemm status");
-  fp4k::GemmLaunch L{nv, M, N, K, Aq, As, Bq, Bs, nv ? Ag : nullptr, nv ? Bg : nullptr, C, ldc, status};
+  fp4k::GemmLaunch L{nv, false, M, N, K, Aq, As, Bq, Bs, nv ? Ag : nullptr, nv ? Bg : nullptr, C, ldc, status};
   e = fp4k::launch_gemm(L, s);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_block_gemm launch");
+}
+
+fp4_status fp4_to_e4m3(const unsigned char* q, long rows, long cols, unsigned char* out, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 32)
+    return fail(FP4_EINVAL, "bad shape [%ld, %ld]: cols must be a positive multiple of 32", rows, cols);
+  if ((long long)rows * cols > kMaxElems) return fail(FP4_EUNSUPPORTED, "tensor larger than 2^40 elements");
+  if (rows == 0) return FP4_OK;
+  if (!q || !out) return fail(FP4_EINVAL, "NULL q or out");
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(FP4_EINVAL, "q and out must be 16-byte aligned");
+  cudaError_t e = fp4k::launch_e2m1_to_e4m3(q, (long long)rows * cols / 2, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_to_e4m3 launch");
+}
+
+fp4_status fp4_block_gemm_e4m3(int M, int N, int K, const unsigned char* A8, const unsigned char* As,
+                               const unsigned char* B8, const unsigned char* Bs, void* C, long ldc,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return fail(FP4_EINVAL, "bad GEMM shape %d x %d x %d", M, N, K);
+  if (M % 128 || N % 256 || K % 128)
+    return fail(FP4_EUNSUPPORTED, "GEMM shape %d x %d x %d: needs M %% 128, N %% 256, K %% 128 == 0", M, N, K);
+  if (!A8 || !As || !B8 || !Bs || !C) return fail(FP4_EINVAL, "NULL operand pointer");
+  if (ldc < N || ldc % 8) return fail(FP4_EINVAL, "ldc %ld must be >= N and a multiple of 8", ldc);
+  if (!aligned(A8, 16) || !aligned(B8, 16) || !aligned(As, 16) || !aligned(Bs, 16) || !aligned(C, 16))
+    return fail(FP4_EINVAL, "GEMM operands must be 16-byte aligned");
+  if (!workspace || ws_bytes < kGemmWorkspace || !aligned(workspace, 16))
+    return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required", kGemmWorkspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "zeroing gemm status");
+  fp4k::GemmLaunch L{false, true, M, N, K, A8, As, B8, Bs, nullptr, nullptr, C, ldc, status};
+  e = fp4k::launch_gemm(L, s);
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_block_gemm_e4m3 launch");
 }
 
 }  // extern "C"

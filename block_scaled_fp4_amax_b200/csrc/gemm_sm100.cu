@@ -132,6 +132,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdes
   }
 }
 
+// The FP8 route for MXFP4 operands expanded to E4M3: kind::mxf8f6f4, one UE8M0 scale per 32 values
+// (scale_vec::1X), K = 32 per instruction.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                          uint32_t sfb, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+               ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate) : "memory");
+}
+
 // Two fp32 accumulator words scaled by alpha and rounded to bf16 (RNE), the first in the low half.
 __device__ __forceinline__ uint32_t bf16x2_scaled(uint32_t lo, uint32_t hi, float alpha) {
   uint32_t b;
@@ -168,11 +177,25 @@ __host__ __device__ constexpr uint32_t idesc(bool nv, uint32_t sfa_id, uint32_t 
          ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
 }
 
+// Instruction descriptor, kind::mxf8f6f4: E4M3 x E4M3 (format code 0 in bits 7-9 and 10-12),
+// K-major A and B, M = 128, N = 256, UE8M0 scales (bit 23), scale byte ids as above.
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
+}
+
+// Operand kinds of the 1-SM kernel.
+constexpr int kMxFp4 = 0, kNvFp4 = 1, kMxE4m3 = 2;
+
 // ---------------------------------------------------------------------------------------------
-template <bool NV>
+// KIND kMxFp4 / kNvFp4: packed E2M1 operands, 256 values (128 bytes) per row per stage, four K=64
+// MMAs.  kMxE4m3: the E4M3 expansions of MXFP4 operands, 128 values (128 bytes) per stage, four
+// K=32 MMAs of kind::mxf8f6f4, each taking one of the stage's four UE8M0 scales per row (scale
+// byte id 0-3 of the atom's 32-bit tensor-memory column).
+template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
-  constexpr int ATOMS = NV ? 4 : 2;           // scale atoms per 128 rows per stage
+  constexpr bool NV = KIND == kNvFp4, F8 = KIND == kMxE4m3;
+  constexpr int ATOMS = NV ? 4 : (F8 ? 1 : 2);  // scale atoms per 128 rows per stage
   constexpr int SFA_BYTES = ATOMS * 512;
   constexpr int SFB_BYTES = 2 * ATOMS * 512;  // two 128-row groups
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
@@ -218,7 +241,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
   const int tiles_m = p.M / BM, tiles_n = p.N / BN;
   const int num_tiles = tiles_m * tiles_n;
-  const int kt_count = p.K / 256;
+  const int kt_count = p.K / (F8 ? 128 : 256);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -290,11 +313,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             tc_cp_sf(tmem + SFB_COL + 8 * a + 4, desc_sf(fbs + (ATOMS + a) * 512));
           }
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {  // four K=64 MMAs per 256-value stage
-            const int atom = NV ? t : (t >> 1);
-            const uint32_t sf_id = NV ? 0u : (uint32_t)((t & 1) * 2);
-            tc_mma<NV>(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc(NV, sf_id, sf_id),
-                       tmem + SFA_COL + 4 * atom, tmem + SFB_COL + 8 * atom, (kt > 0 || t > 0) ? 1u : 0u);
+          for (int t = 0; t < 4; ++t) {  // four MMAs of 32 bytes of K per stage
+            const uint32_t acc = (kt > 0 || t > 0) ? 1u : 0u;
+            if constexpr (F8) {
+              tc_mma_f8(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc_f8(t, t),
+                        tmem + SFA_COL, tmem + SFB_COL, acc);
+            } else {
+              const int atom = NV ? t : (t >> 1);
+              const uint32_t sf_id = NV ? 0u : (uint32_t)((t & 1) * 2);
+              tc_mma<NV>(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc(NV, sf_id, sf_id),
+                         tmem + SFA_COL + 4 * atom, tmem + SFB_COL + 8 * atom, acc);
+            }
           }
           tc_commit(empty0 + 8 * s);  // stage free once these MMAs have read it
         }
@@ -314,7 +343,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const float alpha = p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f;
+    // E4M3 operands hold value * 2^-6 each, so their products carry 2^-12
+    const float alpha = F8 ? 4096.0f : (p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f);
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
       const int tm = tile % tiles_m, tn = tile / tiles_m;
@@ -353,9 +383,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
-template <bool NV>
+template <int KIND>
 constexpr int smem_bytes() {
-  constexpr int atoms = NV ? 4 : 2;
+  constexpr int atoms = KIND == kNvFp4 ? 4 : (KIND == kMxE4m3 ? 1 : 2);
   return 1024 + STAGES * (A_BYTES + B_BYTES + atoms * 512 * 3) + 256;
 }
 
@@ -748,28 +778,27 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   using namespace gemm;
   Params p;
   p.M = L.M; p.N = L.N; p.K = L.K; p.nv = L.nv ? 1 : 0;
-  p.atoms = L.nv ? 4 : 2;
+  p.atoms = L.nv ? 4 : (L.e4m3 ? 1 : 2);
   p.atoms_row = L.K / (L.nv ? 16 : 32) / 4;
   p.As = L.As; p.Bs = L.Bs; p.Ag = L.Ag; p.Bg = L.Bg;
   p.C = reinterpret_cast<__nv_bfloat16_raw*>(L.C);
   p.ldc = L.ldc;
   p.status = L.status;
-  if (L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
+  if (!L.e4m3 && L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
+  // operand rows: K/2 packed bytes (FP4) or K bytes (E4M3 expansion)
+  const uint64_t row_bytes = L.e4m3 ? (uint64_t)L.K : (uint64_t)L.K / 2;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, L.Aq, (uint64_t)L.K / 2, (uint64_t)L.M, BM) ||
-      !make_map(&tb, L.Bq, (uint64_t)L.K / 2, (uint64_t)L.N, BN))
+  if (!make_map(&ta, L.Aq, row_bytes, (uint64_t)L.M, BM) || !make_map(&tb, L.Bq, row_bytes, (uint64_t)L.N, BN))
     return cudaErrorInvalidValue;
   const int tiles = (L.M / BM) * (L.N / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  if (L.nv) {
-    auto k = gemm_kernel<true>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<true>());
-    k<<<grid, NUM_THREADS, smem_bytes<true>(), s>>>(ta, tb, p);
-  } else {
-    auto k = gemm_kernel<false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<false>());
-    k<<<grid, NUM_THREADS, smem_bytes<false>(), s>>>(ta, tb, p);
-  }
+  auto go = [&](auto k, int smem) {
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    k<<<grid, NUM_THREADS, smem, s>>>(ta, tb, p);
+  };
+  if (L.e4m3) go(gemm_kernel<kMxE4m3>, smem_bytes<kMxE4m3>());
+  else if (L.nv) go(gemm_kernel<kNvFp4>, smem_bytes<kNvFp4>());
+  else go(gemm_kernel<kMxFp4>, smem_bytes<kMxFp4>());
   return cudaGetLastError();
 }
 

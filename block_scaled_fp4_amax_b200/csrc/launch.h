@@ -85,6 +85,7 @@ struct FwhtLaunch {
 
 struct GemmLaunch {
   bool nv;
+  bool e4m3;  // MXFP4 through the FP8 MMA: Aq/Bq are E4M3 expansions [rows, K] (kind::mxf8f6f4)
   int M, N, K;
   const uint8_t *Aq, *As, *Bq, *Bs;
   const float *Ag, *Bg;
@@ -99,6 +100,8 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
 cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
                         unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
+// E2M1 nibbles -> E4M3 bytes; n_bytes (packed input bytes) a multiple of 16, both 16-byte aligned.
+cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* out, cudaStream_t s);
 cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s);

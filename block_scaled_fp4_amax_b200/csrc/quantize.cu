@@ -426,6 +426,30 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, con
 }
 
 // ---------------------------------------------------------------------------------------------
+// E2M1 -> E4M3 expansion (metrale `hardware::exec`: the exact conversion that lets the FP8 MMA take
+// FP4 operands).  With a nibble in bits 7..4 of a byte b, (b & 0x80) | ((b & 0x70) >> 2) is the E4M3
+// encoding of its value times 2^-6.  Each thread turns 16 packed bytes (32 nibbles) into 32 bytes.
+__global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint4* q, uint4* out, long long n16) {
+  const long long stride = (long long)gridDim.x * kThreads;
+  for (long long i = (long long)blockIdx.x * kThreads + threadIdx.x; i < n16; i += stride) {
+    const uint4 w = q[i];
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t even = (in[k] << 4) & 0xF0F0F0F0u;  // elements 0, 2, 4, 6 of the word, one per byte
+      const uint32_t odd = in[k] & 0xF0F0F0F0u;          // elements 1, 3, 5, 7
+      const uint32_t e = (even & 0x80808080u) | ((even & 0x70707070u) >> 2);
+      const uint32_t d = (odd & 0x80808080u) | ((odd & 0x70707070u) >> 2);
+      o[2 * k] = __byte_perm(e, d, 0x5140);      // elements 0 1 2 3
+      o[2 * k + 1] = __byte_perm(e, d, 0x7362);  // elements 4 5 6 7
+    }
+    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Launchers
 
 static int grid_for(long long work_items, int per_cta) {
@@ -492,6 +516,14 @@ cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* a
   const int grid = grid_for(chunks / 4 + 1, kThreads);
   if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
   else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* out, cudaStream_t s) {
+  const long long n16 = n_bytes / 16;
+  if (n16 == 0) return cudaSuccess;
+  e2m1_to_e4m3_kernel<<<grid_for(n16, kThreads), kThreads, 0, s>>>(reinterpret_cast<const uint4*>(q),
+                                                                   reinterpret_cast<uint4*>(out), n16);
   return cudaGetLastError();
 }
 

@@ -238,6 +238,34 @@ FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
                           void* C, long ldc, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * fp4_to_e4m3 — E2M1 nibbles to E4M3 bytes through the exact identity of [X] (metrale
+ * `hardware::exec`): with a nibble in bits 7..4 of a byte b, (b & 0x80) | ((b & 0x70) >> 2) is the
+ * E4M3 encoding of the nibble's value times 2^-6 (-0 gives 0x80).  It lets the FP8 tensor-core
+ * MMA take FP4 operands exactly (fp4_block_gemm_e4m3).
+ *   q   : device [rows, cols/2] packed E2M1 as the quantisers write (element 2j low nibble), 16-byte aligned.
+ *   out : device [rows, cols] bytes, element k of a row at byte k, 16-byte aligned.  Caller-owned.
+ * Preconditions: rows >= 0, cols > 0, cols % 32 == 0; rows == 0 launches nothing. */
+FP4_API fp4_status fp4_to_e4m3(const unsigned char* q, long rows, long cols, unsigned char* out, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * fp4_block_gemm_e4m3 — the MXFP4 block-scaled GEMM on the FP8 tensor-core path: C = A * B^T with
+ * the operands given as their E4M3 expansions (fp4_to_e4m3 of MXFP4 nibbles) and the MXFP4 E8M0
+ * scales unchanged, run as tcgen05.mma kind::mxf8f6f4 block_scale scale_vec::1X (one scale per 32
+ * values) with FP32 accumulation; the epilogue multiplies by 2^12, undoing the 2^-6 of each
+ * operand, so C equals fp4_block_gemm(FP4_MXFP4, ...) up to the order of the FP32 accumulation.
+ * [X] (FP4 operands on the FP8 MMA through the exact conversion) — an independent second tensor-
+ * core GEMM for cross-checking the FP4 one.  MXFP4 only: the FP8 kind takes UE8M0 scales per 32,
+ * which cannot carry NVFP4's E4M3 scales per 16.
+ *   A8 : device [M, K] E4M3 bytes; B8 : device [N, K] E4M3 bytes (K-major).
+ *   As, Bs : device MXFP4 scales in FP4_SCALES_MMA_TILED layout (as written by mx_quantize).
+ *   C, ldc, workspace, ws_bytes : as in fp4_block_gemm (workspace of FP4_OP_BLOCK_GEMM size).
+ * Preconditions: M % 128 == 0, N % 256 == 0, K % 128 == 0 (else FP4_EUNSUPPORTED), ldc >= N,
+ * ldc % 8 == 0, all pointers 16-byte aligned.  Runs on the 1-SM kernel (128 x 256 tiles). */
+FP4_API fp4_status fp4_block_gemm_e4m3(int M, int N, int K, const unsigned char* A8, const unsigned char* As,
+                                       const unsigned char* B8, const unsigned char* Bs, void* C, long ldc,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * nvfp4_quantize_noalloc — nvfp4_quantize without a caller-supplied workspace, for callers that
  * cannot allocate device memory: for example a plugin inside another runtime that receives only
  * its input and output buffers, or a latency-critical loop that must not call cudaMalloc (which

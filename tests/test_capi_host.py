@@ -95,6 +95,21 @@ def test_if4_rejects(L):
     assert L.fp4_dequantize(FAKE, FAKE, 2, 16, 0, None, 128, 256, 0, FAKE, None) == 1
 
 
+def test_e4m3_route_rejects(L):
+    # expansion: cols % 32, NULL, misalignment; FP8 GEMM: shape rules, ldc, workspace
+    assert L.fp4_to_e4m3(FAKE, 4, 48, FAKE, None) == 1
+    assert L.fp4_to_e4m3(None, 4, 64, FAKE, None) == 1
+    assert L.fp4_to_e4m3(FAKE, 4, 64, ctypes.c_void_p(0x10008), None) == 1
+    assert L.fp4_to_e4m3(FAKE, 0, 64, FAKE, None) == 0  # empty: nothing launched
+    g = L.fp4_block_gemm_e4m3
+    assert g(100, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2  # M % 128
+    assert g(128, 128, 128, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2  # N % 256
+    assert g(128, 256, 96, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2   # K % 128
+    assert g(128, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 256, None) == 1  # ldc < N
+    assert g(128, 256, 128, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None, 0, None) == 1    # workspace
+    assert g(128, 256, 128, None, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 1  # NULL A
+
+
 def test_fwht_rejects(L):
     # d not a power of two / out of range, MXFP4 with four-over-six, block mismatch
     assert L.fwht_quantize(FAKE, 1, 4, 3000, None, 1, 16, 0, 0, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
