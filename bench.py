@@ -336,6 +336,16 @@ def secondary(args, dev, flush, td, pk):
     out.append({"workload": "randomised FWHT (c*H*D) d=8192 + NVFP4 + stochastic rounding, 16384x8192 bf16",
                 "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
                 "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    # the same randomised rotation into IF4 blocks (round to nearest)
+
+    def c3i():
+        fp4.fwht_quantize(x3, fmt=fp4.NVFP4, if4=True, workspace=ws, signs=sg)
+
+    ms = timed(c3i, K, W, flush, td)
+    t = statistics.median(ms)
+    out.append({"workload": "randomised FWHT (c*H*D) d=8192 + IF4 (E2M1 or INT4 per 16-block), 16384x8192 bf16",
+                "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1),
+                "frac_hbm": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     del x3
     # SwiGLU fused ahead of the rotation: g, u bf16 [16384, 8192] read in both passes
     gg, uu = (t_.to(dev) for t_ in synth.swiglu_inputs(16384, 8192, seed=3))

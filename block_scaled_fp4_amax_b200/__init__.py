@@ -175,9 +175,10 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = F
 def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
                   layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, want_rotated: bool = False,
                   block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
-                  signs: torch.Tensor | None = None):
+                  signs: torch.Tensor | None = None, if4: bool = False):
     """Walsh-Hadamard rotation of each row fused with the quantiser of `fmt`; with `signs` (device
-    int32/uint32 [d/32], bit i negates channel i first) the randomised rotation c*H*D.
+    int32/uint32 [d/32], bit i negates channel i first) the randomised rotation c*H*D; with `if4`
+    (NVFP4, round to nearest) IF4 blocks.
     Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
     _need_cuda(x, global_in, signs)
     rows, d = x.shape
@@ -188,7 +189,7 @@ def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six:
     ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, x.device, rows, d)
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
         raise ValueError("signs must hold d/32 32-bit words")
-    _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, _ptr(signs), fmt, B, round, int(bool(four_six)), seed,
+    _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, _ptr(signs), fmt, B, round, _nv_mode(four_six, if4), seed,
                                layout, _ptr(global_in), _ptr(g), _ptr(rot), _ptr(q), _ptr(s), _ptr(c),
                                _ptr(ws), ws.numel(), _stream(stream)))
     return q, s, g, c, rot
@@ -198,8 +199,9 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
                          four_six: bool = False, seed: int = 0, layout: int = ROWMAJOR,
                          global_in: torch.Tensor | None = None, want_rotated: bool = False,
                          block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
-                         signs: torch.Tensor | None = None):
-    """fl(SiLU(g) * u) in fp32 (never stored), rotated (randomised with `signs`) and quantised to `fmt`.
+                         signs: torch.Tensor | None = None, if4: bool = False):
+    """fl(SiLU(g) * u) in fp32 (never stored), rotated (randomised with `signs`) and quantised to `fmt`
+    (IF4 blocks with `if4`).
     g, u: bf16 [rows, d].  Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
     _need_cuda(g, u, global_in, signs)
     if g.shape != u.shape:
@@ -213,7 +215,7 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
         raise ValueError("signs must hold d/32 32-bit words")
     _check(lib().swiglu_fwht_quantize(_ptr(g), _ptr(u), _dtype_code(g), rows, d, _ptr(signs), fmt, B, round,
-                                      int(bool(four_six)), seed, layout, _ptr(global_in), _ptr(gs), _ptr(rot),
+                                      _nv_mode(four_six, if4), seed, layout, _ptr(global_in), _ptr(gs), _ptr(rot),
                                       _ptr(q), _ptr(s), _ptr(c), _ptr(ws), ws.numel(), _stream(stream)))
     return q, s, gs, c, rot
 

@@ -173,8 +173,8 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   if (st != FP4_OK) return st;
   if (four_six != FP4_NV_PLAIN && four_six != FP4_NV_FOUR_SIX && four_six != FP4_NV_IF4)
     return fail(FP4_EINVAL, "NVFP4 block mode %d unknown", four_six);
-  if (!nv && four_six) return fail(FP4_EUNSUPPORTED, "four-over-six is defined for NVFP4 only");
-  if (four_six == FP4_NV_IF4) return fail(FP4_EUNSUPPORTED, "the rotation path has no IF4 mode");
+  if (!nv && four_six) return fail(FP4_EUNSUPPORTED, "four-over-six and IF4 are defined for NVFP4 only");
+  if (four_six == FP4_NV_IF4 && round != FP4_RNE) return fail(FP4_EUNSUPPORTED, "IF4 is defined with round to nearest only");
   if (nv && !global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
   if (rotated_out && !aligned(rotated_out, 16)) return fail(FP4_EINVAL, "rotated_out must be 16-byte aligned");
@@ -186,7 +186,7 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   if (!amax_pass && (st = zero_counts(counts, s)) != FP4_OK) return st;
   fp4k::FwhtLaunch L{};
   L.x = x; L.bf16 = dtype == FP4_BF16; L.rows = rows; L.d = (int)d; L.nv = nv;
-  L.sr = round == FP4_STOCHASTIC; L.four_six = nv && four_six == FP4_NV_FOUR_SIX; L.seed = seed;
+  L.sr = round == FP4_STOCHASTIC; L.mode = nv ? four_six : 0; L.seed = seed;
   L.tiled = layout == FP4_SCALES_MMA_TILED;
   L.global_in = nv ? global_in : nullptr;
   L.amax_bits = static_cast<uint32_t*>(workspace);

@@ -294,8 +294,10 @@ __device__ __forceinline__ void to_consecutive(float* srow, int t, float (&v)[32
 }
 
 // Pass 2: rotate again, normalise, quantise from registers (whole blocks per thread).
-template <typename T, int LOG_D, bool NV, bool SR, bool FOUR_SIX, bool GATED>
+// MODE: 0 plain, 1 four-over-six, 2 IF4 (NVFP4 only).
+template <typename T, int LOG_D, bool NV, bool SR, int MODE, bool GATED>
 __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 : 1) fwht_quant_kernel(FwhtParams p) {
+  constexpr bool FOUR_SIX = MODE == 1, IF4 = MODE == 2;
   using G = Geom<LOG_D>;
   constexpr int D = G::D;
   constexpr int B = NV ? 16 : 32;
@@ -322,7 +324,10 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = s_g;
   }
   __shared__ float2 tab[NV ? kScaleTab : 1];
+  __shared__ float2 tab7[IF4 ? kScaleTab : 1];
+  const float s7 = IF4 ? __fmul_rn(s_g, kSixSevenths) : 0.0f;
   if (NV) fill_scale_tab(tab, s_g);  // first read after the rotation's __syncthreads
+  if (IF4) fill_int4_tab(tab7, s7);
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};
   U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV], rawu[GATED ? RowLoad<T>::NV : 1];
   auto phys = [&](long long r) { return p.reverse ? (p.rows - 1 - r) : r; };
@@ -401,6 +406,37 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
 #pragma unroll
           for (int k = 0; k < W; ++k) w[k] = w4[k];
         }
+      } else if constexpr (IF4) {
+        // E2M1 or INT4 (round to nearest): residual estimates, exact sums inside the margin
+        uint32_t rnd[B];  // unused without stochastic rounding
+        float D6, A6, R6;
+        sc = nv_candidate_resid_n<B, false>(g, amax, inv6, tab, rnd, p.zero, w, sat, D6, A6, &R6);
+        const float2 DR7 = tab7[sc];
+        uint32_t w7[W];
+        const float A7 = int4_encode_resid_n<B>(g, DR7.y, w, w7);
+        const bool eligible = DR7.y != 0.0f;
+        bool pick;
+        const bool undecided = if4_undecided(am, amax, D6, DR7.x, A6, A7, eligible, pick);
+        if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform branch
+          float sq[B];
+          sq_errors_n<B>(g, w, sc, s_g, p.zero, sq);
+          const float sse6 = block_sse_n<B, 1>(sq, 0);
+          uint32_t wx[W];
+          int4_candidate_n<B>(g, DR7.y, e4m3_value(sc), s7, w, wx, sq);
+          const float sse7 = block_sse_n<B, 1>(sq, 0);
+          pick = eligible && sse7 < sse6;
+        }
+        if (pick) {
+          sc |= 0x80u;
+          four = 1;
+          sat = 0;
+          if (__fmul_rn(amax, DR7.y) > 7.0f) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) sat += fabsf(__fmul_rn(g[i], DR7.y)) > 7.0f;
+          }
+#pragma unroll
+          for (int k = 0; k < W; ++k) w[k] = w7[k];
+        }
       } else {
         uint32_t rnd[B];
         if (SR) sr_words<B>(idx0, p.keys, rnd);
@@ -458,7 +494,7 @@ static FwhtParams make_params(const FwhtLaunch& L) {
   p.c = (float)(1.0 / sqrt((double)L.d));
   p.tiled = L.tiled; p.reverse = 0; p.keys = philox_keys(L.seed); p.zero = 0u;
   p.global_in = L.global_in; p.amax_bits = L.amax_bits; p.global_out = L.global_out;
-  p.six_m = L.four_six ? 1536.0f : 2688.0f;
+  p.six_m = L.mode == 1 ? 1536.0f : 2688.0f;
   p.rotated_out = L.rotated_out; p.signs = L.signs; p.u = L.u; p.q = L.q; p.scales = L.scales; p.counts = L.counts;
   return p;
 }
@@ -473,7 +509,7 @@ static cudaError_t amax_d(const FwhtParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <typename T, int LOG_D, bool NV, bool SR, bool FS, bool GATED>
+template <typename T, int LOG_D, bool NV, bool SR, int FS, bool GATED>
 static cudaError_t quant_d(const FwhtParams& p, bool pdl, cudaStream_t s) {
   using G = Geom<LOG_D>;
   const int smem = G::ROWS * G::D * 4;
@@ -488,10 +524,11 @@ template <typename T, int LOG_D, bool GATED>
 static cudaError_t quant_sel(const FwhtParams& p, const FwhtLaunch& L, cudaStream_t s) {
   const bool d = L.pdl;
   if (!L.nv)
-    return L.sr ? quant_d<T, LOG_D, false, true, false, GATED>(p, d, s) : quant_d<T, LOG_D, false, false, false, GATED>(p, d, s);
-  if (L.four_six)
-    return L.sr ? quant_d<T, LOG_D, true, true, true, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, true, GATED>(p, d, s);
-  return L.sr ? quant_d<T, LOG_D, true, true, false, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, false, GATED>(p, d, s);
+    return L.sr ? quant_d<T, LOG_D, false, true, 0, GATED>(p, d, s) : quant_d<T, LOG_D, false, false, 0, GATED>(p, d, s);
+  if (L.mode == 2) return quant_d<T, LOG_D, true, false, 2, GATED>(p, d, s);  // IF4: round to nearest only
+  if (L.mode == 1)
+    return L.sr ? quant_d<T, LOG_D, true, true, 1, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, 1, GATED>(p, d, s);
+  return L.sr ? quant_d<T, LOG_D, true, true, 0, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, 0, GATED>(p, d, s);
 }
 
 template <typename T, bool GATED>

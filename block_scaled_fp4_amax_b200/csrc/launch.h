@@ -68,7 +68,7 @@ struct FwhtLaunch {
   int d;
   bool nv;
   bool sr;
-  bool four_six;
+  int mode;       // NVFP4 block mode: 0 plain, 1 four-over-six, 2 IF4
   unsigned long long seed;
   int tiled;
   const float* global_in;

@@ -173,8 +173,9 @@ FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, lon
  *   d           : power of two, 1024 <= d <= 16384.
  *   signs       : device uint32 [d / 32], 4-byte aligned, or NULL (plain rotation); caller-owned.
  *   rotated_out : device float [rows, d] or NULL; receives the rotated values (diagnostics).
- *   other arguments as in nvfp4_quantize; four_six (FP4_NV_PLAIN or FP4_NV_FOUR_SIX; FP4_NV_IF4
- *   is FP4_EUNSUPPORTED here) and global_in/out apply to FP4_NVFP4 only. */
+ *   other arguments as in nvfp4_quantize; four_six is the NVFP4 block mode (fp4_nv_mode:
+ *   FP4_NV_PLAIN, FP4_NV_FOUR_SIX, or FP4_NV_IF4 with FP4_RNE only) and, with global_in/out,
+ *   applies to FP4_NVFP4 only. */
 FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d,
                          const unsigned int* signs, fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,

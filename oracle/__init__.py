@@ -301,18 +301,18 @@ def silu_mul(g, u) -> np.ndarray:
 
 
 def swiglu_fwht_quantize(g, u, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
-                         global_in=None, signs=None):
+                         global_in=None, signs=None, if4: bool = False):
     """SiLU(g) * u in fp32 (no storage rounding), then the rotation and quantiser of fwht_quantize."""
     return fwht_quantize(silu_mul(g, u), fmt=fmt, round=round, four_six=four_six, seed=seed,
-                         global_in=global_in, signs=signs)
+                         global_in=global_in, signs=signs, if4=if4)
 
 
 def fwht_quantize(x, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
-                  global_in=None, signs=None):
+                  global_in=None, signs=None, if4: bool = False):
     """Rotation (randomised with `signs`) followed by the quantiser of `fmt` on the rotated fp32 tensor."""
     y = fwht(x, signs)
     if fmt == NVFP4:
-        q, s, sg, c = nvfp4_quantize(y, round=round, four_six=four_six, seed=seed, global_in=global_in)
+        q, s, sg, c = nvfp4_quantize(y, round=round, four_six=four_six, seed=seed, global_in=global_in, if4=if4)
         return y, q, s, sg, c
     q, s, c = mx_quantize(y, policy=OCP_FLOOR, round=round, seed=seed)
     return y, q, s, 1.0, c

@@ -84,10 +84,11 @@ def test_nvfp4_rejects(L):
 
 
 def test_if4_rejects(L):
-    # IF4 is round-to-nearest only; block modes beyond IF4; no IF4 in the rotation path or the GEMM
+    # IF4 is round-to-nearest NVFP4 only (also in the rotation path); block modes beyond IF4; no IF4 GEMM
     assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 1, 2, 0, 0, FAKE, None, FAKE, FAKE, None, None, 0, None) == 2
     assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 0, 3, 0, 0, FAKE, None, FAKE, FAKE, None, None, 0, None) == 1
-    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 1, 16, 0, 2, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 2
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 1, 16, 1, 2, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 2
+    assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 0, 32, 0, 2, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 2
     assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 1, 16, 0, 3, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
     assert L.fp4_block_gemm(2, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2
     # IF4 dequantisation: block 16 and a global scale

@@ -94,3 +94,59 @@ def test_if4_edges(cuda):
 def test_if4_full_outliers(cuda):
     """8192 x 8192 bf16 N(0,1) with 8 outlier columns x U(50,100), seed 5, two-pass global scale."""
     run_if4(synth.nv_outliers(), cuda, dequant=False)
+
+
+# ---------------------------------------------------------------------------------------------
+# IF4 behind the Walsh-Hadamard rotation (plain and randomised) and the SwiGLU fusion
+
+def _signs_dev(d, seed, cuda):
+    return torch.from_numpy(synth.rht_signs(d, seed).view(np.int32)).to(cuda)
+
+
+@pytest.mark.parametrize("d", [1024, 8192, 16384])
+@pytest.mark.parametrize("rht", [False, True])
+def test_if4_rotation_small(cuda, d, rht):
+    rows = 37
+    x = synth.fwht_laplace(rows, d, seed=6)
+    sg = synth.rht_signs(d, 31) if rht else None
+    q, s, g, c, rot = fp4.fwht_quantize(x.to(cuda), if4=True, want_rotated=True,
+                                        signs=_signs_dev(d, 31, cuda) if rht else None)
+    y, qo, so, go, co = O.fwht_quantize(synth.as_f32_numpy(x), if4=True, signs=sg)
+    assert np.array_equal(npy(rot), y)
+    assert np.float32(npy(g)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo)
+    assert np.array_equal(npy(s), so.ravel())
+    assert counts_of(c) == co and co["blocks_four"] > 0
+    # one pass under a caller-fixed global scale (half the derived one: more saturation)
+    gi = float(go) * 0.5
+    q, s, _, c, _ = fp4.fwht_quantize(x.to(cuda), if4=True, global_in=torch.tensor([gi], device=cuda),
+                                      signs=_signs_dev(d, 31, cuda) if rht else None)
+    _, qo, so, _, co = O.fwht_quantize(synth.as_f32_numpy(x), if4=True, signs=sg, global_in=gi)
+    assert np.array_equal(npy(q), qo) and np.array_equal(npy(s), so.ravel()) and counts_of(c) == co
+
+
+@pytest.mark.parametrize("d", [1024, 8192])
+def test_if4_swiglu_rotation_small(cuda, d):
+    rows = 37
+    g, u = synth.swiglu_inputs(rows, d, seed=3)
+    q, s, gs, c, _ = fp4.swiglu_fwht_quantize(g.to(cuda), u.to(cuda), if4=True, signs=_signs_dev(d, 34, cuda))
+    _, qo, so, go, co = O.swiglu_fwht_quantize(synth.as_f32_numpy(g), synth.as_f32_numpy(u), if4=True,
+                                               signs=synth.rht_signs(d, 34))
+    assert np.float32(npy(gs)[0]) == np.float32(go)
+    assert np.array_equal(npy(q), qo) and np.array_equal(npy(s), so.ravel()) and counts_of(c) == co
+
+
+def test_if4_rotation_full_sampled_rows(cuda):
+    """16384 x 8192 bf16 Laplace with spiked channels (seed 6), randomised rotation, IF4, a
+    caller-fixed global scale (so each row quantises on its own): 12 sampled rows bit-exact."""
+    x = synth.fwht_laplace()
+    d = x.shape[1]
+    gi = 0.0125
+    q, s, _, c, _ = fp4.fwht_quantize(x.to(cuda), if4=True, global_in=torch.tensor([gi], device=cuda),
+                                      signs=_signs_dev(d, 33, cuda))
+    rows = np.sort(np.random.default_rng(44).choice(x.shape[0], 12, replace=False))
+    _, qo, so, _, _ = O.fwht_quantize(synth.as_f32_numpy(x[rows]), if4=True, signs=synth.rht_signs(d, 33),
+                                      global_in=gi)
+    assert np.array_equal(npy(q)[rows], qo)
+    assert np.array_equal(npy(s).reshape(x.shape[0], d // 16)[rows], so)
+    assert counts_of(c)["blocks_four"] > 0
