@@ -63,3 +63,23 @@ def test_reference_arm_other_ranks_exit_without_work():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_profiles_are_consistent_with_the_bench():
+    """Every committed ncu summary names a command that runs committed files (a `--case` the bench
+    has), and the roofline kernel's recorded traffic equals its DRAM read + write rows."""
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+    pdir = os.path.join(ROOT, "profiles")
+    for f in sorted(os.listdir(pdir)):
+        text = open(os.path.join(pdir, f)).read()
+        for case in re.findall(r"python bench\.py --case (\w+)", text):
+            assert case in bench.CASES, (f, case)
+        assert "_work" not in text, f
+    t = bench.profile_traffic("nvfp4_quantize_8192x8192")
+    text = open(os.path.join(pdir, "nvfp4_quantize_8192x8192.md")).read()
+    four_six = text[text.index("## four-over-six"):text.index("## plain")]
+    rd = float(re.search(r"DRAM read \(`dram__bytes_read\.sum`\) \| ([0-9.]+) MB", four_six).group(1))
+    wr = float(re.search(r"DRAM write \(`dram__bytes_write\.sum`\) \| ([0-9.]+) MB", four_six).group(1))
+    assert abs(t - (rd + wr) * 1e6) < 0.02e6
