@@ -261,8 +261,9 @@ void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round
  * y_i = fl(x_i * R).
  * Four over six ([P] Four Over Six segment): each block is encoded with T = 6 and with T = 4 and
  * keeps T = 4 iff its fp32 sum of squared errors is strictly lower; the global scale uses M = 256
- * ("shrinking the whole tensor's global scale", 1 - 256/448 = 42.9%, "nearly 43 percent"), which
- * keeps the T = 4 code of the largest block (384) inside E4M3's range.                          */
+ * (the segment's smaller per-tensor scale that avoids overflow and costs about 43% of the dynamic
+ * range: 1 - 256/448 = 42.9%), which keeps the T = 4 code of the largest block (384) inside
+ * E4M3's range.                                                                                */
 
 float ora_nvfp4_global_scale(float amax_t, int four_six) {
   if (amax_t == 0.0f) return 1.0f;

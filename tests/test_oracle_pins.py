@@ -255,8 +255,8 @@ def test_nvfp4_exact_block():
 
 
 def test_nvfp4_scale_is_amax_over_six_cast_to_e4m3():
-    """The block scale is amax_b/(6 s_g) cast to E4M3 (podcast IF4 segment: "largest value over six,
-    cast to FP8 E4M3"), checked against torch's float8 cast of the fp64 ratio."""
+    """The block scale is amax_b/(6 s_g) cast to E4M3 (podcast IF4 segment: the block maximum over
+    six, in FP8 E4M3), checked against torch's float8 cast of the fp64 ratio."""
     x = O._f32(np.random.default_rng(4).standard_normal((64, 256)) * 3)
     q, s, sg, _ = O.nvfp4_quantize(x)
     amax_b = np.abs(x.reshape(64, 16, 16)).max(-1)
