@@ -254,7 +254,7 @@ FP4_API fp4_status fp4_to_e4m3(const unsigned char* q, long rows, long cols, uns
  * scales unchanged, run as tcgen05.mma kind::mxf8f6f4 block_scale scale_vec::1X (one scale per 32
  * values) with FP32 accumulation; the epilogue multiplies by 2^12, undoing the 2^-6 of each
  * operand, so C equals fp4_block_gemm(FP4_MXFP4, ...) up to the order of the FP32 accumulation.
- * [X] (FP4 operands on the FP8 MMA through the exact conversion) — an independent second tensor-
+ * [X] (FP4 operands run exactly on the FP8 MMA after that conversion) — an independent second tensor-
  * core GEMM for cross-checking the FP4 one.  MXFP4 only: the FP8 kind takes UE8M0 scales per 32,
  * which cannot carry NVFP4's E4M3 scales per 16.
  *   A8 : device [M, K] E4M3 bytes; B8 : device [N, K] E4M3 bytes (K-major).

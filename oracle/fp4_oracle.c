@@ -222,8 +222,8 @@ static float block_amax(const float* x, int n) {
 }
 
 /* Pack element 2j into the low nibble and 2j+1 into the high nibble of byte j
- * ([A] "Encode one MXFP4 block step by step": values 0 and 1 occupy the low and high half of the
- * first byte). */
+ * ([A] "Encode one MXFP4 block step by step": the first byte holds element 0 in its low half and
+ * element 1 in its high half). */
 static void pack_pairs(const uint8_t* codes, int n, uint8_t* out) {
   for (int j = 0; j < n / 2; ++j) out[j] = (uint8_t)((codes[2 * j] & 15) | ((codes[2 * j + 1] & 15) << 4));
 }
@@ -471,7 +471,7 @@ void ora_dequantize(const uint8_t* q, const uint8_t* scales, int format, long ro
 }
 
 /* E2M1 nibbles to E4M3 bytes ([X]: devices without the FP4 MMA run the operands on the FP8 MMA
- * after an exact conversion whose 2^6 folds into the scale).  Definition: the E4M3 encoding of
+ * after an exact conversion, the factor 2^6 being absorbed by the scale).  Definition: the E4M3 encoding of
  * value(n) * 2^-6 (exact: at most 2 significant bits, magnitude in [2^-7, 6 * 2^-6]), with the
  * nibble's sign bit, so -0 maps to 0x80.  q: [rows, cols/2] packed as the quantisers write;
  * out: [rows, cols], one byte per element.                                                      */

@@ -1,5 +1,5 @@
 """GPU parity of the FP8 tensor-core route for MXFP4 operands (metrale `hardware::exec`: FP4
-operands on the FP8 MMA through the exact E2M1 -> E4M3 conversion): the expansion kernel bit-exact
+operands run exactly on the FP8 MMA after the E2M1 -> E4M3 conversion): the expansion kernel bit-exact
 against the oracle's E4M3 encode of value * 2^-6, and the kind::mxf8f6f4 GEMM against the same fp64
 reference as the FP4 GEMM (|C - C64| <= 1e-3 * sum |ab|, plus 2^-8 |C64| on small shapes for the bf16
 output rounding) and against the FP4 GEMM itself.
