@@ -461,6 +461,38 @@ def test_if4_never_worse_than_nvfp4_and_keeps_its_fp4_blocks():
     assert abs((s >> 7).mean() - frac["gauss"]) < 0.1
 
 
+def test_if4_picks_lower_error_candidate_brute_force():
+    """Independent brute force: per block, the E2M1 candidate from torch's E4M3 cast and a numpy
+    nearest-lattice search, the INT4 candidate from numpy's round-half-even on the 6/7 step; the
+    oracle's reconstruction must be at least as good as the better of the two, and its flag must
+    name the candidate whose error it has."""
+    rng = np.random.default_rng(15)
+    x = O._f32(np.concatenate([rng.standard_normal((4, 64)), rng.uniform(-1, 1, (4, 64))]))
+    q, s, sg, c = O.nvfp4_quantize(x, if4=True)
+    lat = np.array(LATTICE)
+    xh = O.dequantize(q, s, O.IF4, sg).astype(np.float64)
+    step7 = np.float32(np.float32(sg) * (np.float32(6) / np.float32(7)))
+    for r in range(8):
+        for b in range(4):
+            blk = x[r, 16 * b:16 * b + 16]
+            inv = np.float32(1) / (np.float32(6) * np.float32(sg))
+            code = torch.tensor([np.float32(np.abs(blk).max()) * inv]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+            d = np.float32(O.e4m3_value(code))
+            R = np.float32(1) / (d * np.float32(sg))
+            y = (blk * R).astype(np.float64)
+            mags = np.array([lat[np.argmin(np.abs(lat - min(abs(v), 6.0)) + (np.arange(8) % 2) * 1e-12)] for v in y])
+            rec6 = np.sign(y) * mags * float(d) * sg
+            R7 = np.float32(1) / np.float32(d * step7)
+            k = np.clip(np.rint(np.abs((blk * R7).astype(np.float64))), 0, 7) * np.sign(blk)
+            rec7 = (k * float(d)).astype(np.float32) * step7
+            e6 = float(((blk.astype(np.float64) - rec6) ** 2).sum())
+            e7 = float(((blk.astype(np.float64) - rec7.astype(np.float64)) ** 2).sum())
+            got = float(((blk.astype(np.float64) - xh[r, 16 * b:16 * b + 16]) ** 2).sum())
+            assert got <= min(e6, e7) * (1 + 1e-5) + 1e-30
+            flagged = bool(s[r, b] & 0x80)
+            assert abs(got - (e7 if flagged else e6)) <= 1e-5 * max(got, 1e-30)
+
+
 def test_if4_nonfinite_blocks_keep_fp4():
     x = O._f32(np.random.default_rng(13).uniform(-1, 1, (1, 48)))
     x[0, 3], x[0, 20], x[0, 40] = np.inf, np.nan, -np.inf
