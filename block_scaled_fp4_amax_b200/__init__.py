@@ -7,7 +7,10 @@ libfp4mx.so; there is no CPU path.  If the shared library is missing or was buil
 process can load, the first call raises.
 
     from block_scaled_fp4_amax_b200 import mx_quantize, nvfp4_quantize, fwht_quantize, \
-        fp4_dequantize, fp4_block_gemm
+        swiglu_fwht_quantize, fp4_dequantize, fp4_block_gemm, fp4_to_e4m3, fp4_block_gemm_e4m3
+
+NVFP4 block modes: nvfp4_quantize / fwht_quantize take four_six=True (four over six) or if4=True
+(IF4: E2M1 or INT4 per block, flagged in scale bit 7; read back with fp4_dequantize(fmt=IF4)).
 """
 from __future__ import annotations
 
