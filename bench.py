@@ -282,8 +282,20 @@ def run_ours(args, td, rank, world, local):
     return line
 
 
-def cpu_baseline(x_cpu, rows=4096):
-    """The oracle as it stands, single-threaded, on the first `rows` rows of the workload."""
+def _oracle_chunk(xs):
+    """One thread's share of the all-cores oracle timing: plain then 4/6 on its rows."""
+    import oracle as O
+    O.nvfp4_quantize(xs, four_six=False)
+    O.nvfp4_quantize(xs, four_six=True)
+    return xs.shape[0]
+
+
+def cpu_baseline(x_cpu, rows=4096, max_workers=64):
+    """The oracle as it stands on the first `rows` rows of the workload: single-threaded, then the
+    same rows split over one thread per host core.  The oracle is C called through ctypes, which
+    releases the GIL for the call and keeps no global state, so the threads run in parallel; each
+    handles its rows as a tensor of its own."""
+    import concurrent.futures as cf
     import oracle as O
     xs = synth.as_f32_numpy(x_cpu[:rows])
     t = time.perf_counter()
@@ -291,8 +303,18 @@ def cpu_baseline(x_cpu, rows=4096):
     O.nvfp4_quantize(xs, four_six=True)
     dt = time.perf_counter() - t
     b = 2 * NV_BYTES_2PASS * xs.size
-    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of 8192 rows (plain + 4/6), {dt:.1f} s single-threaded C oracle"}
+    out = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"first {rows} of 8192 rows (plain + 4/6), {dt:.1f} s single-threaded C oracle"}
+    n = max(1, min(os.cpu_count() or 1, max_workers, rows))
+    chunks = np.array_split(xs, n)
+    with cf.ThreadPoolExecutor(max_workers=n) as ex:
+        t = time.perf_counter()
+        done = sum(ex.map(_oracle_chunk, chunks))
+        dt_all = time.perf_counter() - t
+    assert done == rows
+    out["all_cores"] = {"value": round(b / dt_all / 1e9, 4), "unit": "GB/s", "cores": n,
+                        "sample": f"the same rows over {n} threads, {dt_all:.2f} s"}
+    return out
 
 
 # ---------------------------------------------------------------------------------------------

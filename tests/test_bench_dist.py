@@ -83,3 +83,19 @@ def test_profiles_are_consistent_with_the_bench():
     rd = float(re.search(r"DRAM read \(`dram__bytes_read\.sum`\) \| ([0-9.]+) MB", four_six).group(1))
     wr = float(re.search(r"DRAM write \(`dram__bytes_write\.sum`\) \| ([0-9.]+) MB", four_six).group(1))
     assert abs(t - (rd + wr) * 1e6) < 0.02e6
+
+
+def test_oracle_is_thread_safe_for_the_all_cores_baseline():
+    """The all-cores CPU baseline runs the oracle from several threads at once: each thread's
+    result equals the same call made alone."""
+    import concurrent.futures as cf
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    rng = np.random.default_rng(3)
+    chunks = [rng.standard_normal((16, 256)).astype(np.float32) for _ in range(8)]
+    serial = [O.nvfp4_quantize(c, four_six=True) for c in chunks]
+    with cf.ThreadPoolExecutor(max_workers=8) as ex:
+        par = list(ex.map(lambda c: O.nvfp4_quantize(c, four_six=True), chunks))
+    for a, b in zip(serial, par):
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and a[2] == b[2] and a[3] == b[3]
