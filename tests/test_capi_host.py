@@ -156,3 +156,37 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fp4, "_lib", None)
     with pytest.raises(ImportError):
         fp4.lib()
+
+
+def test_header_is_plain_c_and_links_from_c(L, tmp_path):
+    """include/fp4mx.h is a C header: a C99 program includes it, links libfp4mx.so and gets the
+    synchronous argument checks without a GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_fp4mx.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "fp4mx.h"
+int main(void) {
+  if (strcmp(fp4_status_str(FP4_OK), "FP4_OK") != 0) return 1;
+  if (fp4_workspace_size(FP4_OP_NVFP4_QUANTIZE, 8192, 8192) < 4) return 2;
+  /* block 16 is not MXFP4's block: rejected before any CUDA call */
+  if (mx_quantize((const void*)0x10000, FP4_BF16, 128, 256, 16, FP4_MX_OCP_FLOOR, FP4_RNE, 0,
+                  FP4_SCALES_ROWMAJOR, (unsigned char*)0x10000, (unsigned char*)0x10000, 0, 0) != FP4_EINVAL)
+    return 3;
+  if (fp4_block_gemm_e4m3(100, 256, 128, 0, 0, 0, 0, 0, 256, 0, 0, 0) != FP4_EUNSUPPORTED) return 4;
+  printf("ok %s\n", fp4_last_error());
+  return 0;
+}
+''')
+    exe = tmp_path / "use_fp4mx"
+    libdir = os.path.dirname(fp4.LIB_PATH)
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                           "-L", libdir, "-lfp4mx", "-Wl,-rpath," + libdir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    assert out.stdout.startswith("ok ")
