@@ -275,7 +275,7 @@ def run_ours(args, td, rank, world, local):
                        "parallelism": f"replicas x{world}"},
             "roofline": roof, "e2e": e2e, "gpu_launches": NvStep.launches_per_step * args.steps,
             "clocks": clk}
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the oracle baseline is a 1-GPU figure
         line["cpu_baseline"] = cpu_baseline(x_cpu)
     if not args.no_secondary:
         line["secondary"] = secondary(args, dev, flush, td, pk)
