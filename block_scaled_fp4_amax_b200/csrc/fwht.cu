@@ -447,20 +447,22 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
 #pragma unroll
           for (int i = 0; i < B; ++i) cnt[2] += !isfinite(g[i]);
         }
+        // a block holding Inf or NaN is rejected: only its non-finite values are counted
+        const bool audit = am < 0x7F800000u;
         const int zc = zero_codes_n<B>(w);
         int zx = 0;  // a +-0 input always gives a zero code: count inputs only when both occur
         if (zc > 0 && mn == 0u) {
 #pragma unroll
           for (int i = 0; i < B; ++i) zx += g[i] == 0.0f;
         }
-        cnt[0] += (uint32_t)(zc - zx);
-        cnt[1] += sat;
+        cnt[0] += audit ? (uint32_t)(zc - zx) : 0u;
+        cnt[1] += audit ? sat : 0u;
         uint2* q2 = reinterpret_cast<uint2*>(p.q + prow * (D / 2) + i0 / 2);
 #pragma unroll
         for (int k = 0; k < W; k += 2) q2[k / 2] = make_uint2(w[k], w[k + 1]);
         const unsigned long long blk = (unsigned long long)prow * nb + (unsigned)(i0 / B);
         p.scales[scale_offset(blk, nb, p.tiled)] = (uint8_t)sc;
-        cnt[3] += four;
+        cnt[3] += audit ? four : 0u;
       }
     }
     if (!GATED) {

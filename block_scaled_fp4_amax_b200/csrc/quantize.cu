@@ -9,7 +9,8 @@
 //
 // Per-element work is kept to the encode itself: the block amax is an integer max over the
 // magnitude bits (which also exposes Inf/NaN: a block with a non-finite value has amax bits
-// >= 0x7F800000 and only then counts per element); saturation is counted per element only when
+// >= 0x7F800000, is rejected from the audit counters and only then counts its non-finite values
+// per element); saturation is counted per element only when
 // the block's normalised maximum exceeds 6; underflow = zero codes minus zero inputs, both from
 // popcounts over the packed bits.
 //
@@ -297,10 +298,13 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         }
       }
       if (valid) {
+        // a block holding Inf or NaN is rejected: it adds only to the non-finite count, and its
+        // codes and scale byte are unspecified
+        const bool audit = am < 0x7F800000u;
         const int zc = zero_codes_n<E>(w);
         // a +-0 input always gives a zero code, so inputs are counted only when both occur
-        cnt[0] += (uint32_t)(zc - ((zc > 0 && any_zero) ? Vec32<T>::zeros(raw[u]) : 0));
-        cnt[1] += sat;
+        cnt[0] += audit ? (uint32_t)(zc - ((zc > 0 && any_zero) ? Vec32<T>::zeros(raw[u]) : 0)) : 0u;
+        cnt[1] += audit ? sat : 0u;
         if (W == 2) {
           reinterpret_cast<uint2*>(p.q)[c] = make_uint2(w[0], w[W - 1]);
         } else {
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         if ((lane & (G - 1)) == 0) {
           const unsigned long long blk = (unsigned long long)c / G;
           p.scales[scale_offset(blk, p.nb, p.tiled)] = (uint8_t)sc;
-          cnt[3] += four;
+          cnt[3] += audit ? four : 0u;
         }
       }
     }

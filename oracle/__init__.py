@@ -55,62 +55,71 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        L.ora_e2m1_value.restype = ctypes.c_double
-        L.ora_e2m1_value.argtypes = [ctypes.c_int]
-        L.ora_e2m1_encode_rne.restype = ctypes.c_int
-        L.ora_e2m1_encode_rne.argtypes = [ctypes.c_float]
-        L.ora_e2m1_encode_sr.restype = ctypes.c_int
-        L.ora_e2m1_encode_sr.argtypes = [ctypes.c_float, ctypes.c_uint32]
-        L.ora_int4_value.restype = ctypes.c_double
-        L.ora_int4_value.argtypes = [ctypes.c_int]
-        L.ora_int4_encode_rne.restype = ctypes.c_int
-        L.ora_int4_encode_rne.argtypes = [ctypes.c_float]
-        L.ora_e4m3_value.restype = ctypes.c_double
-        L.ora_e4m3_value.argtypes = [ctypes.c_int]
-        L.ora_e4m3_encode_rne_satfinite.restype = ctypes.c_int
-        L.ora_e4m3_encode_rne_satfinite.argtypes = [ctypes.c_float]
-        L.ora_f32_to_bf16_rne.restype = ctypes.c_uint16
-        L.ora_f32_to_bf16_rne.argtypes = [ctypes.c_float]
-        L.ora_philox4x32_10.restype = None
-        L.ora_philox4x32_10.argtypes = [P, P, P]
-        L.ora_sr_word.restype = ctypes.c_uint32
-        L.ora_sr_word.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
-        L.ora_mx_exponent.restype = ctypes.c_int
-        L.ora_mx_exponent.argtypes = [ctypes.c_float, ctypes.c_int]
-        L.ora_mx_encode_block.restype = None
-        L.ora_mx_encode_block.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
-                                          ctypes.c_uint64, P, P]
-        L.ora_mx_quantize.restype = None
-        L.ora_mx_quantize.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_uint64, P, P, P]
-        L.ora_mx_quantize_at.restype = None
-        L.ora_mx_quantize_at.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_uint64, ctypes.c_uint64, P, P, P]
-        L.ora_nvfp4_global_scale.restype = ctypes.c_float
-        L.ora_nvfp4_global_scale.argtypes = [ctypes.c_float, ctypes.c_int]
-        L.ora_nvfp4_quantize.restype = None
-        L.ora_nvfp4_quantize.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_uint64, P, P, P, P, P]
-        L.ora_dequantize.restype = None
-        L.ora_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
-        L.ora_dequantize_f64.restype = None
-        L.ora_dequantize_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
-        L.ora_e2m1_to_e4m3.restype = None
-        L.ora_e2m1_to_e4m3.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
-        L.ora_fwht_norm_const.restype = ctypes.c_float
-        L.ora_fwht_norm_const.argtypes = [ctypes.c_long]
-        L.ora_fwht_rows.restype = None
-        L.ora_fwht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
-        L.ora_rht_rows.restype = None
-        L.ora_rht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P, P]
-        L.ora_exp_cw.restype = ctypes.c_float
-        L.ora_exp_cw.argtypes = [ctypes.c_float]
-        L.ora_silu_mul_rows.restype = None
-        L.ora_silu_mul_rows.argtypes = [P, P, ctypes.c_long, P]
-        _lib = L
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
+
+
+def configure(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C signatures on a loaded copy of the oracle library."""
+    P = ctypes.c_void_p
+    L.ora_e2m1_value.restype = ctypes.c_double
+    L.ora_e2m1_value.argtypes = [ctypes.c_int]
+    L.ora_e2m1_encode_rne.restype = ctypes.c_int
+    L.ora_e2m1_encode_rne.argtypes = [ctypes.c_float]
+    L.ora_e2m1_encode_sr.restype = ctypes.c_int
+    L.ora_e2m1_encode_sr.argtypes = [ctypes.c_float, ctypes.c_uint32]
+    L.ora_int4_value.restype = ctypes.c_double
+    L.ora_int4_value.argtypes = [ctypes.c_int]
+    L.ora_int4_encode_rne.restype = ctypes.c_int
+    L.ora_int4_encode_rne.argtypes = [ctypes.c_float]
+    L.ora_e4m3_value.restype = ctypes.c_double
+    L.ora_e4m3_value.argtypes = [ctypes.c_int]
+    L.ora_e4m3_encode_rne_satfinite.restype = ctypes.c_int
+    L.ora_e4m3_encode_rne_satfinite.argtypes = [ctypes.c_float]
+    L.ora_f32_to_bf16_rne.restype = ctypes.c_uint16
+    L.ora_f32_to_bf16_rne.argtypes = [ctypes.c_float]
+    L.ora_philox4x32_10.restype = None
+    L.ora_philox4x32_10.argtypes = [P, P, P]
+    L.ora_sr_word.restype = ctypes.c_uint32
+    L.ora_sr_word.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+    L.ora_mx_exponent.restype = ctypes.c_int
+    L.ora_mx_exponent.argtypes = [ctypes.c_float, ctypes.c_int]
+    L.ora_mx_encode_block.restype = None
+    L.ora_mx_encode_block.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                      ctypes.c_uint64, P, P]
+    L.ora_mx_quantize.restype = None
+    L.ora_mx_quantize.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_uint64, P, P, P]
+    L.ora_mx_quantize_at.restype = None
+    L.ora_mx_quantize_at.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_uint64, ctypes.c_uint64, P, P, P, P]
+    L.ora_nvfp4_global_scale.restype = ctypes.c_float
+    L.ora_nvfp4_global_scale.argtypes = [ctypes.c_float, ctypes.c_int]
+    L.ora_nvfp4_quantize.restype = None
+    L.ora_nvfp4_quantize.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_uint64, P, P, P, P, P]
+    L.ora_nvfp4_quantize_spec.restype = None
+    L.ora_nvfp4_quantize_spec.argtypes = [P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_uint64, P, P, P, P, P, P]
+    L.ora_block_nonfinite.restype = ctypes.c_int
+    L.ora_block_nonfinite.argtypes = [P, ctypes.c_int]
+    L.ora_dequantize.restype = None
+    L.ora_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
+    L.ora_dequantize_f64.restype = None
+    L.ora_dequantize_f64.argtypes = [P, P, ctypes.c_int, ctypes.c_long, ctypes.c_long, ctypes.c_float, P]
+    L.ora_e2m1_to_e4m3.restype = None
+    L.ora_e2m1_to_e4m3.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
+    L.ora_fwht_norm_const.restype = ctypes.c_float
+    L.ora_fwht_norm_const.argtypes = [ctypes.c_long]
+    L.ora_fwht_rows.restype = None
+    L.ora_fwht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P]
+    L.ora_rht_rows.restype = None
+    L.ora_rht_rows.argtypes = [P, ctypes.c_long, ctypes.c_long, P, P]
+    L.ora_exp_cw.restype = ctypes.c_float
+    L.ora_exp_cw.argtypes = [ctypes.c_float]
+    L.ora_silu_mul_rows.restype = None
+    L.ora_silu_mul_rows.argtypes = [P, P, ctypes.c_long, P]
+    return L
 
 
 def _p(a: np.ndarray):
@@ -196,19 +205,15 @@ def mx_encode_block(x, e: int, round: int = RNE, seed: int = 0, idx0: int = 0):
     return codes, c.as_dict()
 
 
-def mx_quantize(x, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0):
-    """MXFP4 quantise a [rows, cols] array. Returns (q [rows, cols/2] u8, scales [rows, cols/32] u8, counts)."""
-    x = _f32(x)
-    rows, cols = x.shape
-    assert cols % 32 == 0
-    q = np.zeros((rows, cols // 2), dtype=np.uint8)
-    s = np.zeros((rows, cols // 32), dtype=np.uint8)
-    c = _Counts()
-    lib().ora_mx_quantize(_p(x), rows, cols, int(policy), int(round), int(seed), _p(q), _p(s), ctypes.byref(c))
-    return q, s, c.as_dict()
+def mx_quantize(x, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0, spec: bool = False):
+    """MXFP4 quantise a [rows, cols] array. Returns (q [rows, cols/2] u8, scales [rows, cols/32] u8,
+    counts), and with `spec` also the bool [rows, cols/32] mask of blocks whose outputs are defined
+    (False for a rejected block, one holding Inf or NaN: its codes and scale are left open)."""
+    return mx_quantize_rows_at(x, 0, policy=policy, round=round, seed=seed, spec=spec)
 
 
-def mx_quantize_rows_at(x, idx_base: int, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0):
+def mx_quantize_rows_at(x, idx_base: int, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0,
+                        spec: bool = False):
     """mx_quantize of rows that start at flat element index `idx_base` of a larger tensor (the
     random words of stochastic rounding follow the flat index)."""
     x = _f32(x)
@@ -216,15 +221,18 @@ def mx_quantize_rows_at(x, idx_base: int, policy: int = OCP_FLOOR, round: int = 
     assert cols % 32 == 0
     q = np.zeros((rows, cols // 2), dtype=np.uint8)
     s = np.zeros((rows, cols // 32), dtype=np.uint8)
+    m = np.zeros((rows, cols // 32), dtype=np.uint8)
     c = _Counts()
     lib().ora_mx_quantize_at(_p(x), rows, cols, int(policy), int(round), int(seed), int(idx_base), _p(q), _p(s),
-                             ctypes.byref(c))
-    return q, s, c.as_dict()
+                             ctypes.byref(c), _p(m))
+    return (q, s, c.as_dict(), m.astype(bool)) if spec else (q, s, c.as_dict())
 
 
-def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, global_in=None, if4: bool = False):
+def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, global_in=None, if4: bool = False,
+                   spec: bool = False):
     """NVFP4 quantise (with `if4`, IF4: each block E2M1 or INT4, the choice in scale bit 7).
-    Returns (q, scales [rows, cols/16], s_g, counts)."""
+    Returns (q, scales [rows, cols/16], s_g, counts), and with `spec` also the bool [rows, cols/16]
+    mask of blocks whose outputs are defined (see ora_nvfp4_quantize_spec)."""
     assert not (four_six and if4)
     mode = 2 if if4 else int(bool(four_six))
     x = _f32(x)
@@ -234,10 +242,12 @@ def nvfp4_quantize(x, round: int = RNE, four_six: bool = False, seed: int = 0, g
     s = np.zeros((rows, cols // 16), dtype=np.uint8)
     gin = None if global_in is None else np.array([global_in], dtype=np.float32)
     gout = np.zeros(1, dtype=np.float32)
+    m = np.zeros((rows, cols // 16), dtype=np.uint8)
     c = _Counts()
-    lib().ora_nvfp4_quantize(_p(x), rows, cols, int(round), mode, int(seed),
-                             None if gin is None else _p(gin), _p(gout), _p(q), _p(s), ctypes.byref(c))
-    return q, s, float(gout[0]), c.as_dict()
+    lib().ora_nvfp4_quantize_spec(_p(x), rows, cols, int(round), mode, int(seed),
+                                  None if gin is None else _p(gin), _p(gout), _p(q), _p(s), ctypes.byref(c), _p(m))
+    out = (q, s, float(gout[0]), c.as_dict())
+    return out + (m.astype(bool),) if spec else out
 
 
 def dequantize(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
@@ -301,21 +311,22 @@ def silu_mul(g, u) -> np.ndarray:
 
 
 def swiglu_fwht_quantize(g, u, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
-                         global_in=None, signs=None, if4: bool = False):
+                         global_in=None, signs=None, if4: bool = False, spec: bool = False):
     """SiLU(g) * u in fp32 (no storage rounding), then the rotation and quantiser of fwht_quantize."""
     return fwht_quantize(silu_mul(g, u), fmt=fmt, round=round, four_six=four_six, seed=seed,
-                         global_in=global_in, signs=signs, if4=if4)
+                         global_in=global_in, signs=signs, if4=if4, spec=spec)
 
 
 def fwht_quantize(x, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
-                  global_in=None, signs=None, if4: bool = False):
-    """Rotation (randomised with `signs`) followed by the quantiser of `fmt` on the rotated fp32 tensor."""
+                  global_in=None, signs=None, if4: bool = False, spec: bool = False):
+    """Rotation (randomised with `signs`) followed by the quantiser of `fmt` on the rotated fp32
+    tensor.  Returns (y, q, s, s_g, counts) and, with `spec`, the defined-block mask."""
     y = fwht(x, signs)
     if fmt == NVFP4:
-        q, s, sg, c = nvfp4_quantize(y, round=round, four_six=four_six, seed=seed, global_in=global_in, if4=if4)
-        return y, q, s, sg, c
-    q, s, c = mx_quantize(y, policy=OCP_FLOOR, round=round, seed=seed)
-    return y, q, s, 1.0, c
+        r = nvfp4_quantize(y, round=round, four_six=four_six, seed=seed, global_in=global_in, if4=if4, spec=spec)
+        return (y,) + r
+    r = mx_quantize(y, policy=OCP_FLOOR, round=round, seed=seed, spec=spec)
+    return (y,) + r[:2] + (1.0,) + r[2:]
 
 
 def bf16_bits(x) -> np.ndarray:

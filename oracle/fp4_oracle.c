@@ -52,12 +52,14 @@ static int e2m1_nearest_mag(double a) {
   return best;
 }
 
-/* RNE encode of a normalised value y.  Magnitudes strictly above 6 clamp to 6 ([A]: "the lab
- * clamps them to signed 6").  The sign bit always follows signbit(y), so a negative value that
- * rounds to zero encodes -0 (0x8).  E2M1 has no NaN ([E] §1); reading: a NaN encodes as +6 (0x7),
- * its sign carrying no meaning.  Returns the 4-bit code. */
+/* RNE encode of a normalised value y.  Magnitudes strictly above 6, infinities included, clamp to
+ * 6 ([A]: "the lab clamps them to signed 6").  The sign bit always follows signbit(y), so a
+ * negative value that rounds to zero encodes -0 (0x8).  Returns the 4-bit code.
+ * Domain: y is not NaN.  E2M1 has no NaN ([E] §1) and [A]'s receipt rejects non-finite input, so
+ * the quantisers never encode a block that holds one (see ora_block_rejected); a NaN here gets
+ * the placeholder -1, which no caller stores. */
 int ora_e2m1_encode_rne(float y) {
-  if (isnan(y)) return 7;
+  if (isnan(y)) return -1;
   double a = fabs((double)y);
   int mag = (a > 6.0) ? 7 : e2m1_nearest_mag(a);
   return (signbit(y) ? 8 : 0) | mag;
@@ -104,7 +106,7 @@ uint32_t ora_sr_word(uint64_t seed, uint64_t idx) {
  * lattice magnitudes (lo = a when a is a lattice point); p = (a-lo)/(hi-lo) is exact; the value
  * rounds up iff r < ceil(p * 2^32).  a > 6 clamps to 6 (saturation, as for RNE).             */
 int ora_e2m1_encode_sr(float y, uint32_t r) {
-  if (isnan(y)) return 7; /* as for RNE */
+  if (isnan(y)) return -1; /* outside the domain, as for RNE */
   double a = fabs((double)y);
   int sign = signbit(y) ? 8 : 0;
   if (a > 6.0) return sign | 7;
@@ -132,10 +134,11 @@ double ora_e4m3_value(int code) {
 }
 
 /* Round-to-nearest-even onto the positive E4M3 lattice, saturating to 448 (the "satfinite"
- * reading: a magnitude above 448, Inf included, becomes 448).  u >= 0.  Ties take the even code.
- * A NaN u (a block holding a NaN) gives E4M3's NaN byte 0x7F, so the block decodes to NaN.   */
+ * reading: a magnitude above 448, Inf included, becomes 448).  Ties take the even code.
+ * Domain: u >= 0 and not NaN (a block maximum of a finite block times a per-tensor factor); a
+ * NaN gets the placeholder -1, which no caller stores.                                       */
 int ora_e4m3_encode_rne_satfinite(float u) {
-  if (isnan(u)) return 0x7F;
+  if (isnan(u)) return -1;
   double a = (double)u;
   if (!(a <= 448.0)) return 0x7E;
   int best = 0;
@@ -174,11 +177,10 @@ static int floor_log2(double a) { /* a > 0 finite: exact via frexp (a = f * 2^x,
   return x - 1;
 }
 
-/* A non-finite block maximum (a block holding Inf or NaN) counts as 2^128, just above every
- * float: e = 126 under both rules (reading; the pages leave non-finite input open).          */
+/* Domain: amax finite (a block holding Inf or NaN is rejected before its exponent is taken); a
+ * non-finite amax gets the placeholder 0.                                                      */
 int ora_mx_exponent(float amax, int policy) {
-  if (amax == 0.0f) return 0;
-  if (!isfinite(amax)) return 126;
+  if (amax == 0.0f || !isfinite(amax)) return 0;
   double a = (double)amax;
   int e;
   if (policy == 0) {
@@ -192,25 +194,45 @@ int ora_mx_exponent(float amax, int policy) {
   return e;
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* Rejected blocks.  [A] "Publish the MXFP4 audit receipt" lists non-finite input among the inputs
+ * to reject, and E2M1 has no Inf or NaN ([E] §1).  Reading: a block holding an Inf or a NaN is
+ * rejected.  Its non-finite values are counted in `nonfinite`; its codes and scale byte are left
+ * unspecified (the oracle writes zeros there as placeholders, not as a definition) and it adds
+ * nothing to the underflow, saturation and blocks_four counters, which audit encoded values.
+ * Returns the number of non-finite values among the n (0: the block is encoded).              */
+int ora_block_nonfinite(const float* x, int n) {
+  int k = 0;
+  for (int i = 0; i < n; ++i)
+    if (!isfinite(x[i])) k += 1;
+  return k;
+}
+
 /* Encode one block with a given shared exponent e (the manual path of the audit page, and the
  * inner step of ora_mx_quantize): y = x * 2^-e in fp32 (exact unless it underflows), then RNE
  * or stochastic E2M1.  idx0 is the flat index of x[0] (for the random word).  Codes land in
  * codes[0..n-1] (one per byte, unpacked). */
 void ora_mx_encode_block(const float* x, int n, int e, int round, uint64_t seed, uint64_t idx0,
                          uint8_t* codes, ora_counts* cnt) {
+  int bad = ora_block_nonfinite(x, n);
+  if (bad) { /* rejected: placeholder codes, only the non-finite count */
+    cnt->nonfinite += (uint64_t)bad;
+    memset(codes, 0, (size_t)n);
+    return;
+  }
   float inv_scale = ldexpf(1.0f, -e);
   for (int i = 0; i < n; ++i) {
-    if (!isfinite(x[i])) cnt->nonfinite += 1;
     float y = x[i] * inv_scale;
     int c = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
-    if (fabsf(y) > 6.0f) cnt->saturation += 1; /* Inf included, NaN not */
+    if (fabsf(y) > 6.0f) cnt->saturation += 1;
     if (x[i] != 0.0f && (c & 7) == 0) cnt->underflow += 1;
     codes[i] = (uint8_t)c;
   }
 }
 
 /* Largest magnitude of n values; a NaN anywhere makes it NaN (the IEEE maximum that propagates
- * NaN, as torch.amax does).                                                                    */
+ * NaN, as torch.amax does).  Only the tensor maximum of the two-pass NVFP4 scale depends on the
+ * NaN rule: a rejected block's own maximum is never used.                                       */
 static float block_amax(const float* x, int n) {
   float m = 0.0f;
   for (int i = 0; i < n; ++i) {
@@ -230,17 +252,21 @@ static void pack_pairs(const uint8_t* codes, int n, uint8_t* out) {
 
 /* x: [rows, cols] fp32 row-major; q: [rows, cols/2]; scales: [rows, cols/32] row-major bytes. */
 /* idx_base: flat element index of x[0] in the tensor the rows belong to (the random words of
- * stochastic rounding are indexed by it; 0 for a whole tensor). */
+ * stochastic rounding are indexed by it; 0 for a whole tensor).  spec (nullable): one byte per
+ * block, 1 where the block's outputs are defined (every value finite), 0 for a rejected block.
+ * With a finite block the normalised values x * 2^-e are finite, so nothing else is left open. */
 void ora_mx_quantize_at(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
-                        uint64_t idx_base, uint8_t* q, uint8_t* scales, ora_counts* cnt) {
+                        uint64_t idx_base, uint8_t* q, uint8_t* scales, ora_counts* cnt, uint8_t* spec) {
   const int B = 32;
   long nb = cols / B;
   uint8_t codes[32];
   for (long r = 0; r < rows; ++r) {
     for (long j = 0; j < nb; ++j) {
       const float* xb = x + r * cols + j * B;
-      int e = ora_mx_exponent(block_amax(xb, B), policy);
-      scales[r * nb + j] = (uint8_t)(e + 127);
+      int bad = ora_block_nonfinite(xb, B);
+      int e = bad ? 0 : ora_mx_exponent(block_amax(xb, B), policy);
+      scales[r * nb + j] = bad ? 0 : (uint8_t)(e + 127); /* rejected block: placeholder byte */
+      if (spec) spec[r * nb + j] = bad ? 0 : 1;
       ora_mx_encode_block(xb, B, e, round, seed, idx_base + (uint64_t)(r * cols + j * B), codes, cnt);
       pack_pairs(codes, B, q + r * (cols / 2) + j * (B / 2));
     }
@@ -249,7 +275,7 @@ void ora_mx_quantize_at(const float* x, long rows, long cols, int policy, int ro
 
 void ora_mx_quantize(const float* x, long rows, long cols, int policy, int round, uint64_t seed,
                      uint8_t* q, uint8_t* scales, ora_counts* cnt) {
-  ora_mx_quantize_at(x, rows, cols, policy, round, seed, 0, q, scales, cnt);
+  ora_mx_quantize_at(x, rows, cols, policy, round, seed, 0, q, scales, cnt, 0);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -271,17 +297,27 @@ float ora_nvfp4_global_scale(float amax_t, int four_six) {
   return amax_t / six_m;
 }
 
-/* One candidate encoding of a 16-block: returns the sum of squared dequantisation errors.     */
+/* One candidate encoding of a 16-block of finite values: returns the sum of squared
+ * dequantisation errors.  *defined is cleared when one of the reading's fp32 steps gives a NaN
+ * (the scale argument u, or a normalised value y): E4M3 and E2M1 encodings of a NaN are not
+ * fixed by the pages.  That needs a per-tensor scale outside its domain (fl(T*s_g) rounding to
+ * zero or overflowing, or a reciprocal of fl(d*s_g) that overflows), never a normal one.      */
 static float nv_candidate(const float* x, int n, float amax_b, float s_g, float T, int round,
                           uint64_t seed, uint64_t idx0, uint8_t* codes, int* scale_code,
-                          ora_counts* c) {
+                          ora_counts* c, int* defined) {
   float ts = T * s_g;
   float inv_t = 1.0f / ts;
   float u = amax_b * inv_t;
+  memset(c, 0, sizeof(*c));
+  memset(codes, 0, (size_t)n);
+  *scale_code = 0;
+  if (isnan(u)) {
+    *defined = 0;
+    return NAN;
+  }
   int sc = ora_e4m3_encode_rne_satfinite(u);
   float d = (float)ora_e4m3_value(sc);
   *scale_code = sc;
-  memset(c, 0, sizeof(*c));
   if (sc == 0) {
     for (int i = 0; i < n; ++i) {
       codes[i] = (uint8_t)(signbit(x[i]) ? 8 : 0);
@@ -292,8 +328,12 @@ static float nv_candidate(const float* x, int n, float amax_b, float s_g, float 
     float R = 1.0f / ds;
     for (int i = 0; i < n; ++i) {
       float y = x[i] * R;
+      if (isnan(y)) {
+        *defined = 0;
+        return NAN;
+      }
       int code = (round == 0) ? ora_e2m1_encode_rne(y) : ora_e2m1_encode_sr(y, ora_sr_word(seed, idx0 + i));
-      if (fabsf(y) > 6.0f) c->saturation += 1; /* Inf included, NaN not */
+      if (fabsf(y) > 6.0f) c->saturation += 1; /* an overflowed (infinite) y included */
       if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
       codes[i] = (uint8_t)code;
     }
@@ -322,7 +362,8 @@ static float nv_candidate(const float* x, int n, float amax_b, float s_g, float 
  *     the reconstruction is fl(fl(k * d) * s7) (k * d is exact), the INT4 analogue of
  *     fl(fl(v * d) * s_g);
  *   - INT4 is kept iff its fp32 sequential error sum is strictly lower (a tie or a NaN keeps E2M1),
- *     and a block whose scale code is 0 keeps E2M1 (both reconstructions are zero);
+ *     and only when R7 is a finite nonzero number: a block whose scale code is 0 (both
+ *     reconstructions are zero) or whose INT4 step has no usable reciprocal keeps E2M1;
  *   - the global scale is plain NVFP4's (M = 448); round to nearest only;
  *   - counters of an INT4 block: saturation |y| > 7, underflow x != 0 with k = 0.               */
 
@@ -332,10 +373,10 @@ double ora_int4_value(int code) {
 }
 
 /* Nearest of the integers 0..7 to |y| (ties to the even one), by enumerating the lattice; a
- * magnitude above 7, Inf included, clamps to 7.  The sign bit follows signbit(y); a NaN gives +7
- * (as E2M1 gives +6).                                                                          */
+ * magnitude above 7, Inf included, clamps to 7.  The sign bit follows signbit(y).  Domain as
+ * for E2M1: y is not NaN (placeholder -1 otherwise).                                           */
 int ora_int4_encode_rne(float y) {
-  if (isnan(y)) return 7;
+  if (isnan(y)) return -1;
   double a = fabs((double)y);
   int best = 7;
   if (!(a > 7.0)) {
@@ -353,7 +394,8 @@ int ora_int4_encode_rne(float y) {
 }
 
 /* The INT4 candidate of one block with E4M3 scale code sc (nonzero): codes, counters and the
- * fp32 sequential sum of squared errors.                                                       */
+ * fp32 sequential sum of squared errors.  Returns NaN (the candidate is not taken) when R7 is not
+ * a finite nonzero number.                                                                     */
 static float if4_int_candidate(const float* x, int n, int sc, float s_g, uint8_t* codes, ora_counts* c) {
   float six_sevenths = 6.0f / 7.0f;
   float s7 = s_g * six_sevenths;
@@ -361,10 +403,11 @@ static float if4_int_candidate(const float* x, int n, int sc, float s_g, uint8_t
   float D7 = d * s7;
   float R7 = 1.0f / D7;
   memset(c, 0, sizeof(*c));
+  if (!isfinite(R7) || R7 == 0.0f) return NAN;
   for (int i = 0; i < n; ++i) {
     float y = x[i] * R7;
     int code = ora_int4_encode_rne(y);
-    if (fabsf(y) > 7.0f) c->saturation += 1; /* Inf included, NaN not */
+    if (fabsf(y) > 7.0f) c->saturation += 1; /* an overflowed (infinite) y included */
     if (x[i] != 0.0f && (code & 7) == 0) c->underflow += 1;
     codes[i] = (uint8_t)code;
   }
@@ -381,10 +424,16 @@ static float if4_int_candidate(const float* x, int n, int sc, float s_g, uint8_t
 
 /* x: [rows, cols] fp32; q: [rows, cols/2]; scales: [rows, cols/16] row-major E4M3 bytes.
  * mode: 0 plain NVFP4, 1 four over six, 2 IF4.
- * global_in: NULL -> s_g from the tensor amax; else s_g = *global_in.                          */
-void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mode, uint64_t seed,
-                        const float* global_in, float* global_out, uint8_t* q, uint8_t* scales,
-                        ora_counts* cnt) {
+ * global_in: NULL -> s_g from the tensor amax; else s_g = *global_in.
+ * spec (nullable): one byte per block, 1 where the block's outputs are defined.  A block is left
+ * unspecified (placeholder zeros; only its non-finite values counted) when it is rejected (holds
+ * Inf or NaN), when the per-tensor scale is not finite (the tensor maximum of a tensor holding a
+ * NaN or an Inf), or when a step of a candidate it compares gives a NaN (nv_candidate).  A finite
+ * s_g >= 2^-118 rules the last case out: every nonzero block scale fl(d*s_g) is then at least
+ * 2^-127 and has a finite reciprocal.                                                          */
+void ora_nvfp4_quantize_spec(const float* x, long rows, long cols, int round, int mode, uint64_t seed,
+                             const float* global_in, float* global_out, uint8_t* q, uint8_t* scales,
+                             ora_counts* cnt, uint8_t* spec) {
   const int B = 16;
   long nb = cols / B;
   float s_g;
@@ -405,17 +454,27 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mod
     for (long j = 0; j < nb; ++j) {
       const float* xb = x + r * cols + j * B;
       uint64_t idx0 = (uint64_t)(r * cols + j * B);
-      for (int i = 0; i < B; ++i)
-        if (!isfinite(xb[i])) cnt->nonfinite += 1;
-      float amax_b = block_amax(xb, B);
+      int bad = ora_block_nonfinite(xb, B);
+      cnt->nonfinite += (uint64_t)bad;
+      int defined = !bad && isfinite(s_g);
+      float amax_b = 0.0f, sse6 = 0.0f, sse4 = 0.0f;
       ora_counts k6, k4;
-      int sc6, sc4;
-      float sse6 = nv_candidate(xb, B, amax_b, s_g, 6.0f, round, seed, idx0, c6, &sc6, &k6);
+      int sc6 = 0, sc4 = 0;
+      if (defined) {
+        amax_b = block_amax(xb, B);
+        sse6 = nv_candidate(xb, B, amax_b, s_g, 6.0f, round, seed, idx0, c6, &sc6, &k6, &defined);
+        if (mode == 1) sse4 = nv_candidate(xb, B, amax_b, s_g, 4.0f, round, seed, idx0, c4, &sc4, &k4, &defined);
+      }
+      if (spec) spec[r * nb + j] = (uint8_t)defined;
+      if (!defined) { /* placeholders: the outputs of this block are not fixed */
+        scales[r * nb + j] = 0;
+        memset(q + r * (cols / 2) + j * (B / 2), 0, B / 2);
+        continue;
+      }
       const uint8_t* pick = c6;
       int sc = sc6;
       ora_counts k = k6;
       if (mode == 1) {
-        float sse4 = nv_candidate(xb, B, amax_b, s_g, 4.0f, round, seed, idx0, c4, &sc4, &k4);
         if (sse4 < sse6) {
           pick = c4;
           sc = sc4;
@@ -437,6 +496,12 @@ void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mod
       pack_pairs(pick, B, q + r * (cols / 2) + j * (B / 2));
     }
   }
+}
+
+void ora_nvfp4_quantize(const float* x, long rows, long cols, int round, int mode, uint64_t seed,
+                        const float* global_in, float* global_out, uint8_t* q, uint8_t* scales,
+                        ora_counts* cnt) {
+  ora_nvfp4_quantize_spec(x, rows, cols, round, mode, seed, global_in, global_out, q, scales, cnt, 0);
 }
 
 /* ------------------------------------------------------------------------------------------ */

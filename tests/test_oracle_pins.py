@@ -195,11 +195,20 @@ def test_mx_ramp_fixtures():
 
 
 def test_e8m0_limits():
+    """The E8M0 limits ("MXFP4 Quantization: Audit", "Read the shared E8M0 scale"): exponent -127
+    is byte 0 and 127 is byte 254.  A block encoded at each limit exponent and reconstructed from
+    the printed byte gives its values back exactly (2^-127 * v and 2^127 * v are representable)."""
     for e, byte in golden_rows("e8m0_limits.txt"):
         e, byte = int(e), int(byte)
-        x = np.full(32, 1.0, dtype=np.float32)
-        codes, _ = O.mx_encode_block(x, e)
-        assert e + 127 == byte  # the byte mapping the oracle stores
+        # the whole lattice, both signs; at e = 127 only the magnitudes below 2 (2 * 2^127 overflows fp32)
+        lat = [0, 0.5, 1, 1.5] if e == 127 else [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+        mags = np.resize(np.array(lat, dtype=np.float64), 16)
+        x = (np.concatenate([mags, -mags]) * 2.0 ** e).astype(np.float32)
+        codes, c = O.mx_encode_block(x, e)
+        q = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)[None, :]
+        rec = O.dequantize(q, np.array([[byte]], dtype=np.uint8), O.MXFP4)[0]
+        assert np.array_equal(rec, x), (e, rec, x)
+        assert c["saturation"] == 0 and c["underflow"] == 0
     # data-driven exponent clamps at -127 (byte 0) and never yields byte 255
     tiny = np.full((1, 32), 2.0 ** -140, dtype=np.float32)
     assert O.mx_quantize(tiny)[1][0, 0] == 0
@@ -256,15 +265,23 @@ def test_nvfp4_exact_block():
 
 def test_nvfp4_scale_is_amax_over_six_cast_to_e4m3():
     """The block scale is amax_b/(6 s_g) cast to E4M3 (podcast IF4 segment: the block maximum over
-    six, in FP8 E4M3), checked against torch's float8 cast of the fp64 ratio."""
+    six, in FP8 E4M3) under the FP32 global amax_t/(6*448) ("Sub-4-Bit Microscaling" §2).  Every
+    block is compared exactly with the reading's fp32 steps restated in numpy, s_g = fl(amax_t /
+    2688), inv6 = fl(1/fl(6 s_g)), u = fl(amax_b * inv6), the code from torch's float8_e4m3fn
+    cast; and, through the fp64 ratio, never more than one code from the real amax_b/(6 s_g)."""
     x = O._f32(np.random.default_rng(4).standard_normal((64, 256)) * 3)
     q, s, sg, _ = O.nvfp4_quantize(x)
-    amax_b = np.abs(x.reshape(64, 16, 16)).max(-1)
-    ideal = torch.from_numpy((amax_b / (6.0 * sg)).astype(np.float32)).to(torch.float8_e4m3fn)
-    ideal = ideal.view(torch.uint8).numpy()
-    # fp32 rounding of 1/(6 s_g) may move a value across an E4M3 midpoint: at most one code apart
+    f = np.float32
+    amax_t = np.abs(x).max()
+    assert sg == f(amax_t) / f(2688.0)
+    inv6 = f(1.0) / (f(6.0) * f(sg))
+    amax_b = np.abs(x.reshape(64, 16, 16)).max(-1).astype(np.float32)
+    u = (amax_b * inv6).astype(np.float32)
+    code = torch.from_numpy(u).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(s, code)
+    ideal = torch.from_numpy((amax_b.astype(np.float64) / (6.0 * float(sg))).astype(np.float32))
+    ideal = ideal.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.abs(s.astype(int) - ideal.astype(int)).max() <= 1
-    assert (s == ideal).mean() > 0.99
     assert s.max() <= 0x7E
 
 
@@ -285,15 +302,26 @@ def test_four_over_six_pins():
     q, s, sg, c = O.nvfp4_quantize(x, four_six=True, global_in=1.0 / 16)
     assert c["blocks_four"] == 1
     assert np.array_equal(O.dequantize(q, s, O.NVFP4, sg), x)
-    # in T=4 blocks the +-6 codes (the two values given up) never appear
+    # in T=4 blocks the +-6 codes (the two values the segment says are given up) never appear.
+    # The T=4 blocks are found independently of the oracle's choice: the stored scale byte equals
+    # the E4M3 cast (torch) of fl(amax_b * fl(1/fl(4 s_g))) and differs from the T=6 one.
     y = O._f32(np.random.default_rng(6).standard_normal((256, 256)))
     q, s, sg, c = O.nvfp4_quantize(y, four_six=True)
-    assert c["blocks_four"] > 0
-    q6, s6, _, _ = O.nvfp4_quantize(y, four_six=False, global_in=sg)
+    f = np.float32
+    amax_b = np.abs(y.reshape(256, 16, 16)).max(-1).astype(np.float32)
+
+    def code_for(T):
+        u = (amax_b * (f(1.0) / (f(T) * f(sg)))).astype(np.float32)
+        return torch.from_numpy(u).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    c4, c6 = code_for(4.0), code_for(6.0)
+    four_blocks = (s == c4) & (c4 != c6)
+    assert four_blocks.sum() > 0 and four_blocks.sum() <= c["blocks_four"]
+    assert np.all((s == c4) | (s == c6))
     codes = np.stack([q & 15, q >> 4], -1).reshape(256, 16, 16)
-    four_blocks = (s.reshape(256, 16) != s6.reshape(256, 16)) | np.any(codes != np.stack([q6 & 15, q6 >> 4], -1).reshape(256, 16, 16), -1)
-    assert four_blocks.sum() > 0
-    assert not np.isin(codes[four_blocks] & 7, [7]).any() or int(gave) == 2
+    mags = codes[four_blocks] & 7
+    assert not (mags == 7).any()                             # no +-6 in a T=4 block
+    assert int(gave) == len(set(LATTICE[-1:] + [-v for v in LATTICE[-1:]]))  # the two values: +-6
 
 
 def test_four_over_six_picks_lower_error_candidate_brute_force():
@@ -326,31 +354,63 @@ def test_four_over_six_picks_lower_error_candidate_brute_force():
 
 
 # ---------------------------------------------------------------------------------------------
-# Non-finite inputs (the pages leave them open; these are the readings the library follows)
+# Non-finite inputs ("MXFP4 Quantization: Audit", "Publish the MXFP4 audit receipt": non-finite
+# input is among the inputs to reject).  A block holding Inf or NaN is rejected: its codes and
+# scale byte are left open, its non-finite values are counted, and it adds nothing to the other
+# counters.  The tensor maximum propagates NaN as torch.amax does.
 
-def test_nonfinite_readings():
-    """NaN propagates through the block and tensor maxima as in torch.amax; an E4M3 scale of a NaN
-    maximum is the NaN byte torch's float8_e4m3fn cast gives (0x7F); Inf saturates to 448 (0x7E);
-    E2M1 and INT4 have no NaN and encode one as their largest positive code."""
-    nan_e4m3 = torch.tensor([float("nan")]).to(torch.float8_e4m3fn).view(torch.uint8).item()
-    assert O.e4m3_encode(float("nan")) == (nan_e4m3 & 0x7F) == 0x7F
-    assert O.e4m3_encode(float("inf")) == 0x7E
-    assert O.e2m1_encode_rne(float("nan")) == 7 and O.e2m1_encode_sr(float("nan"), 0) == 7
-    assert O.e2m1_encode_rne(float("-inf")) == 15 and O.int4_encode_rne(float("nan")) == 7
-    assert O.mx_exponent(float("inf")) == 126 and O.mx_exponent(float("nan"), O.NOSAT_CEIL) == 126
-    x = O._f32(np.random.default_rng(14).standard_normal((4, 64)))
+def _nonfinite_tensor():
+    x = O._f32(np.random.default_rng(14).standard_normal((8, 64)) * 2)
     x[1, 5] = np.nan
     x[2, 40] = -np.inf
+    x[5, 0], x[5, 1] = np.inf, -np.nan
+    return x
+
+
+def test_rejected_blocks_and_counts():
+    x = _nonfinite_tensor()
+    finite16 = np.isfinite(x).reshape(8, 4, 16).all(-1)
+    finite32 = np.isfinite(x).reshape(8, 2, 32).all(-1)
+    n_bad = int(np.count_nonzero(~np.isfinite(x)))
+    clean = np.where(np.repeat(finite16, 16, axis=1), x, np.float32(0)).astype(np.float32)
+    clean32 = np.where(np.repeat(finite32, 32, axis=1), x, np.float32(0)).astype(np.float32)
+    for mode in ({}, {"four_six": True}, {"if4": True}, {"round": O.STOCHASTIC, "seed": 3}):
+        q, s, sg, c, spec = O.nvfp4_quantize(x, global_in=0.01, spec=True, **mode)
+        assert np.array_equal(spec, finite16) and c["nonfinite"] == n_bad
+        # every other block is encoded as it would be with the rejected blocks' values zeroed (all-zero
+        # blocks add no counts), so the blocks are independent and the rejected ones add no counts
+        q2, s2, _, c2 = O.nvfp4_quantize(clean, global_in=0.01, **mode)
+        assert np.array_equal(s[spec], s2[spec])
+        assert np.array_equal(q[np.repeat(spec, 8, axis=1)], q2[np.repeat(spec, 8, axis=1)])
+        assert {k: v for k, v in c.items() if k != "nonfinite"} == {k: v for k, v in c2.items() if k != "nonfinite"}
+    q, s, c, spec = O.mx_quantize(x, spec=True)
+    q2, s2, c2 = O.mx_quantize(clean32)
+    assert np.array_equal(spec, finite32) and c["nonfinite"] == n_bad
+    assert np.array_equal(s[spec], s2[spec]) and c["underflow"] == c2["underflow"]
+    assert c["saturation"] == c2["saturation"]
+
+
+def test_tensor_scale_of_nonfinite_tensors():
+    """The two-pass global scale follows torch.amax: NaN with a NaN present, +Inf with only
+    infinities; every block is then left open and only the non-finite values are counted."""
+    x = _nonfinite_tensor()
     assert torch.isnan(torch.from_numpy(x).abs().amax())
-    q, s, sg, c = O.nvfp4_quantize(x)
-    assert np.isnan(sg) and (s == 0x7F).all() and c["nonfinite"] == 2
-    q, s, sg, c = O.nvfp4_quantize(x, global_in=0.01)
-    blk = torch.from_numpy(x).abs().reshape(4, 4, 16).amax(-1).numpy()
-    assert (s[np.isnan(blk)] == 0x7F).all() and (s[np.isinf(blk)] == 0x7E).all()
-    codes = np.stack([q & 15, q >> 4], -1).reshape(4, 64)
-    assert (codes[1, :16] == 7).all() and codes[2, 40] == 15
-    q, s, c = O.mx_quantize(x)
-    assert s[1, 0] == s[2, 1] == 126 + 127 and c["nonfinite"] == 2
+    q, s, sg, c, spec = O.nvfp4_quantize(x, spec=True)
+    assert np.isnan(sg) and not spec.any() and c == {"underflow": 0, "saturation": 0, "nonfinite": 4,
+                                                     "blocks_four": 0}
+    y = np.where(np.isnan(x), np.float32(1), x).astype(np.float32)
+    amax = torch.from_numpy(y).abs().amax().item()
+    q, s, sg, c, spec = O.nvfp4_quantize(y, spec=True)
+    assert amax == math.inf and sg == math.inf and not spec.any()
+    assert c["nonfinite"] == int(np.count_nonzero(~np.isfinite(y))) == 2
+
+
+def test_encoders_on_infinite_values():
+    """Infinities are values beyond the largest magnitude: they saturate (E2M1 to +-6, INT4 to
+    +-7, E4M3 scales to 448), with the sign kept."""
+    assert O.e2m1_encode_rne(float("-inf")) == 15 and O.e2m1_encode_rne(float("inf")) == 7
+    assert O.e2m1_encode_sr(float("inf"), 0) == 7 and O.int4_encode_rne(float("-inf")) == 15
+    assert O.e4m3_encode(float("inf")) == 0x7E and O.e4m3_value(0x7E) == 448.0
 
 
 # ---------------------------------------------------------------------------------------------
@@ -493,11 +553,11 @@ def test_if4_picks_lower_error_candidate_brute_force():
             assert abs(got - (e7 if flagged else e6)) <= 1e-5 * max(got, 1e-30)
 
 
-def test_if4_nonfinite_blocks_keep_fp4():
-    x = O._f32(np.random.default_rng(13).uniform(-1, 1, (1, 48)))
+def test_if4_rejected_blocks():
+    x = O._f32(np.random.default_rng(13).uniform(-1, 1, (1, 64)))
     x[0, 3], x[0, 20], x[0, 40] = np.inf, np.nan, -np.inf
-    q, s, _, c = O.nvfp4_quantize(x, global_in=1.0, if4=True)
-    assert c["nonfinite"] == 3 and (s >> 7 == 0).all()
+    q, s, _, c, spec = O.nvfp4_quantize(x, global_in=1.0, if4=True, spec=True)
+    assert c["nonfinite"] == 3 and spec.tolist() == [[False, False, False, True]]
 
 
 # ---------------------------------------------------------------------------------------------
