@@ -11,8 +11,10 @@ block-scaled GEMMs and the down_proj quantise + GEMM pipeline).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-secondary]
 
-Under torchrun every rank quantises its own copy of the workload (independent problems, weak
-scaling, no collective on the data path); the step time is the max over ranks.
+With --gpus N > 1 the bench runs one process per GPU: under torchrun it reads RANK, LOCAL_RANK and
+WORLD_SIZE (which must equal N); started alone it spawns the N ranks itself (127.0.0.1 rendezvous).
+Every rank quantises its own copy of the workload (independent problems, weak scaling, no
+collective on the data path); the step time is the max over ranks.
 Timing: CUDA events on the launching stream per step, L2 flushed (a 256 MiB write) before every
 timed step, outside the events; clocks sampled with nvidia-smi during the timed loop.
 """
@@ -113,6 +115,26 @@ class Clocks:
         reasons = sorted({names[i] for p in load for i in range(4) if p[6 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(load)}
+
+
+def _free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _rank_main(local, world, port, argv):
+    os.environ.update(RANK=str(local), LOCAL_RANK=str(local), WORLD_SIZE=str(world),
+                      LOCAL_WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    main(argv)
+
+
+def spawn_ranks(n, argv):
+    """One process per GPU without an external launcher: N spawned ranks (no CUDA call in this
+    parent before they start), each running main() with the torchrun environment set."""
+    import torch.multiprocessing as tmp
+    tmp.start_processes(_rank_main, args=(n, _free_port(), argv), nprocs=n, join=True, start_method="spawn")
 
 
 def dist():
@@ -230,6 +252,7 @@ def run_ours(args, td, rank, world, local):
     bytes_step = 2 * NV_BYTES_2PASS * n
     value = job_throughput(world, bytes_step, ms_step)
 
+    traffic = profile_traffic("nvfp4_quantize_8192x8192")  # read before any timing
     # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g
     g = step.g[1].clone()
     kms = timed(lambda: step.call(1, True, global_in=g), args.steps, args.warmup, flush, td)
@@ -239,7 +262,9 @@ def run_ours(args, td, rank, world, local):
     roof = {"kernel": "quantize_kernel<bf16, NVFP4, RNE, 4/6> (one launch, 8192x8192)", "bound": "hbm",
             "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
-            "traffic": profile_traffic("nvfp4_quantize_8192x8192"),
+            "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
+            "traffic": traffic, "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of "
+                                                  "this kernel on this workload, profiles/nvfp4_quantize_8192x8192.md",
             "algorithmic_bytes_per_launch": k_bytes}
 
     # end to end through the public binding: pinned host input -> device -> both calls -> host
@@ -282,45 +307,50 @@ def run_ours(args, td, rank, world, local):
     return line
 
 
-def _oracle_chunk(xs):
-    """One thread's share of the all-cores oracle timing: plain then 4/6 on its rows."""
+def _oracle_chunk(xs, g_plain, g46):
+    """One thread's share of the all-cores oracle timing: plain then 4/6 on its rows, under the
+    global scales of the whole sample (the single-threaded leg's), so the codes are the same."""
     import oracle as O
-    O.nvfp4_quantize(xs, four_six=False)
-    O.nvfp4_quantize(xs, four_six=True)
+    O.nvfp4_quantize(xs, four_six=False, global_in=g_plain)
+    O.nvfp4_quantize(xs, four_six=True, global_in=g46)
     return xs.shape[0]
 
 
 def cpu_baseline(x_cpu, rows=4096, max_workers=64):
-    """The oracle as it stands on the first `rows` rows of the workload: single-threaded, then the
-    same rows split over one thread per host core.  The oracle is C called through ctypes, which
-    releases the GIL for the call and keeps no global state, so the threads run in parallel; each
-    handles its rows as a tensor of its own."""
+    """The oracle as it stands on the first `rows` rows of the workload: single-threaded (both
+    passes of each call), then the quantise passes of the same rows split over one thread per host
+    core, each thread given the sample's global scales from the single-threaded run.  The oracle is
+    C called through ctypes, which releases the GIL for the call and keeps no global state, so the
+    threads run in parallel."""
     import concurrent.futures as cf
     import oracle as O
     xs = synth.as_f32_numpy(x_cpu[:rows])
     t = time.perf_counter()
-    O.nvfp4_quantize(xs, four_six=False)
-    O.nvfp4_quantize(xs, four_six=True)
+    g_plain = O.nvfp4_quantize(xs, four_six=False)[2]
+    g46 = O.nvfp4_quantize(xs, four_six=True)[2]
     dt = time.perf_counter() - t
     b = 2 * NV_BYTES_2PASS * xs.size
     out = {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-           "sample": f"first {rows} of 8192 rows (plain + 4/6), {dt:.1f} s single-threaded C oracle"}
+           "sample": f"first {rows} of 8192 rows (plain + 4/6, two passes each), {dt:.1f} s single-threaded C oracle"}
     n = max(1, min(os.cpu_count() or 1, max_workers, rows))
     chunks = np.array_split(xs, n)
     with cf.ThreadPoolExecutor(max_workers=n) as ex:
         t = time.perf_counter()
-        done = sum(ex.map(_oracle_chunk, chunks))
+        done = sum(ex.map(lambda c: _oracle_chunk(c, g_plain, g46), chunks))
         dt_all = time.perf_counter() - t
     assert done == rows
-    out["all_cores"] = {"value": round(b / dt_all / 1e9, 4), "unit": "GB/s", "cores": n,
-                        "sample": f"the same rows over {n} threads, {dt_all:.2f} s"}
+    b1 = 2 * NV_BYTES_1PASS * xs.size
+    out["all_cores"] = {"value": round(b1 / dt_all / 1e9, 4), "unit": "GB/s", "cores": n,
+                        "sample": f"the same rows' quantise passes (plain + 4/6) over {n} threads under the "
+                                  f"single-threaded run's global scales, {dt_all:.2f} s; bytes counted for one "
+                                  f"pass per call"}
     return out
 
 
 # ---------------------------------------------------------------------------------------------
 def secondary(args, dev, flush, td, pk):
     out = []
-    K = max(5, args.steps // 10)
+    K = max(10, args.steps // 4)
     W = args.warmup
     # config 1: MXFP4 quantise + dequantise, 256 x 512 fp32
     x1 = synth.mx_small().to(dev)
@@ -409,9 +439,25 @@ def secondary(args, dev, flush, td, pk):
                 "quantise_pass_gaussian_ms": round(tn, 4),
                 "quantise_pass_gaussian_frac_hbm":
                     round(NV_BYTES_1PASS * xn.numel() / (tn * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
-    del xi, xn
+    # dequantisation of the headline tensor's NVFP4 encoding (4/6 codes), to bf16 and to fp32
+    xd = synth.nv_outliers().to(dev)
+    qd, sd, gd, _ = fp4.nvfp4_quantize(xd, four_six=True, workspace=ws)
+    del xd
+    od = {torch.bfloat16: torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev),
+          torch.float32: torch.empty((8192, 8192), dtype=torch.float32, device=dev)}
+    for dt_, nbytes in ((torch.bfloat16, 2), (torch.float32, 4)):
+        ms = timed(lambda: fp4.fp4_dequantize(qd, sd, fp4.NVFP4, gd, out=od[dt_]), K, W, flush, td)
+        t = statistics.median(ms)
+        bd = qd.numel() * 2 * (0.5 + 1 / 16 + nbytes)
+        out.append({"workload": f"NVFP4 dequantisation 8192x8192 to {'bf16' if nbytes == 2 else 'fp32'}",
+                    "ms": round(t, 4), "GB/s": round(bd / (t * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(bd / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
+    del qd, sd, od
 
-    fp4_peak = 4.0 * pk["bf16_tflops"]  # dense FP4 / BF16 nominal ratio 9 / 2.25 on the measured bf16 peak
+    # The FP4 dense peak is derived, not measured: the measured bf16 cuBLAS peak times the nominal
+    # dense FP4 / BF16 ratio (9 / 2.25 PFLOP/s).  The datasheet's dense FP4 figure is given beside it.
+    fp4_peak = 4.0 * pk["bf16_tflops"]
+    fp4_datasheet = 9000.0
     # config 4: NVFP4 GEMM 8192^3
     A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), layout=fp4.MMA_TILED)
     B = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 2).to(dev), layout=fp4.MMA_TILED)
@@ -423,7 +469,10 @@ def secondary(args, dev, flush, td, pk):
     tf = 2 * 8192 ** 3 / (t * 1e-3) / 1e12
     out.append({"workload": "NVFP4 block-scaled GEMM M=N=K=8192 (E4M3 per 16, fp32 accumulate, bf16 out)",
                 "ms": round(t, 4), "TFLOP/s": round(tf, 1), "frac_fp4_peak": round(tf / fp4_peak, 4),
-                "fp4_peak": fp4_peak, "peak_source": pk["source"] + " bf16 x 4 (nominal FP4/BF16 ratio)"})
+                "fp4_peak": fp4_peak,
+                "peak_source": f"derived: {pk['source']} bf16 burst x 4 (nominal dense FP4/BF16 ratio)",
+                "frac_fp4_datasheet": round(tf / fp4_datasheet, 4),
+                "fp4_datasheet": fp4_datasheet, "datasheet_source": "B200 dense FP4 9 PFLOP/s (NVIDIA, without sparsity)"})
     del A, B, C
     # config 5: MXFP4 down_proj, activations and weights quantised then GEMM, timed end to end
     a = synth.swiglu_act().to(dev)
@@ -450,6 +499,7 @@ def secondary(args, dev, flush, td, pk):
                 "ms_end_to_end": round(t_all, 4), "gemm_ms": round(t_g, 4),
                 "gemm_TFLOP/s": round(flop / (t_g * 1e-3) / 1e12, 1),
                 "gemm_frac_fp4_peak": round(flop / (t_g * 1e-3) / 1e12 / fp4_peak, 4),
+                "gemm_frac_fp4_datasheet": round(flop / (t_g * 1e-3) / 1e12 / fp4_datasheet, 4),
                 "weight_quantise_GB/s": round(qbytes / (t_w * 1e-3) / 1e9, 1),
                 "weight_quantise_frac_hbm": round(qbytes / (t_w * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                 "end_to_end_TFLOP/s": round(flop / (t_all * 1e-3) / 1e12, 1)})
@@ -468,7 +518,8 @@ def secondary(args, dev, flush, td, pk):
                 "expand_frac_hbm": round(xbytes / (t_x * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                 "gemm_ms": round(t_8, 4), "gemm_TFLOP/s": round(flop / (t_8 * 1e-3) / 1e12, 1),
                 "gemm_frac_fp8_peak": round(flop / (t_8 * 1e-3) / 1e12 / fp8_peak, 4), "fp8_peak": fp8_peak,
-                "peak_source": pk["source"] + " bf16 x 2 (nominal FP8/BF16 ratio)"})
+                "peak_source": f"derived: {pk['source']} bf16 burst x 2 (nominal dense FP8/BF16 ratio)",
+                "gemm_frac_fp8_datasheet": round(flop / (t_8 * 1e-3) / 1e12 / 4500.0, 4)})
     return out
 
 
@@ -549,7 +600,21 @@ def run_case(name, reps):
     print(json.dumps({"case": name, "reps": reps, "ok": True}))
 
 
-def main():
+def dist_check(args):
+    """The multi-rank plumbing alone (no GPU work): every rank reports a step time of 1 + rank/2 ms;
+    rank 0 prints the world size, the max over ranks and the whole-job throughput of 1 GB per rank."""
+    td, rank, world, _ = dist()
+    try:
+        barrier(td)
+        m = max_over_ranks(td, 1.0 + 0.5 * rank)
+        if rank == 0:
+            print(json.dumps({"world": world, "max_ms": m, "GB/s": job_throughput(world, 1e9, m)}))
+    finally:
+        if td is not None:
+            td.destroy_process_group()
+
+
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", choices=CASES, help="run one kernel on its workload (profiling)")
     ap.add_argument("--reps", type=int, default=3)
@@ -559,7 +624,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    ap.add_argument("--dist-check", action="store_true", help="run only the multi-rank helpers (no GPU work)")
+    args = ap.parse_args(argv)
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        spawn_ranks(args.gpus, sys.argv[1:] if argv is None else argv)
+        return
+    if env_world is not None and int(env_world) != args.gpus:
+        raise SystemExit(f"bench.py: WORLD_SIZE={env_world} but --gpus {args.gpus}")
+    if args.dist_check:
+        dist_check(args)
+        return
     if args.case:
         run_case(args.case, args.reps)
         return

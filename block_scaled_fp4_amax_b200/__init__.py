@@ -225,12 +225,15 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
 
 def fp4_dequantize(q: torch.Tensor, scales: torch.Tensor, fmt: int, global_scale: torch.Tensor | None = None,
                    layout: int = ROWMAJOR, out_dtype: torch.dtype = torch.float32, block: int | None = None,
-                   stream=None):
-    """x_hat [rows, 2*q.shape[1]] in out_dtype."""
-    _need_cuda(q, scales, global_scale)
+                   stream=None, out: torch.Tensor | None = None):
+    """x_hat [rows, 2*q.shape[1]] in out_dtype (or in `out`, whose dtype then decides)."""
+    _need_cuda(q, scales, global_scale, out)
     rows, half = q.shape
     B = block if block is not None else (32 if fmt == MXFP4 else 16)
-    out = torch.empty((rows, 2 * half), dtype=out_dtype, device=q.device)
+    if out is None:
+        out = torch.empty((rows, 2 * half), dtype=out_dtype, device=q.device)
+    elif out.shape != (rows, 2 * half) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [rows, 2 * q.shape[1]] tensor")
     _check(lib().fp4_dequantize(_ptr(q), _ptr(scales), fmt, B, layout, _ptr(global_scale), rows, 2 * half,
                                 _dtype_code(out), _ptr(out), _stream(stream)))
     return out

@@ -59,7 +59,7 @@ def test_job_throughput_single_rank():
 
 def test_reference_arm_other_ranks_exit_without_work():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
@@ -99,3 +99,24 @@ def test_oracle_is_thread_safe_for_the_all_cores_baseline():
         par = list(ex.map(lambda c: O.nvfp4_quantize(c, four_six=True), chunks))
     for a, b in zip(serial, par):
         assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and a[2] == b[2] and a[3] == b[3]
+
+
+def test_gpus_flag_spawns_the_ranks_itself():
+    """`bench.py --gpus 2` without a launcher starts both ranks (gloo on a machine without a GPU);
+    the helpers then see world size 2 and the slower rank's time."""
+    import json
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_PORT")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dist-check"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    assert out["world"] == 2 and out["max_ms"] == pytest.approx(1.5)
+    assert out["GB/s"] == pytest.approx(2 * 1e9 / 1.5e-3 / 1e9)
+
+
+def test_world_size_must_match_gpus():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4", "--dist-check"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE=2 but --gpus 4" in r.stderr

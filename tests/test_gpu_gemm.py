@@ -1,11 +1,16 @@
 """GPU parity: the tcgen05 block-scaled GEMM against the fp64 oracle.
 
 Bar: |C_gpu - C64| <= 1e-3 * sum_k |a_k b_k| per element, C64 the fp64 dot product of the exactly
-dequantised operands.  The bf16 output rounding alone can reach 2^-9 |C|, which exceeds that bound
-whenever |C| is a sizeable fraction of sum |a b| — small K, or same-sign data — so the small-shape
-cases add the bf16 rounding term 2^-8 |C64|; the full-size workloads (K = 8192 and 28672) are held
-to the bound alone.  Operands are quantised on the GPU (checked bit-exact
-against the oracle elsewhere) while the reference quantises independently on the CPU.
+dequantised operands.  On zero-mean data the tests also hold the result to one bf16 rounding step
+of the exact value plus the fp32 accumulation term: |C_gpu - bf16(C64)| <= ulp(bf16(C64)) +
+K * 2^-23 * sum |a b|.  Only the same-sign test adds the bf16 rounding term 2^-8 |C64| to the first
+bar (there |C| is close to sum |a b|, and the output rounding alone reaches 2^-9 |C|).
+
+Structured operands make the pipeline's bookkeeping exact: every output is a single product, so a
+dropped, repeated or stale K stage, a wrong barrier phase, an accumulator not reset between the
+tiles a CTA takes in turn, or a misplaced scale changes C, and C must equal bf16(C64) bit for bit.
+Operands are quantised on the GPU (checked bit-exact against the oracle elsewhere) while the
+reference quantises independently on the CPU.
 """
 import numpy as np
 import pytest
@@ -38,11 +43,35 @@ def quant(x_cpu, fmt, cuda):
     return (q, s, None), (qo, so, 1.0)
 
 
-def check(C, C64, S, extra_rel=2.0 ** -8):
-    err = np.abs(npy(C.float()).astype(np.float64) - C64)
+def check(C, C64, S, extra_rel=0.0, K=None):
+    """The 1e-3 * sum|ab| bar (plus `extra_rel` * |C64| for same-sign data); with K, also the
+    bf16-aware bar |C - bf16(C64)| <= ulp(bf16(C64)) + K * 2^-23 * S."""
+    got = npy(C.float()).astype(np.float64)
+    err = np.abs(got - C64)
     bound = 1e-3 * S + extra_rel * np.abs(C64)
     bad = err > bound
     assert not bad.any(), f"{bad.sum()} of {bad.size} outside the bound; worst excess {float((err - bound).max())}"
+    if K is not None:
+        check_bf16_tight(got, C64, S, K)
+
+
+def bf16_of(C64):
+    """Round-to-nearest-even bf16 of fp64 values (through fp32: exact for values with few bits)."""
+    return torch.from_numpy(np.ascontiguousarray(C64, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def bf16_ulp(v):
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def check_bf16_tight(got, C64, S, K):
+    ref = bf16_of(C64)
+    err = np.abs(got - ref)
+    bound = bf16_ulp(ref) + K * 2.0 ** -23 * S
+    bad = err > bound
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside ulp + K 2^-23 S; worst excess {float((err - bound).max())}"
 
 
 def gemm(fmt, A, B):
@@ -101,7 +130,61 @@ def test_gemm_small_random(cuda, fmt, shape):
     B, Bo = quant(synth.gemm_operand(N, K, 2), fmt, cuda)
     C = gemm(fmt, A, B)
     C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fmt)
-    check(C, C64, S)
+    check(C, C64, S, K=K)
+
+
+def structured_operands(M, N, K, fmt, seed):
+    """Codes and row-major scales with exactly one nonzero product per output.  K = 8192 is 32
+    groups of 256 values.  In group g, row m of A holds one nonzero value at 8 ((g - m) mod 32) +
+    (g mod 8) and row n of B one at 8 (n mod 32) + (g mod 8): they meet only in the group
+    g = (m + n) mod 32, so C[m, n] is that single product (exact in fp32), every output is nonzero,
+    and every group and every 16- or 32-value block position takes part somewhere.  Values are
+    lattice points of both signs; every block scale is drawn independently."""
+    assert K == 8192
+    G = K // 256
+    rng = np.random.default_rng(seed)
+    Bk = 16 if fmt == fp4.NVFP4 else 32
+    g = np.arange(G)
+    ca = np.zeros((M, K), np.uint8)
+    cb = np.zeros((N, K), np.uint8)
+    m = np.arange(M)[:, None]
+    n = np.arange(N)[:, None]
+    pa = g * 256 + 8 * ((g - m) % 32) + (g % 8)
+    pb = g * 256 + 8 * (n % 32) + (g % 8)
+    code = lambda shape: (rng.integers(1, 8, shape) | (rng.integers(0, 2, shape) << 3)).astype(np.uint8)
+    np.put_along_axis(ca, pa, code((M, G)), axis=1)
+    np.put_along_axis(cb, np.broadcast_to(pb, (N, G)), code((N, G)), axis=1)
+    if fmt == fp4.NVFP4:
+        sa = rng.integers(0x20, 0x50, size=(M, K // Bk)).astype(np.uint8)   # E4M3 2^-3 .. 7.5
+        sb = rng.integers(0x20, 0x50, size=(N, K // Bk)).astype(np.uint8)
+    else:
+        sa = rng.integers(120, 134, size=(M, K // Bk)).astype(np.uint8)     # E8M0 2^-7 .. 2^6
+        sb = rng.integers(120, 134, size=(N, K // Bk)).astype(np.uint8)
+    return packed_from_codes(ca), sa, packed_from_codes(cb), sb
+
+
+def structured_reference(Aq, sa, Bq, sb, fmt):
+    C64, S = O.gemm_f64(Aq, sa, 1.0, Bq, sb, 1.0, fmt)
+    assert np.all(C64 != 0) and np.array_equal(np.abs(C64), S)  # one product per output
+    return bf16_of(C64)
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
+@pytest.mark.parametrize("M", [4096, 3968])  # 2-SM pair tiles (256 x 256); 1-SM tiles (M % 256 == 128)
+def test_gemm_structured_exact_many_tiles(cuda, fmt, M):
+    """K = 8192 (32 stages of 256 values through a 4-6 deep ring, so its barriers change phase many
+    times per tile); N = 4096, so every cluster (pair kernel: 256 tiles over 74 clusters) or CTA
+    (1-SM kernel: 496 tiles over 148 CTAs) computes three or more tiles in turn, re-using its
+    accumulator and scale slots.  C must equal bf16 of the exact product everywhere."""
+    N, K = 4096, 8192
+    Aq, sa, Bq, sb = structured_operands(M, N, K, fmt, seed=M + fmt)
+    want = structured_reference(Aq, sa, Bq, sb, fmt)
+    one = torch.ones(1, dtype=torch.float32, device=cuda)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(cuda)
+    C = gemm(fmt, (dev(Aq), dev(O.scales_to_mma_tiled(sa)), one), (dev(Bq), dev(O.scales_to_mma_tiled(sb)), one))
+    got = npy(C.float()).astype(np.float64)
+    bad = got != want
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ (first at {np.argwhere(bad)[0]})"
 
 
 def test_gemm_positive_data_bf16_rounding(cuda):
@@ -162,12 +245,15 @@ def check_sampled(C, a_cpu, b_cpu, fmt, rows, cols):
     Aq, As, Ag = oq(a_cpu)
     Bq, Bs, Bg = oq(b_cpu)
     Cn = npy(C.float()).astype(np.float64)
+    K = 2 * Aq.shape[1]
     C64, S = O.gemm_f64(Aq, As, Ag, Bq, Bs, Bg, fmt, rows=rows)
     err = np.abs(Cn[rows] - C64)
     assert np.all(err <= 1e-3 * S), float((err - 1e-3 * S).max())
+    check_bf16_tight(Cn[rows], C64, S, K)
     C64, S = O.gemm_f64(Aq, As, Ag, Bq, Bs, Bg, fmt, cols=cols)
     err = np.abs(Cn[:, cols] - C64)
     assert np.all(err <= 1e-3 * S), float((err - 1e-3 * S).max())
+    check_bf16_tight(Cn[:, cols], C64, S, K)
 
 
 def test_gemm_ldc_and_status_word(cuda):
@@ -180,7 +266,7 @@ def test_gemm_ldc_and_status_word(cuda):
     assert status_ok(ws)
     assert torch.all(big[:, N:] == 7.0)
     C64, S = O.gemm_f64(Ao[0], Ao[1], Ao[2], Bo[0], Bo[1], Bo[2], fp4.NVFP4)
-    check(big[:, :N], C64, S)
+    check(big[:, :N], C64, S, K=K)
 
 
 def test_gemm_output_beyond_2p31_elements(cuda):
@@ -201,5 +287,5 @@ def test_gemm_output_beyond_2p31_elements(cuda):
     B64 = O.dequantize(qbo, sbo, O.NVFP4, gbo).astype(np.float64)
     C64 = A64 @ B64.T
     S = np.abs(A64) @ np.abs(B64).T
-    check(C[rows], C64, S)
+    check(C[rows], C64, S, K=K)
     del C

@@ -11,7 +11,8 @@ import torch
 import block_scaled_fp4_amax_b200 as fp4
 import oracle as O
 from block_scaled_fp4_amax_b200 import synth
-from tests.test_gpu_gemm import check, check_sampled, npy, packed_from_codes, status_ok
+from tests.test_gpu_gemm import (check, check_sampled, npy, packed_from_codes, status_ok, structured_operands,
+                                  structured_reference)
 
 pytestmark = pytest.mark.gpu
 
@@ -73,12 +74,26 @@ def test_gemm_e4m3_small_random_and_against_fp4(cuda, shape):
     Aq, As, _ = O.mx_quantize(synth.as_f32_numpy(a))
     Bq, Bs, _ = O.mx_quantize(synth.as_f32_numpy(b))
     C64, S = O.gemm_f64(Aq, As, 1.0, Bq, Bs, 1.0, O.MXFP4)
-    check(C, C64, S)
+    check(C, C64, S, K=K)
     if K % 256 == 0:  # the FP4 GEMM's stage is 256 values
         C4, ws = fp4.fp4_block_gemm(fp4.MXFP4, A[0], A[1], B[0], B[1])
         assert status_ok(ws)
         diff = np.abs(npy(C.float()).astype(np.float64) - npy(C4.float()).astype(np.float64))
         assert np.all(diff <= 2 * (1e-3 * S + 2.0 ** -8 * np.abs(C64)))
+
+
+def test_gemm_e4m3_structured_exact_many_tiles(cuda):
+    """Single-product operands (see tests/test_gpu_gemm.py) at K = 8192: 64 stages of 128 values
+    through the 4-deep ring, 512 tiles of 128 x 256 over 148 CTAs (three or more per CTA).  C must
+    equal bf16 of the exact product everywhere."""
+    M, N, K = 4096, 4096, 8192
+    Aq, sa, Bq, sb = structured_operands(M, N, K, fp4.MXFP4, seed=77)
+    want = structured_reference(Aq, sa, Bq, sb, fp4.MXFP4)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(cuda)
+    C = gemm_e4m3((dev(Aq), dev(O.scales_to_mma_tiled(sa))), (dev(Bq), dev(O.scales_to_mma_tiled(sb))))
+    got = npy(C.float()).astype(np.float64)
+    bad = got != want
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ (first at {np.argwhere(bad)[0]})"
 
 
 def test_gemm_e4m3_down_proj_sampled(cuda):
