@@ -29,7 +29,7 @@ NV_PLAIN, NV_FOUR_SIX, NV_IF4 = 0, 1, 2  # fp4_nv_mode
 RNE, STOCHASTIC = 0, 1
 OCP_FLOOR, NOSAT_CEIL = 0, 1
 ROWMAJOR, MMA_TILED = 0, 1
-OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEMM = range(5)
+OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEMM, OP_FWHT_QUANTIZE_STORED = range(6)
 STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 
 # Every symbol include/fp4mx.h declares.
@@ -175,6 +175,14 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = F
     return q, s, g, c
 
 
+def _fwht_op(fmt, global_in, want_rotated):
+    """The workspace to allocate by default: room for the fp32 rotation when a two-pass NVFP4 call
+    would otherwise rotate twice (a requested rotated_out serves that purpose itself)."""
+    if fmt == NVFP4 and global_in is None and not want_rotated:
+        return OP_FWHT_QUANTIZE_STORED
+    return OP_FWHT_QUANTIZE
+
+
 def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
                   layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, want_rotated: bool = False,
                   block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
@@ -189,7 +197,7 @@ def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six:
     q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, x.device)
     g = torch.empty(1, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
     rot = torch.empty((rows, d), dtype=torch.float32, device=x.device) if want_rotated else None
-    ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, x.device, rows, d)
+    ws = workspace if workspace is not None else _workspace(_fwht_op(fmt, global_in, want_rotated), x.device, rows, d)
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
         raise ValueError("signs must hold d/32 32-bit words")
     _check(lib().fwht_quantize(_ptr(x), _dtype_code(x), rows, d, _ptr(signs), fmt, B, round, _nv_mode(four_six, if4), seed,
@@ -214,7 +222,7 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
     q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, g.device)
     gs = torch.empty(1, dtype=torch.float32, device=g.device) if fmt == NVFP4 else None
     rot = torch.empty((rows, d), dtype=torch.float32, device=g.device) if want_rotated else None
-    ws = workspace if workspace is not None else _workspace(OP_FWHT_QUANTIZE, g.device, rows, d)
+    ws = workspace if workspace is not None else _workspace(_fwht_op(fmt, global_in, want_rotated), g.device, rows, d)
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
         raise ValueError("signs must hold d/32 32-bit words")
     _check(lib().swiglu_fwht_quantize(_ptr(g), _ptr(u), _dtype_code(g), rows, d, _ptr(signs), fmt, B, round,

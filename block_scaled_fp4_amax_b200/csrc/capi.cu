@@ -99,6 +99,9 @@ size_t fp4_workspace_size(fp4_op op, long rows, long cols) {
   switch (op) {
     case FP4_OP_NVFP4_QUANTIZE:
     case FP4_OP_FWHT_QUANTIZE: return kAmaxWorkspace;
+    case FP4_OP_FWHT_QUANTIZE_STORED:
+      // the amax word, padding to a 256-byte boundary, and the fp32 rotation
+      return rows > 0 && cols > 0 ? 2 * kAmaxWorkspace + (size_t)rows * (size_t)cols * sizeof(float) : kAmaxWorkspace;
     case FP4_OP_BLOCK_GEMM: return kGemmWorkspace;
     default: return 0;
   }
@@ -197,8 +200,34 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
   L.pdl = amax_pass;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   cudaError_t e;
+  // Stored-rotation route for the two-pass call: the first pass keeps the fp32 rotation (in
+  // rotated_out, or in the workspace past the amax word) and the second pass quantises it, so the
+  // butterflies run once.  Both routes give the same bytes.
+  float* rot = nullptr;
+  if (amax_pass) {
+    const size_t rot_bytes = (size_t)rows * (size_t)d * sizeof(float);
+    if (rotated_out && aligned(rotated_out, 32)) {
+      rot = rotated_out;
+    } else if (!rotated_out && ws_bytes >= 2 * kAmaxWorkspace + rot_bytes) {
+      // the first 256-byte boundary past the amax word's 256 bytes
+      const uintptr_t w = reinterpret_cast<uintptr_t>(workspace);
+      rot = reinterpret_cast<float*>((w + 2 * kAmaxWorkspace) & ~(uintptr_t)(kAmaxWorkspace - 1));
+    }
+  }
   if (amax_pass) {
     if ((e = cudaMemsetAsync(L.amax_bits, 0, sizeof(uint32_t), s)) != cudaSuccess) return cuda_fail(e, "zeroing amax");
+    if (rot) {
+      L.rotated_out = rot;
+      if ((e = fp4k::launch_fwht_store(L, s)) != cudaSuccess) return cuda_fail(e, "fwht store launch");
+      fp4k::QuantLaunch Q{};
+      Q.x = rot; Q.bf16 = false; Q.rows = rows; Q.cols = d; Q.nv = true;
+      Q.policy = 0; Q.sr = L.sr; Q.mode = L.mode; Q.seed = seed;
+      Q.tiled = L.tiled; Q.reverse = 1;  // start on the rows the first pass left in L2
+      Q.global_in = nullptr; Q.amax_bits = L.amax_bits; Q.global_out = L.global_out;
+      Q.q = q; Q.scales = scales; Q.counts = L.counts; Q.pdl = true;
+      e = fp4k::launch_quantize(Q, s);
+      return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fwht_quantize stored-rotation launch");
+    }
     if ((e = fp4k::launch_fwht_amax(L, s)) != cudaSuccess) return cuda_fail(e, "fwht amax launch");
   }
   e = fp4k::launch_fwht_quantize(L, s);

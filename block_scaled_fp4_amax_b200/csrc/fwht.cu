@@ -293,6 +293,66 @@ __device__ __forceinline__ void to_consecutive(float* srow, int t, float (&v)[32
   __syncthreads();  // row buffer free for the next row
 }
 
+// Pass 1 of the stored-rotation path (NVFP4 without a caller scale, given room for the rotated
+// tensor): rotate once, normalise, store the fp32 rotation row-major to p.rotated_out and reduce
+// the tensor amax.  The quantise pass then reads the stored values (quantize_kernel on fp32 input),
+// so the butterflies run once instead of twice, for 4 more bytes per element of traffic each way.
+// The maximum is an integer max over the magnitude bits, which keeps a NaN (its bits lie above
+// every finite value's and Inf's), as the tensor maximum does in the two-rotation path's reading.
+template <typename T, int LOG_D, bool GATED>
+__global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_store_kernel(FwhtParams p) {
+  using G = Geom<LOG_D>;
+  constexpr int D = G::D;
+  grid_dep_trigger();
+  if (p.counts && blockIdx.x == 0 && threadIdx.x < 4) p.counts[threadIdx.x] = 0ull;
+  extern __shared__ __align__(16) float smem[];
+  const int slot = threadIdx.x / G::T, t = threadIdx.x % G::T;
+  float* srow = smem + slot * D;
+  const T* x = reinterpret_cast<const T*>(p.x);
+  const uint32_t sgn = p.signs ? p.signs[t] : 0u;
+  const long long step = (long long)gridDim.x * G::ROWS;
+  uint32_t m = 0u;
+  U8 raw[RowLoad<T>::NV], nxt[RowLoad<T>::NV], rawu[GATED ? RowLoad<T>::NV : 1];
+  long long row = (long long)blockIdx.x * G::ROWS + slot;
+  if (!GATED) load_row<T, LOG_D>(x, row, p.rows, t, raw);
+  for (long long base = (long long)blockIdx.x * G::ROWS; base < p.rows; base += step) {
+    if constexpr (GATED) {
+      load_row<T, LOG_D>(x, row, p.rows, t, raw);
+      load_row<T, LOG_D>(reinterpret_cast<const T*>(p.u), row, p.rows, t, rawu);
+    } else {
+      load_row<T, LOG_D>(x, row + step, p.rows, t, nxt);
+    }
+    float v[32];
+    rotate_row<T, LOG_D, GATED>(raw, rawu, srow, t, sgn, v);
+    to_consecutive<LOG_D>(srow, t, v);
+    if (row < p.rows) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        v[j] = __fmul_rn(v[j], p.c);
+        m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+      }
+      float4* dst = reinterpret_cast<float4*>(p.rotated_out + row * D + (t << 5));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    if (!GATED) {
+#pragma unroll
+      for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];
+    }
+    row += step;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t wm[32];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0u;
+    for (int w = 0; w < G::CTA / 32; ++w) b = max(b, wm[w]);
+    atomicMax(p.amax_bits, b);
+  }
+}
+
 // Pass 2: rotate again, normalise, quantise from registers (whole blocks per thread).
 // MODE: 0 plain, 1 four-over-six, 2 IF4 (NVFP4 only).
 template <typename T, int LOG_D, bool NV, bool SR, int MODE, bool GATED>
@@ -533,6 +593,29 @@ static cudaError_t quant_sel(const FwhtParams& p, const FwhtLaunch& L, cudaStrea
   return L.sr ? quant_d<T, LOG_D, true, true, 0, GATED>(p, d, s) : quant_d<T, LOG_D, true, false, 0, GATED>(p, d, s);
 }
 
+template <typename T, int LOG_D, bool GATED>
+static cudaError_t store_d(const FwhtParams& p, cudaStream_t s) {
+  using G = Geom<LOG_D>;
+  const int smem = G::ROWS * G::D * 4;
+  auto k = fwht_store_kernel<T, LOG_D, GATED>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  k<<<fwht_grid<LOG_D>(k, p.rows), G::CTA, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, bool GATED>
+static cudaError_t dispatch_store(const FwhtParams& p, int d, cudaStream_t s) {
+  switch (d) {
+    case 1024: return store_d<T, 10, GATED>(p, s);
+    case 2048: return store_d<T, 11, GATED>(p, s);
+    case 4096: return store_d<T, 12, GATED>(p, s);
+    case 8192: return store_d<T, 13, GATED>(p, s);
+    case 16384: return store_d<T, 14, GATED>(p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <typename T, bool GATED>
 static cudaError_t dispatch_amax(const FwhtParams& p, int d, cudaStream_t s) {
   switch (d) {
@@ -563,6 +646,13 @@ cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s) {
   FwhtParams p = make_params(L);
   if (L.u) return L.bf16 ? dispatch_amax<__nv_bfloat16, true>(p, L.d, s) : cudaErrorInvalidValue;
   return L.bf16 ? dispatch_amax<__nv_bfloat16, false>(p, L.d, s) : dispatch_amax<float, false>(p, L.d, s);
+}
+
+cudaError_t launch_fwht_store(const FwhtLaunch& L, cudaStream_t s) {
+  if (L.rows == 0) return cudaSuccess;
+  FwhtParams p = make_params(L);
+  if (L.u) return L.bf16 ? dispatch_store<__nv_bfloat16, true>(p, L.d, s) : cudaErrorInvalidValue;
+  return L.bf16 ? dispatch_store<__nv_bfloat16, false>(p, L.d, s) : dispatch_store<float, false>(p, L.d, s);
 }
 
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s) {

@@ -103,6 +103,10 @@ cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
 // E2M1 nibbles -> E4M3 bytes; n_bytes (packed input bytes) a multiple of 16, both 16-byte aligned.
 cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* out, cudaStream_t s);
 cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);
+// Rotate once, store the normalised fp32 rotation to L.rotated_out ([rows, d]) and reduce the
+// tensor amax into *L.amax_bits; zeroes L.counts.  The quantise pass is then launch_quantize on
+// the stored values.
+cudaError_t launch_fwht_store(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s);
 

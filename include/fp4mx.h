@@ -106,9 +106,11 @@ typedef struct fp4_counts {
   unsigned long long blocks_four;
 } fp4_counts;
 
-/* Operation ids for fp4_workspace_size. */
+/* Operation ids for fp4_workspace_size.  FP4_OP_FWHT_QUANTIZE is the minimum for fwht_quantize and
+ * swiglu_fwht_quantize (the amax word); FP4_OP_FWHT_QUANTIZE_STORED the size that also holds the
+ * fp32 rotation of a [rows, cols] tensor, which lets the two-pass NVFP4 call rotate once. */
 typedef enum fp4_op { FP4_OP_MX_QUANTIZE = 0, FP4_OP_NVFP4_QUANTIZE = 1, FP4_OP_FWHT_QUANTIZE = 2,
-                      FP4_OP_DEQUANTIZE = 3, FP4_OP_BLOCK_GEMM = 4 } fp4_op;
+                      FP4_OP_DEQUANTIZE = 3, FP4_OP_BLOCK_GEMM = 4, FP4_OP_FWHT_QUANTIZE_STORED = 5 } fp4_op;
 
 /* ---------------------------------------------------------------------------------------------
  * mx_quantize — MXFP4 quantisation of a row-major [rows, cols] tensor, blocks of 32 along rows.
@@ -172,10 +174,17 @@ FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, lon
  * unchanged up to quantisation.
  *   d           : power of two, 1024 <= d <= 16384.
  *   signs       : device uint32 [d / 32], 4-byte aligned, or NULL (plain rotation); caller-owned.
- *   rotated_out : device float [rows, d] or NULL; receives the rotated values (diagnostics).
+ *   rotated_out : device float [rows, d] or NULL; receives the rotated values.
+ *   workspace   : device, 16-byte aligned; >= fp4_workspace_size(FP4_OP_FWHT_QUANTIZE) bytes when
+ *                 NVFP4 runs without global_in (two passes).  Clobbered.
  *   other arguments as in nvfp4_quantize; four_six is the NVFP4 block mode (fp4_nv_mode:
  *   FP4_NV_PLAIN, FP4_NV_FOUR_SIX, or FP4_NV_IF4 with FP4_RNE only) and, with global_in/out,
- *   applies to FP4_NVFP4 only. */
+ *   applies to FP4_NVFP4 only.
+ * The two-pass NVFP4 call (global_in NULL) takes one of two routes with the same results: when
+ * rotated_out is 32-byte aligned, or the workspace holds fp4_workspace_size(
+ * FP4_OP_FWHT_QUANTIZE_STORED, rows, d) bytes, the first pass rotates once and stores the fp32
+ * rotation there, and the second quantises the stored values; otherwise each pass rotates (no
+ * extra memory, more arithmetic). */
 FP4_API fp4_status fwht_quantize(const void* x, fp4_dtype dtype, long rows, long d,
                          const unsigned int* signs, fp4_format format,
                          int block, fp4_round round, int four_six, unsigned long long seed,

@@ -286,6 +286,38 @@ def test_fwht_small(cuda, d, fmt, rnd, four_six):
     assert counts_of(c) == co
 
 
+@pytest.mark.parametrize("d", [1024, 8192, 16384])
+@pytest.mark.parametrize("mode", ["sr", "four_six", "if4"])
+@pytest.mark.parametrize("gated", [False, True])
+def test_fwht_two_pass_routes(cuda, d, mode, gated):
+    """The two-pass NVFP4 rotation has two routes with the same bytes: a workspace of
+    fp4_workspace_size(FP4_OP_FWHT_QUANTIZE_STORED) keeps the fp32 rotation from the first pass and
+    the second pass quantises it; the minimal workspace makes both passes rotate.  Each route is
+    compared with the oracle (37 ragged rows; the randomised rotation; SwiGLU inputs when gated)."""
+    rows = 37
+    kw = dict(round=fp4.STOCHASTIC if mode == "sr" else fp4.RNE, four_six=mode == "four_six", if4=mode == "if4",
+              seed=7)
+    sg_np = synth.rht_signs(d, 5)
+    sg = torch.from_numpy(sg_np.view(np.int32)).to(cuda)
+    if gated:
+        g, u = synth.swiglu_inputs(rows, d, seed=9)
+        want = O.swiglu_fwht_quantize(f32(g), f32(u), signs=sg_np, **kw)
+        run = lambda ws: fp4.swiglu_fwht_quantize(g.to(cuda), u.to(cuda), signs=sg, workspace=ws, **kw)
+    else:
+        x = synth.fwht_laplace(rows, d, seed=8)
+        want = O.fwht_quantize(f32(x), signs=sg_np, **kw)
+        run = lambda ws: fp4.fwht_quantize(x.to(cuda), signs=sg, workspace=ws, **kw)
+    y, qo, so, go, co = want
+    small = torch.empty(fp4.workspace_size(fp4.OP_FWHT_QUANTIZE), dtype=torch.uint8, device=cuda)
+    big = torch.empty(fp4.workspace_size(fp4.OP_FWHT_QUANTIZE_STORED, rows, d), dtype=torch.uint8, device=cuda)
+    assert big.numel() >= rows * d * 4 + 256
+    for ws in (small, big):
+        q, s, gg, c, _ = run(ws)
+        assert np.float32(npy(gg)[0]) == np.float32(go)
+        assert np.array_equal(npy(q), qo) and np.array_equal(npy(s), so.ravel())
+        assert counts_of(c) == co
+
+
 def test_fwht_fp32_input_and_tiled_scales(cuda):
     x = synth.fwht_laplace(128, 8192, seed=12).float()
     q, s, g, c, _ = fp4.fwht_quantize(x.to(cuda), layout=fp4.MMA_TILED)
