@@ -473,7 +473,21 @@ def secondary(args, dev, flush, td, pk):
                 "peak_source": f"derived: {pk['source']} bf16 burst x 4 (nominal dense FP4/BF16 ratio)",
                 "frac_fp4_datasheet": round(tf / fp4_datasheet, 4),
                 "fp4_datasheet": fp4_datasheet, "datasheet_source": "B200 dense FP4 9 PFLOP/s (NVIDIA, without sparsity)"})
-    del A, B, C
+    # the IF4 GEMM on the same operands quantised to IF4 blocks: fp16 expansion of both operands,
+    # then the kind::f16 tensor-core GEMM (against the fp16/bf16 dense peak, the measured bf16 burst)
+    del A, B
+    A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), if4=True, layout=fp4.MMA_TILED)
+    B = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 2).to(dev), if4=True, layout=fp4.MMA_TILED)
+    iws = torch.empty(fp4.workspace_size(fp4.OP_BLOCK_GEMM_IF4, 16384, 8192), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: fp4.fp4_block_gemm(fp4.IF4, A[0], A[1], B[0], B[1], A[2], B[2], out=C, workspace=iws),
+               K, W, flush, td)
+    t = statistics.median(ms)
+    tf = 2 * 8192 ** 3 / (t * 1e-3) / 1e12
+    out.append({"workload": "IF4 GEMM M=N=K=8192 (IF4-quantised N(0,1) operands; fp16 expansion + kind::f16 GEMM)",
+                "ms": round(t, 4), "TFLOP/s": round(tf, 1), "frac_f16_peak": round(tf / pk["bf16_tflops"], 4),
+                "f16_peak": pk["bf16_tflops"],
+                "peak_source": f"{pk['source']} bf16 burst (the fp16 dense rate is the same)"})
+    del A, B, C, iws
     # config 5: MXFP4 down_proj, activations and weights quantised then GEMM, timed end to end
     a = synth.swiglu_act().to(dev)
     w = synth.weight().to(dev)
@@ -552,7 +566,8 @@ def run_reference(args, rank):
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-CASES = ("nv", "nv46", "nv_amax", "if4", "mx", "fwht", "gemm_nv", "gemm_mx", "gemm_e4m3", "dequant")
+CASES = ("nv", "nv46", "nv_amax", "if4", "mx", "fwht", "fwht_rht_if4", "swiglu_fwht", "gemm_nv", "gemm_mx",
+         "gemm_e4m3", "gemm_if4", "dequant")
 
 
 def run_case(name, reps):
@@ -574,6 +589,20 @@ def run_case(name, reps):
         x = synth.fwht_laplace().to(dev)
         for _ in range(reps):
             fp4.fwht_quantize(x, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7)
+    elif name == "fwht_rht_if4":
+        x = synth.fwht_laplace().to(dev)
+        sg = torch.from_numpy(synth.rht_signs(8192, 33).view(np.int32)).to(dev)
+        for _ in range(reps):
+            fp4.fwht_quantize(x, fmt=fp4.NVFP4, if4=True, signs=sg)
+    elif name == "swiglu_fwht":
+        g, u = (t_.to(dev) for t_ in synth.swiglu_inputs(16384, 8192, seed=3))
+        for _ in range(reps):
+            fp4.swiglu_fwht_quantize(g, u, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=7)
+    elif name == "gemm_if4":
+        A = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 1).to(dev), if4=True, layout=fp4.MMA_TILED)
+        B = fp4.nvfp4_quantize(synth.gemm_operand(8192, 8192, 2).to(dev), if4=True, layout=fp4.MMA_TILED)
+        for _ in range(reps):
+            fp4.fp4_block_gemm(fp4.IF4, A[0], A[1], B[0], B[1], A[2], B[2])
     elif name == "dequant":
         x = synth.nv_outliers().to(dev)
         q, s, g, _ = fp4.nvfp4_quantize(x)

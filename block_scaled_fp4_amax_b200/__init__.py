@@ -29,7 +29,8 @@ NV_PLAIN, NV_FOUR_SIX, NV_IF4 = 0, 1, 2  # fp4_nv_mode
 RNE, STOCHASTIC = 0, 1
 OCP_FLOOR, NOSAT_CEIL = 0, 1
 ROWMAJOR, MMA_TILED = 0, 1
-OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEMM, OP_FWHT_QUANTIZE_STORED = range(6)
+(OP_MX_QUANTIZE, OP_NVFP4_QUANTIZE, OP_FWHT_QUANTIZE, OP_DEQUANTIZE, OP_BLOCK_GEMM, OP_FWHT_QUANTIZE_STORED,
+ OP_BLOCK_GEMM_IF4) = range(7)
 STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 
 # Every symbol include/fp4mx.h declares.
@@ -250,15 +251,21 @@ def fp4_dequantize(q: torch.Tensor, scales: torch.Tensor, fmt: int, global_scale
 def fp4_block_gemm(fmt: int, Aq: torch.Tensor, As: torch.Tensor, Bq: torch.Tensor, Bs: torch.Tensor,
                    Ag: torch.Tensor | None = None, Bg: torch.Tensor | None = None, out: torch.Tensor | None = None,
                    stream=None, workspace: torch.Tensor | None = None):
-    """C = alpha * A @ B^T in bf16 from packed operands with MMA-tiled scales.  Returns (C, workspace);
-    workspace[0:4] holds the kernel status word (0 = ok)."""
+    """C = alpha * A @ B^T in bf16 from packed operands with MMA-tiled scales (IF4: through fp16
+    expansions held in the workspace).  Returns (C, workspace); workspace[0:4] holds the kernel
+    status word (0 = ok)."""
     _need_cuda(Aq, As, Bq, Bs, Ag, Bg)
     M, K = Aq.shape[0], Aq.shape[1] * 2
     N = Bq.shape[0]
     if Bq.shape[1] * 2 != K:
         raise ValueError("A and B disagree on K")
     C = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=Aq.device)
-    ws = workspace if workspace is not None else _workspace(OP_BLOCK_GEMM, Aq.device, M, N)
+    if workspace is not None:
+        ws = workspace
+    elif fmt == IF4:
+        ws = _workspace(OP_BLOCK_GEMM_IF4, Aq.device, M + N, K)
+    else:
+        ws = _workspace(OP_BLOCK_GEMM, Aq.device, M, N)
     _check(lib().fp4_block_gemm(fmt, M, N, K, _ptr(Aq), _ptr(As), _ptr(Ag), _ptr(Bq), _ptr(Bs), _ptr(Bg),
                                 _ptr(C), C.stride(0), _ptr(ws), ws.numel(), _stream(stream)))
     return C, ws

@@ -103,6 +103,9 @@ size_t fp4_workspace_size(fp4_op op, long rows, long cols) {
       // the amax word, padding to a 256-byte boundary, and the fp32 rotation
       return rows > 0 && cols > 0 ? 2 * kAmaxWorkspace + (size_t)rows * (size_t)cols * sizeof(float) : kAmaxWorkspace;
     case FP4_OP_BLOCK_GEMM: return kGemmWorkspace;
+    case FP4_OP_BLOCK_GEMM_IF4:
+      // rows = M + N, cols = K: the status word, padding, and both fp16 operands
+      return rows > 0 && cols > 0 ? 2 * kGemmWorkspace + 2 * (size_t)rows * (size_t)cols : kGemmWorkspace;
     default: return 0;
   }
 }
@@ -279,13 +282,37 @@ fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* scales, f
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_dequantize launch");
 }
 
+// IF4 GEMM: both operands expanded to fp16 in the workspace (E2M1 blocks exact, INT4 blocks with
+// their six-sevenths step), then the kind::f16 tensor-core GEMM with alpha = (*Ag) * (*Bg).
+static fp4_status if4_block_gemm(int M, int N, int K, const unsigned char* Aq, const unsigned char* As,
+                                 const float* Ag, const unsigned char* Bq, const unsigned char* Bs, const float* Bg,
+                                 void* C, long ldc, void* workspace, size_t ws_bytes, cudaStream_t s) {
+  if (M % 128 || N % 256 || K % 64)
+    return fail(FP4_EUNSUPPORTED, "IF4 GEMM shape %d x %d x %d: needs M %% 128, N %% 256, K %% 64 == 0", M, N, K);
+  if (!Ag || !Bg) return fail(FP4_EINVAL, "IF4 GEMM needs both global scales");
+  const size_t need = fp4_workspace_size(FP4_OP_BLOCK_GEMM_IF4, (long)M + N, K);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 16))
+    return fail(FP4_EINVAL, "the IF4 GEMM needs a 16-byte aligned workspace of %zu bytes "
+                "(fp4_workspace_size(FP4_OP_BLOCK_GEMM_IF4, M + N, K))", need);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  const uintptr_t w = reinterpret_cast<uintptr_t>(workspace);
+  uint8_t* a16 = reinterpret_cast<uint8_t*>((w + 2 * kGemmWorkspace) & ~(uintptr_t)(kGemmWorkspace - 1));
+  uint8_t* b16 = a16 + 2 * (size_t)M * (size_t)K;
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "zeroing gemm status");
+  if ((e = fp4k::launch_if4_to_f16(Aq, As, M, K, a16, s)) != cudaSuccess) return cuda_fail(e, "IF4 operand A expansion");
+  if ((e = fp4k::launch_if4_to_f16(Bq, Bs, N, K, b16, s)) != cudaSuccess) return cuda_fail(e, "IF4 operand B expansion");
+  fp4k::GemmLaunch L{true, false, true, M, N, K, a16, nullptr, b16, nullptr, Ag, Bg, C, ldc, status};
+  e = fp4k::launch_gemm(L, s);
+  return e == cudaSuccess ? FP4_OK : cuda_fail(e, "IF4 fp16 GEMM launch");
+}
+
 fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K, const unsigned char* Aq,
                           const unsigned char* As, const float* Ag, const unsigned char* Bq,
                           const unsigned char* Bs, const float* Bg, void* C, long ldc,
                           void* workspace, size_t ws_bytes, void* stream) {
-  if (format == FP4_IF4)
-    return fail(FP4_EUNSUPPORTED, "IF4 operands have no tensor-core path (the block-scaled MMA reads E2M1 only)");
-  if (format != FP4_MXFP4 && format != FP4_NVFP4) return fail(FP4_EINVAL, "format %d unknown", (int)format);
+  if (format != FP4_MXFP4 && format != FP4_NVFP4 && format != FP4_IF4)
+    return fail(FP4_EINVAL, "format %d unknown", (int)format);
   const bool nv = format == FP4_NVFP4;
   if (M <= 0 || N <= 0 || K <= 0) return fail(FP4_EINVAL, "bad GEMM shape %d x %d x %d", M, N, K);
   if (M % 128 || N % 256 || K % 256)
@@ -295,13 +322,14 @@ fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K, const unsigned
   if (ldc < N || ldc % 8) return fail(FP4_EINVAL, "ldc %ld must be >= N and a multiple of 8", ldc);
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(As, 16) || !aligned(Bs, 16) || !aligned(C, 16))
     return fail(FP4_EINVAL, "GEMM operands must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (format == FP4_IF4) return if4_block_gemm(M, N, K, Aq, As, Ag, Bq, Bs, Bg, C, ldc, workspace, ws_bytes, s);
   if (!workspace || ws_bytes < kGemmWorkspace || !aligned(workspace, 16))
     return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required", kGemmWorkspace);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* status = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return cuda_fail(e, "zeroing gemm status");
-  fp4k::GemmLaunch L{nv, false, M, N, K, Aq, As, Bq, Bs, nv ? Ag : nullptr, nv ? Bg : nullptr, C, ldc, status};
+  fp4k::GemmLaunch L{nv, false, false, M, N, K, Aq, As, Bq, Bs, nv ? Ag : nullptr, nv ? Bg : nullptr, C, ldc, status};
   e = fp4k::launch_gemm(L, s);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_block_gemm launch");
 }
@@ -333,7 +361,7 @@ fp4_status fp4_block_gemm_e4m3(int M, int N, int K, const unsigned char* A8, con
   uint32_t* status = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return cuda_fail(e, "zeroing gemm status");
-  fp4k::GemmLaunch L{false, true, M, N, K, A8, As, B8, Bs, nullptr, nullptr, C, ldc, status};
+  fp4k::GemmLaunch L{false, true, false, M, N, K, A8, As, B8, Bs, nullptr, nullptr, C, ldc, status};
   e = fp4k::launch_gemm(L, s);
   return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fp4_block_gemm_e4m3 launch");
 }

@@ -132,6 +132,14 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdes
   }
 }
 
+// fp16 operands without block scales (the IF4 GEMM's expanded operands): kind::f16, K = 16 per
+// instruction, FP32 accumulation.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+               ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // The FP8 route for MXFP4 operands expanded to E4M3: kind::mxf8f6f4, one UE8M0 scale per 32 values
 // (scale_vec::1X), K = 32 per instruction.
 __device__ __forceinline__ void tc_mma_f8(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
@@ -183,19 +191,26 @@ __host__ __device__ constexpr uint32_t idesc_f8(uint32_t sfa_id, uint32_t sfb_id
   return (sfb_id << 4) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) | (sfa_id << 29);
 }
 
+// Instruction descriptor, kind::f16: F32 accumulator (bits 4-5 = 1), F16 x F16 (format 0 in bits
+// 7-9 and 10-12), K-major A and B, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t idesc_f16() {
+  return (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
 // Operand kinds of the 1-SM kernel.
-constexpr int kMxFp4 = 0, kNvFp4 = 1, kMxE4m3 = 2;
+constexpr int kMxFp4 = 0, kNvFp4 = 1, kMxE4m3 = 2, kF16 = 3;
 
 // ---------------------------------------------------------------------------------------------
 // KIND kMxFp4 / kNvFp4: packed E2M1 operands, 256 values (128 bytes) per row per stage, four K=64
 // MMAs.  kMxE4m3: the E4M3 expansions of MXFP4 operands, 128 values (128 bytes) per stage, four
 // K=32 MMAs of kind::mxf8f6f4, each taking one of the stage's four UE8M0 scales per row (scale
-// byte id 0-3 of the atom's 32-bit tensor-memory column).
+// byte id 0-3 of the atom's 32-bit tensor-memory column).  kF16: fp16 operands, 64 values (128
+// bytes) per stage, four K=16 MMAs of kind::f16, no scales.
 template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
-  constexpr bool NV = KIND == kNvFp4, F8 = KIND == kMxE4m3;
-  constexpr int ATOMS = NV ? 4 : (F8 ? 1 : 2);  // scale atoms per 128 rows per stage
+  constexpr bool NV = KIND == kNvFp4, F8 = KIND == kMxE4m3, F16 = KIND == kF16;
+  constexpr int ATOMS = F16 ? 0 : (NV ? 4 : (F8 ? 1 : 2));  // scale atoms per 128 rows per stage
   constexpr int SFA_BYTES = ATOMS * 512;
   constexpr int SFB_BYTES = 2 * ATOMS * 512;  // two 128-row groups
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
@@ -241,7 +256,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
   const int tiles_m = p.M / BM, tiles_n = p.N / BN;
   const int num_tiles = tiles_m * tiles_n;
-  const int kt_count = p.K / (F8 ? 128 : 256);
+  const int kt_count = p.K / (F16 ? 64 : (F8 ? 128 : 256));
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -265,12 +280,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           last_parity[s] = ph;
           tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, kt * BKB, tm * BM, fb);
           tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, kt * BKB, tn * BN, fb);
-          const uint8_t* sfa = p.As + ((size_t)tm * p.atoms_row + (size_t)kt * ATOMS) * 512;
-          bulk_load(smem_u32(sSFA + s * SFA_BYTES), sfa, SFA_BYTES, fb);
+          if constexpr (!F16) {
+            const uint8_t* sfa = p.As + ((size_t)tm * p.atoms_row + (size_t)kt * ATOMS) * 512;
+            bulk_load(smem_u32(sSFA + s * SFA_BYTES), sfa, SFA_BYTES, fb);
 #pragma unroll
-          for (int rg = 0; rg < 2; ++rg) {
-            const uint8_t* sfb = p.Bs + ((size_t)(2 * tn + rg) * p.atoms_row + (size_t)kt * ATOMS) * 512;
-            bulk_load(smem_u32(sSFB + s * SFB_BYTES + rg * ATOMS * 512), sfb, ATOMS * 512, fb);
+            for (int rg = 0; rg < 2; ++rg) {
+              const uint8_t* sfb = p.Bs + ((size_t)(2 * tn + rg) * p.atoms_row + (size_t)kt * ATOMS) * 512;
+              bulk_load(smem_u32(sSFB + s * SFB_BYTES + rg * ATOMS * 512), sfb, ATOMS * 512, fb);
+            }
           }
         }
       }
@@ -315,7 +332,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 #pragma unroll
           for (int t = 0; t < 4; ++t) {  // four MMAs of 32 bytes of K per stage
             const uint32_t acc = (kt > 0 || t > 0) ? 1u : 0u;
-            if constexpr (F8) {
+            if constexpr (F16) {
+              tc_mma_f16(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc_f16(), acc);
+            } else if constexpr (F8) {
               tc_mma_f8(tmem + ACC_COL, desc_sw128(a0 + 32 * t), desc_sw128(b0 + 32 * t), idesc_f8(t, t),
                         tmem + SFA_COL, tmem + SFB_COL, acc);
             } else {
@@ -385,7 +404,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
 template <int KIND>
 constexpr int smem_bytes() {
-  constexpr int atoms = KIND == kNvFp4 ? 4 : (KIND == kMxE4m3 ? 1 : 2);
+  constexpr int atoms = KIND == kF16 ? 0 : (KIND == kNvFp4 ? 4 : (KIND == kMxE4m3 ? 1 : 2));
   return 1024 + STAGES * (A_BYTES + B_BYTES + atoms * 512 * 3) + 256;
 }
 
@@ -784,9 +803,9 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   p.C = reinterpret_cast<__nv_bfloat16_raw*>(L.C);
   p.ldc = L.ldc;
   p.status = L.status;
-  if (!L.e4m3 && L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
-  // operand rows: K/2 packed bytes (FP4) or K bytes (E4M3 expansion)
-  const uint64_t row_bytes = L.e4m3 ? (uint64_t)L.K : (uint64_t)L.K / 2;
+  if (!L.e4m3 && !L.f16 && L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
+  // operand rows: K/2 packed bytes (FP4), K bytes (E4M3 expansion) or 2K bytes (fp16)
+  const uint64_t row_bytes = L.f16 ? 2 * (uint64_t)L.K : (L.e4m3 ? (uint64_t)L.K : (uint64_t)L.K / 2);
   CUtensorMap ta, tb;
   if (!make_map(&ta, L.Aq, row_bytes, (uint64_t)L.M, BM) || !make_map(&tb, L.Bq, row_bytes, (uint64_t)L.N, BN))
     return cudaErrorInvalidValue;
@@ -796,7 +815,8 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     k<<<grid, NUM_THREADS, smem, s>>>(ta, tb, p);
   };
-  if (L.e4m3) go(gemm_kernel<kMxE4m3>, smem_bytes<kMxE4m3>());
+  if (L.f16) go(gemm_kernel<kF16>, smem_bytes<kF16>());
+  else if (L.e4m3) go(gemm_kernel<kMxE4m3>, smem_bytes<kMxE4m3>());
   else if (L.nv) go(gemm_kernel<kNvFp4>, smem_bytes<kNvFp4>());
   else go(gemm_kernel<kMxFp4>, smem_bytes<kMxFp4>());
   return cudaGetLastError();

@@ -86,6 +86,7 @@ struct FwhtLaunch {
 struct GemmLaunch {
   bool nv;
   bool e4m3;  // MXFP4 through the FP8 MMA: Aq/Bq are E4M3 expansions [rows, K] (kind::mxf8f6f4)
+  bool f16;   // fp16 operands [rows, K] (kind::f16, no block scales; alpha = (*Ag) * (*Bg))
   int M, N, K;
   const uint8_t *Aq, *As, *Bq, *Bs;
   const float *Ag, *Bg;
@@ -100,6 +101,10 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
 cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
                         unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
+// IF4 operand [rows, cols] (packed nibbles, MMA-tiled scales) -> fp16 [rows, cols] without the
+// per-tensor scale: v * d for E2M1 blocks, RNE fp16 of fl(fl(k * d) * fl(6/7)) for INT4 blocks.
+cudaError_t launch_if4_to_f16(const uint8_t* q, const uint8_t* scales, long long rows, long long cols, void* out,
+                              cudaStream_t s);
 // E2M1 nibbles -> E4M3 bytes; n_bytes (packed input bytes) a multiple of 16, both 16-byte aligned.
 cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* out, cudaStream_t s);
 cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);

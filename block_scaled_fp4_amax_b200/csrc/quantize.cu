@@ -454,6 +454,49 @@ __global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint4* q, 
 }
 
 // ---------------------------------------------------------------------------------------------
+// IF4 -> fp16 GEMM operand (the IF4 GEMM: "Adaptive Block-Scaled Data Types" podcast, IF4 segment).
+// An E2M1 block gives v * d, exact in fp16 (at most 6 significant bits, magnitudes 2^-10 .. 2688);
+// an INT4 block (scale bit 7) gives the RNE fp16 of fl(fl(k * d) * fl(6/7)): its integer step is six
+// sevenths of the E2M1 unit, so a mixed block pair carries 6/7 and an INT4 pair 36/49 into the
+// product.  The per-tensor scale stays out of the element (fp16 range); the GEMM epilogue applies
+// both.  Scales are read in the MMA tile layout; each thread expands one 16-block (8 packed bytes).
+__global__ void __launch_bounds__(kThreads) if4_to_f16_kernel(const uint8_t* q, const uint8_t* scales,
+                                                              long long n_groups, DivU32 nb, uint4* out) {
+  const long long stride = (long long)gridDim.x * kThreads;
+  for (long long g = (long long)blockIdx.x * kThreads + threadIdx.x; g < n_groups; g += stride) {
+    const uint2 w = *reinterpret_cast<const uint2*>(q + g * 8);
+    const uint8_t sb = scales[scale_offset((unsigned long long)g, nb, true)];
+    const uint32_t code = sb & 0x7Fu;
+    uint32_t h[8];
+    if (sb & 0x80u) {
+      const float d = e4m3_value(code);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float f[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int e = 2 * i + j;
+          const uint32_t c = ((e < 8 ? w.x : w.y) >> (4 * (e & 7))) & 15u;
+          const float k = (c & 8u) ? -(float)(c & 7u) : (float)(c & 7u);
+          f[j] = __fmul_rn(__fmul_rn(k, d), kSixSevenths);  // k * d exact, then one rounding
+        }
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(f[1]), "f"(f[0]));
+      }
+    } else {
+      uint32_t dh2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(dh2) : "h"((uint16_t)(code | (code << 8))));
+      uint32_t v[8];
+      e2m1x8_to_f16x2(w.x, v);
+      e2m1x8_to_f16x2(w.y, v + 4);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(v[i]), "r"(dh2));
+    }
+    out[2 * g] = make_uint4(h[0], h[1], h[2], h[3]);
+    out[2 * g + 1] = make_uint4(h[4], h[5], h[6], h[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Launchers
 
 static int grid_for(long long work_items, int per_cta) {
@@ -528,6 +571,15 @@ cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* ou
   if (n16 == 0) return cudaSuccess;
   e2m1_to_e4m3_kernel<<<grid_for(n16, kThreads), kThreads, 0, s>>>(reinterpret_cast<const uint4*>(q),
                                                                    reinterpret_cast<uint4*>(out), n16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_if4_to_f16(const uint8_t* q, const uint8_t* scales, long long rows, long long cols, void* out,
+                              cudaStream_t s) {
+  const long long groups = rows * cols / 16;
+  if (groups == 0) return cudaSuccess;
+  if4_to_f16_kernel<<<grid_for(groups, kThreads), kThreads, 0, s>>>(q, scales, groups, make_divu32((uint32_t)(cols / 16)),
+                                                                    reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }
 

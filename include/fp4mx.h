@@ -110,7 +110,8 @@ typedef struct fp4_counts {
  * swiglu_fwht_quantize (the amax word); FP4_OP_FWHT_QUANTIZE_STORED the size that also holds the
  * fp32 rotation of a [rows, cols] tensor, which lets the two-pass NVFP4 call rotate once. */
 typedef enum fp4_op { FP4_OP_MX_QUANTIZE = 0, FP4_OP_NVFP4_QUANTIZE = 1, FP4_OP_FWHT_QUANTIZE = 2,
-                      FP4_OP_DEQUANTIZE = 3, FP4_OP_BLOCK_GEMM = 4, FP4_OP_FWHT_QUANTIZE_STORED = 5 } fp4_op;
+                      FP4_OP_DEQUANTIZE = 3, FP4_OP_BLOCK_GEMM = 4, FP4_OP_FWHT_QUANTIZE_STORED = 5,
+                      FP4_OP_BLOCK_GEMM_IF4 = 6 } fp4_op;
 
 /* ---------------------------------------------------------------------------------------------
  * mx_quantize — MXFP4 quantisation of a row-major [rows, cols] tensor, blocks of 32 along rows.
@@ -239,9 +240,17 @@ FP4_API fp4_status fp4_dequantize(const unsigned char* q, const unsigned char* s
  *   workspace : device, >= fp4_workspace_size(FP4_OP_BLOCK_GEMM, M, N) bytes, 16-byte aligned; the
  *               kernel's status word (0 = ok, nonzero = a bounded pipeline wait gave up) is its
  *               first 4 bytes; see fp4_gemm_status_word.
+ * FP4_IF4 ([P] IF4 segment): blocks whose scale byte has bit 7 set hold INT4 integers k whose step
+ * is six sevenths of the E2M1 unit, so a mixed FP4 x INT4 block pair carries the factor 6/7 and an
+ * INT4 x INT4 pair 36/49.  No block-scaled MMA kind carries those factors (E4M3 and UE8M0 block
+ * scales cannot hold d * 6/7), so both operands are first expanded into the workspace as fp16
+ * without the per-tensor scale: v * d for an E2M1 block (exact) and the RNE fp16 of
+ * fl(fl(k * d) * fl(6/7)) for an INT4 block (relative error below 2^-11).  Then tcgen05.mma
+ * kind::f16 computes C = (*Ag) * (*Bg) * A16 * B16^T with FP32 accumulation.  An NVFP4 operand is
+ * an IF4 operand without INT4 blocks.  Ag and Bg are required; the workspace must hold
+ * fp4_workspace_size(FP4_OP_BLOCK_GEMM_IF4, M + N, K) bytes (the status word first).
  * Preconditions: M % 128 == 0, N % 256 == 0, K % 256 == 0, ldc >= N, ldc % 8 == 0, all pointers
- * 16-byte aligned.  Other shapes return FP4_EUNSUPPORTED, as does FP4_IF4 (the block-scaled MMA
- * reads E2M1 only; dequantise IF4 operands first). */
+ * 16-byte aligned.  Other shapes return FP4_EUNSUPPORTED. */
 FP4_API fp4_status fp4_block_gemm(fp4_format format, int M, int N, int K,
                           const unsigned char* Aq, const unsigned char* As, const float* Ag,
                           const unsigned char* Bq, const unsigned char* Bs, const float* Bg,

@@ -262,7 +262,7 @@ def dequantize(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
 
 
 def dequantize_f64(q, scales, fmt: int, s_g: float = 1.0) -> np.ndarray:
-    """Exact fp64 reconstruction v*d*s_g."""
+    """Exact fp64 reconstruction v*d*s_g (MXFP4 v*2^e; IF4 INT4 blocks k*d*s_g*6/7)."""
     q = np.ascontiguousarray(q, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     rows, half = q.shape
@@ -370,6 +370,6 @@ def gemm_f64(Aq, As, Ag, Bq, Bs, Bg, fmt: int, rows=None, cols=None):
         Aq, As = np.asarray(Aq)[rows], np.asarray(As)[rows]
     if cols is not None:
         Bq, Bs = np.asarray(Bq)[cols], np.asarray(Bs)[cols]
-    a = dequantize_f64(Aq, As, fmt, Ag if fmt == NVFP4 else 1.0)
-    b = dequantize_f64(Bq, Bs, fmt, Bg if fmt == NVFP4 else 1.0)
+    a = dequantize_f64(Aq, As, fmt, 1.0 if fmt == MXFP4 else Ag)
+    b = dequantize_f64(Bq, Bs, fmt, 1.0 if fmt == MXFP4 else Bg)
     return a @ b.T, np.abs(a) @ np.abs(b).T

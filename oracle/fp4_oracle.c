@@ -552,7 +552,13 @@ void ora_e2m1_to_e4m3(const uint8_t* q, long rows, long cols, uint8_t* out) {
   }
 }
 
-/* Exact fp64 dequantisation (for the GEMM reference): v * d * s_g with no rounding.            */
+/* Exact fp64 dequantisation (for the GEMM reference), with no rounding: v * 2^(byte-127) (MXFP4),
+ * v * d * s_g (NVFP4, and IF4 blocks whose scale byte has bit 7 clear), k * d * s_g * 6/7 (IF4
+ * INT4 blocks, d from the low 7 bits).  [P] IF4 segment: an INT4 block's integer step is 6/7 of the
+ * E2M1 unit (its maximum lands on 7), so in a product of two blocks a mixed FP4 x INT4 pair carries
+ * the factor 6/7 and an INT4 x INT4 pair 36/49, applied once in full precision before the sum; here
+ * the factor is the exact ratio 6/7 (the fp32 quantiser's s7 = fl(s_g * fl(6/7)) is a rounding of
+ * it).  The product of two reconstructions carries exactly those factors.                       */
 void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, long rows, long cols,
                         float s_g, double* out) {
   int B = (format == 0) ? 32 : 16;
@@ -563,7 +569,13 @@ void ora_dequantize_f64(const uint8_t* q, const uint8_t* scales, int format, lon
       int code = (k & 1) ? (byte >> 4) : (byte & 15);
       uint8_t sb = scales[r * nb + k / B];
       double v = ora_e2m1_value(code);
-      out[r * cols + k] = (format == 0) ? ldexp(v, (int)sb - 127) : v * ora_e4m3_value(sb) * (double)s_g;
+      if (format == 0) {
+        out[r * cols + k] = ldexp(v, (int)sb - 127);
+      } else if (format == 2 && (sb & 0x80)) {
+        out[r * cols + k] = ora_int4_value(code) * ora_e4m3_value(sb & 0x7F) * (double)s_g * 6.0 / 7.0;
+      } else {
+        out[r * cols + k] = v * ora_e4m3_value(sb) * (double)s_g;
+      }
     }
   }
 }

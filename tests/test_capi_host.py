@@ -84,13 +84,21 @@ def test_nvfp4_rejects(L):
 
 
 def test_if4_rejects(L):
-    # IF4 is round-to-nearest NVFP4 only (also in the rotation path); block modes beyond IF4; no IF4 GEMM
+    # IF4 is round-to-nearest NVFP4 only (also in the rotation path); block modes beyond IF4
     assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 1, 2, 0, 0, FAKE, None, FAKE, FAKE, None, None, 0, None) == 2
     assert L.nvfp4_quantize(FAKE, 1, 128, 256, 16, 0, 3, 0, 0, FAKE, None, FAKE, FAKE, None, None, 0, None) == 1
     assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 1, 16, 1, 2, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 2
     assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 0, 32, 0, 2, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 2
     assert L.fwht_quantize(FAKE, 1, 4, 8192, None, 1, 16, 0, 3, 0, 0, FAKE, None, None, FAKE, FAKE, None, FAKE, 256, None) == 1
-    assert L.fp4_block_gemm(2, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 2
+    # IF4 GEMM: the fp16 operands need fp4_workspace_size(FP4_OP_BLOCK_GEMM_IF4, M + N, K) bytes, both
+    # global scales, and the FP4 GEMM's shape rules
+    need = L.fp4_workspace_size(6, 128 + 256, 256)
+    assert need == 512 + 2 * (128 + 256) * 256
+    assert L.fp4_block_gemm(2, 128, 256, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, 256, None) == 1
+    assert L.fp4_block_gemm(2, 128, 256, 256, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 256, FAKE, need, None) == 1
+    assert L.fp4_block_gemm(2, 128, 256, 192, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, need, None) == 2
+    # the stored-rotation workspace: the amax word, padding and the fp32 rotation
+    assert L.fp4_workspace_size(5, 64, 8192) == 512 + 64 * 8192 * 4 and L.fp4_workspace_size(2, 64, 8192) == 256
     # IF4 dequantisation: block 16 and a global scale
     assert L.fp4_dequantize(FAKE, FAKE, 2, 32, 0, FAKE, 128, 256, 0, FAKE, None) == 1
     assert L.fp4_dequantize(FAKE, FAKE, 2, 16, 0, None, 128, 256, 0, FAKE, None) == 1

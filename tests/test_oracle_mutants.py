@@ -36,6 +36,8 @@ MUTANTS = [
      [pins.test_rejected_blocks_and_counts]),
     ("E2M1 exponent bias dropped", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e)",
      [pins.test_e2m1_decode_table_matches_printed_lattice]),
+    ("IF4 INT4 blocks without the six-sevenths step in the GEMM reference",
+     "(double)s_g * 6.0 / 7.0;", "(double)s_g;", [pins.test_if4_gemm_reference_alignment_factors]),
     ("Hadamard butterfly difference reversed", "        v[i + h] = a - b;", "        v[i + h] = b - a;",
      [pins.test_fwht_matches_sylvester_hadamard_matrix]),
 ]

@@ -745,6 +745,31 @@ def test_gemm_reference_closed_forms():
     assert np.array_equal(C, want)
 
 
+def test_if4_gemm_reference_alignment_factors():
+    """IF4 block products (podcast IF4 segment, tests/golden/if4.txt): an FP4 x INT4 block pair
+    carries six sevenths, an INT4 x INT4 pair thirty-six forty-ninths.  Rows of one 16-block: FP4
+    blocks of code 7 (6.0) or 5 (3.0), INT4 blocks of code 7 (+7) or 13 (-5); every product is
+    checked against the exact rational value."""
+    from fractions import Fraction
+    _, _, _, _, _, mix_n, mix_d, ii_n, ii_d = [int(v) for v in golden_rows("if4.txt")[0]]
+    rows = [(0x77, 0x38, Fraction(6)), (0x55, 0x38, Fraction(3)),        # FP4 blocks, scale 1.0
+            (0x77, 0xB8, Fraction(7)), (0xDD, 0xC0, Fraction(-5))]       # INT4 blocks, scale 1.0 / 2.0
+    Aq = np.array([[b] * 8 for b, _, _ in rows], dtype=np.uint8)
+    As = np.array([[sb] for _, sb, _ in rows], dtype=np.uint8)
+    sga, sgb = 0.5, 0.25
+    C, S = O.gemm_f64(Aq, As, sga, Aq, As, sgb, O.IF4)
+    for i, (_, sa, va) in enumerate(rows):
+        for j, (_, sb, vb) in enumerate(rows):
+            int_a, int_b = bool(sa & 0x80), bool(sb & 0x80)
+            f = {0: Fraction(1), 1: Fraction(mix_n, mix_d), 2: Fraction(ii_n, ii_d)}[int_a + int_b]
+            da = Fraction(O.e4m3_value(sa & 0x7F)).limit_denominator()
+            db = Fraction(O.e4m3_value(sb & 0x7F)).limit_denominator()
+            want = 16 * va * vb * da * db * f * Fraction(sga) * Fraction(sgb)
+            assert abs(C[i, j] - float(want)) <= 1e-12 * abs(float(want)), (i, j, C[i, j], want)
+    # the stretch: an INT4 block at its maximum (7) reconstructs an FP4 block at its maximum (6)
+    assert C[2, 2] == C[0, 0] == C[0, 2]
+
+
 def test_scale_tile_layout_is_a_bijection_with_the_documented_offsets():
     rows, nb = 256, 8
     s = np.arange(rows * nb, dtype=np.int64).reshape(rows, nb) % 251
