@@ -36,7 +36,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_EINVAL", 2: "FP4_EUNSUPPORTED", 3: "FP4_ECUDA"}
 # Every symbol include/fp4mx.h declares.
 EXPORTS = ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize", "fp4_block_gemm",
            "fp4_workspace_size", "fp4_gemm_status_word", "fp4_status_str", "fp4_last_error",
-           "nvfp4_quantize_noalloc", "fp4_to_e4m3", "fp4_block_gemm_e4m3")
+           "nvfp4_quantize_noalloc", "fp4_to_e4m3", "fp4_block_gemm_e4m3", "fp4_set_gemm_wait_limit")
 
 
 class Fp4Error(RuntimeError):
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.fp4_status_str.restype = ctypes.c_char_p
     L.fp4_last_error.argtypes = []
     L.fp4_last_error.restype = ctypes.c_char_p
+    L.fp4_set_gemm_wait_limit.argtypes = [ULL]
+    L.fp4_set_gemm_wait_limit.restype = ULL
     for name in ("mx_quantize", "nvfp4_quantize", "fwht_quantize", "swiglu_fwht_quantize", "fp4_dequantize",
                  "fp4_block_gemm", "fp4_to_e4m3", "fp4_block_gemm_e4m3"):
         getattr(L, name).restype = I
@@ -269,6 +271,12 @@ def fp4_block_gemm(fmt: int, Aq: torch.Tensor, As: torch.Tensor, Bq: torch.Tenso
     _check(lib().fp4_block_gemm(fmt, M, N, K, _ptr(Aq), _ptr(As), _ptr(Ag), _ptr(Bq), _ptr(Bs), _ptr(Bg),
                                 _ptr(C), C.stride(0), _ptr(ws), ws.numel(), _stream(stream)))
     return C, ws
+
+
+def set_gemm_wait_limit(ns: int) -> int:
+    """Limit (ns) of each pipeline wait in GEMM launches made from now on; returns the previous one
+    (default 2 s).  A tiny limit makes the kernel give up early and report it in its status word."""
+    return int(lib().fp4_set_gemm_wait_limit(ns))
 
 
 def fp4_to_e4m3(q: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

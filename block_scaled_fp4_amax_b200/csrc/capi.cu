@@ -112,6 +112,8 @@ size_t fp4_workspace_size(fp4_op op, long rows, long cols) {
 
 size_t fp4_gemm_status_word(void) { return 0; }
 
+unsigned long long fp4_set_gemm_wait_limit(unsigned long long ns) { return fp4k::set_gemm_wait_limit(ns); }
+
 fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
                        fp4_mx_policy policy, fp4_round round, unsigned long long seed,
                        fp4_scale_layout layout, unsigned char* q, unsigned char* scales,

@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "launch.h"
@@ -40,7 +41,7 @@ constexpr int NUM_THREADS = 192;
 constexpr int A_BYTES = BM * BKB, B_BYTES = BN * BKB;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0, SFA_COL = 256, SFB_COL = 288;
-constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s: default pipeline wait limit, and every drain wait
 
 struct Params {
   int M, N, K;
@@ -54,6 +55,7 @@ struct Params {
   __nv_bfloat16_raw* C;
   long long ldc;
   uint32_t* status;
+  unsigned long long wait_ns;  // limit of each pipeline wait (kTimeoutNs unless set otherwise)
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -82,19 +84,27 @@ __device__ __forceinline__ unsigned long long now_ns() {
   return t;
 }
 
-// Bounded wait: true when the phase completed; false when this or another role gave up.
+// Bounded wait: true when the phase completed; false when this or another role gave up.  A wait
+// longer than `limit` ns records its site in the status word and tells the other roles to stop.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t site) {
+                                          uint32_t* status, uint32_t site, unsigned long long limit) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
   while (true) {
     if (mbar_try(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (now_ns() - t0 > kTimeoutNs) {
+    if (now_ns() - t0 > limit) {
       atomicOr(status, 1u << site);
       *abort_flag = 1;
       return false;
     }
+  }
+}
+
+// Drain wait (exit paths): until the phase completes or kTimeoutNs passes, whatever the flags say.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try(bar, parity) && now_ns() - t0 < kTimeoutNs) {
   }
 }
 
@@ -273,7 +283,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         for (int kt = 0; kt < kt_count; ++kt, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0)) { ok = false; break; }
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0, p.wait_ns)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * s;
           mbar_expect_tx(fb, TX_BYTES);
           pending[s] = true;
@@ -291,21 +301,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           }
         }
       }
-      if (!ok) {
-        // drain: every fill issued must land before the CTA's shared memory goes away
-        for (int s = 0; s < STAGES; ++s) {
-          if (!pending[s]) continue;
-          const unsigned long long t0 = now_ns();
-          while (!mbar_try(full0 + 8 * s, last_parity[s]) && now_ns() - t0 < kTimeoutNs) {
-          }
-        }
-      } else {
+      if (ok) {
         // wait for the MMA side to release the last STAGES fills, so that no tcgen05.commit
         // arrival is still in flight towards this CTA's barriers when it exits
         for (int i = 0; i < STAGES; ++i, ++g) {
           const int s = g % STAGES;
-          if (!mbar_wait(empty0 + 8 * s, ((g / STAGES) & 1) ^ 1, abort_flag, p.status, 4)) break;
+          if (!mbar_wait(empty0 + 8 * s, ((g / STAGES) & 1) ^ 1, abort_flag, p.status, 4, p.wait_ns)) {
+            ok = false;
+            break;
+          }
         }
+      }
+      if (!ok) {
+        // a wait gave up: every fill issued must still land before the CTA's shared memory goes
+        // away (the last fill of each stage completes that stage's full-barrier phase)
+        for (int s = 0; s < STAGES; ++s)
+          if (pending[s]) mbar_drain(full0 + 8 * s, last_parity[s]);
       }
     }
   } else if (warp == 1) {
@@ -313,12 +324,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint32_t g = 0, j = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++j) {
-      if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1)) { ok = false; break; }
+      if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       for (int kt = 0; kt < kt_count; ++kt, ++g) {
         const int s = g % STAGES;
         const uint32_t ph = (g / STAGES) & 1;
-        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.status, 2)) { ok = false; break; }
+        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sA + s * A_BYTES), b0 = smem_u32(sB + s * B_BYTES);
@@ -353,10 +364,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       __syncwarp();
     }
     if (!ok && lane == 0) {
-      tc_commit(drain);
-      const unsigned long long t0 = now_ns();
-      while (!mbar_try(drain, 0) && now_ns() - t0 < kTimeoutNs) {
-      }
+      tc_commit(drain);  // arrives once every MMA and scale copy this thread issued has completed
+      mbar_drain(drain, 0);
     }
     __syncwarp();
   } else {
@@ -367,7 +376,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
       const int tm = tile % tiles_m, tn = tile / tiles_m;
-      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3)) break;
+      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const int row = tm * BM + q * 32 + lane;
       uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN);
@@ -556,12 +565,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
       uint32_t g = 0;
       bool ok = true, issued = false;
+      bool pending[S];
+      uint32_t last_parity[S];
+      for (int s = 0; s < S; ++s) { pending[s] = false; last_parity[s] = 0; }
       for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
         const int tm = tile % tiles_m, tn = tile / tiles_m;
         for (int kt = 0; kt < kt_count; ++kt, ++g) {
           const int s = g % S;
           const uint32_t ph = (g / S) & 1;
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0)) { ok = false; break; }
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0, p.wait_ns)) { ok = false; break; }
           const uint32_t fb = map_rank(full0 + 8 * s, 0);  // the leader's barrier
           if (leader) mbar_expect_tx(full0 + 8 * s, TX_PAIR);
           tma_pair_2d(smem_u32(sA + s * C::A_HALF), &tmA, kt * BKB, tm * 256 + (int)rank * 128, fb);
@@ -569,19 +581,32 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           tma_pair_3d(smem_u32(sSFA + s * C::SFA_BYTES), &tmSA, 0, kt * ATOMS, tm * 2 + (int)rank, fb);
           tma_pair_3d(smem_u32(sSFB + s * C::SFB_BYTES), &tmSB, 0, kt * ATOMS, tn * 2, fb);
           issued = true;
+          pending[s] = true;
+          last_parity[s] = ph;
         }
       }
       if (ok) {
         // the last S releases: no tcgen05.commit arrival is still on its way to this CTA
         for (int i = 0; i < S; ++i, ++g) {
           const int s = g % S;
-          if (!mbar_wait(empty0 + 8 * s, ((g / S) & 1) ^ 1, abort_flag, p.status, 4)) break;
+          if (!mbar_wait(empty0 + 8 * s, ((g / S) & 1) ^ 1, abort_flag, p.status, 4, p.wait_ns)) {
+            ok = false;
+            break;
+          }
         }
-      } else if (issued) {
-        // loads in flight complete on the leader's barrier, which this CTA cannot observe:
-        // give them a fixed, bounded time to land before shared memory is released
-        const unsigned long long t0 = now_ns();
-        while (now_ns() - t0 < 2000000ull) {
+      }
+      if (!ok && issued) {
+        if (leader) {
+          // both CTAs' fills complete on the leader's barriers: wait (bounded) for the last phase
+          // of every stage issued, so that they have landed before the final cluster barrier
+          for (int s = 0; s < S; ++s)
+            if (pending[s]) mbar_drain(full0 + 8 * s, last_parity[s]);
+        } else {
+          // this CTA cannot observe its fills (they complete on the leader's barrier): give them a
+          // fixed, bounded time to land before shared memory is released
+          const unsigned long long t0 = now_ns();
+          while (now_ns() - t0 < 2000000ull) {
+          }
         }
       }
     }
@@ -600,8 +625,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t g = 0;
       for (; g < total && ok; ++g) {
         const int s = g % S, b = g % NB;
-        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 6)) { ok = false; break; }
-        if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 7)) { ok = false; break; }
+        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 6, p.wait_ns)) { ok = false; break; }
+        if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 7, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t fa = smem_u32(sSFA + s * C::SFA_BYTES), fbs = smem_u32(sSFB + s * C::SFB_BYTES);
@@ -621,14 +646,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // the MMA warp's last releases of the scale buffers have landed
         for (int i = 0; i < NB; ++i, ++g) {
           const int b = g % NB;
-          if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8)) break;
+          if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8, p.wait_ns)) break;
         }
       } else if (lane == 0) {
         const uint32_t dr = drain0 + 8 * (1 + ci);
-        tc_commit_local_pair(dr);
-        const unsigned long long t0 = now_ns();
-        while (!mbar_try(dr, 0) && now_ns() - t0 < kTimeoutNs) {
-        }
+        tc_commit_local_pair(dr);  // arrives once this warp's scale copies have completed
+        mbar_drain(dr, 0);
       }
       __syncwarp();
     }
@@ -642,10 +665,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int s = g % S, b = g % NB;
         j = g / (uint32_t)kt_count;
         if (kt == 0) {
-          if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1)) { ok = false; break; }
+          if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
         }
-        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 2)) { ok = false; break; }
-        if (!mbar_wait(sf_full0 + 8 * b, (g / NB) & 1, abort_flag, p.status, 9)) { ok = false; break; }
+        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
+        if (!mbar_wait(sf_full0 + 8 * b, (g / NB) & 1, abort_flag, p.status, 9, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sA + s * C::A_HALF), b0 = smem_u32(sB + s * C::B_HALF);
@@ -667,12 +690,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       j = my_tiles;
       if (ok) {
         // both epilogues have released the last accumulator (all their arrivals have landed)
-        mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 5);
+        mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 5, p.wait_ns);
       } else if (lane == 0) {
-        tc_commit_local_pair(drain0);
-        const unsigned long long t0 = now_ns();
-        while (!mbar_try(drain0, 0) && now_ns() - t0 < kTimeoutNs) {
-        }
+        tc_commit_local_pair(drain0);  // arrives once every MMA issued has completed
+        mbar_drain(drain0, 0);
       }
       __syncwarp();
     }
@@ -687,7 +708,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint32_t j = 0;
     for (int tile = cid; tile < num_tiles; tile += ncl, ++j) {
       const int tm = tile % tiles_m, tn = tile / tiles_m;
-      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3)) break;
+      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
       uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -769,6 +790,10 @@ static bool make_sf_map(CUtensorMap* m, const void* base, uint64_t atoms_row, ui
 
 }  // namespace gemm
 
+static std::atomic<unsigned long long> g_wait_ns{gemm::kTimeoutNs};
+
+unsigned long long set_gemm_wait_limit(unsigned long long ns) { return g_wait_ns.exchange(ns); }
+
 static cudaError_t launch_gemm_pair(const GemmLaunch& L, const gemm::Params& p, cudaStream_t s) {
   using namespace gemm;
   const uint32_t atoms = L.nv ? 4 : 2;
@@ -803,6 +828,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   p.C = reinterpret_cast<__nv_bfloat16_raw*>(L.C);
   p.ldc = L.ldc;
   p.status = L.status;
+  p.wait_ns = g_wait_ns.load();
   if (!L.e4m3 && !L.f16 && L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
   // operand rows: K/2 packed bytes (FP4), K bytes (E4M3 expansion) or 2K bytes (fp16)
   const uint64_t row_bytes = L.f16 ? 2 * (uint64_t)L.K : (L.e4m3 ? (uint64_t)L.K : (uint64_t)L.K / 2);

@@ -114,5 +114,7 @@ cudaError_t launch_fwht_amax(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_store(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_fwht_quantize(const FwhtLaunch& L, cudaStream_t s);
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s);
+// Limit (ns) of each pipeline wait in GEMM launches made after the call; returns the previous one.
+unsigned long long set_gemm_wait_limit(unsigned long long ns);
 
 }  // namespace fp4k

@@ -309,8 +309,21 @@ FP4_API fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, long r
 /* Bytes of device workspace `op` needs for the given sizes (rows/cols; M/N for the GEMM). */
 FP4_API size_t fp4_workspace_size(fp4_op op, long rows, long cols);
 
-/* Byte offset, inside fp4_block_gemm's workspace, of its 32-bit device status word. */
+/* Byte offset, inside fp4_block_gemm's workspace, of its 32-bit device status word.  Bit i set
+ * means the pipeline wait at site i gave up: 0 a stage slot to refill, 1 the accumulator to be
+ * released, 2 a stage to land, 3 the accumulator to be ready, 4 the last stage releases, 5 the last
+ * accumulator release, 6-9 the scale-copy stages of the 2-SM kernel.  The kernel then stops every
+ * role, waits (bounded) for the copies and MMAs it issued, frees tensor memory and returns; its
+ * output is incomplete.  A failure of this kind is reported, never trapped ([H]: refuse, never
+ * substitute). */
 FP4_API size_t fp4_gemm_status_word(void);
+
+/* Limit, in nanoseconds, of each pipeline wait inside the GEMM kernels launched after this call
+ * (fp4_block_gemm, fp4_block_gemm_e4m3); returns the previous limit.  The default is 2000000000
+ * (2 s), far above any wait of a working pipeline.  A small limit makes the kernel give up early,
+ * which is how the fault path is exercised without faulting: 0 gives up at the first wait that has
+ * not completed already.  Process-wide; launches already enqueued keep their limit. */
+FP4_API unsigned long long fp4_set_gemm_wait_limit(unsigned long long ns);
 
 /* Static description of a status code. */
 FP4_API const char* fp4_status_str(fp4_status s);

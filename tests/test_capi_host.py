@@ -23,7 +23,8 @@ def L():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^FP4_API\s+(?:const\s+)?[a-z0-9_]+\s*\*?\s*([a-z0-9_]+)\s*\(", src, flags=re.M)
+    # the identifier right before the parameter list: the return type may be several words
+    names = re.findall(r"^FP4_API\s+[^(;]*[\s*]([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
     return sorted(set(n for n in names if n not in ("if", "while")))
 
 
@@ -41,6 +42,9 @@ def test_status_strings_and_workspace(L):
     assert L.fp4_workspace_size(fp4.OP_BLOCK_GEMM, 8192, 8192) >= 4
     assert L.fp4_workspace_size(fp4.OP_MX_QUANTIZE, 8192, 8192) == 0
     assert L.fp4_gemm_status_word() == 0
+    # the GEMM wait limit: default 2 s, returned by the next call that sets it
+    old = L.fp4_set_gemm_wait_limit(12345)
+    assert old == 2000000000 and L.fp4_set_gemm_wait_limit(old) == 12345
 
 
 FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced
