@@ -101,6 +101,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// mbar_wait for code that every lane of a warp runs: the lanes vote, so all of them see the same
+// outcome (one lane giving up while another passes would leave the warp diverged at its next
+// warp-collective instruction: __syncwarp, tcgen05.ld.sync.aligned).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                                          uint32_t site, unsigned long long limit) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, status, site, limit));
+}
+
 // Drain wait (exit paths): until the phase completes or kTimeoutNs passes, whatever the flags say.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const unsigned long long t0 = now_ns();
@@ -324,12 +332,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint32_t g = 0, j = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++j) {
-      if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
+      if (!warp_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       for (int kt = 0; kt < kt_count; ++kt, ++g) {
         const int s = g % STAGES;
         const uint32_t ph = (g / STAGES) & 1;
-        if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
+        if (!warp_wait(full0 + 8 * s, ph, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sA + s * A_BYTES), b0 = smem_u32(sB + s * B_BYTES);
@@ -363,8 +371,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       if (lane == 0) tc_commit(tmem_full);
       __syncwarp();
     }
-    if (!ok && lane == 0) {
-      tc_commit(drain);  // arrives once every MMA and scale copy this thread issued has completed
+    if (lane == 0) {
+      // on every path: the barrier arrives once every MMA and scale copy this thread issued has
+      // completed, so none is still running when tensor memory is freed (the epilogue may have
+      // given up on a tile whose MMAs are in flight)
+      tc_commit(drain);
       mbar_drain(drain, 0);
     }
     __syncwarp();
@@ -376,7 +387,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
       const int tm = tile % tiles_m, tn = tile / tiles_m;
-      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
+      if (!warp_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const int row = tm * BM + q * 32 + lane;
       uint4* crow = reinterpret_cast<uint4*>(p.C + (size_t)row * p.ldc + (size_t)tn * BN);
@@ -625,8 +636,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t g = 0;
       for (; g < total && ok; ++g) {
         const int s = g % S, b = g % NB;
-        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 6, p.wait_ns)) { ok = false; break; }
-        if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 7, p.wait_ns)) { ok = false; break; }
+        if (!warp_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 6, p.wait_ns)) { ok = false; break; }
+        if (!warp_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 7, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t fa = smem_u32(sSFA + s * C::SFA_BYTES), fbs = smem_u32(sSFB + s * C::SFB_BYTES);
@@ -646,11 +657,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // the MMA warp's last releases of the scale buffers have landed
         for (int i = 0; i < NB; ++i, ++g) {
           const int b = g % NB;
-          if (!mbar_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8, p.wait_ns)) break;
+          if (!warp_wait(sf_empty0 + 8 * b, ((g / NB) & 1) ^ 1, abort_flag, p.status, 8, p.wait_ns)) break;
         }
-      } else if (lane == 0) {
+      }
+      if (lane == 0) {
+        // on every path: arrives once this warp's scale copies have completed
         const uint32_t dr = drain0 + 8 * (1 + ci);
-        tc_commit_local_pair(dr);  // arrives once this warp's scale copies have completed
+        tc_commit_local_pair(dr);
         mbar_drain(dr, 0);
       }
       __syncwarp();
@@ -665,10 +678,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int s = g % S, b = g % NB;
         j = g / (uint32_t)kt_count;
         if (kt == 0) {
-          if (!mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
+          if (!warp_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 1, p.wait_ns)) { ok = false; break; }
         }
-        if (!mbar_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
-        if (!mbar_wait(sf_full0 + 8 * b, (g / NB) & 1, abort_flag, p.status, 9, p.wait_ns)) { ok = false; break; }
+        if (!warp_wait(full0 + 8 * s, (g / S) & 1, abort_flag, p.status, 2, p.wait_ns)) { ok = false; break; }
+        if (!warp_wait(sf_full0 + 8 * b, (g / NB) & 1, abort_flag, p.status, 9, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sA + s * C::A_HALF), b0 = smem_u32(sB + s * C::B_HALF);
@@ -690,9 +703,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       j = my_tiles;
       if (ok) {
         // both epilogues have released the last accumulator (all their arrivals have landed)
-        mbar_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 5, p.wait_ns);
-      } else if (lane == 0) {
-        tc_commit_local_pair(drain0);  // arrives once every MMA issued has completed
+        warp_wait(tmem_empty, (j & 1) ^ 1, abort_flag, p.status, 5, p.wait_ns);
+      }
+      if (lane == 0) {
+        // on every path: arrives once every MMA issued has completed (an epilogue that gave up
+        // may have left a tile's MMAs running)
+        tc_commit_local_pair(drain0);
         mbar_drain(drain0, 0);
       }
       __syncwarp();
@@ -708,7 +724,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint32_t j = 0;
     for (int tile = cid; tile < num_tiles; tile += ncl, ++j) {
       const int tm = tile % tiles_m, tn = tile / tiles_m;
-      if (!mbar_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
+      if (!warp_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
       uint32_t r0[32], r1[32], r2[32], r3[32];
