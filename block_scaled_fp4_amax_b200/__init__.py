@@ -164,14 +164,19 @@ def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, se
 
 def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
                            layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
-                           stream=None, if4: bool = False):
+                           stream=None, if4: bool = False, out=None):
     """nvfp4_quantize for callers that cannot hand the library a device workspace: the amax word
     between the two passes lives in a fixed area of the library's own device memory.  Calls that
-    overlap on the GPU share that area and must be serialised.  Returns (q, scales, s_g, counts)."""
+    overlap on the GPU share that area and must be serialised.  `out` = (q, scales, s_g, counts)
+    preallocated by the caller (else allocated here).  Returns (q, scales, s_g, counts)."""
     _need_cuda(x, global_in)
     rows, cols = x.shape
-    q, s, c = _alloc_outputs(rows, cols, 16, x.device)
-    g = torch.empty(1, dtype=torch.float32, device=x.device)
+    if out is None:
+        q, s, c = _alloc_outputs(rows, cols, 16, x.device)
+        g = torch.empty(1, dtype=torch.float32, device=x.device)
+    else:
+        q, s, g, c = out
+        _need_cuda(q, s, g, c)
     _check(lib().nvfp4_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, block, round, _nv_mode(four_six, if4),
                                         seed, layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c),
                                         _stream(stream)))

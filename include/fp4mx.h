@@ -296,7 +296,10 @@ FP4_API fp4_status fp4_block_gemm_e4m3(int M, int N, int K, const unsigned char*
  *   FP4_EUNSUPPORTED; today every shape needs one amax word and fits.
  *   Allocation: none (no cudaMalloc, no cudaFree, no allocating library call).
  *   First call on a device: looks up the array's device address with cudaGetSymbolAddress, with
- *   that device current; make that first call before any stream capture.
+ *   that device current; make that first call before any stream capture.  The address is kept for
+ *   the life of the process: after a cudaDeviceReset (or anything else that tears down and
+ *   re-creates the device's primary context) it is stale, so such a process must not call this
+ *   entry point again.
  *   Sharing: all calls on a device share the one array and it keeps the last call's contents; the
  *   amax word is zeroed on `stream` at the start of each call.  Calls that overlap on the GPU (in
  *   flight at the same time on different streams) race on it: serialise them. */

@@ -25,14 +25,27 @@ def _same(a, b):
         assert torch.equal(u.cpu(), v.cpu())
 
 
-@pytest.mark.parametrize("four_six", [False, True])
-def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda, four_six):
+@pytest.mark.parametrize("mode", ["plain", "four_six", "if4"])
+@pytest.mark.parametrize("on_stream", [False, True])
+def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda, mode, on_stream):
+    kw = {"four_six": mode == "four_six", "if4": mode == "if4"}
     big = synth.nv_outliers(512, 2048, seed=5).to(cuda)        # amax ~ 100s (outlier columns)
     small = (synth.normal_f32(512, 2048, 9) * 0.01).to(torch.bfloat16).to(cuda)
+    stream = torch.cuda.Stream() if on_stream else None
+    fp4.nvfp4_quantize_noalloc(big, stream=stream, **kw)        # warm: the per-device set-up is done
+    torch.cuda.synchronize()
     for x in (big, small, big):
-        want = fp4.nvfp4_quantize(x, four_six=four_six)
-        got = fp4.nvfp4_quantize_noalloc(x, four_six=four_six)
+        want = fp4.nvfp4_quantize(x, **kw)
+        # the outputs are allocated before the free-memory reading: the call itself allocates nothing
+        q = torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=cuda)
+        s = torch.empty(x.numel() // 16, dtype=torch.uint8, device=cuda)
+        g = torch.empty(1, dtype=torch.float32, device=cuda)
+        c = torch.empty(4, dtype=torch.int64, device=cuda)
         torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        got = fp4.nvfp4_quantize_noalloc(x, stream=stream, out=(q, s, g, c), **kw)
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free0
         _same(got, want)
 
 
