@@ -261,6 +261,30 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_amax_kernel(FwhtParams 
   }
 }
 
+// Last-round order -> natural order in the (free) row buffer: the thread writes its 2^NH groups of
+// 2^L consecutive values (consecutive 16-byte chunks across a warp, conflict-free), then syncs.
+template <int LOG_D>
+__device__ __forceinline__ void to_row_buffer(float* srow, int t, const float (&v)[32]) {
+  using G = Geom<LOG_D>;
+  constexpr int L = G::L, NH = G::NH, HI = G::HI;
+#pragma unroll
+  for (int h = 0; h < (1 << NH); ++h) {
+    const int i0 = (t << L) | (h << HI);
+    if constexpr (L >= 2) {
+#pragma unroll
+      for (int q = 0; q < (1 << L) / 4; ++q) {
+        const float* f = v + (h << L) + 4 * q;
+        *reinterpret_cast<float4*>(srow + swz(i0 + 4 * q)) = make_float4(f[0], f[1], f[2], f[3]);
+      }
+    } else if constexpr (L == 1) {
+      *reinterpret_cast<float2*>(srow + swz(i0)) = make_float2(v[h << 1], v[(h << 1) + 1]);
+    } else {
+      srow[swz(i0)] = v[h];
+    }
+  }
+  __syncthreads();
+}
+
 // Last-round order -> 32 consecutive values per thread, through the (free) row buffer: the thread
 // writes its 2^NH groups of 2^L consecutive values and reads back elements [32 t, 32 t + 32), so
 // that every quantisation block lies inside one thread.  Both the writes (consecutive 16-byte
@@ -324,17 +348,23 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA) fwht_store_kernel(FwhtParams
     }
     float v[32];
     rotate_row<T, LOG_D, GATED>(raw, rawu, srow, t, sgn, v);
-    to_consecutive<LOG_D>(srow, t, v);
+    // through the row buffer in natural order, then out in 512-byte warp-contiguous pieces: thread
+    // t stores the 16-byte groups t, t + T, t + 2T, ... of the row
+    to_row_buffer<LOG_D>(srow, t, v);
     if (row < p.rows) {
+      float4* dst = reinterpret_cast<float4*>(p.rotated_out + row * D);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        v[j] = __fmul_rn(v[j], p.c);
-        m = max(m, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+      for (int q = 0; q < 8; ++q) {
+        const int grp = t + q * G::T;
+        float4 f = *reinterpret_cast<const float4*>(srow + swz(4 * grp));
+        f.x = __fmul_rn(f.x, p.c); f.y = __fmul_rn(f.y, p.c);
+        f.z = __fmul_rn(f.z, p.c); f.w = __fmul_rn(f.w, p.c);
+        m = max(m, max(max(__float_as_uint(f.x) & 0x7FFFFFFFu, __float_as_uint(f.y) & 0x7FFFFFFFu),
+                       max(__float_as_uint(f.z) & 0x7FFFFFFFu, __float_as_uint(f.w) & 0x7FFFFFFFu)));
+        dst[grp] = f;
       }
-      float4* dst = reinterpret_cast<float4*>(p.rotated_out + row * D + (t << 5));
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
+    __syncthreads();  // row buffer free for the next row
     if (!GATED) {
 #pragma unroll
       for (int c = 0; c < RowLoad<T>::NV; ++c) raw[c] = nxt[c];

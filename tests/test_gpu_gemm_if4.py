@@ -5,7 +5,7 @@ to fp16 (E2M1 blocks exact, INT4 blocks rounded once to fp16) and runs the kind:
 GEMM; the reference is the oracle's exact fp64 product with the exact factor 6/7.
 
 Bars: the benchmark spec's |C - C64| <= 1e-3 * sum |a b| on quantised data; on single-product operands
-|C - C64| <= (2^-9 + 2^-10 + 2^-18) |C64| (bf16 output rounding plus the fp16 rounding of two INT4
+|C - C64| <= (2^-8 + 2^-10 + 2^-16) |C64| (bf16 output rounding plus the fp16 rounding of two INT4
 elements), and bit-exact bf16(C64) wherever neither block is INT4.
 """
 import numpy as np
@@ -44,7 +44,7 @@ def test_if4_gemm_structured(cuda, M):
     assert np.all(C64 != 0) and np.allclose(np.abs(C64), S, rtol=1e-15, atol=0)
     got = npy(C.float()).astype(np.float64)
     rel = np.abs(got - C64) / np.abs(C64)
-    assert rel.max() <= 2.0 ** -9 + 2.0 ** -10 + 2.0 ** -18, float(rel.max())
+    assert rel.max() <= 2.0 ** -8 + 2.0 ** -10 + 2.0 ** -16, float(rel.max())
     # which block pair each output used: group g = (m + n) mod 32, position 8 ((g - m) mod 32) + (g mod 8)
     m = np.arange(M)[:, None]
     n = np.arange(N)[None, :]
