@@ -631,12 +631,13 @@ __device__ __forceinline__ float int4_encode_resid_n(const float* v, float R7, c
 
 
 // sum over N values of (q_i - y_i)^2: q_i decoded from the packed nibbles (exact in f16), the
-// difference formed in fp32 from the f16 operand directly.  `opaque0` is a kernel-parameter zero
+// difference formed in fp32 from the f16 operand directly, the squares accumulated by packed FMAs
+// into two partial sums (the estimate's bound allows any rounding order).  `opaque0` is a kernel-parameter zero
 // (see sq_errors_n).
 template <int N>
 __device__ __forceinline__ float resid_sq_n(const uint32_t* w, const float* y, uint32_t opaque0) {
   static_assert(N % 2 == 0, "pairs");
-  float acc0 = 0.0f, acc1 = 0.0f;
+  f32x2 acc = 0ull;  // even and odd values in the two halves: one packed FMA per pair
 #pragma unroll
   for (int k = 0; k < (N + 7) / 8; ++k) {
     uint32_t h[4];
@@ -645,16 +646,17 @@ __device__ __forceinline__ float resid_sq_n(const uint32_t* w, const float* y, u
     for (int b = 0; b < 4; ++b) {
       const int j = 8 * k + 2 * b;
       if (j < N) {
-        float rl, rh;
-        asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
-            "sub.rn.f32.f16 %0, l, %3;\n\tsub.rn.f32.f16 %1, u, %4;\n\t}"
-            : "=f"(rl), "=f"(rh) : "r"(h[b]), "f"(y[j]), "f"(y[j + 1]));
-        acc0 = fmaf(rl, rl, acc0);
-        acc1 = fmaf(rh, rh, acc1);
+        f32x2 r;
+        asm("{\n\t.reg .b16 l, u;\n\t.reg .f32 rl, rh;\n\tmov.b32 {l, u}, %1;\n\t"
+            "sub.rn.f32.f16 rl, l, %2;\n\tsub.rn.f32.f16 rh, u, %3;\n\tmov.b64 %0, {rl, rh};\n\t}"
+            : "=l"(r) : "r"(h[b]), "f"(y[j]), "f"(y[j + 1]));
+        asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(r));
       }
     }
   }
-  return acc0 + acc1;
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  return a0 + a1;
 }
 
 // One NVFP4 candidate as nv_candidate_n, plus D = fl(d * s_g) and the residual sum A (both 0

@@ -56,7 +56,17 @@ struct Params {
   long long ldc;
   uint32_t* status;
   unsigned long long wait_ns;  // limit of each pipeline wait (kTimeoutNs unless set otherwise)
+  int group_m;                 // M tiles walked together before the walk moves along N
 };
+
+// Output tile of linear index `tile`: bands of group_m M tiles, M fastest inside a band, the bands
+// one after another, so that the A rows of one band stay in L2 while all of B streams past them.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group_m, int& tm, int& tn) {
+  const int per_group = group_m * tiles_n;
+  const int g = tile / per_group, r = tile - g * per_group;
+  tm = g * group_m + r % group_m;
+  tn = r / group_m;
+}
 
 // ---------------------------------------------------------------------------------------------
 // PTX wrappers
@@ -114,6 +124,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const unsigned long long t0 = now_ns();
   while (!mbar_try(bar, parity) && now_ns() - t0 < kTimeoutNs) {
+  }
+}
+
+// After `issued` fills of a ring of `stages` full barriers (fill g on stage g % stages, phase
+// parity (g / stages) & 1), wait (bounded) until the last fill of every stage has landed.
+__device__ __forceinline__ void drain_fills(uint32_t full0, uint32_t issued, uint32_t stages) {
+  for (uint32_t s = 0; s < stages && s < issued; ++s) {
+    const uint32_t last = s + stages * ((issued - 1 - s) / stages);
+    mbar_drain(full0 + 8 * s, (last / stages) & 1);
   }
 }
 
@@ -283,20 +302,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmA) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
       uint32_t g = 0;  // global k-iteration counter
-      uint32_t last_parity[STAGES];
-      bool pending[STAGES];
-      for (int s = 0; s < STAGES; ++s) { pending[s] = false; last_parity[s] = 0; }
+      uint32_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        int tm, tn;
+        tile_coords(tile, tiles_m, tiles_n, p.group_m, tm, tn);
         for (int kt = 0; kt < kt_count; ++kt, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, p.status, 0, p.wait_ns)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * s;
           mbar_expect_tx(fb, TX_BYTES);
-          pending[s] = true;
-          last_parity[s] = ph;
+          issued = g + 1;
           tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, kt * BKB, tm * BM, fb);
           tma_load_2d(smem_u32(sB + s * B_BYTES), &tmB, kt * BKB, tn * BN, fb);
           if constexpr (!F16) {
@@ -321,12 +338,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           }
         }
       }
-      if (!ok) {
-        // a wait gave up: every fill issued must still land before the CTA's shared memory goes
-        // away (the last fill of each stage completes that stage's full-barrier phase)
-        for (int s = 0; s < STAGES; ++s)
-          if (pending[s]) mbar_drain(full0 + 8 * s, last_parity[s]);
-      }
+      // a wait gave up: every fill issued must still land before the CTA's shared memory goes away
+      if (!ok) drain_fills(full0, issued, STAGES);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (lane 0)
@@ -385,7 +398,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const float alpha = F8 ? 4096.0f : (p.nv ? __fmul_rn(*p.Ag, *p.Bg) : 1.0f);
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
-      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      int tm, tn;
+      tile_coords(tile, tiles_m, tiles_n, p.group_m, tm, tn);
       if (!warp_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const int row = tm * BM + q * 32 + lane;
@@ -575,11 +589,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
       uint32_t g = 0;
       bool ok = true, issued = false;
-      bool pending[S];
-      uint32_t last_parity[S];
-      for (int s = 0; s < S; ++s) { pending[s] = false; last_parity[s] = 0; }
+      uint32_t issued_n = 0;
       for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
-        const int tm = tile % tiles_m, tn = tile / tiles_m;
+        int tm, tn;
+        tile_coords(tile, tiles_m, tiles_n, p.group_m, tm, tn);
         for (int kt = 0; kt < kt_count; ++kt, ++g) {
           const int s = g % S;
           const uint32_t ph = (g / S) & 1;
@@ -591,8 +604,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           tma_pair_3d(smem_u32(sSFA + s * C::SFA_BYTES), &tmSA, 0, kt * ATOMS, tm * 2 + (int)rank, fb);
           tma_pair_3d(smem_u32(sSFB + s * C::SFB_BYTES), &tmSB, 0, kt * ATOMS, tn * 2, fb);
           issued = true;
-          pending[s] = true;
-          last_parity[s] = ph;
+          issued_n = g + 1;
         }
       }
       if (ok) {
@@ -609,8 +621,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (leader) {
           // both CTAs' fills complete on the leader's barriers: wait (bounded) for the last phase
           // of every stage issued, so that they have landed before the final cluster barrier
-          for (int s = 0; s < S; ++s)
-            if (pending[s]) mbar_drain(full0 + 8 * s, last_parity[s]);
+          drain_fills(full0, issued_n, S);
         } else {
           // this CTA cannot observe its fills (they complete on the leader's barrier): give them a
           // fixed, bounded time to land before shared memory is released
@@ -716,7 +727,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t empty_leader = map_rank(tmem_empty, 0);
     uint32_t j = 0;
     for (int tile = cid; tile < num_tiles; tile += ncl, ++j) {
-      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      int tm, tn;
+      tile_coords(tile, tiles_m, tiles_n, p.group_m, tm, tn);
       if (!warp_wait(tmem_full, j & 1, abort_flag, p.status, 3, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ACC_COL + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
@@ -838,6 +850,18 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s) {
   p.ldc = L.ldc;
   p.status = L.status;
   p.wait_ns = g_wait_ns.load();
+  // The largest power-of-two band of M tiles whose A rows fit in 40 MB of L2 (a little under a
+  // third of it, leaving room for the B tiles streaming past).  Tiles are 256 rows in the 2-SM
+  // kernel and 128 in the 1-SM one; A rows hold K/2 bytes (FP4), K (E4M3) or 2K (fp16).
+  {
+    const bool pair = !L.e4m3 && !L.f16 && L.M % 256 == 0 && num_sms() >= 2;
+    const int tile_rows = pair ? 256 : BM;
+    const unsigned long long row_bytes = L.f16 ? 2ull * L.K : (L.e4m3 ? (unsigned long long)L.K : L.K / 2ull);
+    const unsigned long long band = (unsigned long long)tile_rows * row_bytes;
+    const int tiles_m = L.M / tile_rows;
+    p.group_m = 1;
+    while (tiles_m % (2 * p.group_m) == 0 && 2ull * p.group_m * band <= (40ull << 20)) p.group_m *= 2;
+  }
   if (!L.e4m3 && !L.f16 && L.M % 256 == 0 && num_sms() >= 2) return launch_gemm_pair(L, p, s);
   // operand rows: K/2 packed bytes (FP4), K bytes (E4M3 expansion) or 2K bytes (fp16)
   const uint64_t row_bytes = L.f16 ? 2 * (uint64_t)L.K : (L.e4m3 ? (uint64_t)L.K : (uint64_t)L.K / 2);
