@@ -680,7 +680,13 @@ __device__ __forceinline__ uint32_t nv_candidate_resid_n(const float* v, float a
 // pattern and A6/A4 the residual sums of the whole block.  Returns true when the exact sums are
 // needed; otherwise `four` holds the decision.
 __device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, float D6, float D4, float A6,
-                                                   float A4, bool& four) {
+                                                   float A4, uint32_t sc6, uint32_t sc4, bool& four) {
+  // equal scale codes make the two candidates identical (same scale, codes and errors): an exact
+  // tie, which keeps 6 (a clamped scale, for example, under a small caller-supplied global scale)
+  if (sc6 == sc4) {
+    four = false;
+    return false;
+  }
   const float a6 = __fmul_rn(__fmul_rn(D6, D6), A6);
   const float a4 = __fmul_rn(__fmul_rn(D4, D4), A4);
   const float sa = a6 + a4;

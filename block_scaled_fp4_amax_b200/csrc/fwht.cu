@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(Geom<LOG_D>::CTA, Geom<LOG_D>::CTA <= 256 ? 2 
         sc = nv_candidate_resid_n<B, SR>(g, amax, inv6, tab, rnd, p.zero, w, sat, D6, A6);
         const uint32_t sc4 = nv_candidate_resid_n<B, SR>(g, amax, inv4, tab, rnd, p.zero, w4, sat4, D4, A4);
         bool pick4;
-        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
+        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, sc, sc4, pick4);
         if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform branch
           float sq[B];
           sq_errors_n<B>(g, w, sc, s_g, p.zero, sq);

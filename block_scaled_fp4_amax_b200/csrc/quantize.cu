@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
           A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
         }
         bool pick4;
-        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, pick4);
+        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, sc6, sc4, pick4);
         if (__any_sync(0xFFFFFFFFu, undecided))  // warp-uniform call: the exact sums shuffle
           pick4 = four_six_exact<T, G>(xb, c, valid, w[0], w[W - 1], w4[0], w4[W - 1], sc6, sc4, ns.s_g, p.zero) != 0u;
         sc = sc6;
