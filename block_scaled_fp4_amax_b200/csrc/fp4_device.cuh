@@ -589,7 +589,7 @@ template <int N>
 __device__ __forceinline__ float int4_encode_resid_n(const float* v, float R7, const uint32_t* w_e2m1, uint32_t* w7) {
   static_assert(N % 8 == 0, "whole packed words");
   const f32x2 R2 = f2_pack(R7, R7), M2 = f2_pack(0x1p23f, 0x1p23f);
-  float acc0 = 0.0f, acc1 = 0.0f;
+  f32x2 acc2 = 0ull;  // even and odd values in the two halves: one packed FMA per pair
 #pragma unroll
   for (int k = 0; k < N / 8; ++k) {
     uint32_t acc = 0u;
@@ -598,19 +598,21 @@ __device__ __forceinline__ float int4_encode_resid_n(const float* v, float R7, c
       const int j = 8 * k + i;
       float y0, y1;
       f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), R2), y0, y1);
-      const f32x2 t = f2_add(f2_pack(fminf(fabsf(y0), 7.0f), fminf(fabsf(y1), 7.0f)), M2);
-      float t0, t1, m0, m1;
+      const float a0 = fabsf(y0), a1 = fabsf(y1);
+      const f32x2 t = f2_add(f2_pack(fminf(a0, 7.0f), fminf(a1, 7.0f)), M2);
+      float t0, t1;
       f2_unpack(t, t0, t1);
       acc += __float_as_uint(t0) << (4 * i);
       acc += __float_as_uint(t1) << (4 * i + 4);
-      f2_unpack(f2_sub(t, M2), m0, m1);
-      const float r0 = fabsf(y0) - m0, r1 = fabsf(y1) - m1;
-      acc0 = fmaf(r0, r0, acc0);
-      acc1 = fmaf(r1, r1, acc1);
+      // residual |y| - |k|, the clamp's excess above 7 included
+      const f32x2 r = f2_sub(f2_pack(a0, a1), f2_sub(t, M2));
+      asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc2) : "l"(r));
     }
     w7[k] = (acc - int4_pack_fold()) | (w_e2m1[k] & 0x88888888u);
   }
-  return acc0 + acc1;
+  float a0, a1;
+  f2_unpack(acc2, a0, a1);
+  return a0 + a1;
 }
 
 // ---------------------------------------------------------------------------------------------
