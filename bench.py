@@ -209,12 +209,13 @@ class NvStep:
         self.c = [torch.empty(4, dtype=torch.int64, device=dev) for _ in range(2)]
         self.ws = torch.empty(fp4.workspace_size(fp4.OP_NVFP4_QUANTIZE), dtype=torch.uint8, device=dev)
 
-    def call(self, i, four_six, global_in=None):
+    def call(self, i, four_six, global_in=None, counts=True):
         st = self.L.nvfp4_quantize(ctypes.c_void_p(self.x.data_ptr()), fp4.BF16, self.rows, self.cols, 16, fp4.RNE,
                                    int(four_six), 0, fp4.ROWMAJOR,
                                    None if global_in is None else ctypes.c_void_p(global_in.data_ptr()),
                                    ctypes.c_void_p(self.g[i].data_ptr()), ctypes.c_void_p(self.q[i].data_ptr()),
-                                   ctypes.c_void_p(self.s[i].data_ptr()), ctypes.c_void_p(self.c[i].data_ptr()),
+                                   ctypes.c_void_p(self.s[i].data_ptr()),
+                                   ctypes.c_void_p(self.c[i].data_ptr()) if counts else None,
                                    ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         if st != 0:
@@ -253,13 +254,16 @@ def run_ours(args, td, rank, world, local):
     value = job_throughput(world, bytes_step, ms_step)
 
     traffic = profile_traffic("nvfp4_quantize_8192x8192")  # read before any timing
-    # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g
+    # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g (the
+    # one derived in the step).  Without a counter buffer the call enqueues that launch and nothing
+    # else (with one it first zeroes the counters on the stream); the instantiation is the same.
     g = step.g[1].clone()
-    kms = timed(lambda: step.call(1, True, global_in=g), args.steps, args.warmup, flush, td)
+    kms = timed(lambda: step.call(1, True, global_in=g, counts=False), args.steps, args.warmup, flush, td)
     k_ms = max_over_ranks(td, sum(kms) / len(kms))
     k_bytes = NV_BYTES_1PASS * n
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
     roof = {"kernel": "quantize_kernel<bf16, NVFP4, RNE, 4/6> (one launch, 8192x8192)", "bound": "hbm",
+            "timed": "CUDA events around the launch alone (no counter buffer, so no counter memset)",
             "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
             "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
