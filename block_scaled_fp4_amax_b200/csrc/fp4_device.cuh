@@ -47,6 +47,15 @@ __device__ __forceinline__ U8 ld32(const void* p) {
   return r;
 }
 
+// Stores.
+// 32 bytes per lane (sm_100 256-bit store, `p` 32-byte aligned): each lane fills whole 32-byte
+// sectors, where two 16-byte stores from lanes 32 bytes apart would half-fill twice as many.
+__device__ __forceinline__ void st32(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // Element traits for a 32-byte chunk: E values, unpacked to fp32 (exact), and the number of
 // values that are +-0 (from the bit patterns: the magnitude bits of a nonzero value, plus all
 // ones, carry into the top bit of its field).

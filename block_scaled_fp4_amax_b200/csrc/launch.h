@@ -102,7 +102,8 @@ cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* a
                         unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
 // IF4 operand [rows, cols] (packed nibbles, MMA-tiled scales) -> fp16 [rows, cols] without the
-// per-tensor scale: v * d for E2M1 blocks, RNE fp16 of fl(fl(k * d) * fl(6/7)) for INT4 blocks.
+// per-tensor scale: v * d for E2M1 blocks, RNE fp16 of fl(fl(k * d) * fl(6/7)) for INT4 blocks.  `out`
+// must be 32-byte aligned (256-bit stores), else cudaErrorInvalidValue.
 cudaError_t launch_if4_to_f16(const uint8_t* q, const uint8_t* scales, long long rows, long long cols, void* out,
                               cudaStream_t s);
 // E2M1 nibbles -> E4M3 bytes; n_bytes (packed input bytes) a multiple of 16, both 16-byte aligned.

@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long
 // v * 2^(byte-127) (MXFP4, exact); IF4 blocks whose scale byte has bit 7 set hold INT4 nibbles,
 // x_hat = fl(fl(k*d)*s7) with d from the low 7 bits and s7 = fl(s_g * fl(6/7)).  bf16 output is
 // the RNE cast of the fp32 value.
-template <int FMT, bool OUT_BF16>  // FMT: 0 MXFP4, 1 NVFP4, 2 IF4
+template <int FMT, bool OUT_BF16, bool V8>  // FMT: 0 MXFP4, 1 NVFP4, 2 IF4; V8: 256-bit stores
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, const uint8_t* scales,
                                                            const float* global, long long n_groups,
                                                            DivU32 nb, int tiled, void* out) {
@@ -418,13 +418,28 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, con
       uint32_t pw[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) pw[i] = bf16x2_pack(o[2 * i], o[2 * i + 1]);
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + g * 16);
-      dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out) + g * 16;
+      if (V8) {
+        st32(dst, pw);
+      } else {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      }
     } else {
-      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + g * 16);
+      float* dst = reinterpret_cast<float*>(out) + g * 16;
+      if (V8) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(o[8 * h + i]);
+          st32(dst + 8 * h, w8);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(dst)[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      }
     }
   }
 }
@@ -433,6 +448,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* q, con
 // E2M1 -> E4M3 expansion (metrale `hardware::exec`: the exact conversion that lets the FP8 MMA take
 // FP4 operands).  With a nibble in bits 7..4 of a byte b, (b & 0x80) | ((b & 0x70) >> 2) is the E4M3
 // encoding of its value times 2^-6.  Each thread turns 16 packed bytes (32 nibbles) into 32 bytes.
+template <bool V8>
 __global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint4* q, uint4* out, long long n16) {
   const long long stride = (long long)gridDim.x * kThreads;
   for (long long i = (long long)blockIdx.x * kThreads + threadIdx.x; i < n16; i += stride) {
@@ -448,8 +464,12 @@ __global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint4* q, 
       o[2 * k] = __byte_perm(e, d, 0x5140);      // elements 0 1 2 3
       o[2 * k + 1] = __byte_perm(e, d, 0x7362);  // elements 4 5 6 7
     }
-    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    if (V8) {
+      st32(out + 2 * i, o);
+    } else {
+      out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+      out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   }
 }
 
@@ -459,7 +479,8 @@ __global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint4* q, 
 // an INT4 block (scale bit 7) gives the RNE fp16 of fl(fl(k * d) * fl(6/7)): its integer step is six
 // sevenths of the E2M1 unit, so a mixed block pair carries 6/7 and an INT4 pair 36/49 into the
 // product.  The per-tensor scale stays out of the element (fp16 range); the GEMM epilogue applies
-// both.  Scales are read in the MMA tile layout; each thread expands one 16-block (8 packed bytes).
+// both.  Scales are read in the MMA tile layout; each thread expands one 16-block (8 packed bytes)
+// into one 256-bit store.
 __global__ void __launch_bounds__(kThreads) if4_to_f16_kernel(const uint8_t* q, const uint8_t* scales,
                                                               long long n_groups, DivU32 nb, uint4* out) {
   const long long stride = (long long)gridDim.x * kThreads;
@@ -491,13 +512,15 @@ __global__ void __launch_bounds__(kThreads) if4_to_f16_kernel(const uint8_t* q, 
 #pragma unroll
       for (int i = 0; i < 8; ++i) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(v[i]), "r"(dh2));
     }
-    out[2 * g] = make_uint4(h[0], h[1], h[2], h[3]);
-    out[2 * g + 1] = make_uint4(h[4], h[5], h[6], h[7]);
+    st32(out + 2 * g, h);
   }
 }
 
 // ---------------------------------------------------------------------------------------------
 // Launchers
+
+// The 256-bit store variants need 32-byte aligned output (the API promises 16).
+static bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 static int grid_for(long long work_items, int per_cta) {
   const long long want = (work_items + per_cta - 1) / per_cta;
@@ -569,8 +592,11 @@ cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* a
 cudaError_t launch_e2m1_to_e4m3(const uint8_t* q, long long n_bytes, uint8_t* out, cudaStream_t s) {
   const long long n16 = n_bytes / 16;
   if (n16 == 0) return cudaSuccess;
-  e2m1_to_e4m3_kernel<<<grid_for(n16, kThreads), kThreads, 0, s>>>(reinterpret_cast<const uint4*>(q),
-                                                                   reinterpret_cast<uint4*>(out), n16);
+  const int grid = grid_for(n16, kThreads);
+  const uint4* in = reinterpret_cast<const uint4*>(q);
+  uint4* o = reinterpret_cast<uint4*>(out);
+  if (aligned32(out)) e2m1_to_e4m3_kernel<true><<<grid, kThreads, 0, s>>>(in, o, n16);
+  else e2m1_to_e4m3_kernel<false><<<grid, kThreads, 0, s>>>(in, o, n16);
   return cudaGetLastError();
 }
 
@@ -578,8 +604,10 @@ cudaError_t launch_if4_to_f16(const uint8_t* q, const uint8_t* scales, long long
                               cudaStream_t s) {
   const long long groups = rows * cols / 16;
   if (groups == 0) return cudaSuccess;
-  if4_to_f16_kernel<<<grid_for(groups, kThreads), kThreads, 0, s>>>(q, scales, groups, make_divu32((uint32_t)(cols / 16)),
-                                                                    reinterpret_cast<uint4*>(out));
+  const int grid = grid_for(groups, kThreads);
+  const DivU32 nb = make_divu32((uint32_t)(cols / 16));
+  if (!aligned32(out)) return cudaErrorInvalidValue;  // the GEMM workspace places it 256-byte aligned
+  if4_to_f16_kernel<<<grid, kThreads, 0, s>>>(q, scales, groups, nb, reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }
 
@@ -590,13 +618,17 @@ cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s) {
   const int grid = grid_for(groups, kThreads);
   const float* gl = L.format != 0 ? L.global : nullptr;
   auto go = [&](auto kernel) { kernel<<<grid, kThreads, 0, s>>>(L.q, L.scales, gl, groups, nb, L.tiled, L.out); };
-  if (L.format == 2) {
-    if (L.out_bf16) go(dequant_kernel<2, true>); else go(dequant_kernel<2, false>);
-  } else if (L.format == 1) {
-    if (L.out_bf16) go(dequant_kernel<1, true>); else go(dequant_kernel<1, false>);
-  } else {
-    if (L.out_bf16) go(dequant_kernel<0, true>); else go(dequant_kernel<0, false>);
-  }
+  auto pick = [&](auto fmt) {
+    constexpr int F = decltype(fmt)::value;
+    if (aligned32(L.out)) {
+      if (L.out_bf16) go(dequant_kernel<F, true, true>); else go(dequant_kernel<F, false, true>);
+    } else {
+      if (L.out_bf16) go(dequant_kernel<F, true, false>); else go(dequant_kernel<F, false, false>);
+    }
+  };
+  if (L.format == 2) pick(std::integral_constant<int, 2>{});
+  else if (L.format == 1) pick(std::integral_constant<int, 1>{});
+  else pick(std::integral_constant<int, 0>{});
   return cudaGetLastError();
 }
 

@@ -510,3 +510,39 @@ def test_mx_weight_rows_sampled(cuda):
     qo, so, _ = O.mx_quantize(f32(w[torch.from_numpy(rows)]))
     assert np.array_equal(npy(q)[rows], qo)
     assert np.array_equal(npy(s).reshape(8192, -1)[rows], so)
+
+
+def _offset_by_16(shape, dtype, cuda):
+    """A contiguous tensor whose data starts 16 bytes past a 32-byte boundary (the API promises
+    16-byte alignment only; 32-byte aligned outputs take the 256-bit store path)."""
+    n = int(np.prod(shape)) * torch.empty(0, dtype=dtype).element_size()
+    buf = torch.empty(n + 64, dtype=torch.uint8, device=cuda)
+    off = (16 - buf.data_ptr()) % 32
+    t = buf[off:off + n].view(dtype).view(shape)
+    assert t.data_ptr() % 32 == 16
+    return t
+
+
+@pytest.mark.parametrize("fmt", [fp4.MXFP4, fp4.NVFP4, fp4.IF4])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_expansions_on_16_byte_aligned_outputs(cuda, fmt, out_dtype):
+    rows, cols = 136, 1056  # ragged against the launch's chunking: 8976 16-blocks
+    x = synth.nv_outliers(rows, cols, seed=12).to(cuda)
+    if fmt == fp4.MXFP4:
+        q, s = fp4.mx_quantize(x)[:2]
+        g = None
+    else:
+        q, s, g = fp4.nvfp4_quantize(x, if4=(fmt == fp4.IF4))[:3]
+    want = O.dequantize(npy(q), npy(s), fmt, 1.0 if g is None else float(g.item()))
+    want_t = torch.from_numpy(want).to(out_dtype)
+    aligned = fp4.fp4_dequantize(q, s, fmt, g, out_dtype=out_dtype)
+    assert aligned.data_ptr() % 32 == 0
+    shifted = fp4.fp4_dequantize(q, s, fmt, g, out=_offset_by_16((rows, cols), out_dtype, cuda))
+    assert torch.equal(aligned.cpu(), want_t)
+    assert torch.equal(shifted.cpu(), want_t)
+    # the E2M1 -> E4M3 expansion takes the same choice of store
+    if fmt == fp4.MXFP4 and out_dtype == torch.float32:
+        e_al = fp4.fp4_to_e4m3(q)
+        e_sh = fp4.fp4_to_e4m3(q, out=_offset_by_16((rows, cols), torch.uint8, cuda))
+        assert np.array_equal(npy(e_al), O.e2m1_to_e4m3(npy(q)))
+        assert np.array_equal(npy(e_sh), O.e2m1_to_e4m3(npy(q)))
