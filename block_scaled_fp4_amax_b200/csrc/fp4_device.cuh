@@ -87,12 +87,13 @@ template <> struct Vec32<float> {
 };
 template <> struct Vec32<__nv_bfloat16> {
   static constexpr int E = 16;
+  // bf16 -> fp32 as the exact mixed-precision sum x + (-0): it runs on the FMA pipe, where two
+  // shifts/masks per pair would load the integer pipe, the busiest one in the quantisers.
   __device__ __forceinline__ static void unpack(const U8& r, float* v) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = __uint_as_float(r.w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(r.w[i] & 0xFFFF0000u);
-    }
+    for (int i = 0; i < 8; ++i)
+      asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tadd.rn.f32.bf16 %0, l, 0f80000000;\n\t"
+          "add.rn.f32.bf16 %1, u, 0f80000000;\n\t}" : "=f"(v[2 * i]), "=f"(v[2 * i + 1]) : "r"(r.w[i]));
   }
   __device__ __forceinline__ static int zeros(const U8& r) {
     int nz = 0;
@@ -100,15 +101,17 @@ template <> struct Vec32<__nv_bfloat16> {
     for (int i = 0; i < 8; ++i) nz += __popc(((r.w[i] & 0x7FFF7FFFu) + 0x7FFF7FFFu) & 0x80008000u);
     return 16 - nz;
   }
-  // Largest magnitude as an fp32 bit pattern (16-bit lane-wise max of the bf16 magnitudes);
-  // `any_zero` is set if some value is +-0 (lane-wise minimum magnitude 0).
+  // Largest magnitude as an fp32 bit pattern (lane-wise bf16x2 max of the sign-cleared values, on
+  // the half-precision pipe; a NaN makes the result the canonical NaN 0x7FFF, above +Inf, so the
+  // block still reads as non-finite); `any_zero` is set if some value is +-0 (lane-wise minimum
+  // magnitude 0; the bf16 minimum ignores NaN operands).
   __device__ __forceinline__ static uint32_t max_mag(const U8& r, bool& any_zero) {
     uint32_t m = 0u, mn = 0x7FFF7FFFu;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t a = r.w[i] & 0x7FFF7FFFu;
-      asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(a));
-      asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(a));
+      asm("max.NaN.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(a));
+      asm("min.bf16x2 %0, %0, %1;" : "+r"(mn) : "r"(a));
     }
     any_zero = ((mn & 0xFFFFu) == 0u) | ((mn >> 16) == 0u);
     return max(m & 0xFFFFu, m >> 16) << 16;
