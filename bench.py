@@ -370,7 +370,7 @@ def secondary(args, dev, flush, td, pk):
                 "ms": round(t, 5), "GB/s": round(b / (t * 1e-3) / 1e9, 1)})
     # config 3: fused FWHT + NVFP4 + SR, 16384 x 8192 bf16
     x3 = synth.fwht_laplace().to(dev)
-    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    ws = torch.empty(fp4.workspace_size(fp4.OP_FWHT_QUANTIZE), dtype=torch.uint8, device=dev)
     # the workspace that lets the two-pass call keep its fp32 rotation (rotate once)
     wsr = torch.empty(fp4.workspace_size(fp4.OP_FWHT_QUANTIZE_STORED, 16384, 8192), dtype=torch.uint8, device=dev)
 
@@ -429,20 +429,21 @@ def secondary(args, dev, flush, td, pk):
     # IF4 (E2M1 or INT4 per block) on the headline tensor: two passes, and the quantise pass alone
     xi = synth.nv_outliers().to(dev)
     gi = torch.empty(1, dtype=torch.float32, device=dev)
-    fp4.nvfp4_quantize(xi, if4=True, workspace=ws)
+    wsq = torch.empty(fp4.workspace_size(fp4.OP_NVFP4_QUANTIZE), dtype=torch.uint8, device=dev)
+    fp4.nvfp4_quantize(xi, if4=True, workspace=wsq)
 
     def cif4():
-        fp4.nvfp4_quantize(xi, if4=True, workspace=ws)
+        fp4.nvfp4_quantize(xi, if4=True, workspace=wsq)
 
     ms = timed(cif4, K, W, flush, td)
     t = statistics.median(ms)
-    gi.copy_(fp4.nvfp4_quantize(xi, workspace=ws)[2])
+    gi.copy_(fp4.nvfp4_quantize(xi, workspace=wsq)[2])
     ms1 = timed(lambda: fp4.nvfp4_quantize(xi, if4=True, global_in=gi), K, W, flush, td)
     t1 = statistics.median(ms1)
     # the same quantise pass on N(0,1) without outliers (the rotated-data case IF4 is aimed at)
     xn = synth.normal_bf16(8192, 8192, 8)
     xn = xn.to(dev)
-    gn = fp4.nvfp4_quantize(xn, workspace=ws)[2].clone()
+    gn = fp4.nvfp4_quantize(xn, workspace=wsq)[2].clone()
     msn = timed(lambda: fp4.nvfp4_quantize(xn, if4=True, global_in=gn), K, W, flush, td)
     tn = statistics.median(msn)
     out.append({"workload": "IF4 quantisation (E2M1 or INT4 per 16-block) 8192x8192 bf16 outliers, two passes",
@@ -455,7 +456,7 @@ def secondary(args, dev, flush, td, pk):
                     round(NV_BYTES_1PASS * xn.numel() / (tn * 1e-3) / 1e9 / pk["hbm_gbs"], 4)})
     # dequantisation of the headline tensor's NVFP4 encoding (4/6 codes), to bf16 and to fp32
     xd = synth.nv_outliers().to(dev)
-    qd, sd, gd, _ = fp4.nvfp4_quantize(xd, four_six=True, workspace=ws)
+    qd, sd, gd, _ = fp4.nvfp4_quantize(xd, four_six=True, workspace=wsq)
     del xd
     od = {torch.bfloat16: torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev),
           torch.float32: torch.empty((8192, 8192), dtype=torch.float32, device=dev)}

@@ -32,7 +32,9 @@ fp4_status cuda_fail(cudaError_t e, const char* what) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr long long kMaxElems = 1LL << 40;
-constexpr size_t kAmaxWorkspace = 256;  // one 32-bit amax word, padded
+constexpr size_t kAmaxWorkspace = 256;  // the rotations' 32-bit amax word, padded
+// nvfp4_quantize's amax pass: one 32-bit partial maximum per CTA of that pass
+constexpr size_t kAmaxSlotsWorkspace = fp4k::kAmaxSlots * sizeof(uint32_t);
 constexpr size_t kGemmWorkspace = 256;  // one 32-bit status word, padded
 
 fp4_status check_quant_common(const void* x, fp4_dtype dtype, long rows, long cols, int block,
@@ -97,7 +99,7 @@ size_t fp4_workspace_size(fp4_op op, long rows, long cols) {
   (void)rows;
   (void)cols;
   switch (op) {
-    case FP4_OP_NVFP4_QUANTIZE:
+    case FP4_OP_NVFP4_QUANTIZE: return kAmaxSlotsWorkspace;
     case FP4_OP_FWHT_QUANTIZE: return kAmaxWorkspace;
     case FP4_OP_FWHT_QUANTIZE_STORED:
       // the amax word, padding to a 256-byte boundary, and the fp32 rotation
@@ -142,17 +144,19 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   if (mode != FP4_NV_PLAIN && mode != FP4_NV_FOUR_SIX && mode != FP4_NV_IF4)
     return fail(FP4_EINVAL, "NVFP4 block mode %d unknown", mode);
   if (mode == FP4_NV_IF4 && round != FP4_RNE) return fail(FP4_EUNSUPPORTED, "IF4 is defined with round to nearest only");
-  if (!global_in && (!workspace || ws_bytes < kAmaxWorkspace || !aligned(workspace, 16)))
-    return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL", kAmaxWorkspace);
+  if (!global_in && (!workspace || ws_bytes < kAmaxSlotsWorkspace || !aligned(workspace, 16)))
+    return fail(FP4_EINVAL, "a 16-byte aligned workspace of %zu bytes is required when global_in is NULL",
+                kAmaxSlotsWorkspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (counts && !aligned(counts, 8)) return fail(FP4_EINVAL, "counts must be 8-byte aligned");
   // with an amax pass (and a non-empty tensor) that pass zeroes the counters; otherwise a memset does
   const bool amax_pass = !global_in && (long long)rows * cols > 0;
   if (!amax_pass && (st = zero_counts(counts, s)) != FP4_OK) return st;
+  // the amax pass writes one partial maximum per CTA into the workspace (no zeroing needed); the
+  // quantise pass reduces them
   uint32_t* amax = static_cast<uint32_t*>(workspace);
   cudaError_t e;
   if (amax_pass) {
-    if ((e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s)) != cudaSuccess) return cuda_fail(e, "zeroing amax");
     if ((e = fp4k::launch_amax(x, dtype == FP4_BF16, (long long)rows * cols, amax,
                                reinterpret_cast<unsigned long long*>(counts), s)) != cudaSuccess)
       return cuda_fail(e, "nvfp4 amax launch");
@@ -162,6 +166,7 @@ fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, 
   L.policy = 0; L.sr = round == FP4_STOCHASTIC; L.mode = mode; L.seed = seed;
   L.tiled = layout == FP4_SCALES_MMA_TILED; L.reverse = global_in ? 0 : 1;
   L.global_in = global_in; L.amax_bits = amax; L.global_out = global_out;
+  L.amax_slots = amax_pass ? fp4k::amax_grid((long long)rows * cols, dtype == FP4_BF16) : 0;
   L.q = q; L.scales = scales; L.counts = reinterpret_cast<unsigned long long*>(counts);
   L.pdl = amax_pass;
   e = fp4k::launch_quantize(L, s);
@@ -228,7 +233,7 @@ static fp4_status fwht_quantize_impl(const void* x, const void* u, fp4_dtype dty
       Q.x = rot; Q.bf16 = false; Q.rows = rows; Q.cols = d; Q.nv = true;
       Q.policy = 0; Q.sr = L.sr; Q.mode = L.mode; Q.seed = seed;
       Q.tiled = L.tiled; Q.reverse = 1;  // start on the rows the first pass left in L2
-      Q.global_in = nullptr; Q.amax_bits = L.amax_bits; Q.global_out = L.global_out;
+      Q.global_in = nullptr; Q.amax_bits = L.amax_bits; Q.amax_slots = 1; Q.global_out = L.global_out;
       Q.q = q; Q.scales = scales; Q.counts = L.counts; Q.pdl = true;
       e = fp4k::launch_quantize(Q, s);
       return e == cudaSuccess ? FP4_OK : cuda_fail(e, "fwht_quantize stored-rotation launch");

@@ -1,7 +1,7 @@
 // capi_noalloc.cu — nvfp4_quantize for callers that cannot allocate device memory.
 //
-// nvfp4_quantize needs a small device workspace (the word that collects the tensor amax between
-// its two passes).  Some callers cannot provide one: a plugin running inside another runtime that
+// nvfp4_quantize needs a small device workspace (the per-CTA partial maxima that carry the tensor
+// amax between its two passes).  Some callers cannot provide one: a plugin running inside another runtime that
 // hands it only its input and output buffers, or a latency-critical loop in which a cudaMalloc
 // (which may synchronise the device) is not acceptable.  This entry point takes the workspace from
 // a fixed array in this library's device memory instead, and otherwise runs exactly the
@@ -18,7 +18,8 @@
 
 namespace {
 
-constexpr size_t kNoallocScratchBytes = 256;  // holds the amax word (fp4_workspace_size's need)
+// holds the amax pass's partial maxima (fp4_workspace_size's need for every shape)
+constexpr size_t kNoallocScratchBytes = fp4k::kAmaxSlots * sizeof(uint32_t);
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
@@ -65,8 +66,8 @@ extern "C" fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, lon
     }
     scratch = g_scratch_ptr[dev];
   }
-  // nvfp4_quantize zeroes the amax word on `stream` before its first pass, so the contents left by
-  // the previous call do not leak into this one.
+  // the amax pass overwrites every slot the quantise pass reads, so the contents left by the
+  // previous call do not leak into this one.
   return nvfp4_quantize(x, dtype, rows, cols, block, round, mode, seed, layout, global_in, global_out, q, scales,
                         counts, scratch, kNoallocScratchBytes, stream);
 }

@@ -41,8 +41,9 @@ struct QuantLaunch {
   unsigned long long seed;
   int tiled;      // scale layout
   int reverse;    // walk tiles last-to-first
-  const float* global_in;    // NVFP4: caller-fixed s_g, or NULL to derive from *amax_bits
-  const uint32_t* amax_bits;
+  const float* global_in;    // NVFP4: caller-fixed s_g, or NULL to derive from the amax words
+  const uint32_t* amax_bits;  // amax_slots words whose maximum is the tensor amax (magnitude bits)
+  int amax_slots;             // 1 (a single word reduced by atomicMax) or the amax pass's grid
   float* global_out;
   uint8_t* q;
   uint8_t* scales;
@@ -96,9 +97,15 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s);
-// Tensor amax into *amax_bits (zeroed by the caller); also zeroes `counts` (4 words) if non-null.
-// Lets the following quantise pass, launched with QuantLaunch::pdl, be scheduled as it retires.
-cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
+// Upper bound of the tensor-amax pass's grid: the number of 32-bit slots its output needs.
+constexpr int kAmaxSlots = 2048;
+// CTAs of the tensor-amax pass over n_elems values (at most kAmaxSlots; 0 for an empty tensor).
+int amax_grid(long long n_elems, bool bf16);
+// Tensor amax as per-CTA partial maxima: CTA i writes the magnitude bits of its maximum to
+// slots[i], i < amax_grid(n_elems, bf16), so nothing needs zeroing first.  Also zeroes `counts`
+// (4 words) if non-null.  Lets the following quantise pass, launched with QuantLaunch::pdl and
+// amax_slots = amax_grid(...), be scheduled as it retires.
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* slots,
                         unsigned long long* counts, cudaStream_t s);
 cudaError_t launch_dequant(const DequantLaunch& L, cudaStream_t s);
 // IF4 operand [rows, cols] (packed nibbles, MMA-tiled scales) -> fp16 [rows, cols] without the

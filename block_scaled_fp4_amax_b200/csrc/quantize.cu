@@ -47,13 +47,34 @@ struct NvScale {
   float s_g, inv6, inv4;
 };
 
-__device__ __forceinline__ NvScale nv_scales(const float* global_in, const uint32_t* amax_bits,
+// The tensor amax from `n` <= kAmaxSlots words of magnitude bits (the amax pass's per-CTA maxima,
+// or one word): an integer maximum, which orders non-negative floats (NaN patterns above +Inf).
+// Every thread of the CTA (kThreads of them) calls it and gets the result.  The loads have a fixed
+// trip count, so they are all in flight together: one L2 round trip.
+__device__ __forceinline__ uint32_t cta_amax_bits(const uint32_t* slots, int n) {
+  __shared__ uint32_t red;
+  if (threadIdx.x == 0) red = 0u;
+  __syncthreads();
+  uint32_t m = 0u;
+#pragma unroll
+  for (int k = 0; k < kAmaxSlots / kThreads; ++k) {
+    const int i = (int)threadIdx.x + k * kThreads;
+    if (i < n) m = max(m, __ldcg(slots + i));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(&red, m);
+  __syncthreads();
+  return red;
+}
+
+__device__ __forceinline__ NvScale nv_scales(const float* global_in, const uint32_t* amax_bits, int amax_slots,
                                              float six_m) {
   NvScale s;
   if (global_in) {
     s.s_g = *global_in;
   } else {
-    const float amax = __uint_as_float(*amax_bits);
+    const float amax = __uint_as_float(cta_amax_bits(amax_bits, amax_slots));
     s.s_g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, six_m);
   }
   s.inv6 = __frcp_rn(__fmul_rn(6.0f, s.s_g));
@@ -72,6 +93,7 @@ struct QuantParams {
   uint32_t zero;       // 0, read at run time: makes in-register nibble decodes opaque
   const float* global_in;
   const uint32_t* amax_bits;
+  int amax_slots;
   float* global_out;
   float six_m;
   uint8_t* q;
@@ -155,7 +177,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
   __shared__ float2 tab7[IF4 ? kScaleTab : 1];
   float s7 = 0.0f;
   if (NV) {
-    ns = nv_scales(p.global_in, p.amax_bits, p.six_m);
+    ns = nv_scales(p.global_in, p.amax_bits, p.amax_slots, p.six_m);
     if (p.global_out && blockIdx.x == 0 && threadIdx.x == 0) *p.global_out = ns.s_g;
     fill_scale_tab(tab, ns.s_g);
     if (IF4) {
@@ -323,11 +345,13 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
 
 // ---------------------------------------------------------------------------------------------
 // Tensor amax (NVFP4 global scale, first pass): max |x| over the whole tensor as an integer max
-// of the magnitude bits (monotone for non-negative floats), one atomicMax per CTA.  Loads keep
-// their L2 lines so the second pass, walking the tiles in reverse, starts on resident data.
+// of the magnitude bits (monotone for non-negative floats).  Each CTA stores its maximum in its own
+// slot, so the word needs no zeroing before the pass (a memset on the stream costs about as much
+// as 7% of this kernel); the quantise pass reduces the slots.  Loads keep their L2 lines so the
+// second pass, walking the tiles in reverse, starts on resident data.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long n_chunks,
-                                                        uint32_t* amax_bits, unsigned long long* counts) {
+                                                        uint32_t* slots, unsigned long long* counts) {
   grid_dep_trigger();  // the quantise pass may take SMs as this grid's CTAs retire
   // the counters the following quantise pass accumulates into start at zero (stream order)
   if (counts && blockIdx.x == 0 && threadIdx.x < 4) counts[threadIdx.x] = 0ull;
@@ -364,7 +388,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long
     uint32_t b = 0u;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) b = max(b, wm[w]);
-    atomicMax(amax_bits, b);
+    slots[blockIdx.x] = b;
   }
 }
 
@@ -569,6 +593,7 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
   p.zero = 0u;
   p.global_in = L.global_in;
   p.amax_bits = L.amax_bits;
+  p.amax_slots = L.amax_slots;
   p.global_out = L.global_out;
   p.six_m = L.mode == kFourSix ? 1536.0f : 2688.0f;
   p.q = L.q;
@@ -579,13 +604,20 @@ cudaError_t launch_quantize(const QuantLaunch& L, cudaStream_t s) {
                 : dispatch_q<float>(p, L.nv, L.sr, L.mode, L.pdl, s);
 }
 
-cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* amax_bits,
+int amax_grid(long long n_elems, bool bf16) {
+  const long long chunks = n_elems / (bf16 ? 16 : 8);
+  if (chunks == 0) return 0;
+  const int grid = grid_for(chunks / 4 + 1, kThreads);
+  return grid < kAmaxSlots ? grid : kAmaxSlots;
+}
+
+cudaError_t launch_amax(const void* x, bool bf16, long long n_elems, uint32_t* slots,
                         unsigned long long* counts, cudaStream_t s) {
   const long long chunks = n_elems / (bf16 ? 16 : 8);
-  if (chunks == 0) return cudaSuccess;
-  const int grid = grid_for(chunks / 4 + 1, kThreads);
-  if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
-  else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, amax_bits, counts);
+  const int grid = amax_grid(n_elems, bf16);
+  if (grid == 0) return cudaSuccess;
+  if (bf16) amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(x, chunks, slots, counts);
+  else amax_kernel<float><<<grid, kThreads, 0, s>>>(x, chunks, slots, counts);
   return cudaGetLastError();
 }
 

@@ -106,7 +106,9 @@ typedef struct fp4_counts {
   unsigned long long blocks_four;
 } fp4_counts;
 
-/* Operation ids for fp4_workspace_size.  FP4_OP_FWHT_QUANTIZE is the minimum for fwht_quantize and
+/* Operation ids for fp4_workspace_size.  FP4_OP_NVFP4_QUANTIZE is nvfp4_quantize's need (8 KiB: one
+ * 32-bit partial maximum per CTA of the amax pass, which the quantise pass reduces, so nothing is
+ * zeroed between calls).  FP4_OP_FWHT_QUANTIZE is the minimum for fwht_quantize and
  * swiglu_fwht_quantize (the amax word); FP4_OP_FWHT_QUANTIZE_STORED the size that also holds the
  * fp32 rotation of a [rows, cols] tensor, which lets the two-pass NVFP4 call rotate once. */
 typedef enum fp4_op { FP4_OP_MX_QUANTIZE = 0, FP4_OP_NVFP4_QUANTIZE = 1, FP4_OP_FWHT_QUANTIZE = 2,
@@ -151,7 +153,8 @@ FP4_API fp4_status mx_quantize(const void* x, fp4_dtype dtype, long rows, long c
  *   global_out : device float or NULL; receives the s_g used.
  *   q, scales, counts : as in mx_quantize (E4M3 scale bytes).
  *   workspace  : device, >= fp4_workspace_size(FP4_OP_NVFP4_QUANTIZE, rows, cols) bytes, 16-byte
- *                aligned; required when global_in == NULL.  Clobbered.
+ *                aligned; required when global_in == NULL.  Clobbered; needs no initialisation (the
+ *                amax pass writes every word the quantise pass reads).
  * Preconditions: block == 16, cols % 16 == 0. */
 FP4_API fp4_status nvfp4_quantize(const void* x, fp4_dtype dtype, long rows, long cols, int block,
                           fp4_round round, int mode, unsigned long long seed,
@@ -291,18 +294,18 @@ FP4_API fp4_status fp4_block_gemm_e4m3(int M, int N, int K, const unsigned char*
  * can synchronise the device).  The source pages have no counterpart; this is a library
  * convenience.
  *   Arguments, results and errors are those of nvfp4_quantize, minus `workspace`/`ws_bytes`.
- *   Scratch: a fixed 256-byte array in this library's device memory (per GPU, kept until the
- *   process exits).  A shape whose workspace need (fp4_workspace_size) exceeds it is rejected with
- *   FP4_EUNSUPPORTED; today every shape needs one amax word and fits.
+ *   Scratch: a fixed 8 KiB array in this library's device memory (per GPU, kept until the process
+ *   exits).  A shape whose workspace need (fp4_workspace_size) exceeds it is rejected with
+ *   FP4_EUNSUPPORTED; today every shape needs the same 8 KiB and fits.
  *   Allocation: none (no cudaMalloc, no cudaFree, no allocating library call).
  *   First call on a device: looks up the array's device address with cudaGetSymbolAddress, with
  *   that device current; make that first call before any stream capture.  The address is kept for
  *   the life of the process: after a cudaDeviceReset (or anything else that tears down and
  *   re-creates the device's primary context) it is stale, so such a process must not call this
  *   entry point again.
- *   Sharing: all calls on a device share the one array and it keeps the last call's contents; the
- *   amax word is zeroed on `stream` at the start of each call.  Calls that overlap on the GPU (in
- *   flight at the same time on different streams) race on it: serialise them. */
+ *   Sharing: all calls on a device share the one array and it keeps the last call's contents; each
+ *   call's amax pass overwrites every word its quantise pass reads.  Calls that overlap on the GPU
+ *   (in flight at the same time on different streams) race on it: serialise them. */
 FP4_API fp4_status nvfp4_quantize_noalloc(const void* x, fp4_dtype dtype, long rows, long cols, int block,
                                           fp4_round round, int mode, unsigned long long seed,
                                           fp4_scale_layout layout, const float* global_in, float* global_out,
