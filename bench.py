@@ -58,16 +58,21 @@ def peaks():
     return d
 
 
-def profile_traffic(name):
-    """Per-launch DRAM bytes (read + write) recorded in profiles/<name>.md, if any."""
+def profile_value(name, key):
+    """A `key: value` figure recorded in profiles/<name>.md (from that kernel's ncu capture), if any."""
     path = os.path.join(PROFILE_DIR, name + ".md")
     if not os.path.exists(path):
         return None
     for ln in open(path):
-        if ln.startswith("traffic_bytes_per_launch:"):
+        if ln.startswith(key + ":"):
             v = ln.split(":", 1)[1].strip()
             return None if v in ("", "null") else float(v)
     return None
+
+
+def profile_traffic(name):
+    """Per-launch DRAM bytes (read + write) recorded in profiles/<name>.md, if any."""
+    return profile_value(name, "traffic_bytes_per_launch")
 
 
 class Clocks:
@@ -254,6 +259,7 @@ def run_ours(args, td, rank, world, local):
     value = job_throughput(world, bytes_step, ms_step)
 
     traffic = profile_traffic("nvfp4_quantize_8192x8192")  # read before any timing
+    ipe = profile_value("nvfp4_quantize_8192x8192", "thread_instructions_per_element")
     # dominant kernel: the quantise launch (4/6 variant), timed alone with a caller-fixed s_g (the
     # one derived in the step).  Without a counter buffer the call enqueues that launch and nothing
     # else (with one it first zeroes the counters on the stream); the instantiation is the same.
@@ -270,6 +276,18 @@ def run_ours(args, td, rank, world, local):
             "traffic": traffic, "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of "
                                                   "this kernel on this workload, profiles/nvfp4_quantize_8192x8192.md",
             "algorithmic_bytes_per_launch": k_bytes}
+    if ipe:
+        # the kernel is issue-bound: its ceiling at one warp instruction per scheduler per clock
+        # (SMs x 4 schedulers x 32 lanes x the SM clock sampled under load), at the thread
+        # instructions per element of its ncu capture
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        tips = torch.cuda.get_device_properties(dev).multi_processor_count * 4 * 32 * mhz * 1e6
+        ceil_gbs = tips / ipe * NV_BYTES_1PASS / 1e9
+        roof["issue_ceiling"] = {"thread_instructions_per_element": ipe,
+                                 "source": "ncu smsp__thread_inst_executed.sum of one launch / elements, "
+                                           "profiles/nvfp4_quantize_8192x8192.md",
+                                 "thread_instructions_per_s": round(tips / 1e12, 2), "unit": "T/s",
+                                 "ceiling_GB/s": round(ceil_gbs, 1), "frac_of_ceiling": round(achieved / ceil_gbs, 4)}
 
     # end to end through the public binding: pinned host input -> device -> both calls -> host
     host_in = x_cpu.pin_memory()
