@@ -546,3 +546,24 @@ def test_expansions_on_16_byte_aligned_outputs(cuda, fmt, out_dtype):
         e_sh = fp4.fp4_to_e4m3(q, out=_offset_by_16((rows, cols), torch.uint8, cuda))
         assert np.array_equal(npy(e_al), O.e2m1_to_e4m3(npy(q)))
         assert np.array_equal(npy(e_sh), O.e2m1_to_e4m3(npy(q)))
+
+
+@pytest.mark.parametrize("mode", ["plain", "four_six", "if4"])
+def test_two_pass_workspace_needs_no_initialisation(cuda, mode):
+    """The amax pass writes one partial maximum per CTA into the workspace and the quantise pass
+    reduces exactly those words, so nothing is zeroed between calls.  A workspace filled with 0xFF
+    bytes (NaN patterns, above every finite magnitude) must not leak into the result: the global
+    scale, nibbles, scales and counters match the oracle.  Sizes: a one-CTA amax grid, and
+    8192 x 2432 (1.2 M 32-byte chunks), whose amax grid is capped at 8 CTAs per SM."""
+    kw = dict(four_six=mode == "four_six", if4=mode == "if4")
+    for rows, cols in ((37, 1024), (8192, 2432)):
+        x_cpu = synth.nv_outliers(rows, cols, seed=21)
+        ws = torch.full((fp4.workspace_size(fp4.OP_NVFP4_QUANTIZE),), 0xFF, dtype=torch.uint8, device=cuda)
+        q, s, g, c = fp4.nvfp4_quantize(x_cpu.to(cuda), workspace=ws, **kw)
+        x = f32(x_cpu)
+        qo, so, go, co, spec = O.nvfp4_quantize(x, spec=True, **kw)
+        assert spec.all()
+        assert np.float32(npy(g)[0]) == np.float32(go)
+        assert np.array_equal(npy(q), qo)
+        assert np.array_equal(npy(s), so.ravel())
+        compare_counts(c, co, x, spec, 16)
