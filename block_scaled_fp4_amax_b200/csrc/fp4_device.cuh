@@ -716,6 +716,74 @@ __device__ __forceinline__ bool four_six_undecided(uint32_t am, float amax, floa
   return (am != 0u) & !(in_range & (fabsf(diff) > m));
 }
 
+// ---------------------------------------------------------------------------------------------
+// Exact decisions for one common shape of undecided block.
+//
+// On tensors with outlier channels the blocks holding an outlier often fall inside the estimate's
+// margin: their small values encode to zero under both candidates, so the two sums differ only in
+// the outlier's term and the estimates differ by rounding noise.  Such a block has, in each
+// candidate, exactly one nonzero code, at the same position.  That element is the block maximum
+// (codes are monotone in |x|), so |x| = amax there, and every other element has x_hat = +-0 in both
+// candidates and the same error term fl(x_i^2).  The fp32 sequential error sums then differ in one
+// term t = fl(fl(amax - xh)^2), xh = fl(fl(|q| d) s), and such a sum is monotone in each term: if the
+// alternative's term is not below the incumbent's, its sum is not below either, and the incumbent
+// stays (ties included).  Only the other outcome still needs the exact sums.  Valid for positive
+// finite scales (s > 0, d > 0), a finite amax and a lane holding the whole block (two words).
+
+// Bit 3 of every nibble whose 3-bit magnitude is nonzero.
+__device__ __forceinline__ uint32_t nonzero_nibbles(uint32_t w) {
+  return ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+}
+
+// If the blocks wa and wb (two words each) both hold exactly one nonzero code, at the same position,
+// their 3-bit magnitudes through ca, cb; false otherwise.
+__device__ __forceinline__ bool single_nonzero_code(const uint32_t* wa, const uint32_t* wb, uint32_t& ca,
+                                                    uint32_t& cb) {
+  const uint32_t m0 = nonzero_nibbles(wa[0]), m1 = nonzero_nibbles(wa[1]);
+  if (m0 != nonzero_nibbles(wb[0]) || m1 != nonzero_nibbles(wb[1]) || __popc(m0) + __popc(m1) != 1) return false;
+  // the words' other nibbles have magnitude 0, so or-folding leaves the one nonzero magnitude
+  uint32_t a = (wa[0] | wa[1]) & 0x77777777u, b = (wb[0] | wb[1]) & 0x77777777u;
+  a |= a >> 16; b |= b >> 16;
+  a |= a >> 8; b |= b >> 8;
+  a |= a >> 4; b |= b >> 4;
+  ca = a & 7u;
+  cb = b & 7u;
+  return true;
+}
+
+// E2M1 magnitude of a 3-bit code: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_magnitude(uint32_t c) {
+  return c < 4u ? 0.5f * (float)c : (c == 7u ? 6.0f : (float)(c - 2u));
+}
+
+// fl(fl(amax - fl(fl(q d) s))^2): the squared error of the block maximum, as the exact sums form it.
+__device__ __forceinline__ float max_term(float amax, float q, float d, float s) {
+  const float e = __fsub_rn(amax, __fmul_rn(__fmul_rn(q, d), s));
+  return __fmul_rn(e, e);
+}
+
+// Four-over-six: true when the single-term shape settles the choice, which is then 6 (kept).
+__device__ __forceinline__ bool four_six_single_term(const uint32_t* w6, const uint32_t* w4, float amax,
+                                                     uint32_t sc6, uint32_t sc4, float s_g) {
+  uint32_t c6, c4;
+  if (!single_nonzero_code(w6, w4, c6, c4)) return false;
+  const float t6 = max_term(amax, e2m1_magnitude(c6), e4m3_value(sc6), s_g);
+  const float t4 = max_term(amax, e2m1_magnitude(c4), e4m3_value(sc4), s_g);
+  return t4 >= t6;
+}
+
+// IF4: the same for the E2M1 candidate (words w, scale code sc) against the INT4 one (words w7, the
+// same scale, integer magnitudes, factor s7 = fl(s_g * fl(6/7))): true when E2M1 is kept.
+__device__ __forceinline__ bool if4_single_term(const uint32_t* w, const uint32_t* w7, float amax, uint32_t sc,
+                                                float s_g, float s7) {
+  uint32_t c, k;
+  if (!single_nonzero_code(w, w7, c, k)) return false;
+  const float d = e4m3_value(sc);
+  const float te = max_term(amax, e2m1_magnitude(c), d, s_g);
+  const float ti = max_term(amax, (float)k, d, s7);
+  return ti >= te;
+}
+
 // IF4: the same test for the E2M1 candidate (D, A) against the INT4 one (D7, A7).  The INT4
 // reconstruction fl(fl(k*d)*s7), its step D7 = fl(d*s7) and y = fl(v*fl(1/D7)) take the rounded
 // steps of the E2M1 ones (k*d exact, then one product with a per-tensor factor), so the bound

@@ -260,10 +260,19 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
         }
         const bool eligible = DR7.y != 0.0f;
         bool pick;
-        const bool undecided = if4_undecided(am, amax, D, DR7.x, A, A7, eligible, pick);
-        if (__any_sync(0xFFFFFFFFu, undecided)) {  // warp-uniform call: the exact sums shuffle
-          const uint32_t lower = if4_exact<T, G>(xb, c, valid, w[0], w[W - 1], sc, ns.s_g, DR7.y, s7, p.zero);
-          pick = eligible && lower != 0u;
+        bool undecided = if4_undecided(am, amax, D, DR7.x, A, A7, eligible, pick);
+        if (__any_sync(0xFFFFFFFFu, undecided)) {  // rare: warp-uniform, so the common path is unchanged
+          if constexpr (G == 1) {
+            if (undecided && eligible && ns.s_g > 0.0f && s7 > 0.0f && am < 0x7F800000u &&
+                if4_single_term(w, w7, amax, sc, ns.s_g, s7)) {
+              undecided = false;
+              pick = false;
+            }
+          }
+          if (__any_sync(0xFFFFFFFFu, undecided)) {  // the exact sums shuffle: the whole warp calls
+            const uint32_t lower = if4_exact<T, G>(xb, c, valid, w[0], w[W - 1], sc, ns.s_g, DR7.y, s7, p.zero);
+            pick = eligible && lower != 0u;
+          }
         }
         if (pick) {
           sc |= 0x80u;
@@ -307,9 +316,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
           A4 += __shfl_xor_sync(0xFFFFFFFFu, A4, o);
         }
         bool pick4;
-        const bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, sc6, sc4, pick4);
-        if (__any_sync(0xFFFFFFFFu, undecided))  // warp-uniform call: the exact sums shuffle
-          pick4 = four_six_exact<T, G>(xb, c, valid, w[0], w[W - 1], w4[0], w4[W - 1], sc6, sc4, ns.s_g, p.zero) != 0u;
+        bool undecided = four_six_undecided(am, amax, D6, D4, A6, A4, sc6, sc4, pick4);
+        if (__any_sync(0xFFFFFFFFu, undecided)) {  // rare: warp-uniform, so the common path is unchanged
+          if constexpr (G == 1) {
+            // the outlier-block shape: one nonzero code per candidate, decided from one term
+            if (undecided && ns.s_g > 0.0f && am < 0x7F800000u && four_six_single_term(w, w4, amax, sc6, sc4, ns.s_g)) {
+              undecided = false;
+              pick4 = false;
+            }
+          }
+          if (__any_sync(0xFFFFFFFFu, undecided))  // the exact sums shuffle: the whole warp calls
+            pick4 = four_six_exact<T, G>(xb, c, valid, w[0], w[W - 1], w4[0], w4[W - 1], sc6, sc4, ns.s_g, p.zero) != 0u;
+        }
         sc = sc6;
         if (pick4) {
           sc = sc4;
