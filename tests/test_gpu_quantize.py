@@ -567,3 +567,44 @@ def test_two_pass_workspace_needs_no_initialisation(cuda, mode):
         assert np.array_equal(npy(q), qo)
         assert np.array_equal(npy(s), so.ravel())
         compare_counts(c, co, x, spec, 16)
+
+
+def test_four_six_decided_by_upper_bytes_of_each_word(cuda):
+    """The four-over-six estimate decodes each packed word in registers, and bytes 2-3 of a word (values
+    4-7 and 12-15 of a block) are the ones that once decoded to zeros when the word came straight
+    from the encoder.  Blocks whose estimated choice would flip if those values decoded to zero (and
+    that the estimate decides by at least four times its margin) are picked from a seeded N(0,1)
+    pool; both choices occur among them.  The GPU must choose exactly as the oracle does: nibbles,
+    scale bytes and the 4-count.  A caller-fixed global scale (the pool's) keeps the scales the
+    selection assumed."""
+    rng = np.random.default_rng(41)
+    pool = torch.from_numpy(rng.standard_normal((200000, 16), dtype=np.float32)).to(torch.bfloat16)
+    x = pool.float().numpy()
+    s_g = np.float32(np.float32(np.abs(x).max()) / np.float32(1536.0))
+    lat = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+
+    def rne(y):  # E2M1 round to nearest, ties to the even code (the selection's own model)
+        a = np.minimum(np.abs(y.astype(np.float64)), 6.0)
+        i = np.clip(np.searchsorted(lat, a), 1, 7)
+        lo, hi = lat[i - 1], lat[i]
+        return np.where((a - lo > hi - a) | ((a - lo == hi - a) & (i % 2 == 0)), hi, lo) * (a > 0)
+
+    amax = np.abs(x).max(1)
+    upper = np.zeros(16, bool)
+    upper[4:8] = upper[12:16] = True
+    est, est0 = {}, {}
+    for T in (6, 4):
+        d = torch.from_numpy(amax * (np.float32(1) / (np.float32(T) * s_g))).to(torch.float8_e4m3fn).float().numpy()
+        D = (d * s_g).astype(np.float32)
+        y = np.abs(x * (np.float32(1) / D)[:, None]).astype(np.float32)
+        r2 = (rne(y) - y) ** 2
+        est[T] = D.astype(np.float64) ** 2 * r2.sum(1)
+        est0[T] = D.astype(np.float64) ** 2 * np.where(upper, y.astype(np.float64) ** 2, r2).sum(1)
+    margin = 2.0 ** -17 * (1.02 * amax.astype(np.float64) ** 2 + 2 * (est[6] + est[4]))
+    pick = (np.abs(est[4] - est[6]) > 4 * margin) & (np.sign(est0[4] - est0[6]) != np.sign(est[4] - est[6]))
+    blocks = pool[torch.from_numpy(np.nonzero(pick)[0][:8192])]
+    assert blocks.shape[0] == 8192
+    xs = blocks.reshape(256, 512)
+    q, s, g, qo, so, go = run_nv(xs, cuda, four_six=True, global_in=float(s_g))
+    co = O.nvfp4_quantize(f32(xs), four_six=True, global_in=float(s_g))[3]
+    assert 1000 < co["blocks_four"] < 7000  # both choices are exercised
