@@ -372,7 +372,7 @@ def cpu_baseline(x_cpu, rows=4096, max_workers=64):
 # ---------------------------------------------------------------------------------------------
 def secondary(args, dev, flush, td, pk):
     out = []
-    K = max(10, args.steps // 4)
+    K = max(20, args.steps // 4)
     W = args.warmup
     # config 1: MXFP4 quantise + dequantise, 256 x 512 fp32
     x1 = synth.mx_small().to(dev)
