@@ -165,8 +165,8 @@ def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, se
 def nvfp4_quantize_noalloc(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
                            layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
                            stream=None, if4: bool = False, out=None):
-    """nvfp4_quantize for callers that cannot hand the library a device workspace: the amax word
-    between the two passes lives in a fixed area of the library's own device memory.  Calls that
+    """nvfp4_quantize for callers that cannot hand the library a device workspace: the amax pass's
+    per-CTA partial maxima live in a fixed area of the library's own device memory.  Calls that
     overlap on the GPU share that area and must be serialised.  `out` = (q, scales, s_g, counts)
     preallocated by the caller (else allocated here).  Returns (q, scales, s_g, counts)."""
     _need_cuda(x, global_in)

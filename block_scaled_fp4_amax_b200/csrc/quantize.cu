@@ -364,8 +364,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QuantParams p) {
 // ---------------------------------------------------------------------------------------------
 // Tensor amax (NVFP4 global scale, first pass): max |x| over the whole tensor as an integer max
 // of the magnitude bits (monotone for non-negative floats).  Each CTA stores its maximum in its own
-// slot, so the word needs no zeroing before the pass (a memset on the stream costs about as much
-// as 7% of this kernel); the quantise pass reduces the slots.  Loads keep their L2 lines so the
+// slot, so nothing needs zeroing before the pass (a memset on the stream costs about as much as 7%
+// of this kernel); the quantise pass reduces the slots.  Loads keep their L2 lines so the
 // second pass, walking the tiles in reverse, starts on resident data.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const void* x, long long n_chunks,
