@@ -538,7 +538,9 @@ def secondary(args, dev, flush, td, pk):
     Aq, Bq = st["ab"]
     ms = timed(lambda: fp4.fp4_block_gemm(fp4.MXFP4, Aq[0], Aq[1], Bq[0], Bq[1], out=C, workspace=gws), K, W, flush, td)
     t_g = statistics.median(ms)
-    ms = timed(lambda: fp4.mx_quantize(w, layout=fp4.MMA_TILED), K, W, flush, td)
+    # the weight quantise launch into preallocated outputs (no allocation in the timed region)
+    wout = (torch.empty_like(Bq[0]), torch.empty_like(Bq[1]), None, torch.empty_like(Bq[2]))
+    ms = timed(lambda: fp4.mx_quantize(w, layout=fp4.MMA_TILED, out=wout), K, W, flush, td)
     t_w = statistics.median(ms)
     flop = 2 * 4096 * 8192 * 28672
     qbytes = w.numel() * (2 + 0.5 + 1 / 32)

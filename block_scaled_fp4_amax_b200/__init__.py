@@ -128,13 +128,31 @@ def _alloc_outputs(rows, cols, block, device):
     return q, s, c
 
 
+def _outputs(out, rows, cols, block, device, with_scale):
+    """The quantisers' outputs: the caller's `out` (checked: contiguous, on `device`, the sizes the
+    call writes) or new tensors.  Returns (q, scales, s_g or None, counts)."""
+    if out is None:
+        q, s, c = _alloc_outputs(rows, cols, block, device)
+        g = torch.empty(1, dtype=torch.float32, device=device) if with_scale else None
+        return q, s, g, c
+    q, s, g, c = out
+    want = [(q, rows * cols // 2, torch.uint8), (s, rows * cols // block, torch.uint8), (c, 4, torch.int64)]
+    if with_scale:
+        want.append((g, 1, torch.float32))
+    for t, n, dt in want:
+        if t is None or t.device != device or t.dtype != dt or t.numel() != n or not t.is_contiguous():
+            raise ValueError(f"out: expected a contiguous {dt} tensor of {n} elements on {device}")
+    return q, s, (g if with_scale else None), c
+
+
 def mx_quantize(x: torch.Tensor, policy: int = OCP_FLOOR, round: int = RNE, seed: int = 0,
-                layout: int = ROWMAJOR, block: int = 32, stream=None):
+                layout: int = ROWMAJOR, block: int = 32, stream=None, out=None):
     """MXFP4: returns (q uint8 [rows, cols/2], scales uint8 [rows*cols/32] in `layout`,
-    counts int64[4] on device: underflow, saturation, nonfinite, blocks_four)."""
+    counts int64[4] on device: underflow, saturation, nonfinite, blocks_four).  `out` = (q, scales,
+    None, counts) preallocated by the caller (else allocated here)."""
     _need_cuda(x)
     rows, cols = x.shape
-    q, s, c = _alloc_outputs(rows, cols, 32, x.device)
+    q, s, _, c = _outputs(out, rows, cols, 32, x.device, False)
     _check(lib().mx_quantize(_ptr(x), _dtype_code(x), rows, cols, block, policy, round, seed, layout,
                              _ptr(q), _ptr(s), _ptr(c), _stream(stream)))
     return q, s, c
@@ -148,13 +166,12 @@ def _nv_mode(four_six: bool, if4: bool) -> int:
 
 def nvfp4_quantize(x: torch.Tensor, round: int = RNE, four_six: bool = False, seed: int = 0,
                    layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, block: int = 16,
-                   stream=None, workspace: torch.Tensor | None = None, if4: bool = False):
+                   stream=None, workspace: torch.Tensor | None = None, if4: bool = False, out=None):
     """NVFP4 (with `if4`, IF4: E2M1 or INT4 per block, flagged in scale bit 7): returns
-    (q, scales, s_g float32[1] on device, counts)."""
+    (q, scales, s_g float32[1] on device, counts); `out` = those four preallocated by the caller."""
     _need_cuda(x, global_in)
     rows, cols = x.shape
-    q, s, c = _alloc_outputs(rows, cols, 16, x.device)
-    g = torch.empty(1, dtype=torch.float32, device=x.device)
+    q, s, g, c = _outputs(out, rows, cols, 16, x.device, True)
     ws = workspace if workspace is not None else _workspace(OP_NVFP4_QUANTIZE, x.device, rows, cols)
     _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, round, _nv_mode(four_six, if4), seed,
                                 layout, _ptr(global_in), _ptr(g), _ptr(q), _ptr(s), _ptr(c), _ptr(ws),
@@ -194,16 +211,15 @@ def _fwht_op(fmt, global_in, want_rotated):
 def fwht_quantize(x: torch.Tensor, fmt: int = NVFP4, round: int = RNE, four_six: bool = False, seed: int = 0,
                   layout: int = ROWMAJOR, global_in: torch.Tensor | None = None, want_rotated: bool = False,
                   block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
-                  signs: torch.Tensor | None = None, if4: bool = False):
+                  signs: torch.Tensor | None = None, if4: bool = False, out=None):
     """Walsh-Hadamard rotation of each row fused with the quantiser of `fmt`; with `signs` (device
     int32/uint32 [d/32], bit i negates channel i first) the randomised rotation c*H*D; with `if4`
-    (NVFP4, round to nearest) IF4 blocks.
+    (NVFP4, round to nearest) IF4 blocks.  `out` = (q, scales, s_g or None, counts) preallocated.
     Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
     _need_cuda(x, global_in, signs)
     rows, d = x.shape
     B = block if block is not None else (32 if fmt == MXFP4 else 16)
-    q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, x.device)
-    g = torch.empty(1, dtype=torch.float32, device=x.device) if fmt == NVFP4 else None
+    q, s, g, c = _outputs(out, rows, d, 16 if fmt == NVFP4 else 32, x.device, fmt == NVFP4)
     rot = torch.empty((rows, d), dtype=torch.float32, device=x.device) if want_rotated else None
     ws = workspace if workspace is not None else _workspace(_fwht_op(fmt, global_in, want_rotated), x.device, rows, d)
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):
@@ -218,17 +234,16 @@ def swiglu_fwht_quantize(g: torch.Tensor, u: torch.Tensor, fmt: int = NVFP4, rou
                          four_six: bool = False, seed: int = 0, layout: int = ROWMAJOR,
                          global_in: torch.Tensor | None = None, want_rotated: bool = False,
                          block: int | None = None, stream=None, workspace: torch.Tensor | None = None,
-                         signs: torch.Tensor | None = None, if4: bool = False):
+                         signs: torch.Tensor | None = None, if4: bool = False, out=None):
     """fl(SiLU(g) * u) in fp32 (never stored), rotated (randomised with `signs`) and quantised to `fmt`
-    (IF4 blocks with `if4`).
+    (IF4 blocks with `if4`).  `out` = (q, scales, s_g or None, counts) preallocated.
     g, u: bf16 [rows, d].  Returns (q, scales, s_g (NVFP4; None for MXFP4), counts, rotated fp32 or None)."""
     _need_cuda(g, u, global_in, signs)
     if g.shape != u.shape:
         raise ValueError("g and u must have the same shape")
     rows, d = g.shape
     B = block if block is not None else (32 if fmt == MXFP4 else 16)
-    q, s, c = _alloc_outputs(rows, d, 16 if fmt == NVFP4 else 32, g.device)
-    gs = torch.empty(1, dtype=torch.float32, device=g.device) if fmt == NVFP4 else None
+    q, s, gs, c = _outputs(out, rows, d, 16 if fmt == NVFP4 else 32, g.device, fmt == NVFP4)
     rot = torch.empty((rows, d), dtype=torch.float32, device=g.device) if want_rotated else None
     ws = workspace if workspace is not None else _workspace(_fwht_op(fmt, global_in, want_rotated), g.device, rows, d)
     if signs is not None and (signs.numel() != d // 32 or signs.element_size() != 4):

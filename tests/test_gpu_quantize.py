@@ -608,3 +608,26 @@ def test_four_six_decided_by_upper_bytes_of_each_word(cuda):
     q, s, g, qo, so, go = run_nv(xs, cuda, four_six=True, global_in=float(s_g))
     co = O.nvfp4_quantize(f32(xs), four_six=True, global_in=float(s_g))[3]
     assert 1000 < co["blocks_four"] < 7000  # both choices are exercised
+
+
+def test_quantisers_write_into_preallocated_outputs(cuda):
+    """`out=` hands the quantisers the caller's buffers: the bytes match the allocating call, and a
+    buffer of the wrong size is refused before any launch."""
+    x = synth.nv_outliers(64, 2048, seed=31).to(cuda)
+    ref = fp4.mx_quantize(x)
+    out = (torch.empty_like(ref[0]), torch.empty_like(ref[1]), None, torch.empty_like(ref[2]))
+    got = fp4.mx_quantize(x, out=out)
+    assert got[0].data_ptr() == out[0].data_ptr()
+    assert all(torch.equal(a, b) for a, b in zip(ref, got))
+    ref = fp4.nvfp4_quantize(x, four_six=True)
+    out = tuple(torch.empty_like(t) for t in ref)
+    got = fp4.nvfp4_quantize(x, four_six=True, out=out)
+    assert got[1].data_ptr() == out[1].data_ptr()
+    assert all(torch.equal(a, b) for a, b in zip(ref, got))
+    ref = fp4.fwht_quantize(x, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=3)
+    out = tuple(torch.empty_like(t) for t in ref[:4])
+    got = fp4.fwht_quantize(x, fmt=fp4.NVFP4, round=fp4.STOCHASTIC, seed=3, out=out)
+    assert all(torch.equal(a, b) for a, b in zip(ref[:4], got[:4]))
+    bad = (torch.empty(10, dtype=torch.uint8, device=cuda), out[1], out[2], out[3])
+    with pytest.raises(ValueError):
+        fp4.nvfp4_quantize(x, out=bad)
